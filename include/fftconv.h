@@ -1,0 +1,169 @@
+/*
+ * fftconv.h -- C ABI of the B200 (sm_100a) exact causal long-convolution
+ * library.
+ *
+ * Operation (page "FlashFFTConv: Efficient Convolutions for Long Sequences
+ * with Tensor Cores", summary paragraph, "Approach" and "Key results"): for
+ * every batch row b and channel h,
+ *
+ *     y[b,h,t] = v[b,h,t] * sum_{s=0}^{min(t, L-1)} k[h,s] * u[b,h,t-s] * w[b,h,t-s]
+ *
+ * for 0 <= t < N, computed as irfft(rfft(u*w, 2N) * K_f, 2N)[:N] with
+ * K_f = rfft(k zero-padded to 2N).  The gates w and v are optional ("gated
+ * convolution", Key results); a filter shorter than the sequence (L < N) is
+ * the "partial convolution" and a block mask on K_f the "frequency-sparse
+ * convolution" (Approach; measured-effects table, 75% / 79% sparsity rows).
+ * The length-2N transform is evaluated as a product of small DFT factors (a
+ * Monarch decomposition, Approach) inside the library's kernels.
+ *
+ * Conventions shared by every entry point:
+ *   - Every data pointer is a DEVICE pointer unless its name ends in _host.
+ *     The caller owns and allocates every buffer passed in; the library owns
+ *     only what a plan allocates (its tables and its workspace).
+ *   - Tensors are row-major with the sequence index fastest: u, w, v, y are
+ *     [B, H, N]; k is [H, L].  Their element type is the plan dtype.
+ *   - Device pointers must be 16-byte aligned.
+ *   - All calls return an fftconv_status_t (0 = success).  On failure nothing
+ *     has been launched and fftconv_last_error() describes the cause
+ *     (thread-local).  Nothing throws across the ABI.
+ *   - Calls taking a cudaStream_t are asynchronous on that stream, allocate
+ *     no memory and do not synchronise (except where noted).
+ */
+#ifndef FFTCONV_H_
+#define FFTCONV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FFTCONV_API __attribute__((visibility("default")))
+#else
+#define FFTCONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque stream handle; identical to cudaStream_t (NULL = legacy default). */
+typedef struct CUstream_st* fftconv_stream_t;
+
+typedef struct fftconv_plan_s* fftconv_plan_t;
+
+typedef enum {
+    FFTCONV_F32 = 0,   /* float                    */
+    FFTCONV_F16 = 1,   /* IEEE binary16 (__half)   */
+    FFTCONV_BF16 = 2   /* bfloat16 (__nv_bfloat16) */
+} fftconv_dtype_t;
+
+typedef enum {
+    FFTCONV_OK = 0,
+    FFTCONV_ERR_INVALID_ARG = -1,   /* null/negative/mismatched argument      */
+    FFTCONV_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. N=3000) */
+    FFTCONV_ERR_ALIGNMENT = -3,     /* pointer not 16-byte aligned            */
+    FFTCONV_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed   */
+    FFTCONV_ERR_OOM = -5,           /* plan allocation failed                 */
+    FFTCONV_ERR_TIMEOUT = -6        /* a bounded device wait gave up          */
+} fftconv_status_t;
+
+/* Kernel family a plan uses (fftconv_plan_path). */
+typedef enum {
+    FFTCONV_PATH_SIMT_FUSED = 1,    /* fp32 FFT in shared memory, one kernel  */
+    FFTCONV_PATH_SIMT_STAGED = 2,   /* fp32, column/row passes via workspace  */
+    FFTCONV_PATH_TC_FUSED = 3       /* tcgen05 tensor-core Monarch, one kernel */
+} fftconv_path_t;
+
+/* Create a plan for sequences of length N (a power of two, 256 <= N <= 2^22)
+ * and H channels with full-length filters (L = N).  `order` selects the
+ * decomposition: 0 = automatic; 2 or 3 = fused on-chip kernel (N <= 8192);
+ * 4 = the staged path with one workspace round trip (any N); other values are
+ * FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
+ * (a few hundred KB) and its workspace (staged path only) on the current
+ * device.  *out receives the plan, or NULL on failure. */
+FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
+                        fftconv_dtype_t dtype, int order);
+
+/* As fftconv_plan_create with a filter of length L (1 <= L <= N): the
+ * partial convolution, defined as the convolution with k zero-padded to N. */
+FFTCONV_API int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H,
+                           fftconv_dtype_t dtype, int order, int64_t L);
+
+/* Release a plan and its device memory (synchronises the device first).
+ * NULL is accepted. */
+FFTCONV_API int fftconv_plan_destroy(fftconv_plan_t plan);
+
+/* Bytes of the opaque transformed filter K_f for this plan (0 for NULL). */
+FFTCONV_API size_t fftconv_filter_bytes(fftconv_plan_t plan);
+
+/* Bytes of the plan's own device workspace (0 on the fused paths). */
+FFTCONV_API size_t fftconv_workspace_bytes(fftconv_plan_t plan);
+
+/* The kernel family this plan dispatches to (an fftconv_path_t), or <0. */
+FFTCONV_API int fftconv_plan_path(fftconv_plan_t plan);
+
+/* K_f <- rfft(k zero-padded to 2N) in the plan's internal (digit-permuted)
+ * layout with the 1/(2N) normalisation folded in.  k: [H, L] device, plan
+ * dtype.  K_f: device, fftconv_filter_bytes(plan) bytes, written completely.
+ * Run once per filter; the result is reused by every forward call. */
+FFTCONV_API int fftconv_filter_precompute(fftconv_plan_t plan, const void* k, void* K_f,
+                              fftconv_stream_t stream);
+
+/* y <- causal convolution of u (gated by w and v) with the filter K_f.
+ *   u, y       : [B, H, N] device, plan dtype.  y must not overlap u, w or v.
+ *   K_f        : from fftconv_filter_precompute on this plan.
+ *   B, H, N    : B >= 0; H and N must equal the plan's.  B == 0 is a no-op.
+ *   w, v       : [B, H, N] device or NULL (absent gate = all ones).
+ *   block_mask : NULL, or [mask_h, N/32] device bytes; block m covers rfft
+ *                bins [32m, 32m+32) of each channel's filter (the last block
+ *                also holds the Nyquist bin N); 0 zeroes those bins (and their
+ *                Hermitian mirrors), anything else keeps them.
+ *   mask_h     : 1 (one mask row for all channels) or H; ignored when
+ *                block_mask is NULL.
+ * Asynchronous on `stream`; allocates nothing.  Calls on the staged path
+ * share the plan's workspace and must be serialised on one stream. */
+FFTCONV_API int fftconv_forward(fftconv_plan_t plan, const void* u, const void* K_f, void* y,
+                    int64_t B, int64_t H, int64_t N, const void* w, const void* v,
+                    const uint8_t* block_mask, int64_t mask_h,
+                    fftconv_stream_t stream);
+
+/* Device bytes fftconv_forward_host needs as staging for B rows with the
+ * given gates and mask present (nonzero = present). */
+FFTCONV_API size_t fftconv_forward_host_staging_bytes(fftconv_plan_t plan, int64_t B, int has_w,
+                                          int has_v, int has_mask, int64_t mask_h);
+
+/* fftconv_forward on HOST buffers: copies u_host (and w_host, v_host,
+ * mask_host) into the caller's device staging buffer, runs the forward pass
+ * and copies y back into y_host, all asynchronously on `stream` (page-locked
+ * host memory makes the copies asynchronous; pageable memory works but
+ * blocks).  K_f stays a device pointer.  staging: device, at least
+ * fftconv_forward_host_staging_bytes(...) bytes, 256-byte aligned. */
+FFTCONV_API int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, const void* K_f,
+                         void* y_host, int64_t B, int64_t H, int64_t N,
+                         const void* w_host, const void* v_host,
+                         const uint8_t* mask_host, int64_t mask_h, void* staging,
+                         size_t staging_bytes, fftconv_stream_t stream);
+
+/* Test hook: export K_f in natural order as out[h, f, 0..1] = (Re, Im) of
+ * rfft(k)[f] for f in [0, N] (normalisation undone), fp32, device. */
+FFTCONV_API int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out,
+                           fftconv_stream_t stream);
+
+/* Synchronise `stream` and return the plan's device status word:
+ * FFTCONV_OK, or FFTCONV_ERR_TIMEOUT if a bounded device-side wait gave up
+ * since the last call (the word is reset to OK by this call). */
+FFTCONV_API int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream);
+
+/* Static description of a status code. */
+FFTCONV_API const char* fftconv_status_string(int status);
+
+/* Detail of the last failure on the calling thread ("" if none). */
+FFTCONV_API const char* fftconv_last_error(void);
+
+/* Library version string. */
+FFTCONV_API const char* fftconv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FFTCONV_H_ */

@@ -1,0 +1,365 @@
+// api.cu -- the C ABI (include/fftconv.h): plan creation, argument
+// validation, host-side fp64 twiddle tables and dispatch to the kernels.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/fftconv.h"
+#include "internal.h"
+
+using namespace fftconv;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(FFTCONV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ilog2(int64_t v) {
+    int l = 0;
+    while ((int64_t(1) << l) < v) ++l;
+    return l;
+}
+
+size_t dtype_size(int dt) { return dt == kF32 ? 4 : 2; }
+
+// exp(-2 pi i e / L) for e < count (scaled by `mult`: exp(-2 pi i e*mult / L)),
+// evaluated in double with the angle reduced exactly, then rounded to fp32.
+std::vector<float2> host_twiddles(int64_t L, int64_t count, int64_t mult) {
+    std::vector<float2> t((size_t)count);
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int64_t e = 0; e < count; ++e) {
+        const int64_t r = (e * mult) % L;
+        const double a = two_pi * (double)r / (double)L;
+        t[(size_t)e] = make_float2((float)std::cos(a), (float)-std::sin(a));
+    }
+    return t;
+}
+
+cudaError_t upload(float2** dst, const std::vector<float2>& v) {
+    cudaError_t e = cudaMalloc((void**)dst, v.size() * sizeof(float2));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpy(*dst, v.data(), v.size() * sizeof(float2), cudaMemcpyHostToDevice);
+}
+
+void free_plan(Plan* p) {
+    if (!p) return;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(p->device);
+    if (p->tc) tc_plan_free(*p);
+    cudaFree(p->tw);
+    cudaFree(p->twLo);
+    cudaFree(p->twHi);
+    cudaFree(p->work);
+    cudaFree(p->status);
+    cudaSetDevice(cur);
+    delete p;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || !na || !nb) return false;
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+}  // namespace
+
+struct fftconv_plan_s {
+    Plan p;
+};
+
+extern "C" {
+
+const char* fftconv_version(void) { return "fftconv-b200 0.1"; }
+
+const char* fftconv_status_string(int status) {
+    switch (status) {
+        case FFTCONV_OK: return "ok";
+        case FFTCONV_ERR_INVALID_ARG: return "invalid argument";
+        case FFTCONV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case FFTCONV_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case FFTCONV_ERR_CUDA: return "CUDA error";
+        case FFTCONV_ERR_OOM: return "out of device memory";
+        case FFTCONV_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* fftconv_last_error(void) { return g_last_error.c_str(); }
+
+int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dtype_t dtype,
+                           int order, int64_t L) {
+    g_last_error.clear();
+    if (!out) return fail(FFTCONV_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (N <= 0 || H <= 0) return fail(FFTCONV_ERR_INVALID_ARG, "N=%lld and H=%lld must be positive",
+                                      (long long)N, (long long)H);
+    if (dtype != FFTCONV_F32 && dtype != FFTCONV_F16 && dtype != FFTCONV_BF16)
+        return fail(FFTCONV_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (L <= 0 || L > N) return fail(FFTCONV_ERR_INVALID_ARG, "filter length L=%lld not in [1, N]", (long long)L);
+    if ((N & (N - 1)) != 0) return fail(FFTCONV_ERR_UNSUPPORTED, "N=%lld is not a power of two", (long long)N);
+    if (N < 256 || N > (int64_t(1) << 22))
+        return fail(FFTCONV_ERR_UNSUPPORTED, "N=%lld outside [256, 2^22]", (long long)N);
+    if (order < 0 || order > 4) return fail(FFTCONV_ERR_UNSUPPORTED, "order %d not in {0,1,2,3,4}", order);
+    if (H > (int64_t(1) << 24)) return fail(FFTCONV_ERR_UNSUPPORTED, "H=%lld too large", (long long)H);
+
+    Plan* p = new (std::nothrow) Plan();
+    if (!p) return fail(FFTCONV_ERR_OOM, "host allocation failed");
+    p->N = N; p->H = H; p->L = L; p->M = 2 * N; p->logM = ilog2(2 * N);
+    p->dtype = (int)dtype; p->order = order;
+    cudaGetDevice(&p->device);
+
+    const bool tc_ok = tc_supported(N, L, (int)dtype);
+    if (order == 4 || (order == 0 && !tc_ok && !simt_fused_supported(p->logM))) {
+        p->path = kPathSimtStaged;
+    } else if (order == 1) {
+        if (!simt_fused_supported(p->logM)) { delete p; return fail(FFTCONV_ERR_UNSUPPORTED, "order 1 needs N <= 8192"); }
+        p->path = kPathSimtFused;
+    } else if (tc_ok) {
+        p->path = kPathTcFused;
+    } else if (simt_fused_supported(p->logM)) {
+        p->path = kPathSimtFused;
+    } else {
+        delete p;
+        return fail(FFTCONV_ERR_UNSUPPORTED, "order %d: no fused kernel for N=%lld; use order 4 or 0", order,
+                    (long long)N);
+    }
+
+    cudaError_t e = cudaMalloc((void**)&p->status, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(p->status, 0, sizeof(int));
+    if (e != cudaSuccess) { free_plan(p); return e == cudaErrorMemoryAllocation ? fail(FFTCONV_ERR_OOM, "status word") : cuda_fail(e, "plan status"); }
+
+    if (p->path == kPathSimtFused) {
+        p->logTab = p->logM;
+        e = upload(&p->tw, host_twiddles(p->M, p->M, 1));
+        p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
+    } else if (p->path == kPathSimtStaged) {
+        p->logC = p->logM - 1 < 14 ? p->logM - 1 : 14;
+        p->logR = p->logM - p->logC;
+        p->logTab = p->logC;
+        const int64_t C = int64_t(1) << p->logC;
+        e = upload(&p->tw, host_twiddles(C, C, 1));
+        p->twSplit = (p->logM + 1) / 2;
+        if (e == cudaSuccess) e = upload(&p->twLo, host_twiddles(p->M, int64_t(1) << p->twSplit, 1));
+        if (e == cudaSuccess)
+            e = upload(&p->twHi, host_twiddles(p->M, p->M >> p->twSplit, int64_t(1) << p->twSplit));
+        // workspace: a chunk of pairs of about 64 MB (L2-sized), at least one
+        const size_t per_pair = (size_t)p->M * sizeof(float2);
+        p->chunkPairs = (int64_t)((size_t(64) << 20) / per_pair);
+        if (p->chunkPairs < 1) p->chunkPairs = 1;
+        p->workBytes = per_pair * (size_t)p->chunkPairs;
+        if (e == cudaSuccess) e = cudaMalloc((void**)&p->work, p->workBytes);
+        p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
+    } else {
+        e = tc_plan_init(*p);
+        p->filter_bytes = tc_filter_bytes(*p);
+    }
+    if (e != cudaSuccess) {
+        free_plan(p);
+        if (e == cudaErrorMemoryAllocation) return fail(FFTCONV_ERR_OOM, "plan tables/workspace");
+        return cuda_fail(e, "plan tables");
+    }
+    fftconv_plan_s* h = new (std::nothrow) fftconv_plan_s();
+    if (!h) { free_plan(p); return fail(FFTCONV_ERR_OOM, "host allocation failed"); }
+    h->p = *p;
+    delete p;   // shallow copy moved into the handle (device pointers now owned by h)
+    *out = h;
+    return FFTCONV_OK;
+}
+
+int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dtype_t dtype, int order) {
+    return fftconv_plan_create_ex(out, N, H, dtype, order, N);
+}
+
+int fftconv_plan_destroy(fftconv_plan_t plan) {
+    g_last_error.clear();
+    if (!plan) return FFTCONV_OK;
+    cudaDeviceSynchronize();
+    Plan* p = new (std::nothrow) Plan(plan->p);
+    if (p) free_plan(p);
+    delete plan;
+    return FFTCONV_OK;
+}
+
+size_t fftconv_filter_bytes(fftconv_plan_t plan) { return plan ? plan->p.filter_bytes : 0; }
+
+size_t fftconv_workspace_bytes(fftconv_plan_t plan) { return plan ? plan->p.workBytes : 0; }
+
+int fftconv_plan_path(fftconv_plan_t plan) {
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    return plan->p.path;
+}
+
+int fftconv_filter_precompute(fftconv_plan_t plan, const void* k, void* K_f, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan || !k || !K_f) return fail(FFTCONV_ERR_INVALID_ARG, "plan, k and K_f must be non-NULL");
+    if (!aligned16(k) || !aligned16(K_f)) return fail(FFTCONV_ERR_ALIGNMENT, "k or K_f not 16-byte aligned");
+    const Plan& p = plan->p;
+    if (ranges_overlap(k, (size_t)(p.H * p.L) * dtype_size(p.dtype), K_f, p.filter_bytes))
+        return fail(FFTCONV_ERR_INVALID_ARG, "k and K_f overlap");
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (p.path) {
+        case kPathSimtFused: e = simt_fused_precompute(p, k, K_f, s); break;
+        case kPathSimtStaged: e = simt_staged_precompute(p, k, K_f, s); break;
+        default: e = tc_precompute(p, k, K_f, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "filter precompute launch");
+    return FFTCONV_OK;
+}
+
+static int validate_forward(const Plan& p, const void* u, const void* K_f, void* y, int64_t B,
+                            int64_t H, int64_t N, const void* w, const void* v, const uint8_t* mask,
+                            int64_t mask_h) {
+    if (B < 0) return fail(FFTCONV_ERR_INVALID_ARG, "B=%lld is negative", (long long)B);
+    if (H != p.H || N != p.N)
+        return fail(FFTCONV_ERR_INVALID_ARG, "H=%lld N=%lld do not match the plan (H=%lld N=%lld)",
+                    (long long)H, (long long)N, (long long)p.H, (long long)p.N);
+    if (B == 0) return FFTCONV_OK;
+    if (!u || !K_f || !y) return fail(FFTCONV_ERR_INVALID_ARG, "u, K_f and y must be non-NULL");
+    if (!aligned16(u) || !aligned16(K_f) || !aligned16(y) || !aligned16(w) || !aligned16(v))
+        return fail(FFTCONV_ERR_ALIGNMENT, "u, K_f, y, w and v must be 16-byte aligned");
+    if (mask && mask_h != 1 && mask_h != H)
+        return fail(FFTCONV_ERR_INVALID_ARG, "mask_h=%lld must be 1 or H=%lld", (long long)mask_h, (long long)H);
+    if (mask && N < 32) return fail(FFTCONV_ERR_UNSUPPORTED, "block mask needs N >= 32");
+    if (B > (int64_t(1) << 30) / 1) {
+        if ((double)B * (double)H > 4.0e9) return fail(FFTCONV_ERR_UNSUPPORTED, "B*H too large");
+    }
+    const size_t bytes = (size_t)B * (size_t)H * (size_t)N * dtype_size(p.dtype);
+    if (ranges_overlap(y, bytes, u, bytes) || ranges_overlap(y, bytes, w, bytes) ||
+        ranges_overlap(y, bytes, v, bytes) || ranges_overlap(y, bytes, K_f, p.filter_bytes))
+        return fail(FFTCONV_ERR_INVALID_ARG, "y overlaps an input");
+    if ((double)H * (double)((B + 1) / 2) > 2147483647.0)
+        return fail(FFTCONV_ERR_UNSUPPORTED, "too many sequence pairs for one launch");
+    return FFTCONV_OK;
+}
+
+static int run_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s) {
+    cudaError_t e;
+    switch (p.path) {
+        case kPathSimtFused: e = simt_fused_forward(p, a, s); break;
+        case kPathSimtStaged: e = simt_staged_forward(p, a, s); break;
+        default: e = tc_forward(p, a, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return FFTCONV_OK;
+}
+
+int fftconv_forward(fftconv_plan_t plan, const void* u, const void* K_f, void* y, int64_t B, int64_t H,
+                    int64_t N, const void* w, const void* v, const uint8_t* block_mask, int64_t mask_h,
+                    fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    const Plan& p = plan->p;
+    int rc = validate_forward(p, u, K_f, y, B, H, N, w, v, block_mask, mask_h);
+    if (rc != FFTCONV_OK || B == 0) return rc;
+    ForwardArgs a{u, w, v, y, K_f, block_mask, block_mask ? mask_h : 0, B};
+    return run_forward(p, a, (cudaStream_t)stream);
+}
+
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t fftconv_forward_host_staging_bytes(fftconv_plan_t plan, int64_t B, int has_w, int has_v, int has_mask,
+                                          int64_t mask_h) {
+    if (!plan || B < 0) return 0;
+    const Plan& p = plan->p;
+    const size_t t = round256((size_t)B * (size_t)p.H * (size_t)p.N * dtype_size(p.dtype));
+    size_t total = 2 * t;                          // u, y
+    if (has_w) total += t;
+    if (has_v) total += t;
+    if (has_mask) total += round256((size_t)(mask_h > 0 ? mask_h : 1) * (size_t)(p.N / 32));
+    return total;
+}
+
+int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, const void* K_f, void* y_host, int64_t B,
+                         int64_t H, int64_t N, const void* w_host, const void* v_host, const uint8_t* mask_host,
+                         int64_t mask_h, void* staging, size_t staging_bytes, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    const Plan& p = plan->p;
+    if (B < 0 || H != p.H || N != p.N) return validate_forward(p, u_host, K_f, y_host, B, H, N, nullptr, nullptr,
+                                                               nullptr, 1);
+    if (B == 0) return FFTCONV_OK;
+    if (!u_host || !y_host || !K_f || !staging)
+        return fail(FFTCONV_ERR_INVALID_ARG, "u_host, y_host, K_f and staging must be non-NULL");
+    if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0)
+        return fail(FFTCONV_ERR_ALIGNMENT, "staging must be 256-byte aligned");
+    const size_t need = fftconv_forward_host_staging_bytes(plan, B, w_host != nullptr, v_host != nullptr,
+                                                           mask_host != nullptr, mask_h);
+    if (staging_bytes < need)
+        return fail(FFTCONV_ERR_INVALID_ARG, "staging has %zu bytes, %zu needed", staging_bytes, need);
+    const size_t bytes = (size_t)B * (size_t)p.H * (size_t)p.N * dtype_size(p.dtype);
+    const size_t t = round256(bytes);
+    char* base = (char*)staging;
+    void* du = base; base += t;
+    void* dy = base; base += t;
+    void* dw = nullptr; void* dv = nullptr; uint8_t* dm = nullptr;
+    if (w_host) { dw = base; base += t; }
+    if (v_host) { dv = base; base += t; }
+    const size_t mbytes = mask_host ? (size_t)mask_h * (size_t)(p.N / 32) : 0;
+    if (mask_host) { dm = (uint8_t*)base; }
+    cudaStream_t s = (cudaStream_t)stream;
+    int rc = validate_forward(p, du, K_f, dy, B, H, N, dw, dv, dm, mask_h);
+    if (rc != FFTCONV_OK) return rc;
+    cudaError_t e = cudaMemcpyAsync(du, u_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && w_host) e = cudaMemcpyAsync(dw, w_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && v_host) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && mask_host) e = cudaMemcpyAsync(dm, mask_host, mbytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    ForwardArgs a{du, dw, dv, dy, K_f, dm, mask_host ? mask_h : 0, B};
+    rc = run_forward(p, a, s);
+    if (rc != FFTCONV_OK) return rc;
+    e = cudaMemcpyAsync(y_host, dy, bytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    return FFTCONV_OK;
+}
+
+int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan || !K_f || !out) return fail(FFTCONV_ERR_INVALID_ARG, "plan, K_f and out must be non-NULL");
+    if (!aligned16(K_f) || ((uintptr_t)out & 7u)) return fail(FFTCONV_ERR_ALIGNMENT, "K_f/out misaligned");
+    const Plan& p = plan->p;
+    cudaError_t e = (p.path == kPathTcFused) ? tc_export_rfft(p, K_f, out, (cudaStream_t)stream)
+                                             : simt_export_rfft(p, K_f, out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "export launch");
+    return FFTCONV_OK;
+}
+
+int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    cudaStream_t s = (cudaStream_t)stream;
+    int host = 0;
+    cudaError_t e = cudaMemcpyAsync(&host, plan->p.status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (host != 0) {
+        int zero = 0;
+        cudaMemcpy(plan->p.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(host, "a bounded device wait timed out");
+    }
+    return FFTCONV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// internal.h -- plan structure and kernel launchers shared by the C ABI
+// implementation (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fftconv {
+
+enum Path : int { kPathSimtFused = 1, kPathSimtStaged = 2, kPathTcFused = 3 };
+enum DType : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
+
+struct Plan {
+    int64_t N = 0, H = 0, L = 0, M = 0;
+    int logM = 0;
+    int dtype = 0;
+    int order = 0;
+    int path = 0;
+    int device = 0;
+    size_t filter_bytes = 0;
+
+    // fp32 twiddle table exp(-2 pi i e / Ltab), e < Ltab (fused: Ltab = M;
+    // staged: Ltab = C).
+    float2* tw = nullptr;
+    int logTab = 0;
+
+    // staged path: M = R * C, two-level table for exp(-2 pi i e / M)
+    int logR = 0, logC = 0;
+    int twSplit = 0;            // bits of the low table
+    float2* twLo = nullptr;     // exp(-2 pi i e / M), e < 2^twSplit
+    float2* twHi = nullptr;     // exp(-2 pi i (e << twSplit) / M)
+    float2* work = nullptr;     // [chunkPairs][R][C] complex fp32
+    int64_t chunkPairs = 0;
+    size_t workBytes = 0;
+
+    // tensor-core path resources (owned by the tc translation unit)
+    void* tc = nullptr;
+
+    int* status = nullptr;      // device status word (timeouts)
+};
+
+struct ForwardArgs {
+    const void* u;
+    const void* w;
+    const void* v;
+    void* y;
+    const void* Kf;
+    const uint8_t* mask;
+    int64_t mask_h;
+    int64_t B;
+};
+
+// SIMT fp32 path (simt_kernels.cu)
+cudaError_t simt_fused_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
+cudaError_t simt_fused_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t simt_staged_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
+cudaError_t simt_staged_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t simt_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s);
+bool simt_fused_supported(int logM);
+
+// tensor-core path (tc_kernels.cu)
+bool tc_supported(int64_t N, int64_t L, int dtype);
+cudaError_t tc_plan_init(Plan& p);
+void tc_plan_free(Plan& p);
+size_t tc_filter_bytes(const Plan& p);
+cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t tc_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
+cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s);
+
+}  // namespace fftconv

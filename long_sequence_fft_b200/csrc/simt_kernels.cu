@@ -1,0 +1,540 @@
+// simt_kernels.cu -- fp32 FFT-convolution kernels on the FP32 lanes.
+//
+// Fused path (one launch): one CTA per pair of batch rows of one channel.  The
+// two real sequences ride in the real and imaginary parts of one complex
+// sequence ("two for one": the filter is real, so its spectrum is Hermitian
+// and the real/imaginary parts of the result are the two convolutions).  The
+// whole length-M (= 2N) transform stays in shared memory: the first stage
+// reads u*w straight from global memory (only the nonzero half), the last
+// forward stage, the product with K_f and the first inverse stage are fused
+// in registers, and the last inverse stage writes y*v for t < N only.
+//
+// Staged path (three launches per chunk of pairs, any N): M = R*C with a
+// column pass (length-R DFTs at stride C plus the exp(-2 pi i c r/M)
+// twiddle), a row pass (length-C forward DFT, product with K_f, inverse) and
+// an inverse column pass, through a plan-owned workspace.  This is the
+// "I/O between memory levels" regime of the FlashFFTConv page (Limitations).
+#include "internal.h"
+#include "simt_fft.cuh"
+
+namespace fftconv {
+
+namespace {
+
+constexpr int kMaskBlock = 32;
+
+// ------------------------------------------------------------ pair I/O ---
+
+template <typename T>
+struct PairRows {
+    const T* u0 = nullptr; const T* u1 = nullptr;
+    const T* w0 = nullptr; const T* w1 = nullptr;
+    const T* v0 = nullptr; const T* v1 = nullptr;
+    T* y0 = nullptr; T* y1 = nullptr;
+    int nvalid = 0;   // inputs at t >= nvalid read as zero (filter length)
+
+    __device__ __forceinline__ float2 load(int t) const {
+        if (t >= nvalid) return make_float2(0.f, 0.f);
+        float a = to_f32(u0[t]);
+        if (w0) a *= to_f32(w0[t]);
+        float b = 0.f;
+        if (u1) {
+            b = to_f32(u1[t]);
+            if (w1) b *= to_f32(w1[t]);
+        }
+        return make_float2(a, b);
+    }
+    __device__ __forceinline__ void store(int t, float2 z) const {
+        float a = z.x, b = z.y;
+        if (v0) a *= to_f32(v0[t]);
+        y0[t] = from_f32<T>(a);
+        if (y1) {
+            if (v1) b *= to_f32(v1[t]);
+            y1[t] = from_f32<T>(b);
+        }
+    }
+};
+
+// Rows of pair `pair` (pairs are channel-major: all batch pairs of channel 0
+// first, so consecutive CTAs share the channel's K_f in L2).
+template <typename T>
+__device__ __forceinline__ PairRows<T> pair_rows(const ForwardArgs& a, int64_t H, int64_t N,
+                                                 int64_t pair, int* h_out) {
+    const int64_t PB = (a.B + 1) / 2;
+    const int64_t h = pair / PB;
+    const int64_t b0 = 2 * (pair % PB), b1 = b0 + 1;
+    const int64_t o0 = (b0 * H + h) * N, o1 = (b1 * H + h) * N;
+    const bool has1 = b1 < a.B;
+    PairRows<T> r;
+    r.u0 = (const T*)a.u + o0;
+    r.u1 = has1 ? (const T*)a.u + o1 : nullptr;
+    if (a.w) { r.w0 = (const T*)a.w + o0; r.w1 = has1 ? (const T*)a.w + o1 : nullptr; }
+    if (a.v) { r.v0 = (const T*)a.v + o0; r.v1 = has1 ? (const T*)a.v + o1 : nullptr; }
+    r.y0 = (T*)a.y + o0;
+    r.y1 = has1 ? (T*)a.y + o1 : nullptr;
+    r.nvalid = (int)N;
+    *h_out = (int)h;
+    return r;
+}
+
+// 1 if rfft bin of full-spectrum frequency f survives the mask row.
+__device__ __forceinline__ bool bin_kept(const uint8_t* __restrict__ mrow, int64_t f, int64_t N) {
+    const int64_t M = 2 * N;
+    const int64_t g = f <= N ? f : M - f;
+    int64_t blk = g / kMaskBlock;
+    const int64_t nblk = N / kMaskBlock;
+    if (blk >= nblk) blk = nblk - 1;
+    return __ldg(&mrow[blk]) != 0;
+}
+
+__device__ __forceinline__ float2 tw_M(const float2* __restrict__ lo, const float2* __restrict__ hi,
+                                       int split, int64_t e) {
+    return cmul(__ldg(&hi[e >> split]), __ldg(&lo[e & ((1LL << split) - 1)]));
+}
+
+// ------------------------------------------------------- fused kernel ---
+
+template <int LOGM>
+constexpr int fused_threads() {
+    return (1 << LOGM) / 32 < 128 ? 128 : ((1 << LOGM) / 32 > 512 ? 512 : (1 << LOGM) / 32);
+}
+
+// Stage 0 of the fused transform, reading the zero-padded input from global
+// memory: position j*S + r, j < R/2 (t < N); the upper half is zero.
+template <int LOGM, int NT, typename T>
+__device__ __forceinline__ void first_stage_global(float2* s, const float2* __restrict__ tw,
+                                                   const PairRows<T>& io, int tid) {
+    constexpr int LB = Sched<LOGM>::bits(0);
+    constexpr int R = 1 << LB;
+    constexpr int S = 1 << (LOGM - LB);
+    for (int r = tid; r < S; r += NT) {
+        float2 x[R];
+#pragma unroll
+        for (int j = 0; j < R / 2; ++j) x[j] = io.load(j * S + r);
+        Dft<R, -1>::run_half_input(x);
+#pragma unroll
+        for (int c = 1; c < R; ++c) x[c] = cmul(x[c], __ldg(&tw[c * r]));
+#pragma unroll
+        for (int c = 0; c < R; ++c) s[sidx<1>(c * S + r, 0)] = x[c];
+    }
+}
+
+// Inverse of stage 0, writing y = v * z for t < N only.
+template <int LOGM, int NT, typename T>
+__device__ __forceinline__ void last_stage_global(const float2* s, const float2* __restrict__ tw,
+                                                  const PairRows<T>& io, int tid) {
+    constexpr int LB = Sched<LOGM>::bits(0);
+    constexpr int R = 1 << LB;
+    constexpr int S = 1 << (LOGM - LB);
+    for (int r = tid; r < S; r += NT) {
+        float2 x[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) x[c] = s[sidx<1>(c * S + r, 0)];
+#pragma unroll
+        for (int c = 1; c < R; ++c) x[c] = cmulc(x[c], __ldg(&tw[c * r]));
+        Dft<R, +1>::run(x);
+#pragma unroll
+        for (int j = 0; j < R / 2; ++j) io.store(j * S + r, x[j]);
+    }
+}
+
+// Last forward stage (unit stride), product with the filter spectrum and
+// first inverse stage, fused in registers.  freq(p) maps a permuted position
+// to its full-spectrum frequency for the mask; Krow is indexed by position.
+template <int LOGL, int NT, typename FreqFn>
+__device__ __forceinline__ void middle_stage(float2* s, const float2* __restrict__ Krow,
+                                             const uint8_t* __restrict__ mrow, int64_t N,
+                                             FreqFn freq, int tid) {
+    constexpr int I = Sched<LOGL>::K - 1;
+    constexpr int LB = Sched<LOGL>::bits(I);
+    constexpr int R = 1 << LB;
+    static_assert(Sched<LOGL>::stride_bits(I) == 0, "middle stage must have unit stride");
+    constexpr int G = (1 << LOGL) / R;
+    for (int g = tid; g < G; g += NT) {
+        const int base = g * R;
+        float2 x[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) x[c] = s[sidx<1>(base + c, 0)];
+        Dft<R, -1>::run(x);
+        const float4* K4 = reinterpret_cast<const float4*>(Krow + base);
+#pragma unroll
+        for (int c = 0; c < R; c += 2) {
+            float4 kk = __ldg(&K4[c / 2]);
+            float2 k0 = make_float2(kk.x, kk.y), k1 = make_float2(kk.z, kk.w);
+            if (mrow) {
+                if (!bin_kept(mrow, freq(base + c), N)) k0 = make_float2(0.f, 0.f);
+                if (!bin_kept(mrow, freq(base + c + 1), N)) k1 = make_float2(0.f, 0.f);
+            }
+            x[c] = cmul(x[c], k0);
+            x[c + 1] = cmul(x[c + 1], k1);
+        }
+        Dft<R, +1>::run(x);
+#pragma unroll
+        for (int j = 0; j < R; ++j) s[sidx<1>(base + j, 0)] = x[j];
+    }
+}
+
+template <int LOGM, typename T>
+__global__ void __launch_bounds__(fused_threads<LOGM>())
+simt_fused_kernel(ForwardArgs a, int64_t H, const float2* __restrict__ tw) {
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    static_assert(K >= 2, "fused path needs at least two stages");
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int64_t N = (int64_t)1 << (LOGM - 1);
+    int h;
+    const PairRows<T> io = pair_rows<T>(a, H, N, blockIdx.x, &h);
+    const float2* Krow = (const float2*)a.Kf + (int64_t)h * (1 << LOGM);
+    const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : h) * (N / kMaskBlock) : nullptr;
+
+    first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K - 1, 1, NT>(s, tw, 0, tid);
+    middle_stage<LOGM, NT>(s, Krow, mrow, N, [](int p) { return perm_to_freq(p, LOGM); }, tid);
+    __syncthreads();
+    inv_stages<LOGM, 1, K - 1, 1, NT>(s, tw, 0, tid);
+    last_stage_global<LOGM, NT, T>(s, tw, io, tid);
+}
+
+// K_f[h, p] = FFT_M(k_h zero-padded)[freq(p)] / M, one channel per CTA.
+template <int LOGM, typename T>
+__global__ void __launch_bounds__(fused_threads<LOGM>())
+simt_fused_precompute_kernel(const T* __restrict__ k, int64_t L, float2* __restrict__ Kf,
+                             const float2* __restrict__ tw) {
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x;
+    PairRows<T> io;
+    io.u0 = k + (int64_t)h * L;
+    io.nvalid = (int)L;
+    first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
+    const float inv = 1.0f / (float)(1 << LOGM);
+    float2* out = Kf + (int64_t)h * (1 << LOGM);
+    for (int p = tid; p < (1 << LOGM); p += NT) out[p] = cscale(s[sidx<1>(p, 0)], inv);
+}
+
+template <int LOGM, typename T>
+cudaError_t launch_fused(const Plan& p, const ForwardArgs& a, cudaStream_t st) {
+    constexpr int NT = fused_threads<LOGM>();
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << LOGM);
+    auto kern = simt_fused_kernel<LOGM, T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t pairs = p.H * ((a.B + 1) / 2);
+    kern<<<(unsigned)pairs, NT, smem, st>>>(a, p.H, p.tw);
+    return cudaGetLastError();
+}
+
+template <int LOGM, typename T>
+cudaError_t launch_fused_pre(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    constexpr int NT = fused_threads<LOGM>();
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << LOGM);
+    auto kern = simt_fused_precompute_kernel<LOGM, T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)p.H, NT, smem, st>>>((const T*)k, p.L, (float2*)Kf, p.tw);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------ staged kernels ---
+
+constexpr int kColTile = 32;    // columns per CTA in the column passes
+constexpr int kColThreads = 256;
+
+template <int LOGC>
+constexpr int row_threads() { return (1 << LOGC) / 32 < 128 ? 128 : ((1 << LOGC) / 32 > 512 ? 512 : (1 << LOGC) / 32); }
+
+struct StagedArgs {
+    ForwardArgs fa;
+    int64_t H, N, M;
+    int64_t pair0;          // first pair of this chunk
+    int64_t npairs;         // pairs in this chunk
+    int logC;
+    float2* work;           // [npairs][R][C]
+    const float2* tw;       // exp(-2 pi i e / C)
+    const float2* twLo;
+    const float2* twHi;
+    int twSplit;
+    // precompute mode: input k [H, L] instead of u/w; pair == channel
+    const void* k;
+    int64_t L;
+};
+
+template <typename T>
+__device__ __forceinline__ PairRows<T> staged_rows(const StagedArgs& A, int64_t pair, int* h) {
+    if (A.k) {
+        PairRows<T> r;
+        r.u0 = (const T*)A.k + pair * A.L;
+        r.nvalid = (int)A.L;
+        *h = (int)pair;
+        return r;
+    }
+    return pair_rows<T>(A.fa, A.H, A.N, pair, h);
+}
+
+// Column pass: length-R DFT over j of x[j*C + r] (upper half zero), twiddle
+// exp(-2 pi i c r / M), stored at work[pair][c][r] in natural c order.
+template <int LOGR, typename T>
+__global__ void __launch_bounds__(kColThreads)
+staged_col_fwd_kernel(StagedArgs A) {
+    constexpr int R = 1 << LOGR;
+    constexpr int TC = kColTile;
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int64_t C = (int64_t)1 << A.logC;
+    const int64_t pl = blockIdx.y;
+    const int64_t col0 = (int64_t)blockIdx.x * TC;
+    int h;
+    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    for (int idx = tid; idx < R * TC; idx += kColThreads) {
+        const int j = idx / TC, col = idx % TC;
+        s[sidx<TC>(j, col)] = (j < R / 2) ? io.load((int)(j * C + col0 + col)) : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    float2* W = A.work + pl * (R * C);
+    for (int idx = tid; idx < R * TC; idx += kColThreads) {
+        const int p = idx / TC, col = idx % TC;
+        const int64_t c = perm_to_freq(p, LOGR);
+        const int64_t r = col0 + col;
+        const float2 z = cmul(s[sidx<TC>(p, col)], tw_M(A.twLo, A.twHi, A.twSplit, c * r));
+        W[c * C + r] = z;
+    }
+}
+
+// Row pass.  MODE 0: forward DFT over r, product with K_f row, inverse, back
+// into the workspace.  MODE 1 (filter precompute): forward only, scaled by
+// 1/M, into K_f[h][c][position].
+template <int LOGC, int MODE>
+__global__ void __launch_bounds__(row_threads<LOGC>())
+staged_row_kernel(StagedArgs A) {
+    constexpr int NT = row_threads<LOGC>();
+    constexpr int C = 1 << LOGC;
+    constexpr int K = Sched<LOGC>::K;
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int64_t c = blockIdx.x;
+    const int64_t R = A.M >> LOGC;
+    const int64_t pl = blockIdx.y;
+    float2* row = A.work + (pl * R + c) * C;
+    for (int i = tid; i < C; i += NT) s[sidx<1>(i, 0)] = row[i];
+    __syncthreads();
+    if constexpr (MODE == 0) {
+        const int64_t h = (A.pair0 + pl) / ((A.fa.B + 1) / 2);   // channel of this pair
+        const float2* Krow = (const float2*)A.fa.Kf + ((int64_t)h * R + c) * C;
+        const uint8_t* mrow = A.fa.mask ? A.fa.mask + (A.fa.mask_h == 1 ? 0 : h) * (A.N / kMaskBlock) : nullptr;
+        fwd_stages<LOGC, 0, K - 1, 1, NT>(s, A.tw, 0, tid);
+        middle_stage<LOGC, NT>(s, Krow, mrow, A.N,
+                               [c, R](int p) { return c + R * perm_to_freq(p, LOGC); }, tid);
+        __syncthreads();
+        inv_stages<LOGC, 0, K - 1, 1, NT>(s, A.tw, 0, tid);
+        for (int i = tid; i < C; i += NT) row[i] = s[sidx<1>(i, 0)];
+    } else {
+        fwd_stages<LOGC, 0, K, 1, NT>(s, A.tw, 0, tid);
+        const float inv = 1.0f / (float)A.M;
+        const int64_t h = A.pair0 + pl;
+        float2* out = (float2*)A.fa.y + (h * R + c) * C;   // fa.y carries K_f here
+        for (int i = tid; i < C; i += NT) out[i] = cscale(s[sidx<1>(i, 0)], inv);
+    }
+}
+
+// Inverse column pass: conjugate twiddle, inverse length-R DFT over c, and
+// y = v * z for t = j*C + r < N.
+template <int LOGR, typename T>
+__global__ void __launch_bounds__(kColThreads)
+staged_col_inv_kernel(StagedArgs A) {
+    constexpr int R = 1 << LOGR;
+    constexpr int TC = kColTile;
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int64_t C = (int64_t)1 << A.logC;
+    const int64_t pl = blockIdx.y;
+    const int64_t col0 = (int64_t)blockIdx.x * TC;
+    int h;
+    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    const float2* W = A.work + pl * (R * C);
+    for (int idx = tid; idx < R * TC; idx += kColThreads) {
+        const int p = idx / TC, col = idx % TC;
+        const int64_t c = perm_to_freq(p, LOGR);
+        const int64_t r = col0 + col;
+        s[sidx<TC>(p, col)] = cmulc(W[c * C + r], tw_M(A.twLo, A.twHi, A.twSplit, c * r));
+    }
+    __syncthreads();
+    inv_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads) {
+        const int j = idx / TC, col = idx % TC;
+        io.store((int)(j * C + col0 + col), s[sidx<TC>(j, col)]);
+    }
+}
+
+template <int LOGR, typename T>
+cudaError_t launch_cols(const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
+    const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * kColTile;
+    dim3 grid((unsigned)(C / kColTile), (unsigned)A.npairs);
+    if (!inverse) {
+        auto kern = staged_col_fwd_kernel<LOGR, T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kColThreads, smem, st>>>(A);
+    } else {
+        auto kern = staged_col_inv_kernel<LOGR, T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kColThreads, smem, st>>>(A);
+    }
+    return cudaGetLastError();
+}
+
+template <int LOGC, int MODE>
+cudaError_t launch_rows(const StagedArgs& A, int64_t R, cudaStream_t st) {
+    constexpr int NT = row_threads<LOGC>();
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << LOGC);
+    auto kern = staged_row_kernel<LOGC, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)R, (unsigned)A.npairs);
+    kern<<<grid, NT, smem, st>>>(A);
+    return cudaGetLastError();
+}
+
+// Runtime -> compile-time dispatch helpers.
+template <typename T>
+cudaError_t cols_dispatch(int logR, const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
+    switch (logR) {
+        case 1: return launch_cols<1, T>(A, C, inverse, st);
+        case 2: return launch_cols<2, T>(A, C, inverse, st);
+        case 3: return launch_cols<3, T>(A, C, inverse, st);
+        case 4: return launch_cols<4, T>(A, C, inverse, st);
+        case 5: return launch_cols<5, T>(A, C, inverse, st);
+        case 6: return launch_cols<6, T>(A, C, inverse, st);
+        case 7: return launch_cols<7, T>(A, C, inverse, st);
+        case 8: return launch_cols<8, T>(A, C, inverse, st);
+        case 9: return launch_cols<9, T>(A, C, inverse, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int MODE>
+cudaError_t rows_dispatch(int logC, const StagedArgs& A, int64_t R, cudaStream_t st) {
+    switch (logC) {
+        case 8: return launch_rows<8, MODE>(A, R, st);
+        case 9: return launch_rows<9, MODE>(A, R, st);
+        case 10: return launch_rows<10, MODE>(A, R, st);
+        case 11: return launch_rows<11, MODE>(A, R, st);
+        case 12: return launch_rows<12, MODE>(A, R, st);
+        case 13: return launch_rows<13, MODE>(A, R, st);
+        case 14: return launch_rows<14, MODE>(A, R, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t staged_forward_t(const Plan& p, const ForwardArgs& fa, const void* k, cudaStream_t st) {
+    StagedArgs A{};
+    A.fa = fa;
+    A.H = p.H; A.N = p.N; A.M = p.M;
+    A.logC = p.logC;
+    A.work = p.work;
+    A.tw = p.tw; A.twLo = p.twLo; A.twHi = p.twHi; A.twSplit = p.twSplit;
+    A.k = k; A.L = p.L;
+    const int64_t C = (int64_t)1 << p.logC, R = (int64_t)1 << p.logR;
+    const int64_t total = k ? p.H : p.H * ((fa.B + 1) / 2);
+    for (int64_t first = 0; first < total; first += p.chunkPairs) {
+        A.pair0 = first;
+        A.npairs = total - first < p.chunkPairs ? total - first : p.chunkPairs;
+        cudaError_t e = cols_dispatch<T>(p.logR, A, C, false, st);
+        if (e != cudaSuccess) return e;
+        e = k ? rows_dispatch<1>(p.logC, A, R, st) : rows_dispatch<0>(p.logC, A, R, st);
+        if (e != cudaSuccess) return e;
+        if (!k) {
+            e = cols_dispatch<T>(p.logR, A, C, true, st);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------- export (test hook) ---
+
+__global__ void export_rfft_kernel(const float2* __restrict__ Kf, float* __restrict__ out, int64_t H,
+                                   int64_t N, int logM, int staged, int logR, int logC) {
+    const int64_t M = 2 * N;
+    const int64_t total = H * (N + 1);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t h = i / (N + 1), f = i % (N + 1);
+        int64_t pos;
+        if (!staged) {
+            pos = freq_to_perm(f, logM);
+        } else {
+            const int64_t R = (int64_t)1 << logR;
+            const int64_t c = f & (R - 1), e = f >> logR;
+            pos = (c << logC) + freq_to_perm(e, logC);
+        }
+        const float2 z = Kf[h * M + pos];
+        out[2 * i] = z.x * (float)M;
+        out[2 * i + 1] = z.y * (float)M;
+    }
+}
+
+}  // namespace
+
+bool simt_fused_supported(int logM) { return logM >= 9 && logM <= 14; }
+
+#define FFTCONV_DISPATCH_T(dtype, ...)                                   \
+    switch (dtype) {                                                     \
+        case kF32: { using T = float; __VA_ARGS__; }                     \
+        case kF16: { using T = __half; __VA_ARGS__; }                    \
+        case kBF16: { using T = __nv_bfloat16; __VA_ARGS__; }            \
+        default: return cudaErrorInvalidValue;                           \
+    }
+
+cudaError_t simt_fused_forward(const Plan& p, const ForwardArgs& a, cudaStream_t st) {
+    FFTCONV_DISPATCH_T(p.dtype, switch (p.logM) {
+        case 9: return launch_fused<9, T>(p, a, st);
+        case 10: return launch_fused<10, T>(p, a, st);
+        case 11: return launch_fused<11, T>(p, a, st);
+        case 12: return launch_fused<12, T>(p, a, st);
+        case 13: return launch_fused<13, T>(p, a, st);
+        case 14: return launch_fused<14, T>(p, a, st);
+        default: return cudaErrorInvalidValue;
+    })
+}
+
+cudaError_t simt_fused_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    FFTCONV_DISPATCH_T(p.dtype, switch (p.logM) {
+        case 9: return launch_fused_pre<9, T>(p, k, Kf, st);
+        case 10: return launch_fused_pre<10, T>(p, k, Kf, st);
+        case 11: return launch_fused_pre<11, T>(p, k, Kf, st);
+        case 12: return launch_fused_pre<12, T>(p, k, Kf, st);
+        case 13: return launch_fused_pre<13, T>(p, k, Kf, st);
+        case 14: return launch_fused_pre<14, T>(p, k, Kf, st);
+        default: return cudaErrorInvalidValue;
+    })
+}
+
+cudaError_t simt_staged_forward(const Plan& p, const ForwardArgs& a, cudaStream_t st) {
+    FFTCONV_DISPATCH_T(p.dtype, return staged_forward_t<T>(p, a, nullptr, st))
+}
+
+cudaError_t simt_staged_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    ForwardArgs fa{};
+    fa.y = Kf;      // the row pass in precompute mode writes K_f through fa.y
+    FFTCONV_DISPATCH_T(p.dtype, return staged_forward_t<T>(p, fa, k, st))
+}
+
+cudaError_t simt_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t st) {
+    const int64_t total = p.H * (p.N + 1);
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 65535) blocks = 65535;
+    export_rfft_kernel<<<blocks, 256, 0, st>>>((const float2*)Kf, out, p.H, p.N, p.logM,
+                                               p.path == kPathSimtStaged, p.logR, p.logC);
+    return cudaGetLastError();
+}
+
+}  // namespace fftconv

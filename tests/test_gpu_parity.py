@@ -1,0 +1,213 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded, dtype-rounded inputs.
+
+Element-by-element at sizes the oracle finishes in seconds (several tiles and
+ragged batches: odd B leaves an unpaired sequence), and on sampled outputs at
+the workloads' full sizes, in the launch configuration the benchmark times."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from parity_util import assert_close, rel_l2, run_cuda, to_dev
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(2024)
+
+
+def _rand_inputs(B, H, N, L, dtype, gated, mask_frac=0.0, seed=0):
+    rng = np.random.default_rng(seed)
+    u = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    k = W.round_to((rng.standard_normal((H, L), dtype=np.float32) / np.float32(np.sqrt(L))), dtype)
+    out = {"u": u, "k": k, "w": None, "v": None, "mask": None}
+    if gated:
+        out["w"] = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+        out["v"] = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    if mask_frac > 0:
+        m = (rng.random((H, N // 32)) >= mask_frac).astype(np.uint8)
+        out["mask"] = m
+    return out
+
+
+def _oracle(inp):
+    return oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], mask=inp["mask"])
+
+
+# ------------------------------------------------------ small, full compare ---
+
+CASES = []
+for dtype in ("f32", "f16", "bf16"):
+    for order in (1, 4, 0):
+        for (B, H, N) in ((1, 2, 256), (3, 2, 1024), (2, 3, 4096), (1, 1, 8192)):
+            CASES.append((dtype, order, B, H, N))
+    CASES.append((dtype, 4, 2, 2, 16384))
+    CASES.append((dtype, 0, 3, 1, 32768))
+
+
+@pytest.mark.parametrize("dtype,order,B,H,N", CASES)
+def test_small_shapes_full_compare(dtype, order, B, H, N):
+    inp = _rand_inputs(B, H, N, N, dtype, gated=(B % 2 == 1), seed=B * 131 + H * 7 + N)
+    y, plan = run_cuda(inp, dtype, order=order)
+    ref = _oracle(inp)
+    assert_close(y, ref, dtype, f"{dtype} order={order} path={plan.path_name} B={B} H={H} N={N}")
+
+
+@pytest.mark.parametrize("order", [1, 4, 0])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_partial_and_masked(order, dtype):
+    N = 2048
+    inp = _rand_inputs(3, 2, N, 300, dtype, gated=True, seed=7)
+    y, _ = run_cuda(inp, dtype, order=order)
+    assert_close(y, _oracle(inp), dtype, "partial L=300")
+    inp = _rand_inputs(2, 3, N, N, dtype, gated=True, mask_frac=0.75, seed=8)
+    y, _ = run_cuda(inp, dtype, order=order)
+    assert_close(y, _oracle(inp), dtype, "masked per-channel")
+    inp["mask"] = inp["mask"][:1]
+    y, _ = run_cuda(inp, dtype, order=order)
+    assert_close(y, _oracle(inp), dtype, "masked shared row")
+
+
+# ---------------------------------------------------------- workloads ---
+
+REDUCED = {
+    "fp32_n1k": dict(),                      # already small: full size
+    "gated_bf16_n4k": dict(B=3, H=4),
+    "fp16_n32k": dict(B=2, H=2),
+    "dna_bf16_n1m": dict(H=2),
+    "partial_bf16_n8k": dict(B=3, H=3),
+    "sparse_bf16_n8k": dict(B=3, H=3),
+}
+
+
+@pytest.mark.parametrize("name", sorted(REDUCED))
+def test_workload_reduced_full_compare(name):
+    w = W.WORKLOADS[name].with_shape(**REDUCED[name])
+    inp = W.make_all(w)
+    y, plan = run_cuda(inp, w.dtype)
+    ref = _oracle(inp)
+    assert_close(y, ref, w.dtype, f"{name} ({plan.path_name})")
+
+
+def _sampled_ref(w, inp, seq, ts):
+    if inp["mask"] is None:
+        return oracle.direct_conv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], seq=seq, ts=ts)
+    # frequency-sparse: circular sum with the masked filter's time-domain
+    # response, computed only for the channels that are sampled
+    hs = np.unique(seq % w.H)
+    keff = np.zeros((w.H, 2 * w.N))
+    keff[hs] = oracle.masked_filter(inp["k"][hs], w.N, inp["mask"])
+    return oracle.circular_conv_samples(inp["u"], keff, seq, ts, w=inp["w"], v=inp["v"])
+
+
+@pytest.mark.parametrize("name", sorted(W.WORKLOADS))
+def test_workload_full_size_sampled(name):
+    """Full BASELINE shapes, the benchmark's launch configuration (order 0),
+    compared at seeded sample points against direct sums."""
+    w = W.WORKLOADS[name]
+    inp = W.make_all(w)
+    y, plan = run_cuda(inp, w.dtype)
+    seq, ts = W.sample_points(w, nseq=16, nrand=61)
+    ref = _sampled_ref(w, inp, seq, ts)
+    got = y.reshape(w.B * w.H, w.N)[seq, ts]
+    assert_close(got, ref, w.dtype, f"{name} sampled ({plan.path_name})")
+    # properties that hold at any size: finite everywhere
+    assert np.isfinite(y).all()
+
+
+# -------------------------------------------------------------- edges ---
+
+def test_filter_export_matches_oracle_rfft():
+    import long_sequence_fft_b200 as lsf
+    for dtype, order, N, L in (("f32", 1, 1024, 1024), ("bf16", 4, 4096, 1000), ("f16", 0, 2048, 2048)):
+        k = W.round_to(RNG.standard_normal((3, L), dtype=np.float32), dtype)
+        plan = lsf.Plan(N, 3, dtype, order=order, L=L)
+        Kf = plan.precompute(to_dev(k, dtype))
+        got = plan.export_rfft(Kf).cpu().numpy().astype(np.complex128)
+        ref = oracle.filter_rfft(k, N)
+        err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert err <= 1e-5, (dtype, order, err)
+
+
+@pytest.mark.parametrize("order", [1, 4])
+def test_delta_and_scalar_filters(order):
+    import long_sequence_fft_b200 as lsf
+    import torch
+    N = 1024
+    inp = _rand_inputs(3, 2, N, N, "f32", gated=True, seed=3)
+    inp["k"] = np.zeros((2, N), np.float32)
+    inp["k"][:, 0] = 1.0
+    y, _ = run_cuda(inp, "f32", order=order)
+    assert_close(y, inp["u"] * inp["w"] * inp["v"], "f32", "delta filter")
+    # L = 1 partial filter
+    inp["k"] = np.array([[2.0], [-0.5]], np.float32)
+    y, _ = run_cuda(inp, "f32", order=order)
+    ref = inp["u"] * inp["w"] * inp["v"] * inp["k"][None, :, :1]
+    assert_close(y, ref, "f32", "L=1 filter")
+
+
+@pytest.mark.parametrize("order", [1, 4])
+def test_zero_and_full_masks(order):
+    N = 1024
+    inp = _rand_inputs(2, 2, N, N, "f32", gated=False, seed=5)
+    inp["mask"] = np.zeros((1, N // 32), np.uint8)
+    y, _ = run_cuda(inp, "f32", order=order)
+    assert np.max(np.abs(y)) == 0.0
+    inp["mask"] = np.full((2, N // 32), 7, np.uint8)     # any nonzero byte keeps
+    y1, _ = run_cuda(inp, "f32", order=order)
+    inp["mask"] = None
+    y2, _ = run_cuda(inp, "f32", order=order)
+    assert np.array_equal(y1, y2)
+
+
+def test_empty_batch_is_noop():
+    import long_sequence_fft_b200 as lsf
+    import torch
+    plan = lsf.Plan(1024, 2, "bf16")
+    Kf = plan.precompute(torch.zeros((2, 1024), dtype=torch.bfloat16, device="cuda"))
+    u = torch.zeros((0, 2, 1024), dtype=torch.bfloat16, device="cuda")
+    y = plan.forward(u, Kf)
+    assert y.shape == (0, 2, 1024)
+
+
+def test_forward_host_matches_device_path():
+    import long_sequence_fft_b200 as lsf
+    import torch
+    w = W.WORKLOADS["gated_bf16_n4k"].with_shape(B=3, H=5)
+    inp = W.make_all(w)
+    plan = lsf.Plan(w.N, w.H, "bf16")
+    Kf = plan.precompute(to_dev(inp["k"], "bf16"))
+    yd = plan.forward(to_dev(inp["u"], "bf16"), Kf, w=to_dev(inp["w"], "bf16"), v=to_dev(inp["v"], "bf16"))
+    pin = lambda a: torch.from_numpy(a).to(torch.bfloat16).pin_memory()
+    uh, wh, vh = pin(inp["u"]), pin(inp["w"]), pin(inp["v"])
+    yh = torch.empty_like(uh).pin_memory()
+    staging = torch.empty(plan.staging_bytes(w.B, True, True), dtype=torch.uint8, device="cuda")
+    plan.forward_host(uh, Kf, yh, staging, w_host=wh, v_host=vh)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, yd.cpu())
+
+
+def test_bad_arguments_are_rejected_without_launch():
+    import long_sequence_fft_b200 as lsf
+    import torch
+    plan = lsf.Plan(1024, 2, "f32")
+    k = torch.zeros((2, 1024), device="cuda")
+    Kf = plan.precompute(k)
+    u = torch.zeros((2, 2, 1024), device="cuda")
+    with pytest.raises(lsf.FFTConvError) as e:
+        lib = lsf.library()
+        rc = lib.fftconv_forward(plan.handle, u.data_ptr() + 4, Kf.data_ptr(), u.data_ptr() + 8192 * 4, 2, 2, 1024,
+                                 None, None, None, 0, None)
+        lsf._check(rc)
+    assert e.value.status == lsf.ERR_ALIGNMENT
+    with pytest.raises(lsf.FFTConvError) as e:
+        lsf._check(lsf.library().fftconv_forward(plan.handle, u.data_ptr(), Kf.data_ptr(), u.data_ptr(), 2, 2,
+                                                 1024, None, None, None, 0, None))
+    assert e.value.status == lsf.ERR_INVALID_ARG        # y aliases u
+    with pytest.raises(lsf.FFTConvError) as e:
+        lsf._check(lsf.library().fftconv_forward(plan.handle, u.data_ptr(), Kf.data_ptr(), u.data_ptr(), 2, 3,
+                                                 1024, None, None, None, 0, None))
+    assert e.value.status == lsf.ERR_INVALID_ARG        # H mismatch
+    with pytest.raises(lsf.FFTConvError) as e:
+        lsf.Plan(1000, 2, "f32")
+    assert e.value.status == lsf.ERR_UNSUPPORTED
