@@ -67,7 +67,7 @@ def read_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks/throttle reasons sampled every 20 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -82,7 +82,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -160,26 +160,25 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --------------------------------------------------------------- oracle ---
 
-def time_oracle(w: W.Workload, target_s: float = 10.0, max_seqs: int = 1 << 16):
-    """The fp64 oracle on a bounded sample of the workload: whole sequences
-    (b, h) of the same shape, as many as fit in about `target_s` seconds on
-    all host cores.  Returns (elems/s, cores, description)."""
+def time_oracle(w: W.Workload, target_s: float = 10.0):
+    """The fp64 oracle on a bounded sample of the workload: a block of whole
+    sequences (b, h) of the workload's shape, convolved repeatedly on all host
+    cores until about `target_s` seconds have passed.  Returns (elems/s,
+    cores, description)."""
     import oracle
     cores = os.cpu_count() or 1
-    sub = w.with_shape(B=1, H=min(w.H, 64))
+    sub = w.with_shape(B=min(w.B, 16), H=min(w.H, 64))
     inp = W.make_all(sub)
-    t0 = time.perf_counter()
-    oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], mask=inp["mask"], nthreads=cores)
-    t1 = time.perf_counter()
-    per_seq = (t1 - t0) / sub.H
-    B = max(1, min(int(target_s / max(per_seq, 1e-9) / sub.H), max_seqs // sub.H))
-    sub = w.with_shape(B=B, H=sub.H)
-    inp = W.make_all(sub)
-    t0 = time.perf_counter()
-    oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], mask=inp["mask"], nthreads=cores)
-    dt = time.perf_counter() - t0
-    return sub.elems / dt, cores, f"{sub.B * sub.H} whole sequences (B={sub.B}, H={sub.H}) of N={w.N}, " \
-                                  f"{dt:.1f} s on {cores} threads"
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], mask=inp["mask"], nthreads=cores)
+        done += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            break
+    elems = done * sub.elems
+    return elems / dt, cores, (f"{done} passes over {sub.B * sub.H} whole sequences (B={sub.B}, H={sub.H}) of "
+                               f"N={w.N}: {done * sub.B * sub.H} sequences in {dt:.1f} s on {cores} threads")
 
 
 def run_reference(args):
@@ -221,13 +220,17 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=W.BENCH_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--order", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--B", type=int, default=None,
+                    help="override the batch size (small cases for profiling; not a bench number)")
+    ap.add_argument("--profile", action="store_true",
+                    help="profiling run: skip the host-buffer and CPU-baseline legs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -239,11 +242,13 @@ def main():
 
     world, rank, local = dist_setup()
     w = W.WORKLOADS[args.workload]
+    if args.B is not None:
+        w = w.with_shape(B=args.B)
     if w.B * w.H * w.N == 0:
         raise SystemExit("empty workload")
 
-    # inputs: seeded host generation, copied to HBM once (each rank holds its
-    # own channel shard of the same shape; the seed is offset by rank)
+    # inputs: seeded host generation, copied to HBM once (each rank convolves
+    # its own channel shard; all shards have the workload's shape)
     inp = W.make_all(w)
     dt = W.torch_dtype(w.dtype)
     dev = lambda a: None if a is None else torch.from_numpy(a).to(dt).cuda()
@@ -294,6 +299,12 @@ def main():
         chunk = max(1, plan.workspace_bytes // (2 * w.N * 8))
         pairs = w.H * ((w.B + 1) // 2)
         launches_per_step = 3 * ((pairs + chunk - 1) // chunk)
+
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": ms_per_step, "workload": w.name, "B": w.B,
+                              "path": plan.path_name}), flush=True)
+        return 0
 
     # end to end through the host-buffer entry point (pinned memory, copies in
     # the timed region)

@@ -78,6 +78,51 @@ __device__ __forceinline__ int sidx(int p, int col) {
 template <int TC>
 __host__ __device__ constexpr int smem_elems(int L) { return TC == 1 ? L + L / 16 : L * TC; }
 
+// x[c] *= w^c (or conj(w)^c) for c = 1..R-1, where w = tw[e1] is a table
+// entry.  Instead of gathering R-1 table entries at stride e1 (uncoalesced
+// across a warp), at most three coalesced entries w, w^4, w^16 are loaded and
+// the other powers formed by products of at most four factors, which keeps
+// the rounding error within a few fp32 ulps.
+template <int R, bool CONJ>
+__device__ __forceinline__ void twiddle_powers(float2 (&x)[R], const float2* __restrict__ tw, int e1) {
+    auto mul = [](float2 a, float2 b) { return CONJ ? cmulc(a, b) : cmul(a, b); };
+    const float2 w1 = __ldg(&tw[e1]);
+    if constexpr (R == 2) {
+        x[1] = mul(x[1], w1);
+    } else {
+        float2 p[4];
+        p[1] = w1;
+        p[2] = cmul(w1, w1);
+        p[3] = cmul(p[2], w1);
+        if constexpr (R == 4) {
+#pragma unroll
+            for (int c = 1; c < 4; ++c) x[c] = mul(x[c], p[c]);
+        } else {
+            constexpr int Q = R / 4;
+            float2 q[Q];
+            const float2 w4 = __ldg(&tw[4 * e1]);
+            q[1] = w4;
+            if constexpr (Q > 2) q[2] = cmul(w4, w4);
+            if constexpr (Q > 3) q[3] = cmul(q[2], w4);
+            if constexpr (Q > 4) {
+                const float2 w16 = __ldg(&tw[16 * e1]);
+                q[4] = w16;
+#pragma unroll
+                for (int a = 5; a < Q; ++a) q[a] = cmul(w16, q[a - 4]);
+            }
+#pragma unroll
+            for (int c = 1; c < R; ++c) {
+                const int a = c / 4, b = c % 4;
+                float2 w;
+                if (a == 0) w = p[b];
+                else if (b == 0) w = q[a];
+                else w = cmul(q[a], p[b]);
+                x[c] = mul(x[c], w);
+            }
+        }
+    }
+}
+
 // Forward stage I of a length-2^LOGL transform over TC batch columns held in
 // shared memory.  tw = exp(-2 pi i e / Ltab) for e < Ltab, Ltab = L << twshift.
 template <int LOGL, int I, int TC, int NT>
@@ -96,11 +141,7 @@ __device__ __forceinline__ void fwd_stage(float2* s, const float2* __restrict__ 
 #pragma unroll
         for (int j = 0; j < R; ++j) x[j] = s[sidx<TC>(base + j * S, col)];
         Dft<R, -1>::run(x);
-        if constexpr (S > 1) {
-            const int sh = twshift + (LOGL - SB - LB);
-#pragma unroll
-            for (int c = 1; c < R; ++c) x[c] = cmul(x[c], __ldg(&tw[(c * r) << sh]));
-        }
+        if constexpr (S > 1) twiddle_powers<R, false>(x, tw, r << (twshift + (LOGL - SB - LB)));
 #pragma unroll
         for (int c = 0; c < R; ++c) s[sidx<TC>(base + c * S, col)] = x[c];
     }
@@ -122,11 +163,7 @@ __device__ __forceinline__ void inv_stage(float2* s, const float2* __restrict__ 
         float2 x[R];
 #pragma unroll
         for (int c = 0; c < R; ++c) x[c] = s[sidx<TC>(base + c * S, col)];
-        if constexpr (S > 1) {
-            const int sh = twshift + (LOGL - SB - LB);
-#pragma unroll
-            for (int c = 1; c < R; ++c) x[c] = cmulc(x[c], __ldg(&tw[(c * r) << sh]));
-        }
+        if constexpr (S > 1) twiddle_powers<R, true>(x, tw, r << (twshift + (LOGL - SB - LB)));
         Dft<R, +1>::run(x);
 #pragma unroll
         for (int j = 0; j < R; ++j) s[sidx<TC>(base + j * S, col)] = x[j];

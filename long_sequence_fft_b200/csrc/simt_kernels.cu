@@ -112,8 +112,7 @@ __device__ __forceinline__ void first_stage_global(float2* s, const float2* __re
 #pragma unroll
         for (int j = 0; j < R / 2; ++j) x[j] = io.load(j * S + r);
         Dft<R, -1>::run_half_input(x);
-#pragma unroll
-        for (int c = 1; c < R; ++c) x[c] = cmul(x[c], __ldg(&tw[c * r]));
+        twiddle_powers<R, false>(x, tw, r);
 #pragma unroll
         for (int c = 0; c < R; ++c) s[sidx<1>(c * S + r, 0)] = x[c];
     }
@@ -130,8 +129,7 @@ __device__ __forceinline__ void last_stage_global(const float2* s, const float2*
         float2 x[R];
 #pragma unroll
         for (int c = 0; c < R; ++c) x[c] = s[sidx<1>(c * S + r, 0)];
-#pragma unroll
-        for (int c = 1; c < R; ++c) x[c] = cmulc(x[c], __ldg(&tw[c * r]));
+        twiddle_powers<R, true>(x, tw, r);
         Dft<R, +1>::run(x);
 #pragma unroll
         for (int j = 0; j < R / 2; ++j) io.store(j * S + r, x[j]);
@@ -216,6 +214,32 @@ simt_fused_precompute_kernel(const T* __restrict__ k, int64_t L, float2* __restr
     const float inv = 1.0f / (float)(1 << LOGM);
     float2* out = Kf + (int64_t)h * (1 << LOGM);
     for (int p = tid; p < (1 << LOGM); p += NT) out[p] = cscale(s[sidx<1>(p, 0)], inv);
+}
+
+// Same transform written in the tensor-core kernel's filter layout
+// [h][c2][c3][c1] for M = 8192 (f = c1 + 32 c2 + 1024 c3), unnormalised.
+template <typename T>
+__global__ void __launch_bounds__(fused_threads<13>())
+simt_precompute_tc8192_kernel(const T* __restrict__ k, int64_t L, float2* __restrict__ Kf,
+                              const float2* __restrict__ tw) {
+    constexpr int LOGM = 13;
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    extern __shared__ float2 s[];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x;
+    PairRows<T> io;
+    io.u0 = k + (int64_t)h * L;
+    io.nvalid = (int)L;
+    first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
+    float2* out = Kf + (int64_t)h * (1 << LOGM);
+    for (int p = tid; p < (1 << LOGM); p += NT) {
+        const int f = (int)perm_to_freq(p, LOGM);
+        const int c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
+        out[(c2 * 8 + c3) * 32 + c1] = s[sidx<1>(p, 0)];
+    }
 }
 
 template <int LOGM, typename T>
@@ -503,6 +527,18 @@ cudaError_t simt_fused_forward(const Plan& p, const ForwardArgs& a, cudaStream_t
         case 13: return launch_fused<13, T>(p, a, st);
         case 14: return launch_fused<14, T>(p, a, st);
         default: return cudaErrorInvalidValue;
+    })
+}
+
+cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    if (p.logM != 13) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << 13);
+    FFTCONV_DISPATCH_T(p.dtype, {
+        auto kern = simt_precompute_tc8192_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (float2*)Kf, p.tw);
+        return cudaGetLastError();
     })
 }
 

@@ -119,7 +119,8 @@ def test_workload_full_size_sampled(name):
 
 def test_filter_export_matches_oracle_rfft():
     import long_sequence_fft_b200 as lsf
-    for dtype, order, N, L in (("f32", 1, 1024, 1024), ("bf16", 4, 4096, 1000), ("f16", 0, 2048, 2048)):
+    for dtype, order, N, L in (("f32", 1, 1024, 1024), ("bf16", 4, 4096, 1000), ("f16", 0, 2048, 2048),
+                               ("bf16", 0, 4096, 4096), ("f16", 0, 4096, 3000)):
         k = W.round_to(RNG.standard_normal((3, L), dtype=np.float32), dtype)
         plan = lsf.Plan(N, 3, dtype, order=order, L=L)
         Kf = plan.precompute(to_dev(k, dtype))
