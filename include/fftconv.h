@@ -143,6 +143,33 @@ FFTCONV_API int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, co
                          const uint8_t* mask_host, int64_t mask_h, void* staging,
                          size_t staging_bytes, fftconv_stream_t stream);
 
+/* fftconv_forward without a plan and without allocating: for callers that
+ * may not call cudaMalloc at all (code inside a host framework whose memory
+ * pool owns every byte of device memory, or latency-critical paths that
+ * cannot pay for cudaMalloc's implicit synchronisation).  It runs the staged
+ * passes of an order-4 plan, with their intermediate spectra and twiddle
+ * tables in the library's own statically allocated device arrays (16 MiB of
+ * scratch, held on every GPU that loads the library until the process exits).
+ * The FlashFFTConv page has no counterpart for this entry point.
+ *   u, y, w, v, block_mask, mask_h, B: as for fftconv_forward (device memory,
+ *     16-byte aligned; w, v, block_mask may be NULL).
+ *   K_f : the filter transform that fftconv_filter_precompute wrote for an
+ *     order-4 plan with the same N, H and dtype (made once, by code that may
+ *     allocate, e.g. when the filter is loaded).
+ *   N   : power of two, 256 <= N <= 2^20 (2N complex fp32 values must fit the
+ *     scratch); larger N returns FFTCONV_ERR_UNSUPPORTED with the limit in
+ *     fftconv_last_error().
+ * Calls no cudaMalloc/cudaFree and allocates nothing else.  The first call on
+ * a device resolves the device addresses of the static arrays
+ * (cudaGetSymbolAddress), so that first call should come before any stream
+ * capture.  All calls share the scratch arrays and each call overwrites them,
+ * so calls whose execution overlaps on the GPU (other streams, other host
+ * threads) race; serialise them. */
+FFTCONV_API int fftconv_forward_noalloc(const void* u, const void* K_f, void* y, int64_t B, int64_t H,
+                                        int64_t N, fftconv_dtype_t dtype, const void* w, const void* v,
+                                        const uint8_t* block_mask, int64_t mask_h,
+                                        fftconv_stream_t stream);
+
 /* Test hook: export K_f in natural order as out[h, f, 0..1] = (Re, Im) of
  * rfft(k)[f] for f in [0, N] (normalisation undone), fp32, device. */
 FFTCONV_API int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out,

@@ -85,6 +85,10 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 }  // namespace
 
+namespace fftconv {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace fftconv
+
 struct fftconv_plan_s {
     Plan p;
 };

@@ -51,6 +51,9 @@ struct ForwardArgs {
     int64_t B;
 };
 
+// Thread-local detail string returned by fftconv_last_error (api.cu).
+void set_last_error(const char* msg);
+
 // SIMT fp32 path (simt_kernels.cu)
 cudaError_t simt_fused_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
 cudaError_t simt_fused_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
