@@ -216,16 +216,19 @@ simt_fused_precompute_kernel(const T* __restrict__ k, int64_t L, float2* __restr
     for (int p = tid; p < (1 << LOGM); p += NT) out[p] = cscale(s[sidx<1>(p, 0)], inv);
 }
 
-// Same transform written in the tensor-core kernel's filter layout
-// [h][c2][c3][c1] for M = 8192 (f = c1 + 32 c2 + 1024 c3), unnormalised.
+// Same transform written in the tensor-core kernel's filter format for
+// M = 8192: per channel, 8192 complex fp16 values K[f] / s_h at position
+// ((c2*2 + c3/4)*32 + c1)*4 + c3%4 (f = c1 + 32 c2 + 1024 c3), with
+// s_h = max |Re|, |Im| over the channel stored after the H rows.
 template <typename T>
 __global__ void __launch_bounds__(fused_threads<13>())
-simt_precompute_tc8192_kernel(const T* __restrict__ k, int64_t L, float2* __restrict__ Kf,
-                              const float2* __restrict__ tw) {
+simt_precompute_tc8192_kernel(const T* __restrict__ k, int64_t L, __half2* __restrict__ Kh,
+                              float* __restrict__ scales, const float2* __restrict__ tw) {
     constexpr int LOGM = 13;
     constexpr int NT = fused_threads<LOGM>();
     constexpr int K = Sched<LOGM>::K;
     extern __shared__ float2 s[];
+    __shared__ float red[NT / 32];
     const int tid = threadIdx.x;
     const int h = blockIdx.x;
     PairRows<T> io;
@@ -234,12 +237,26 @@ simt_precompute_tc8192_kernel(const T* __restrict__ k, int64_t L, float2* __rest
     first_stage_global<LOGM, NT, T>(s, tw, io, tid);
     __syncthreads();
     fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
-    float2* out = Kf + (int64_t)h * (1 << LOGM);
+    float m = 0.f;
+    for (int p = tid; p < (1 << LOGM); p += NT) {
+        const float2 z = s[sidx<1>(p, 0)];
+        m = fmaxf(m, fmaxf(fabsf(z.x), fabsf(z.y)));
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int i = 0; i < NT / 32; ++i) m = fmaxf(m, red[i]);
+    const float sc = m > 0.f ? m : 1.f;
+    const float inv = 1.f / sc;
+    __half2* out = Kh + (int64_t)h * (1 << LOGM);
     for (int p = tid; p < (1 << LOGM); p += NT) {
         const int f = (int)perm_to_freq(p, LOGM);
         const int c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
-        out[(c2 * 8 + c3) * 32 + c1] = s[sidx<1>(p, 0)];
+        const float2 z = s[sidx<1>(p, 0)];
+        out[((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + (c3 & 3)] = __floats2half2_rn(z.x * inv, z.y * inv);
     }
+    if (tid == 0) scales[h] = sc;
 }
 
 template <int LOGM, typename T>
@@ -537,7 +554,8 @@ cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf,
         auto kern = simt_precompute_tc8192_kernel<T>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (float2*)Kf, p.tw);
+        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (__half2*)Kf,
+                                                               (float*)((uint8_t*)Kf + (size_t)p.H * (8192 * 4)), p.tw);
         return cudaGetLastError();
     })
 }

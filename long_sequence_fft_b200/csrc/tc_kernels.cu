@@ -62,8 +62,27 @@ using namespace tc;
 constexpr int kN = 4096;
 constexpr int kM = 8192;
 constexpr int kEpiWarps = 16;
-constexpr int kThreads = (kEpiWarps + 1) * 32;
-constexpr int kChunksPerUnit = 22;   // 4 chunks in each of S1..S2', 2 in S1'
+constexpr int kMmaWarps = 4;     // one MMA issuer per SMSP; issuer i owns accumulator buffer i
+constexpr int kThreads = (kEpiWarps + kMmaWarps) * 32;
+constexpr int kDBuf = 4;             // accumulator ring: 4 buffers of 64 TMEM columns
+constexpr int kChunksPerUnit = 44;   // 8 chunks in each of S1..S2', 4 in S1'
+
+// chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
+__host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
+__host__ __device__ __forceinline__ int chunk_index(int c) { return c < 40 ? (c & 7) : c - 40; }
+// Besides its buffer (chunk g waits for epilogue g - 4), a chunk reads data
+// that whole earlier epilogues wrote.  Every S3 chunk needs all of E2 (chunk
+// 15), every S2' chunk all of E3' (chunk 31), and S1''s second chunk E2' for
+// j3 = 4..7 (chunk 39); other chunks are covered by the buffer rule.  Returns
+// how many chunks back that epilogue is (0 = none).  With several MMA
+// issuers this must be explicit: chunks of one stage are issued
+// independently.
+__host__ __device__ __forceinline__ int chunk_extra_lag(int c) {
+    if (c >= 16 && c < 20) return c - 15;
+    if (c >= 32 && c < 36) return c - 31;
+    if (c == 41) return 2;
+    return 0;
+}
 constexpr uint32_t kWaitLimit = 1u << 20;
 
 // shared-memory map (bytes from a 1024-aligned base)
@@ -77,8 +96,11 @@ constexpr int kOffBS2i = kOffBS3i + 16384;   // K=64 N=64   8 KB
 constexpr int kOffBS1i = kOffBS2i + 8192;    // K=64 N=32   4 KB
 constexpr int kOffBEnd = kOffBS1i + 4096;
 constexpr int kBImageBytes = kOffBEnd - kOffBS1;   // 57344
-constexpr int kOffBars = kOffBEnd;           // 8 mbarriers
-constexpr int kOffMisc = kOffBars + 64;      // tmem base, abort flag
+constexpr int kOffK = kOffBEnd;              // the tile's filter spectrum, 8192 x half2
+constexpr int kKBytes = kM * 4;
+constexpr int kOffTwM = kOffK + kKBytes;     // exp(-2 pi i e/8192), 256 x float2
+constexpr int kOffBars = kOffTwM + 2048;     // 16 mbarrier slots
+constexpr int kOffMisc = kOffBars + 128;     // tmem base, abort flag
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;    // + alignment slack
 
 // byte offset of element (n, k) of a K x N B operand in the no-swizzle
@@ -93,12 +115,14 @@ struct TcArgs {
     const void* w;
     const void* v;
     void* y;
-    const float2* Kf;          // [H][c2][c3][c1] complex fp32, unnormalised
+    const __half2* Kh16;       // [H] rows of 8192 complex fp16 (see k16_index), unnormalised / scale
+    const float* Kscale;       // [H] per-channel scale of the fp16 rows
     const uint8_t* mask;
     int64_t mask_h;
     int64_t B, H;
-    int64_t npairs;            // H * ceil(B/2)
-    int64_t nunits;            // ceil(npairs / 4)
+    int64_t pb;                // pairs per channel, ceil(B/2)
+    int64_t tpc;               // tiles per channel, ceil(pb/4)
+    int64_t nunits;            // H * tpc
     const uint4* bimg;         // DFT factors, image of the shared-memory region
     const float2* tw1024;      // exp(-2 pi i e/1024), e < 1024
     const float2* twM;         // exp(-2 pi i e/8192), e < 256
@@ -144,16 +168,24 @@ struct PairInfo {
     bool valid;
 };
 
-__device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t pair) {
+// A tile holds 4 pairs of batch rows of ONE channel: tile u covers channel
+// u / tpc and pairs 4*(u % tpc) + q, q < 4 (pairs past ceil(B/2) are empty).
+__device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t unit, int q) {
     PairInfo p;
-    p.valid = pair < a.npairs;
-    const int64_t PB = (a.B + 1) / 2;
-    const int64_t pp = p.valid ? pair : 0;
-    p.h = pp / PB;
-    const int64_t b0 = 2 * (pp % PB), b1 = b0 + 1;
+    p.h = unit / a.tpc;
+    const int64_t bp = 4 * (unit % a.tpc) + q;
+    p.valid = bp < a.pb;
+    const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
     p.o0 = (b0 * a.H + p.h) * kN;
-    p.o1 = b1 < a.B ? (b1 * a.H + p.h) * kN : -1;
+    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * kN : -1;
     return p;
+}
+
+// position of spectrum value f = c1 + 32 c2 + 1024 c3 in a channel's fp16 row:
+// 16-byte groups of four c3 values, consecutive c1 in consecutive groups, so a
+// warp (c1 = lane) reads 512 contiguous bytes per (c2, c3 half)
+__host__ __device__ __forceinline__ int k16_index(int c1, int c2, int c3) {
+    return ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + (c3 & 3);
 }
 
 template <typename T>
@@ -161,10 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* bar = (uint64_t*)(smem + kOffBars);
-    uint64_t* bar_in = bar + 0;
-    uint64_t* dfull = bar + 1;   // [2]
-    uint64_t* dfree = bar + 3;   // [2]
-    uint64_t* bar_fin = bar + 5;
+    uint64_t* bar_in = bar + 0;    // the tile's input is in TMEM (16 epilogue warps)
+    uint64_t* dfull = bar + 1;     // [kDBuf] accumulator buffer written (tcgen05.commit)
+    uint64_t* dfree = bar + 5;     // [kDBuf] accumulator buffer drained (16 epilogue warps)
+    uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
+    uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
     uint32_t* tmem_base_sh = (uint32_t*)(smem + kOffMisc);
     volatile int* abort_flag = (volatile int*)(smem + kOffMisc + 4);
 
@@ -175,20 +208,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 
     if (tid == 0) {
         mbar_init(bar_in, kEpiWarps);
-        mbar_init(&dfull[0], 1);
-        mbar_init(&dfull[1], 1);
-        mbar_init(&dfree[0], kEpiWarps);
-        mbar_init(&dfree[1], kEpiWarps);
-        mbar_init(bar_fin, 1);
+        for (int i = 0; i < kDBuf; ++i) {
+            mbar_init(&dfull[i], 1);
+            mbar_init(&dfree[i], kEpiWarps);
+        }
+        mbar_init(bar_fin, kMmaWarps);
+        mbar_init(bar_k, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kEpiWarps) tmem_alloc(tmem_base_sh, 512);
-    // DFT factors into shared memory
+    if (warp == kEpiWarps) tmem_alloc(tmem_base_sh, 512);   // the first MMA warp owns TMEM
+    // DFT factors and the w8192 twiddle table into shared memory
     {
         uint4* dst = (uint4*)(smem + kOffBS1);
         for (int i = tid; i < kBImageBytes / 16; i += kThreads) dst[i] = __ldg(&a.bimg[i]);
+        float2* t2 = (float2*)(smem + kOffTwM);
+        for (int i = tid; i < 256; i += kThreads) t2[i] = __ldg(&a.twM[i]);
     }
+    const float2* stwM = (const float2*)(smem + kOffTwM);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -207,337 +244,355 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         }
     };
 
-    if (warp == kEpiWarps) {
-        // ============================ MMA issuer ============================
+    if (warp >= kEpiWarps) {
+        // ============================ MMA issuers ===========================
+        // A single thread can issue a tcgen05.mma only every ~100 cycles, far
+        // slower than the tensor core retires these small MMAs, so four warps
+        // issue: issuer i handles the chunks g = i (mod 4), which all use
+        // accumulator buffer i (44 chunks per tile keeps the assignment fixed).
+        const int issuer = warp - kEpiWarps;
         const uint32_t id64 = idesc_f16_f32(128, 64);
         const uint32_t id16 = idesc_f16_f32(128, 16);
-        uint32_t g = 0;          // global chunk counter
+        // descriptor bases (start address in 16-byte units in the low bits)
+        const uint64_t dS1 = make_desc(sbase + kOffBS1, 1024, 128, 0);    // K-step: +2048 B
+        const uint64_t dS2 = make_desc(sbase + kOffBS2, 1024, 128, 0);    // K-step: +2048 B
+        const uint64_t dS2i = make_desc(sbase + kOffBS2i, 1024, 128, 0);
+        const uint64_t dS3 = make_desc(sbase + kOffBS3, 256, 128, 0);     // per c2: +512 B
+        const uint64_t dS3i = make_desc(sbase + kOffBS3i, 256, 128, 0);
+        const uint64_t dS1i = make_desc(sbase + kOffBS1i, 512, 128, 0);   // N half: +256 B, K-step: +1024 B
+        const uint64_t dA = make_desc(sbase + kOffData, 16, 1024, 2);     // tile: +16384 B, K-step: +32 B
+        uint32_t g = 0;          // global chunk counter (accumulator buffer g % kDBuf)
         int iter = 0;
+        int k_issued = 0;        // filter-row copies issued
         bool ok = true;
+        g = issuer;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
             if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kChunksPerUnit && ok; ++c, ++g) {
-                const int stage = c < 20 ? (c >> 2) : 5, k = c < 20 ? (c & 3) : c - 20;
-                const uint32_t b = g & 1;
-                if (g >= 2 && !wait(&dfree[b], ((g - 2) >> 1) & 1)) {
-                    ok = false; fail(); break;
+            if (issuer == 0) {
+                if (lane == 0) {
+                    // the previous tile is finished with the filter buffer (its
+                    // epilogue warps arrived on bar_in after all their reads)
+                    mbar_expect_tx(bar_k, kKBytes);
+                    bulk_copy_g2s(smem + kOffK, a.Kh16 + (unit / a.tpc) * (int64_t)kM, kKBytes, bar_k);
                 }
-                // stages whose chunks regroup the data need every epilogue of
-                // the previous stage, including the one on the other buffer
-                if ((stage == 2 || stage == 4 || stage == 5) && k == 0 &&
-                    !wait(&dfree[b ^ 1], ((g - 1) >> 1) & 1)) {
+                ++k_issued;
+                __syncwarp();
+            }
+#pragma unroll 1
+            for (int c = issuer; c < kChunksPerUnit && ok; c += kMmaWarps, g += kMmaWarps) {
+                const int stage = chunk_stage(c), k = chunk_index(c);
+                const uint32_t b = g % kDBuf;
+                // the buffer's previous contents must have been drained ...
+                if (g >= kDBuf && !wait(&dfree[b], ((g - kDBuf) / kDBuf) & 1)) { ok = false; fail(); break; }
+                // ... and chunks that regroup the data need more recent
+                // epilogues (each warp finishes its epilogues in order)
+                const int lag = chunk_extra_lag(c);
+                if (lag && !wait(&dfree[(g - lag) % kDBuf], ((g - lag) / kDBuf) & 1)) {
                     ok = false; fail(); break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t d = tbase + 256 + 128 * b;
-                    if (stage == 0) {            // S1: A1 (TMEM) cols j3*16 + j1
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j3 = 2 * k + jj;
-                            for (int s = 0; s < 2; ++s)
-                                mma_ts(d + jj * 64, tbase + j3 * 16 + s * 8,
-                                       make_desc(sbase + kOffBS1 + s * 2 * 1024, 1024, 128, 0), id64, s);
-                        }
-                    } else if (stage == 1) {     // S2: A2 (smem tile j3)
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j3 = 2 * k + jj;
+                    // descriptors are loop-invariant bases plus an offset in
+                    // 16-byte units added to the start-address field
+                    const uint32_t d = tbase + 256 + 64 * b;
+                    if (stage == 0) {            // S1: A1 (TMEM) cols j3*16 + j1, j3 = k
+                        mma_ts(d, tbase + k * 16, dS1, id64, 0);
+                        mma_ts(d, tbase + k * 16 + 8, dS1 + 128, id64, 1);
+                    } else if (stage == 1 || stage == 4) {   // S2 / S2': smem tile j3 = k
+                        const uint64_t db = stage == 1 ? dS2 : dS2i;
+                        const uint64_t da = dA + (uint64_t)(k * (kTile >> 4));
+#pragma unroll
+                        for (int s = 0; s < 4; ++s) mma_ss(d, da + 2 * s, db + 128 * s, id64, s);
+                    } else if (stage == 2 || stage == 3) {   // S3 / S3': TMEM cols c2*8 + j3|c3
+                        const uint64_t db = (stage == 2 ? dS3 : dS3i) + (uint64_t)(4 * k * 32);
+#pragma unroll
+                        for (int cl = 0; cl < 4; ++cl) mma_ts(d + cl * 16, tbase + (4 * k + cl) * 8, db + 32 * cl, id16, 0);
+                    } else {                     // S1': j1 in [8h, 8h+8), j3 in [4jh, 4jh+4)
+                        const int h = k >> 1, jh = k & 1;
+                        const uint64_t db = dS1i + (uint64_t)(16 * h);
+                        const uint64_t da = dA + (uint64_t)(4 * jh * (kTile >> 4));
+#pragma unroll
+                        for (int j3l = 0; j3l < 4; ++j3l) {
+#pragma unroll
                             for (int s = 0; s < 4; ++s)
-                                mma_ss(d + jj * 64, make_desc(sbase + kOffData + j3 * kTile + 32 * s, 16, 1024, 2),
-                                       make_desc(sbase + kOffBS2 + s * 2 * 1024, 1024, 128, 0), id64, s);
-                        }
-                    } else if (stage == 2 || stage == 3) {   // S3 / S3': A (TMEM) cols c2*8 + j3|c3
-                        const int off = stage == 2 ? kOffBS3 : kOffBS3i;
-                        for (int cl = 0; cl < 8; ++cl) {
-                            const int c2 = 8 * k + cl;
-                            mma_ts(d + cl * 16, tbase + c2 * 8,
-                                   make_desc(sbase + off + c2 * 512, 256, 128, 0), id16, 0);
-                        }
-                    } else if (stage == 4) {     // S2': A5 (smem tile j3), K = c2
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j3 = 2 * k + jj;
-                            for (int s = 0; s < 4; ++s)
-                                mma_ss(d + jj * 64, make_desc(sbase + kOffData + j3 * kTile + 32 * s, 16, 1024, 2),
-                                       make_desc(sbase + kOffBS2i + s * 2 * 1024, 1024, 128, 0), id64, s);
-                        }
-                    } else {                     // S1': A6 (smem tile j3), K = c1; chunk k: j1 in [8k, 8k+8)
-                        for (int j3 = 0; j3 < 8; ++j3) {
-                            for (int s = 0; s < 4; ++s)
-                                mma_ss(d + j3 * 16, make_desc(sbase + kOffData + j3 * kTile + 32 * s, 16, 1024, 2),
-                                       make_desc(sbase + kOffBS1i + 256 * k + s * 2 * 512, 512, 128, 0), id16, s);
+                                mma_ss(d + j3l * 16, da + j3l * (kTile >> 4) + 2 * s, db + 64 * s, id16, s);
                         }
                     }
                     tc_commit(&dfull[b]);
                 }
                 __syncwarp();
+                if (c == issuer && issuer == 1) {
+                    // warm L2 with the next tile's rows (u, w, v of both
+                    // sequences of each pair, and the filter spectrum) while
+                    // this tile is being transformed
+                    const int64_t nu = unit + gridDim.x;
+                    if (nu < a.nunits && lane < 28) {
+                        const PairInfo Q = pair_info(a, nu, lane >> 3);
+                        const int which = lane & 7;
+                        const void* src = nullptr;
+                        uint32_t bytes = kN * sizeof(T);
+                        if (Q.valid) {
+                            if (which == 0) src = (const T*)a.u + Q.o0;
+                            else if (which == 1 && a.w) src = (const T*)a.w + Q.o0;
+                            else if (which == 2 && a.v) src = (const T*)a.v + Q.o0;
+                            else if (which == 3 && Q.o1 >= 0) src = (const T*)a.u + Q.o1;
+                            else if (which == 4 && Q.o1 >= 0 && a.w) src = (const T*)a.w + Q.o1;
+                            else if (which == 5 && Q.o1 >= 0 && a.v) src = (const T*)a.v + Q.o1;
+                            else if (which == 6 && (lane >> 3) == 0) { src = a.Kh16 + Q.h * (int64_t)kM; bytes = kKBytes; }
+                        }
+                        if (src) prefetch_l2(src, bytes);
+                    }
+                    __syncwarp();
+                }
             }
         }
-        // drain: every issued MMA must finish before TMEM is released
+        // drain: every issued MMA and the last filter copy must finish before
+        // TMEM and shared memory are released -- bounded, and regardless of
+        // an abort
         if (lane == 0) tc_commit(bar_fin);
         __syncwarp();
-        if (!wait(bar_fin, 0)) fail();
+        bool drained = false;
+        for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(bar_fin, 0);
+        if (!drained) fail();
+        if (issuer == 0 && k_issued > 0) {
+            drained = false;
+            for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(bar_k, (k_issued - 1) & 1);
+            if (!drained) fail();
+        }
+        __syncwarp();
     } else {
         // ========================== epilogue warps ==========================
         const int q = warp & 3;          // lane quarter = pair within the tile
         const int s = warp >> 2;         // column slice
         const uint32_t lq = (uint32_t)(32 * q) << 16;
-        const int64_t N = kN;
-        const int64_t nblk = N / 32;
+        const int64_t nblk = kN / 32;
 
-        // loop-invariant twiddles
-        // (the wM^(c1 j3) twiddles are read from the L1-resident table per use)
-        float2 tw1[8], tw3[8];
+        // w1024^(c1 l) with (c1, l) = (8s + i, lane) in E1 and (lane, 8s + i)
+        // in E2' -- the same eight values, kept in registers; wM^(c1 j3) with
+        // c1 = lane in E2 and E3' comes from the shared-memory table
+        float2 tw[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            tw1[i] = __ldg(&a.tw1024[((8 * s + i) * lane) & 1023]);   // w1024^(c1 l), l = lane
-            tw3[i] = __ldg(&a.tw1024[(lane * (8 * s + i)) & 1023]);   // w1024^(c1 l), c1 = lane
-        }
+        for (int i = 0; i < 8; ++i) tw[i] = __ldg(&a.tw1024[((8 * s + i) * lane) & 1023]);
 
         uint32_t g = 0;
         int iter = 0;
         bool ok = true;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
-            const PairInfo P = pair_info(a, unit * 4 + q);
-            const T* u0 = (const T*)a.u + P.o0;
-            const T* w0 = a.w ? (const T*)a.w + P.o0 : nullptr;
+            const PairInfo P = pair_info(a, unit, q);
+            // row pointers are formed from the kernel parameters on use (they
+            // live in constant memory), keeping registers for the stages
             const bool has1 = P.o1 >= 0;
-            const T* u1 = has1 ? (const T*)a.u + P.o1 : nullptr;
-            const T* w1 = (has1 && a.w) ? (const T*)a.w + P.o1 : nullptr;
 
-            // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [4s, 4s+4)
+            // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [4s, 4s+4).
+            // Loads are issued in batches before any use (absent rows or gates
+            // read a present row and are masked afterwards).
             {
-                uint32_t packed[8][4];   // [j3][j1 - 4s]
+                const int64_t oo1 = has1 ? P.o1 : P.o0;
+                const T* pu0 = (const T*)a.u + P.o0;
+                const T* pw0 = a.w ? (const T*)a.w + P.o0 : pu0;
+                const T* pu1 = (const T*)a.u + oo1;
+                const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
+                const bool has_w = a.w != nullptr;
+                const bool keep0 = P.valid, keep1 = has1;
 #pragma unroll
-                for (int jl = 0; jl < 4; ++jl) {
-                    const int j1 = 4 * s + jl;
-                    const int64_t t0 = 256 * j1 + 8 * lane;
-                    float xa[8], xb[8];
-                    if (P.valid) {
-                        const uint4 ua = __ldg((const uint4*)(u0 + t0));
-                        const uint32_t uw[4] = {ua.x, ua.y, ua.z, ua.w};
-                        uint32_t ww[4] = {0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u};
-                        if (w0) { const uint4 wa = __ldg((const uint4*)(w0 + t0)); ww[0] = wa.x; ww[1] = wa.y; ww[2] = wa.z; ww[3] = wa.w; }
+                for (int jp = 0; jp < 2; ++jp) {
+                    uint4 ld[2][4];
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const int64_t t0 = 256 * (4 * s + 2 * jp + jh) + 8 * lane;
+                        ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
+                        ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
+                        ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
+                        ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+                    }
+                    uint32_t pk[8][2];
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
+                        const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
+                        const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
+                        const uint32_t wb[4] = {ld[jh][3].x, ld[jh][3].y, ld[jh][3].z, ld[jh][3].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 uu = IO<T>::unpack2(uw[e]);
-                            const float2 gg = w0 ? IO<T>::unpack2(ww[e]) : make_float2(1.f, 1.f);
-                            xa[2 * e] = uu.x * gg.x;
-                            xa[2 * e + 1] = uu.y * gg.y;
-                        }
-                        if (u1) {
-                            const uint4 ub = __ldg((const uint4*)(u1 + t0));
-                            const uint32_t ubw[4] = {ub.x, ub.y, ub.z, ub.w};
-                            uint32_t wb[4];
-                            if (w1) { const uint4 t4 = __ldg((const uint4*)(w1 + t0)); wb[0] = t4.x; wb[1] = t4.y; wb[2] = t4.z; wb[3] = t4.w; }
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 uu = IO<T>::unpack2(ubw[e]);
-                                const float2 gg = w1 ? IO<T>::unpack2(wb[e]) : make_float2(1.f, 1.f);
-                                xb[2 * e] = uu.x * gg.x;
-                                xb[2 * e + 1] = uu.y * gg.y;
+                            float2 xa = IO<T>::unpack2(ua[e]), xb = IO<T>::unpack2(ub[e]);
+                            if (has_w) {
+                                const float2 g0 = IO<T>::unpack2(wa[e]), g1 = IO<T>::unpack2(wb[e]);
+                                xa.x *= g0.x; xa.y *= g0.y; xb.x *= g1.x; xb.y *= g1.y;
                             }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) xb[e] = 0.f;
+                            if (!keep0) xa = make_float2(0.f, 0.f);
+                            if (!keep1) xb = make_float2(0.f, 0.f);
+                            pk[2 * e][jh] = pack_h2(xa.x, xb.x);
+                            pk[2 * e + 1][jh] = pack_h2(xa.y, xb.y);
                         }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) { xa[e] = 0.f; xb[e] = 0.f; }
                     }
 #pragma unroll
-                    for (int j3 = 0; j3 < 8; ++j3) packed[j3][jl] = pack_h2(xa[j3], xb[j3]);
+                    for (int j3 = 0; j3 < 8; ++j3) tmem_st2(tbase + lq + j3 * 16 + 4 * s + 2 * jp, pk[j3][0], pk[j3][1]);
                 }
-#pragma unroll
-                for (int j3 = 0; j3 < 8; ++j3) tmem_st4(tbase + lq + j3 * 16 + 4 * s, packed[j3]);
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_in);
             }
 
-            // warm L2 with the next tile's rows (u, w, v of both sequences and
-            // the filter spectrum) while this tile is being transformed
-            if (s == 0 && lane < 7) {
-                const int64_t nu = unit + gridDim.x;
-                if (nu < a.nunits) {
-                    const PairInfo Q = pair_info(a, nu * 4 + q);
-                    if (Q.valid) {
-                        const void* src = nullptr;
-                        uint32_t bytes = kN * sizeof(T);
-                        if (lane == 0) src = (const T*)a.u + Q.o0;
-                        else if (lane == 1 && a.w) src = (const T*)a.w + Q.o0;
-                        else if (lane == 2 && a.v) src = (const T*)a.v + Q.o0;
-                        else if (lane == 3 && Q.o1 >= 0) src = (const T*)a.u + Q.o1;
-                        else if (lane == 4 && Q.o1 >= 0 && a.w) src = (const T*)a.w + Q.o1;
-                        else if (lane == 5 && Q.o1 >= 0 && a.v) src = (const T*)a.v + Q.o1;
-                        else if (lane == 6) { src = a.Kf + Q.h * (int64_t)kM; bytes = kM * sizeof(float2); }
-                        if (src) prefetch_l2(src, bytes);
-                    }
-                }
-            }
-
-            // per-tile epilogue state
-            const float2* Kh = a.Kf + P.h * (int64_t)kM;
+            const __half2* Ks = (const __half2*)(smem + kOffK);
+            // loaded once per tile and pinned in a register (an opaque move
+            // keeps the compiler from re-issuing the global load at each use)
+            float kscale = __ldg(&a.Kscale[P.h]);
+            asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : P.h) * nblk : nullptr;
-            T* y0 = (T*)a.y + P.o0;
-            T* y1 = has1 ? (T*)a.y + P.o1 : nullptr;
-            const T* v0 = a.v ? (const T*)a.v + P.o0 : nullptr;
-            const T* v1 = (has1 && a.v) ? (const T*)a.v + P.o1 : nullptr;
 
 #pragma unroll 1
             for (int c = 0; c < kChunksPerUnit; ++c, ++g) {
-                const int stage = c < 20 ? (c >> 2) : 5, k = c < 20 ? (c & 3) : c - 20;
-                const uint32_t b = g & 1;
-                if (!wait(&dfull[b], (g >> 1) & 1)) { ok = false; fail(); break; }
-                tc_fence_after();
-                const uint32_t dcol = tbase + lq + 256 + 128 * b;
-
-                if (stage == 0) {
-                    // E1: lane = l; columns (jj, c1 = 8s + i); twiddle w1024^(c1 l);
-                    // write A2 tile j3, row 32q + c1, K element pair 2l
+                const int stage = chunk_stage(c), k = chunk_index(c);
+                const uint32_t b = g % kDBuf;
+                // output gate values for an output chunk, requested before the
+                // accumulator wait so the latency overlaps the MMA
+                uint2 va[2], vb[2];
+                if (stage == 5) {
+                    const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+                    const int h = k >> 1, jh = k & 1;
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
-                        uint32_t r[16];
-                        tmem_ld16(dcol + jj * 64 + 16 * s, r);
-                        tc_wait_ld();
-                        uint8_t* tile = smem + kOffData + (2 * k + jj) * kTile;
+                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane + 4 * jh;
+                        va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
+                        vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                    }
+                }
+                if (c == 16 && !wait(bar_k, iter & 1)) { ok = false; fail(); break; }
+                if (!wait(&dfull[b], (g / kDBuf) & 1)) { ok = false; fail(); break; }
+                tc_fence_after();
+                const uint32_t dcol = tbase + lq + 256 + 64 * b;
+
+                if (stage == 0) {
+                    // E1: lane = l; columns c1 = 8s + i of j3 = k; twiddle
+                    // w1024^(c1 l); write A2 tile k, row 32q + c1, K pair 2l
+                    uint32_t r[16];
+                    tmem_ld16(dcol + 16 * s, r);
+                    tc_wait_ld();
+                    uint8_t* tile = smem + kOffData + k * kTile;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), tw1[i]);
-                            const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
-                            *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
-                        }
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), tw[i]);
+                        const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
+                        *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
                     }
                     fence_proxy_async_smem();
                 } else if (stage == 1) {
-                    // E2: lane = c1; columns (jj, c2 = 8s + i); twiddle wM^(c1 j3);
-                    // write A3 (TMEM) col c2*8 + j3
-                    uint32_t h[2][8];
+                    // E2: lane = c1; columns c2 = 8s + i of j3 = k; twiddle
+                    // wM^(c1 j3); write A3 (TMEM) col c2*8 + j3
+                    uint32_t r[16];
+                    tmem_ld16(dcol + 16 * s, r);
+                    const float2 t = stwM[lane * k];
+                    tc_wait_ld();
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        uint32_t r[16];
-                        tmem_ld16(dcol + jj * 64 + 16 * s, r);
-                        tc_wait_ld();
-                        const float2 t = __ldg(&a.twM[lane * (2 * k + jj)]);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), t);
-                            h[jj][i] = pack_h2(z.x, z.y);
-                        }
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), t);
+                        tmem_st1(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z.x, z.y));
                     }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) tmem_st2(tbase + lq + (8 * s + i) * 8 + 2 * k, h[0][i], h[1][i]);
                     tc_wait_st();
                 } else if (stage == 2) {
-                    // EK: lane = c1; columns (c2 = 8k + 2s + cc, c3); times K_f;
-                    // write A4 (TMEM) col c2*8 + c3 (in place)
+                    // EK: lane = c1; columns c3 of c2 = 4k + s; times the filter
+                    // spectrum; write A4 (TMEM) col c2*8 + c3 (in place)
+                    const int c2 = 4 * k + s;
+                    uint32_t r[16];
+                    tmem_ld16(dcol + 16 * s, r);
+                    const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
+                    const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
+                    const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    float2 kv[8];
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const int c2 = 8 * k + 2 * s + cc;
-                        uint32_t r[16];
-                        tmem_ld16(dcol + (2 * s + cc) * 16, r);
-                        float2 kv[8];
-#pragma unroll
-                        for (int c3 = 0; c3 < 8; ++c3) kv[c3] = __ldg(&Kh[(c2 * 8 + c3) * 32 + lane]);
-                        tc_wait_ld();
-                        uint32_t h8[8];
+                    for (int c3 = 0; c3 < 8; ++c3) {
+                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
+                        kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
+                    }
+                    if (mrow) {
+                        // frequency-sparse filter: zero the masked bins (f and
+                        // its mirror M - f share one rfft bin)
 #pragma unroll
                         for (int c3 = 0; c3 < 8; ++c3) {
-                            float2 kk = kv[c3];
-                            if (mrow) {
-                                const int64_t f = lane + 32 * c2 + 1024 * c3;
-                                const int64_t gb = f <= N ? f : kM - f;
-                                int64_t blk = gb >> 5;
-                                if (blk >= nblk) blk = nblk - 1;
-                                if (__ldg(&mrow[blk]) == 0) kk = make_float2(0.f, 0.f);
-                            }
-                            const float2 z = cmul(f2(r[2 * c3], r[2 * c3 + 1]), kk);
-                            h8[c3] = pack_h2(z.x, z.y);
+                            const int f = lane + 32 * c2 + 1024 * c3;
+                            int blk = (f <= kN ? f : kM - f) >> 5;
+                            blk = blk < (int)nblk ? blk : (int)nblk - 1;
+                            if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
                         }
-                        tmem_st8(tbase + lq + c2 * 8, h8);
                     }
+                    tc_wait_ld();
+                    uint32_t h8[8];
+#pragma unroll
+                    for (int c3 = 0; c3 < 8; ++c3) {
+                        const float2 z = cmul(f2(r[2 * c3], r[2 * c3 + 1]), kv[c3]);
+                        h8[c3] = pack_h2(z.x, z.y);
+                    }
+                    tmem_st8(tbase + lq + c2 * 8, h8);
                     tc_wait_st();
                 } else if (stage == 3) {
-                    // E3': lane = c1; columns (c2 = 8k + cl, j3 = 2s + jj); twiddle
-                    // conj wM^(c1 j3); write A5 tile j3, row 32q + c1, K pair 2*c2
-                    uint32_t h[2][8];
-                    const float2 t0 = __ldg(&a.twM[lane * (2 * s)]), t1 = __ldg(&a.twM[lane * (2 * s + 1)]);
+                    // E3': lane = c1; columns (c2 = 4k + cl, j3 = 2s + jj); twiddle
+                    // conj wM^(c1 j3); write A5 tile j3, row 32q + c1, K pairs of
+                    // c2 = 4k..4k+3 as one 16-byte store
+                    uint32_t h[2][4];
+                    const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
 #pragma unroll
-                    for (int cl = 0; cl < 8; ++cl) {
+                    for (int cl = 0; cl < 4; ++cl) {
                         uint32_t r[4];
                         tmem_ld4(dcol + cl * 16 + 4 * s, r);
                         tc_wait_ld();
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const float2 z = cmulc(f2(r[2 * jj], r[2 * jj + 1]), jj ? t1 : t0);
-                            h[jj][cl] = pack_h2(z.x, z.y);
-                        }
+                        const float2 z0 = cmulc(f2(r[0], r[1]), t0);
+                        const float2 z1 = cmulc(f2(r[2], r[3]), t1);
+                        h[0][cl] = pack_h2(z0.x, z0.y);
+                        h[1][cl] = pack_h2(z1.x, z1.y);
                     }
+                    const uint32_t m = 32 * q + lane;
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         uint8_t* tile = smem + kOffData + (2 * s + jj) * kTile;
-                        const uint32_t m = 32 * q + lane;
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + (32 * k + 16 * hh);
-                            *(uint4*)(tile + swz(off)) =
-                                make_uint4(h[jj][4 * hh], h[jj][4 * hh + 1], h[jj][4 * hh + 2], h[jj][4 * hh + 3]);
-                        }
+                        const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * k;
+                        *(uint4*)(tile + swz(off)) = make_uint4(h[jj][0], h[jj][1], h[jj][2], h[jj][3]);
                     }
                     fence_proxy_async_smem();
                 } else if (stage == 4) {
-                    // E2': lane = c1; columns (jj, l = 8s + i); twiddle conj w1024^(c1 l);
-                    // write A6 tile j3 (in place), row 32q + l, K pair 2*c1
+                    // E2': lane = c1; columns l = 8s + i of j3 = k; twiddle conj
+                    // w1024^(c1 l); write A6 tile k (in place), row 32q + l, K pair 2*c1
+                    uint32_t r[16];
+                    tmem_ld16(dcol + 16 * s, r);
+                    tc_wait_ld();
+                    uint8_t* tile = smem + kOffData + k * kTile;
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        uint32_t r[16];
-                        tmem_ld16(dcol + jj * 64 + 16 * s, r);
-                        tc_wait_ld();
-                        uint8_t* tile = smem + kOffData + (2 * k + jj) * kTile;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 z = cmulc(f2(r[2 * i], r[2 * i + 1]), tw3[i]);
-                            const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
-                            *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
-                        }
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 z = cmulc(f2(r[2 * i], r[2 * i + 1]), tw[i]);
+                        const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
+                        *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
                     }
                     fence_proxy_async_smem();
-                } else {
-                    // EO: lane = l; chunk k holds j1 in [8k, 8k+8) for every j3 at
-                    // columns j3*16 + 2*(j1 - 8k); this warp takes j1 = 8k + 2s + jj
-                    // and writes y = v * z at t = 256 j1 + 8 l + j3, 8 consecutive t
-                    // per (row, j1) as one 16-byte store.
-                    if (P.valid) {
-                        uint4 va[2], vb[2];
+                } else if (P.valid) {
+                    // EO: lane = l; chunk k = (h, jh) holds j1 in [8h, 8h+8) for
+                    // j3 in [4jh, 4jh+4) at columns j3l*16 + 2*(j1 - 8h); this warp
+                    // takes j1 = 8h + 2s + jj and writes y = v * z at
+                    // t = 256 j1 + 8 l + 4 jh + j3l, four consecutive t per row
+                    const int h = k >> 1, jh = k & 1;
+                    uint32_t r[4][4];
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int64_t t0 = 256 * (8 * k + 2 * s + jj) + 8 * lane;
-                            va[jj] = v0 ? __ldg((const uint4*)(v0 + t0)) : make_uint4(0, 0, 0, 0);
-                            vb[jj] = v1 ? __ldg((const uint4*)(v1 + t0)) : make_uint4(0, 0, 0, 0);
-                        }
-                        uint32_t r[8][4];
+                    for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dcol + j3l * 16 + 4 * s, r[j3l]);
+                    tc_wait_ld();
 #pragma unroll
-                        for (int j3 = 0; j3 < 8; ++j3) tmem_ld4(dcol + j3 * 16 + 4 * s, r[j3]);
-                        tc_wait_ld();
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane + 4 * jh;
+                        const uint32_t vaw[2] = {va[jj].x, va[jj].y};
+                        const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
+                        uint32_t oa[2], ob[2];
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int64_t t0 = 256 * (8 * k + 2 * s + jj) + 8 * lane;
-                            const uint32_t vaw[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
-                            const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
-                            uint32_t oa[4], ob[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float a0 = __uint_as_float(r[2 * e][2 * jj]), a1 = __uint_as_float(r[2 * e + 1][2 * jj]);
-                                float b0 = __uint_as_float(r[2 * e][2 * jj + 1]), b1 = __uint_as_float(r[2 * e + 1][2 * jj + 1]);
-                                if (v0) { const float2 g = IO<T>::unpack2(vaw[e]); a0 *= g.x; a1 *= g.y; }
-                                if (v1) { const float2 g = IO<T>::unpack2(vbw[e]); b0 *= g.x; b1 *= g.y; }
-                                oa[e] = IO<T>::pack2(a0, a1);
-                                ob[e] = IO<T>::pack2(b0, b1);
+                        for (int e = 0; e < 2; ++e) {
+                            float a0 = __uint_as_float(r[2 * e][2 * jj]), a1 = __uint_as_float(r[2 * e + 1][2 * jj]);
+                            float b0 = __uint_as_float(r[2 * e][2 * jj + 1]), b1 = __uint_as_float(r[2 * e + 1][2 * jj + 1]);
+                            if (a.v) {
+                                const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
+                                a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
                             }
-                            *(uint4*)(y0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-                            if (y1) *(uint4*)(y1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                            oa[e] = IO<T>::pack2(a0, a1);
+                            ob[e] = IO<T>::pack2(b0, b1);
                         }
+                        *(uint2*)((T*)a.y + P.o0 + t0) = make_uint2(oa[0], oa[1]);
+                        if (has1) *(uint2*)((T*)a.y + P.o1 + t0) = make_uint2(ob[0], ob[1]);
                     }
                 }
                 tc_fence_before();
@@ -549,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kEpiWarps) {
+    if (warp == kEpiWarps) {     // the warp that allocated
         tc_fence_after();
         tmem_dealloc(tbase, 512);
         tmem_relinquish();
@@ -637,14 +692,15 @@ std::vector<float2> twiddle_table(int n, int count) {
     return t;
 }
 
-__global__ void tc_export_kernel(const float2* __restrict__ Kf, float* __restrict__ out, int64_t H) {
+__global__ void tc_export_kernel(const __half2* __restrict__ Kh, const float* __restrict__ scale,
+                                 float* __restrict__ out, int64_t H) {
     const int64_t total = H * (kN + 1);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t h = i / (kN + 1), f = i % (kN + 1);
-        const int64_t c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
-        const float2 z = Kf[h * kM + (c2 * 8 + c3) * 32 + c1];
-        out[2 * i] = z.x;
-        out[2 * i + 1] = z.y;
+        const int c1 = (int)(f & 31), c2 = (int)((f >> 5) & 31), c3 = (int)(f >> 10);
+        const float2 z = __half22float2(Kh[h * kM + k16_index(c1, c2, c3)]);
+        out[2 * i] = z.x * scale[h];
+        out[2 * i + 1] = z.y * scale[h];
     }
 }
 
@@ -698,7 +754,9 @@ void tc_plan_free(Plan& p) {
     p.tc = nullptr;
 }
 
-size_t tc_filter_bytes(const Plan& p) { return (size_t)p.H * kM * sizeof(float2); }
+// K_f: [H] rows of 8192 complex fp16 (scaled so the largest component is 1),
+// then [H] fp32 scales.
+size_t tc_filter_bytes(const Plan& p) { return (size_t)p.H * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15)); }
 
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
     return simt_precompute_to_tc_layout(p, k, Kf, s);
@@ -708,11 +766,13 @@ cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     const TcResources* r = (const TcResources*)p.tc;
     TcArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
-    a.Kf = (const float2*)fa.Kf;
+    a.Kh16 = (const __half2*)fa.Kf;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H;
-    a.npairs = p.H * ((fa.B + 1) / 2);
-    a.nunits = (a.npairs + 3) / 4;
+    a.pb = (fa.B + 1) / 2;
+    a.tpc = (a.pb + 3) / 4;
+    a.nunits = p.H * a.tpc;
     a.bimg = (const uint4*)r->bimg;
     a.tw1024 = r->tw1024;
     a.twM = r->twM;
@@ -729,7 +789,8 @@ cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream
     const int64_t total = p.H * (kN + 1);
     int blocks = (int)((total + 255) / 256);
     if (blocks > 65535) blocks = 65535;
-    tc_export_kernel<<<blocks, 256, 0, s>>>((const float2*)Kf, out, p.H);
+    tc_export_kernel<<<blocks, 256, 0, s>>>((const __half2*)Kf,
+                                            (const float*)((const uint8_t*)Kf + (size_t)p.H * kKBytes), out, p.H);
     return cudaGetLastError();
 }
 

@@ -53,10 +53,10 @@ def test_small_shapes_full_compare(dtype, order, B, H, N):
     assert_close(y, ref, dtype, f"{dtype} order={order} path={plan.path_name} B={B} H={H} N={N}")
 
 
+@pytest.mark.parametrize("N", [2048, 4096])
 @pytest.mark.parametrize("order", [1, 4, 0])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_partial_and_masked(order, dtype):
-    N = 2048
+def test_partial_and_masked(order, dtype, N):
     inp = _rand_inputs(3, 2, N, 300, dtype, gated=True, seed=7)
     y, _ = run_cuda(inp, dtype, order=order)
     assert_close(y, _oracle(inp), dtype, "partial L=300")
@@ -127,7 +127,10 @@ def test_filter_export_matches_oracle_rfft():
         got = plan.export_rfft(Kf).cpu().numpy().astype(np.complex128)
         ref = oracle.filter_rfft(k, N)
         err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-        assert err <= 1e-5, (dtype, order, err)
+        # fp32 spectra: 1e-5; the tensor-core path stores fp16 spectra with a
+        # per-channel scale: 1e-3 relative (half-precision storage bound)
+        tol = 1e-3 if plan.path_name == "tc_fused" else 1e-5
+        assert err <= tol, (dtype, order, plan.path_name, err)
 
 
 @pytest.mark.parametrize("order", [1, 4])
