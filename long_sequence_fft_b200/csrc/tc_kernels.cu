@@ -442,148 +442,161 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : P.h) * nblk : nullptr;
 
+            // Chunks are handled in pairs (c, c+1) of the same stage: both
+            // accumulators are waited for and loaded before one TMEM-load
+            // wait, and the fences and barrier arrivals are shared, which
+            // halves the fixed latency per chunk.
 #pragma unroll 1
-            for (int c = 0; c < kChunksPerUnit; ++c, ++g) {
-                const int stage = chunk_stage(c), k = chunk_index(c);
-                const uint32_t b = g % kDBuf;
-                // output gate values for an output chunk, requested before the
-                // accumulator wait so the latency overlaps the MMA
-                uint2 va[2], vb[2];
-                if (stage == 5) {
-                    const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
-                    const int h = k >> 1, jh = k & 1;
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane + 4 * jh;
-                        va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
-                        vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
-                    }
-                }
+            for (int c = 0; c < kChunksPerUnit; c += 2, g += 2) {
+                const int stage = chunk_stage(c), k = chunk_index(c);   // k even; chunks k and k + 1
+                const uint32_t b0 = g % kDBuf, b1 = (g + 1) % kDBuf;
                 if (c == 16 && !wait(bar_k, iter & 1)) { ok = false; fail(); break; }
-                if (!wait(&dfull[b], (g / kDBuf) & 1)) { ok = false; fail(); break; }
+                if (!wait(&dfull[b0], (g / kDBuf) & 1)) { ok = false; fail(); break; }
+                if (!wait(&dfull[b1], ((g + 1) / kDBuf) & 1)) { ok = false; fail(); break; }
                 tc_fence_after();
-                const uint32_t dcol = tbase + lq + 256 + 64 * b;
+                const uint32_t dc[2] = {tbase + lq + 256 + 64 * b0, tbase + lq + 256 + 64 * b1};
 
-                if (stage == 0) {
-                    // E1: lane = l; columns c1 = 8s + i of j3 = k; twiddle
-                    // w1024^(c1 l); write A2 tile k, row 32q + c1, K pair 2l
-                    uint32_t r[16];
-                    tmem_ld16(dcol + 16 * s, r);
+                if (stage == 0 || stage == 4) {
+                    // E1 (S1 -> S2): lane = l; columns c1 = 8s + i of j3 = k + cc;
+                    //   twiddle w1024^(c1 l); A2 tile j3, row 32q + c1, K pair 2l.
+                    // E2' (S2' -> S1'): lane = c1; columns l = 8s + i of j3;
+                    //   twiddle conj w1024^(c1 l); A6 tile j3, row 32q + l, K pair 2c1.
+                    // The same eight twiddles and the same store pattern.
+                    uint32_t r[2][16];
+                    tmem_ld16(dc[0] + 16 * s, r[0]);
+                    tmem_ld16(dc[1] + 16 * s, r[1]);
                     tc_wait_ld();
-                    uint8_t* tile = smem + kOffData + k * kTile;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), tw[i]);
-                        const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
-                        *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint8_t* tile = smem + kOffData + (k + cc) * kTile;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 x = f2(r[cc][2 * i], r[cc][2 * i + 1]);
+                            const float2 z = stage == 0 ? cmul(x, tw[i]) : cmulc(x, tw[i]);
+                            const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
+                            *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
+                        }
                     }
                     fence_proxy_async_smem();
                 } else if (stage == 1) {
-                    // E2: lane = c1; columns c2 = 8s + i of j3 = k; twiddle
-                    // wM^(c1 j3); write A3 (TMEM) col c2*8 + j3
-                    uint32_t r[16];
-                    tmem_ld16(dcol + 16 * s, r);
-                    const float2 t = stwM[lane * k];
+                    // E2: lane = c1; columns c2 = 8s + i of j3 = k, k+1; twiddle
+                    // wM^(c1 j3); A3 (TMEM) cols c2*8 + j3 (two adjacent columns)
+                    uint32_t r[2][16];
+                    tmem_ld16(dc[0] + 16 * s, r[0]);
+                    tmem_ld16(dc[1] + 16 * s, r[1]);
+                    const float2 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
                     tc_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float2 z = cmul(f2(r[2 * i], r[2 * i + 1]), t);
-                        tmem_st1(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z.x, z.y));
+                        const float2 z0 = cmul(f2(r[0][2 * i], r[0][2 * i + 1]), t0);
+                        const float2 z1 = cmul(f2(r[1][2 * i], r[1][2 * i + 1]), t1);
+                        tmem_st2(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z0.x, z0.y), pack_h2(z1.x, z1.y));
                     }
                     tc_wait_st();
                 } else if (stage == 2) {
-                    // EK: lane = c1; columns c3 of c2 = 4k + s; times the filter
-                    // spectrum; write A4 (TMEM) col c2*8 + c3 (in place)
-                    const int c2 = 4 * k + s;
-                    uint32_t r[16];
-                    tmem_ld16(dcol + 16 * s, r);
-                    const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
-                    const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
-                    const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    float2 kv[8];
+                    // EK: lane = c1; columns c3 of c2 = 4(k+cc) + s; times the
+                    // filter spectrum; A4 (TMEM) cols c2*8 + c3 (in place)
+                    uint32_t r[2][16];
+                    tmem_ld16(dc[0] + 16 * s, r[0]);
+                    tmem_ld16(dc[1] + 16 * s, r[1]);
+                    tc_wait_ld();
 #pragma unroll
-                    for (int c3 = 0; c3 < 8; ++c3) {
-                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
-                        kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
-                    }
-                    if (mrow) {
-                        // frequency-sparse filter: zero the masked bins (f and
-                        // its mirror M - f share one rfft bin)
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c2 = 4 * (k + cc) + s;
+                        const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
+                        const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
+                        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                        float2 kv[8];
 #pragma unroll
                         for (int c3 = 0; c3 < 8; ++c3) {
-                            const int f = lane + 32 * c2 + 1024 * c3;
-                            int blk = (f <= kN ? f : kM - f) >> 5;
-                            blk = blk < (int)nblk ? blk : (int)nblk - 1;
-                            if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
+                            const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
+                            kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
                         }
-                    }
-                    tc_wait_ld();
-                    uint32_t h8[8];
+                        if (mrow) {
+                            // frequency-sparse filter: zero the masked bins (f and
+                            // its mirror M - f share one rfft bin)
 #pragma unroll
-                    for (int c3 = 0; c3 < 8; ++c3) {
-                        const float2 z = cmul(f2(r[2 * c3], r[2 * c3 + 1]), kv[c3]);
-                        h8[c3] = pack_h2(z.x, z.y);
+                            for (int c3 = 0; c3 < 8; ++c3) {
+                                const int f = lane + 32 * c2 + 1024 * c3;
+                                int blk = (f <= kN ? f : kM - f) >> 5;
+                                blk = blk < (int)nblk ? blk : (int)nblk - 1;
+                                if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
+                            }
+                        }
+                        uint32_t h8[8];
+#pragma unroll
+                        for (int c3 = 0; c3 < 8; ++c3) {
+                            const float2 z = cmul(f2(r[cc][2 * c3], r[cc][2 * c3 + 1]), kv[c3]);
+                            h8[c3] = pack_h2(z.x, z.y);
+                        }
+                        tmem_st8(tbase + lq + c2 * 8, h8);
                     }
-                    tmem_st8(tbase + lq + c2 * 8, h8);
                     tc_wait_st();
                 } else if (stage == 3) {
-                    // E3': lane = c1; columns (c2 = 4k + cl, j3 = 2s + jj); twiddle
-                    // conj wM^(c1 j3); write A5 tile j3, row 32q + c1, K pairs of
-                    // c2 = 4k..4k+3 as one 16-byte store
-                    uint32_t h[2][4];
-                    const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
+                    // E3': lane = c1; columns (c2 = 4(k+cc) + cl, j3 = 2s + jj);
+                    // twiddle conj wM^(c1 j3); A5 tile j3, row 32q + c1, K pairs of
+                    // c2 = 4k..4k+7 as two 16-byte stores
+                    uint32_t r[2][4][4];
 #pragma unroll
-                    for (int cl = 0; cl < 4; ++cl) {
-                        uint32_t r[4];
-                        tmem_ld4(dcol + cl * 16 + 4 * s, r);
-                        tc_wait_ld();
-                        const float2 z0 = cmulc(f2(r[0], r[1]), t0);
-                        const float2 z1 = cmulc(f2(r[2], r[3]), t1);
-                        h[0][cl] = pack_h2(z0.x, z0.y);
-                        h[1][cl] = pack_h2(z1.x, z1.y);
-                    }
+                    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                        for (int cl = 0; cl < 4; ++cl) tmem_ld4(dc[cc] + cl * 16 + 4 * s, r[cc][cl]);
+                    const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
+                    tc_wait_ld();
                     const uint32_t m = 32 * q + lane;
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         uint8_t* tile = smem + kOffData + (2 * s + jj) * kTile;
-                        const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * k;
-                        *(uint4*)(tile + swz(off)) = make_uint4(h[jj][0], h[jj][1], h[jj][2], h[jj][3]);
-                    }
-                    fence_proxy_async_smem();
-                } else if (stage == 4) {
-                    // E2': lane = c1; columns l = 8s + i of j3 = k; twiddle conj
-                    // w1024^(c1 l); write A6 tile k (in place), row 32q + l, K pair 2*c1
-                    uint32_t r[16];
-                    tmem_ld16(dcol + 16 * s, r);
-                    tc_wait_ld();
-                    uint8_t* tile = smem + kOffData + k * kTile;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float2 z = cmulc(f2(r[2 * i], r[2 * i + 1]), tw[i]);
-                        const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
-                        *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
+                        for (int cc = 0; cc < 2; ++cc) {
+                            uint32_t hq[4];
+#pragma unroll
+                            for (int cl = 0; cl < 4; ++cl) {
+                                const float2 z = cmulc(f2(r[cc][cl][2 * jj], r[cc][cl][2 * jj + 1]), jj ? t1 : t0);
+                                hq[cl] = pack_h2(z.x, z.y);
+                            }
+                            const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * (k + cc);
+                            *(uint4*)(tile + swz(off)) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+                        }
                     }
                     fence_proxy_async_smem();
                 } else if (P.valid) {
-                    // EO: lane = l; chunk k = (h, jh) holds j1 in [8h, 8h+8) for
-                    // j3 in [4jh, 4jh+4) at columns j3l*16 + 2*(j1 - 8h); this warp
-                    // takes j1 = 8h + 2s + jj and writes y = v * z at
-                    // t = 256 j1 + 8 l + 4 jh + j3l, four consecutive t per row
-                    const int h = k >> 1, jh = k & 1;
-                    uint32_t r[4][4];
+                    // EO: lane = l; the pair (h, jh = 0, 1) holds j1 in [8h, 8h+8)
+                    // for all eight j3 at columns (j3 % 4)*16 + 2*(j1 - 8h); this
+                    // warp takes j1 = 8h + 2s + jj and writes y = v * z for the
+                    // eight consecutive t = 256 j1 + 8 l + j3 as one 16-byte store
+                    const int h = k >> 1;
+                    // output gate values: rows j1 = 8h + 2s + jj, eight
+                    // consecutive t each, requested before the TMEM loads
+                    uint4 va[2], vb[2];
+                    {
+                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
-                    for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dcol + j3l * 16 + 4 * s, r[j3l]);
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane;
+                            va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
+                            vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                        }
+                    }
+                    uint32_t r[2][4][4];
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                        for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dc[cc] + j3l * 16 + 4 * s, r[cc][j3l]);
                     tc_wait_ld();
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
-                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane + 4 * jh;
-                        const uint32_t vaw[2] = {va[jj].x, va[jj].y};
-                        const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
-                        uint32_t oa[2], ob[2];
+                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane;
+                        const uint32_t vaw[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
+                        const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
+                        uint32_t oa[4], ob[4];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            float a0 = __uint_as_float(r[2 * e][2 * jj]), a1 = __uint_as_float(r[2 * e + 1][2 * jj]);
-                            float b0 = __uint_as_float(r[2 * e][2 * jj + 1]), b1 = __uint_as_float(r[2 * e + 1][2 * jj + 1]);
+                        for (int e = 0; e < 4; ++e) {
+                            // j3 = 2e, 2e + 1 live in chunk cc = e / 2 at j3l = 2(e % 2), +1
+                            const int cc = e >> 1, j3l = 2 * (e & 1);
+                            float a0 = __uint_as_float(r[cc][j3l][2 * jj]), a1 = __uint_as_float(r[cc][j3l + 1][2 * jj]);
+                            float b0 = __uint_as_float(r[cc][j3l][2 * jj + 1]);
+                            float b1 = __uint_as_float(r[cc][j3l + 1][2 * jj + 1]);
                             if (a.v) {
                                 const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
                                 a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
@@ -591,13 +604,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             oa[e] = IO<T>::pack2(a0, a1);
                             ob[e] = IO<T>::pack2(b0, b1);
                         }
-                        *(uint2*)((T*)a.y + P.o0 + t0) = make_uint2(oa[0], oa[1]);
-                        if (has1) *(uint2*)((T*)a.y + P.o1 + t0) = make_uint2(ob[0], ob[1]);
+                        *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                        if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dfree[b]);
+                if (lane == 0) {
+                    mbar_arrive(&dfree[b0]);
+                    mbar_arrive(&dfree[b1]);
+                }
             }
         }
     }
