@@ -126,38 +126,6 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup():
-    import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 # --------------------------------------------------------------- oracle ---
 
 def time_oracle(w: W.Workload, target_s: float = 10.0):
@@ -240,15 +208,19 @@ def main():
     import torch
     import long_sequence_fft_b200 as lsf
 
-    world, rank, local = dist_setup()
+    from long_sequence_fft_b200 import multigpu as mg
+    ctx = mg.init_from_env()
+    world, rank = ctx.world, ctx.rank
     w = W.WORKLOADS[args.workload]
     if args.B is not None:
         w = w.with_shape(B=args.B)
+    w = W.shard_of(w, rank)                  # this rank's channel shard
     if w.B * w.H * w.N == 0:
         raise SystemExit("empty workload")
 
     # inputs: seeded host generation, copied to HBM once (each rank convolves
-    # its own channel shard; all shards have the workload's shape)
+    # its own channel shard, drawn from its own seeded streams; all shards
+    # have the workload's shape)
     inp = W.make_all(w)
     dt = W.torch_dtype(w.dtype)
     dev = lambda a: None if a is None else torch.from_numpy(a).to(dt).cuda()
@@ -276,7 +248,7 @@ def main():
     assert plan.device_status() == 0
 
     # timed region: K forward calls, barrier + synchronize on both sides
-    barrier(world)
+    mg.barrier(ctx)
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -285,14 +257,14 @@ def main():
             plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
         stop.record(stream)
         torch.cuda.synchronize()
-    barrier(world)
+    mg.barrier(ctx)
     ms_local = start.elapsed_time(stop)
-    ms = max_over_ranks(ms_local, world)
+    ms = mg.max_over_ranks(ctx, ms_local)
     status = plan.device_status()
     if status != 0:
         raise SystemExit(f"device status {status} after the timed region")
     ms_per_step = ms / args.steps
-    value = world * w.elems / (ms_per_step * 1e-3)
+    value = mg.job_throughput(w.elems, ctx, ms_per_step)
 
     launches_per_step = 1
     if plan.path == lsf.PATH_SIMT_STAGED:
@@ -304,6 +276,7 @@ def main():
         if rank == 0:
             print(json.dumps({"profile_run": True, "ms_per_step": ms_per_step, "workload": w.name, "B": w.B,
                               "path": plan.path_name}), flush=True)
+        mg.shutdown(ctx)
         return 0
 
     # end to end through the host-buffer entry point (pinned memory, copies in
@@ -316,14 +289,14 @@ def main():
                           dtype=torch.uint8, device="cuda")
     plan.forward_host(uh, Kf, yh, staging, w_host=gh, v_host=vh, mask_host=mh)
     torch.cuda.synchronize()
-    barrier(world)
+    mg.barrier(ctx)
     s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s2.record(stream)
     for _ in range(args.e2e_steps):
         plan.forward_host(uh, Kf, yh, staging, w_host=gh, v_host=vh, mask_host=mh)
     t2.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(s2.elapsed_time(t2), world) / args.e2e_steps
+    e2e_ms = mg.max_over_ranks(ctx, s2.elapsed_time(t2)) / args.e2e_steps
     esz = uh.element_size()
     h2d = w.elems * esz * (1 + (gh is not None) + (vh is not None)) + (0 if mh is None else mh.numel())
     d2h = w.elems * esz
@@ -349,7 +322,7 @@ def main():
                      "traffic": None if traffic is None else traffic.get("bytes_per_launch"),
                      "algorithmic_bytes": abytes,
                      "kernel": kernel_key},
-        "e2e": {"value": world * w.elems / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": mg.job_throughput(w.elems, ctx, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "filter_precompute_ms": precompute_ms,
@@ -360,9 +333,7 @@ def main():
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    mg.shutdown(ctx)
     return 0
 
 

@@ -46,3 +46,23 @@ def test_sample_points_cover_edges():
     s, t = W.sample_points(w, nseq=4, nrand=5)
     assert len(s) == len(t) == 4 * 8
     assert set([0, 1, w.N - 1]).issubset(set(t.tolist()))
+
+
+def test_channel_shards_own_streams_share_symbols_and_mask():
+    base = W.WORKLOADS["dna_bf16_n1m"].with_shape(H=4, N=4096)
+    s0, s1 = W.shard_of(base, 0), W.shard_of(base, 1)
+    assert np.array_equal(W.make_input(s0), W.make_input(base))     # shard 0 is the workload
+    u0, u1 = W.make_input(s0), W.make_input(s1)
+    assert not np.array_equal(u0, u1)                              # own projection
+    # the symbol stream is shared: positions that carry one symbol on shard 0
+    # (equal columns across all channels) carry one symbol on shard 1 too
+    key0 = [tuple(u0[0, :, t]) for t in range(base.N)]
+    key1 = [tuple(u1[0, :, t]) for t in range(base.N)]
+    first = {}
+    for t, kk in enumerate(key0):
+        first.setdefault(kk, t)
+    for t, kk in enumerate(key0):
+        assert key1[t] == key1[first[kk]]
+    sp = W.WORKLOADS["sparse_bf16_n8k"].with_shape(B=1, H=2)
+    assert np.array_equal(W.make_mask(W.shard_of(sp, 3)), W.make_mask(sp))
+    assert not np.array_equal(W.make_filter(W.shard_of(sp, 3)), W.make_filter(sp))

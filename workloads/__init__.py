@@ -41,6 +41,7 @@ class Workload:
     u_kind: str = "normal"   # "normal" | "dna"
     sparsity: float = 0.0    # fraction of mask blocks zeroed (0 = no mask)
     description: str = ""
+    shard: int = 0           # channel shard (one per rank); 0 = the workload itself
 
     @property
     def seed(self) -> int:
@@ -87,8 +88,28 @@ WORKLOADS = {
 BENCH_WORKLOAD = "gated_bf16_n4k"
 
 
+# Tensors every channel shard shares: the DNA symbol stream (one per batch
+# row, embedded into every channel) and the frequency mask row.
+SHARED_TENSORS = ("sym", "mask")
+
+
 def _rng(w: Workload, tensor: str) -> np.random.Generator:
-    return np.random.default_rng([w.seed, TENSOR_IDS[tensor]])
+    if w.shard == 0 or tensor in SHARED_TENSORS:
+        return np.random.default_rng([w.seed, TENSOR_IDS[tensor]])
+    return np.random.default_rng([w.seed, TENSOR_IDS[tensor], w.shard])
+
+
+def shard_of(w: Workload, rank: int) -> Workload:
+    """Rank `rank`'s channel shard of the multi-GPU problem built on `w`.
+
+    With R ranks the whole problem has H*R channels: shard r holds channels
+    [r*H, (r+1)*H), drawn from its own seeded streams (u, w, v, k and the DNA
+    projection take the shard id as a third seed word), while the DNA symbol
+    stream and the mask row are the same on every shard.  Shard 0 is the
+    workload itself, so a one-rank run is unchanged."""
+    if rank < 0:
+        raise ValueError(rank)
+    return dataclasses.replace(w, shard=rank)
 
 
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
