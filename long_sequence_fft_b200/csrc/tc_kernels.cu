@@ -375,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i) tw[i] = __ldg(&a.tw1024[((8 * s + i) * lane) & 1023]);
 
-        uint32_t g = 0;
         int iter = 0;
         bool ok = true;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
@@ -442,130 +441,174 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : P.h) * nblk : nullptr;
 
-            // Chunks are handled in pairs (c, c+1) of the same stage: both
-            // accumulators are waited for and loaded before one TMEM-load
-            // wait, and the fences and barrier arrivals are shared, which
-            // halves the fixed latency per chunk.
-#pragma unroll 1
-            for (int c = 0; c < kChunksPerUnit; c += 2, g += 2) {
-                const int stage = chunk_stage(c), k = chunk_index(c);   // k even; chunks k and k + 1
-                const uint32_t b0 = g % kDBuf, b1 = (g + 1) % kDBuf;
-                if (c == 16 && !wait(bar_k, iter & 1)) { ok = false; fail(); break; }
-                if (!wait(&dfull[b0], (g / kDBuf) & 1)) { ok = false; fail(); break; }
-                if (!wait(&dfull[b1], ((g + 1) / kDBuf) & 1)) { ok = false; fail(); break; }
+            // Accumulator chunks are handled in pairs (c, c+1) of one stage:
+            // both are waited for and loaded before one TMEM-load wait, and
+            // the fences and barrier arrivals are shared.  Each stage has its
+            // own loop, so the stage, the ring slots (chunk c of a tile uses
+            // buffer c % 4; 44 chunks per tile) and the store patterns are
+            // fixed at compile time.
+            auto begin_pair = [&](int c) -> bool {
+                const uint32_t par = (uint32_t)(iter ^ (c >> 2)) & 1u;   // use number 11*iter + c/4 of the buffer
+                if (!wait(&dfull[c & 3], par) || !wait(&dfull[(c & 3) + 1], par)) {
+                    fail();
+                    return false;
+                }
                 tc_fence_after();
-                const uint32_t dc[2] = {tbase + lq + 256 + 64 * b0, tbase + lq + 256 + 64 * b1};
+                return true;
+            };
+            auto end_pair = [&](int c) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&dfree[c & 3]);
+                    mbar_arrive(&dfree[(c & 3) + 1]);
+                }
+            };
+            auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (c & 3); };
 
-                if (stage == 0 || stage == 4) {
-                    // E1 (S1 -> S2): lane = l; columns c1 = 8s + i of j3 = k + cc;
-                    //   twiddle w1024^(c1 l); A2 tile j3, row 32q + c1, K pair 2l.
-                    // E2' (S2' -> S1'): lane = c1; columns l = 8s + i of j3;
-                    //   twiddle conj w1024^(c1 l); A6 tile j3, row 32q + l, K pair 2c1.
-                    // The same eight twiddles and the same store pattern.
-                    uint32_t r[2][16];
-                    tmem_ld16(dc[0] + 16 * s, r[0]);
-                    tmem_ld16(dc[1] + 16 * s, r[1]);
-                    tc_wait_ld();
+            // E1 (S1 -> S2): lane = l; columns c1 = 8s + i of j3 = k + cc;
+            //   twiddle w1024^(c1 l); A2 tile j3, row 32q + c1, K pair 2l.
+            // E2' (S2' -> S1'): lane = c1; columns l = 8s + i of j3;
+            //   twiddle conj w1024^(c1 l); A6 tile j3, row 32q + l, K pair 2c1.
+            // The same eight twiddles and the same store pattern.
+            auto e_transpose = [&](int c, int k, bool conj) {
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tc_wait_ld();
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        uint8_t* tile = smem + kOffData + (k + cc) * kTile;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 x = f2(r[cc][2 * i], r[cc][2 * i + 1]);
-                            const float2 z = stage == 0 ? cmul(x, tw[i]) : cmulc(x, tw[i]);
-                            const uint32_t off = (uint32_t)(4 * q + s) * 1024 + i * 128 + ((4 * lane) ^ (i << 4));
-                            *(uint32_t*)(tile + off) = pack_h2(z.x, z.y);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                } else if (stage == 1) {
-                    // E2: lane = c1; columns c2 = 8s + i of j3 = k, k+1; twiddle
-                    // wM^(c1 j3); A3 (TMEM) cols c2*8 + j3 (two adjacent columns)
-                    uint32_t r[2][16];
-                    tmem_ld16(dc[0] + 16 * s, r[0]);
-                    tmem_ld16(dc[1] + 16 * s, r[1]);
-                    const float2 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
-                    tc_wait_ld();
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint8_t* tile = smem + kOffData + (k + cc) * kTile + (4 * q + s) * 1024;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float2 z0 = cmul(f2(r[0][2 * i], r[0][2 * i + 1]), t0);
-                        const float2 z1 = cmul(f2(r[1][2 * i], r[1][2 * i + 1]), t1);
-                        tmem_st2(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z0.x, z0.y), pack_h2(z1.x, z1.y));
+                        const float2 x = f2(r[cc][2 * i], r[cc][2 * i + 1]);
+                        const float2 z = conj ? cmulc(x, tw[i]) : cmul(x, tw[i]);
+                        *(uint32_t*)(tile + i * 128 + ((4 * lane) ^ (i << 4))) = pack_h2(z.x, z.y);
                     }
-                    tc_wait_st();
-                } else if (stage == 2) {
-                    // EK: lane = c1; columns c3 of c2 = 4(k+cc) + s; times the
-                    // filter spectrum; A4 (TMEM) cols c2*8 + c3 (in place)
-                    uint32_t r[2][16];
-                    tmem_ld16(dc[0] + 16 * s, r[0]);
-                    tmem_ld16(dc[1] + 16 * s, r[1]);
-                    tc_wait_ld();
+                }
+                fence_proxy_async_smem();
+            };
+
+#pragma unroll 1
+            for (int k = 0; k < 8; k += 2) {
+                if (!(ok = begin_pair(k))) break;
+                e_transpose(k, k, false);
+                end_pair(k);
+            }
+            // E2: lane = c1; columns c2 = 8s + i of j3 = k, k+1; twiddle
+            // wM^(c1 j3); A3 (TMEM) cols c2*8 + j3 (two adjacent columns)
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 8 + k;
+                if (!(ok = begin_pair(c))) break;
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                const float2 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 z0 = cmul(f2(r[0][2 * i], r[0][2 * i + 1]), t0);
+                    const float2 z1 = cmul(f2(r[1][2 * i], r[1][2 * i + 1]), t1);
+                    tmem_st2(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z0.x, z0.y), pack_h2(z1.x, z1.y));
+                }
+                tc_wait_st();
+                end_pair(c);
+            }
+            // EK: lane = c1; columns c3 of c2 = 4(k+cc) + s; times the filter
+            // spectrum; A4 (TMEM) cols c2*8 + c3 (in place)
+            if (ok && !(ok = wait(bar_k, iter & 1))) fail();
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 16 + k;
+                if (!(ok = begin_pair(c))) break;
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tc_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c2 = 4 * (k + cc) + s;
+                    const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
+                    const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
+                    const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    float2 kv[8];
+#pragma unroll
+                    for (int c3 = 0; c3 < 8; ++c3) {
+                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
+                        kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
+                    }
+                    if (mrow) {
+                        // frequency-sparse filter: zero the masked bins (f and
+                        // its mirror M - f share one rfft bin)
+#pragma unroll
+                        for (int c3 = 0; c3 < 8; ++c3) {
+                            const int f = lane + 32 * c2 + 1024 * c3;
+                            int blk = (f <= kN ? f : kM - f) >> 5;
+                            blk = blk < (int)nblk ? blk : (int)nblk - 1;
+                            if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
+                        }
+                    }
+                    uint32_t h8[8];
+#pragma unroll
+                    for (int c3 = 0; c3 < 8; ++c3) {
+                        const float2 z = cmul(f2(r[cc][2 * c3], r[cc][2 * c3 + 1]), kv[c3]);
+                        h8[c3] = pack_h2(z.x, z.y);
+                    }
+                    tmem_st8(tbase + lq + c2 * 8, h8);
+                }
+                tc_wait_st();
+                end_pair(c);
+            }
+            // E3': lane = c1; columns (c2 = 4(k+cc) + cl, j3 = 2s + jj);
+            // twiddle conj wM^(c1 j3); A5 tile j3, row 32q + c1, K pairs of
+            // c2 = 4k..4k+7 as two 16-byte stores
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 24 + k;
+                if (!(ok = begin_pair(c))) break;
+                uint32_t r[2][4][4];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                    for (int cl = 0; cl < 4; ++cl) tmem_ld4(dcol(c + cc) + cl * 16 + 4 * s, r[cc][cl]);
+                const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
+                tc_wait_ld();
+                const uint32_t m = 32 * q + lane;
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    uint8_t* tile = smem + kOffData + (2 * s + jj) * kTile;
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        const int c2 = 4 * (k + cc) + s;
-                        const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
-                        const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
-                        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                        float2 kv[8];
+                        uint32_t hq[4];
 #pragma unroll
-                        for (int c3 = 0; c3 < 8; ++c3) {
-                            const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
-                            kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
+                        for (int cl = 0; cl < 4; ++cl) {
+                            const float2 z = cmulc(f2(r[cc][cl][2 * jj], r[cc][cl][2 * jj + 1]), jj ? t1 : t0);
+                            hq[cl] = pack_h2(z.x, z.y);
                         }
-                        if (mrow) {
-                            // frequency-sparse filter: zero the masked bins (f and
-                            // its mirror M - f share one rfft bin)
-#pragma unroll
-                            for (int c3 = 0; c3 < 8; ++c3) {
-                                const int f = lane + 32 * c2 + 1024 * c3;
-                                int blk = (f <= kN ? f : kM - f) >> 5;
-                                blk = blk < (int)nblk ? blk : (int)nblk - 1;
-                                if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
-                            }
-                        }
-                        uint32_t h8[8];
-#pragma unroll
-                        for (int c3 = 0; c3 < 8; ++c3) {
-                            const float2 z = cmul(f2(r[cc][2 * c3], r[cc][2 * c3 + 1]), kv[c3]);
-                            h8[c3] = pack_h2(z.x, z.y);
-                        }
-                        tmem_st8(tbase + lq + c2 * 8, h8);
+                        const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * (k + cc);
+                        *(uint4*)(tile + swz(off)) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
                     }
-                    tc_wait_st();
-                } else if (stage == 3) {
-                    // E3': lane = c1; columns (c2 = 4(k+cc) + cl, j3 = 2s + jj);
-                    // twiddle conj wM^(c1 j3); A5 tile j3, row 32q + c1, K pairs of
-                    // c2 = 4k..4k+7 as two 16-byte stores
-                    uint32_t r[2][4][4];
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                        for (int cl = 0; cl < 4; ++cl) tmem_ld4(dc[cc] + cl * 16 + 4 * s, r[cc][cl]);
-                    const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
-                    tc_wait_ld();
-                    const uint32_t m = 32 * q + lane;
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        uint8_t* tile = smem + kOffData + (2 * s + jj) * kTile;
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
-                            uint32_t hq[4];
-#pragma unroll
-                            for (int cl = 0; cl < 4; ++cl) {
-                                const float2 z = cmulc(f2(r[cc][cl][2 * jj], r[cc][cl][2 * jj + 1]), jj ? t1 : t0);
-                                hq[cl] = pack_h2(z.x, z.y);
-                            }
-                            const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * (k + cc);
-                            *(uint4*)(tile + swz(off)) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                } else if (P.valid) {
-                    // EO: lane = l; the pair (h, jh = 0, 1) holds j1 in [8h, 8h+8)
-                    // for all eight j3 at columns (j3 % 4)*16 + 2*(j1 - 8h); this
-                    // warp takes j1 = 8h + 2s + jj and writes y = v * z for the
-                    // eight consecutive t = 256 j1 + 8 l + j3 as one 16-byte store
-                    const int h = k >> 1;
+                }
+                fence_proxy_async_smem();
+                end_pair(c);
+            }
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 32 + k;
+                if (!(ok = begin_pair(c))) break;
+                e_transpose(c, k, true);
+                end_pair(c);
+            }
+            // EO: lane = l; the pair (h, jh = 0, 1) holds j1 in [8h, 8h+8) for
+            // all eight j3 at columns (j3 % 4)*16 + 2*(j1 - 8h); this warp takes
+            // j1 = 8h + 2s + jj and writes y = v * z for the eight consecutive
+            // t = 256 j1 + 8 l + j3 as one 16-byte store
+#pragma unroll 1
+            for (int h = 0; h < 2 && ok; ++h) {
+                const int c = 40 + 2 * h;
+                if (!(ok = begin_pair(c))) break;
+                if (P.valid) {
                     // output gate values: rows j1 = 8h + 2s + jj, eight
                     // consecutive t each, requested before the TMEM loads
                     uint4 va[2], vb[2];
@@ -582,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-                        for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dc[cc] + j3l * 16 + 4 * s, r[cc][j3l]);
+                        for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dcol(c + cc) + j3l * 16 + 4 * s, r[cc][j3l]);
                     tc_wait_ld();
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
@@ -608,12 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&dfree[b0]);
-                    mbar_arrive(&dfree[b1]);
-                }
+                end_pair(c);
             }
         }
     }
