@@ -27,11 +27,12 @@
 // lane (S1, S3 and their inverses) take A from TMEM; the two stages that
 // contract the lane digit (S2, S2') and the last inverse stage take A from
 // shared memory, written by the previous epilogue in the transposed order
-// (the "on-chip transpose").  Accumulators are fp32 in TMEM; twiddles and the
-// filter product are applied in fp32 by the epilogue warps, which round to
-// fp16 for the next stage.  Each DFT factor carries 1/sqrt(n), so the forward
-// and inverse transforms are unitary and the filter spectrum is used
-// unnormalised.
+// (the "on-chip transpose").  Accumulators are fp32 in TMEM.  The epilogue
+// warps round them to fp16 and apply the twiddles in packed half precision
+// (the rounding the next stage's operands take anyway, plus one product
+// rounding); the filter product is taken in fp32 before rounding.  Each
+// DFT factor carries 1/sqrt(n), so the forward and inverse transforms are
+// unitary and the filter spectrum is used unnormalised.
 //
 // Warp roles: warps 0..15 are epilogue warps (warp w serves lane quarter
 // w % 4 and the column slice w / 4), warp 16 issues the MMAs.  Accumulators
@@ -159,6 +160,25 @@ __device__ __forceinline__ uint32_t pack_h2(float re, float im) {
 }
 __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
+// Twiddle products in packed half precision.  A twiddle t = (tr, ti) is held
+// as the two half2 values tp = (tr, ti) and tq = (-ti, tr); then
+//   x t = re(x) tp + im(x) tq,   x conj(t) = re(x) tp* + im(x) tq*
+// with tp* = (tr, -ti) and tq* = (ti, tr), each a sign flip of one half.
+struct Tw16 {
+    uint32_t p, q;
+};
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ Tw16 tw16(float2 t) {
+    return {h2u(__floats2half2_rn(t.x, t.y)), h2u(__floats2half2_rn(-t.y, t.x))};
+}
+__device__ __forceinline__ Tw16 tw16_conj(Tw16 t) { return {t.p ^ 0x80000000u, t.q ^ 0x00008000u}; }
+// x (fp32 accumulator pair) rounded to fp16, times t; returns packed fp16
+__device__ __forceinline__ uint32_t cmul_h(uint32_t xr, uint32_t xi, Tw16 t) {
+    const __half2 x = __floats2half2_rn(__uint_as_float(xr), __uint_as_float(xi));
+    return h2u(__hfma2(__low2half2(x), u2h(t.p), __hmul2(__high2half2(x), u2h(t.q))));
+}
+
 // 128-byte swizzle of a logical byte offset inside a 1024-byte-aligned tile
 __device__ __forceinline__ uint32_t swz(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
 
@@ -222,10 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
     {
         uint4* dst = (uint4*)(smem + kOffBS1);
         for (int i = tid; i < kBImageBytes / 16; i += kThreads) dst[i] = __ldg(&a.bimg[i]);
-        float2* t2 = (float2*)(smem + kOffTwM);
-        for (int i = tid; i < 256; i += kThreads) t2[i] = __ldg(&a.twM[i]);
+        Tw16* t2 = (Tw16*)(smem + kOffTwM);
+        for (int i = tid; i < 256; i += kThreads) t2[i] = tw16(__ldg(&a.twM[i]));
     }
-    const float2* stwM = (const float2*)(smem + kOffTwM);
+    const Tw16* stwM = (const Tw16*)(smem + kOffTwM);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -371,9 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         // w1024^(c1 l) with (c1, l) = (8s + i, lane) in E1 and (lane, 8s + i)
         // in E2' -- the same eight values, kept in registers; wM^(c1 j3) with
         // c1 = lane in E2 and E3' comes from the shared-memory table
-        float2 tw[8];
+        Tw16 tw[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) tw[i] = __ldg(&a.tw1024[((8 * s + i) * lane) & 1023]);
+        for (int i = 0; i < 8; ++i) tw[i] = tw16(__ldg(&a.tw1024[((8 * s + i) * lane) & 1023]));
 
         int iter = 0;
         bool ok = true;
@@ -471,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // E2' (S2' -> S1'): lane = c1; columns l = 8s + i of j3;
             //   twiddle conj w1024^(c1 l); A6 tile j3, row 32q + l, K pair 2c1.
             // The same eight twiddles and the same store pattern.
-            auto e_transpose = [&](int c, int k, bool conj) {
+            auto e_transpose = [&](int c, int k) {
                 uint32_t r[2][16];
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
@@ -481,9 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     uint8_t* tile = smem + kOffData + (k + cc) * kTile + (4 * q + s) * 1024;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float2 x = f2(r[cc][2 * i], r[cc][2 * i + 1]);
-                        const float2 z = conj ? cmulc(x, tw[i]) : cmul(x, tw[i]);
-                        *(uint32_t*)(tile + i * 128 + ((4 * lane) ^ (i << 4))) = pack_h2(z.x, z.y);
+                        *(uint32_t*)(tile + i * 128 + ((4 * lane) ^ (i << 4))) = cmul_h(r[cc][2 * i], r[cc][2 * i + 1], tw[i]);
                     }
                 }
                 fence_proxy_async_smem();
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll 1
             for (int k = 0; k < 8; k += 2) {
                 if (!(ok = begin_pair(k))) break;
-                e_transpose(k, k, false);
+                e_transpose(k, k);
                 end_pair(k);
             }
             // E2: lane = c1; columns c2 = 8s + i of j3 = k, k+1; twiddle
@@ -504,14 +522,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 uint32_t r[2][16];
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
-                const float2 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
+                const Tw16 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
                 tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float2 z0 = cmul(f2(r[0][2 * i], r[0][2 * i + 1]), t0);
-                    const float2 z1 = cmul(f2(r[1][2 * i], r[1][2 * i + 1]), t1);
-                    tmem_st2(tbase + lq + (8 * s + i) * 8 + k, pack_h2(z0.x, z0.y), pack_h2(z1.x, z1.y));
-                }
+                for (int i = 0; i < 8; ++i)
+                    tmem_st2(tbase + lq + (8 * s + i) * 8 + k, cmul_h(r[0][2 * i], r[0][2 * i + 1], t0),
+                             cmul_h(r[1][2 * i], r[1][2 * i + 1], t1));
                 tc_wait_st();
                 end_pair(c);
             }
@@ -572,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
                     for (int cl = 0; cl < 4; ++cl) tmem_ld4(dcol(c + cc) + cl * 16 + 4 * s, r[cc][cl]);
-                const float2 t0 = stwM[lane * (2 * s)], t1 = stwM[lane * (2 * s + 1)];
+                const Tw16 t0 = tw16_conj(stwM[lane * (2 * s)]), t1 = tw16_conj(stwM[lane * (2 * s + 1)]);
                 tc_wait_ld();
                 const uint32_t m = 32 * q + lane;
 #pragma unroll
@@ -582,10 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     for (int cc = 0; cc < 2; ++cc) {
                         uint32_t hq[4];
 #pragma unroll
-                        for (int cl = 0; cl < 4; ++cl) {
-                            const float2 z = cmulc(f2(r[cc][cl][2 * jj], r[cc][cl][2 * jj + 1]), jj ? t1 : t0);
-                            hq[cl] = pack_h2(z.x, z.y);
-                        }
+                        for (int cl = 0; cl < 4; ++cl) hq[cl] = cmul_h(r[cc][cl][2 * jj], r[cc][cl][2 * jj + 1], jj ? t1 : t0);
                         const uint32_t off = (m >> 3) * 1024 + (m & 7) * 128 + 16 * (k + cc);
                         *(uint4*)(tile + swz(off)) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
                     }
@@ -593,13 +606,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 fence_proxy_async_smem();
                 end_pair(c);
             }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 32 + k;
                 if (!(ok = begin_pair(c))) break;
-                e_transpose(c, k, true);
+                e_transpose(c, k);
                 end_pair(c);
             }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
             // EO: lane = l; the pair (h, jh = 0, 1) holds j1 in [8h, 8h+8) for
             // all eight j3 at columns (j3 % 4)*16 + 2*(j1 - 8h); this warp takes
             // j1 = 8h + 2s + jj and writes y = v * z for the eight consecutive
