@@ -532,7 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 end_pair(c);
             }
             // EK: lane = c1; columns c3 of c2 = 4(k+cc) + s; times the filter
-            // spectrum; A4 (TMEM) cols c2*8 + c3 (in place)
+            // spectrum row in its fp16 form K/scale (|K/scale| <= 1, so the
+            // inverse stages see values no larger than the forward output);
+            // the channel scale is applied to y in fp32.  A4 (TMEM) cols
+            // c2*8 + c3 (in place)
             if (ok && !(ok = wait(bar_k, iter & 1))) fail();
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
@@ -547,13 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     const int c2 = 4 * (k + cc) + s;
                     const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
                     const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
-                    const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    float2 kv[8];
-#pragma unroll
-                    for (int c3 = 0; c3 < 8; ++c3) {
-                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&kw[c3]));
-                        kv[c3] = make_float2(kk.x * kscale, kk.y * kscale);
-                    }
+                    uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
                     if (mrow) {
                         // frequency-sparse filter: zero the masked bins (f and
                         // its mirror M - f share one rfft bin)
@@ -562,14 +559,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             const int f = lane + 32 * c2 + 1024 * c3;
                             int blk = (f <= kN ? f : kM - f) >> 5;
                             blk = blk < (int)nblk ? blk : (int)nblk - 1;
-                            if (__ldg(&mrow[blk]) == 0) kv[c3] = make_float2(0.f, 0.f);
+                            if (__ldg(&mrow[blk]) == 0) kw[c3] = 0u;
                         }
                     }
                     uint32_t h8[8];
 #pragma unroll
                     for (int c3 = 0; c3 < 8; ++c3) {
-                        const float2 z = cmul(f2(r[cc][2 * c3], r[cc][2 * c3 + 1]), kv[c3]);
-                        h8[c3] = pack_h2(z.x, z.y);
+                        // x K = re(K) (xr, xi) + im(K) (-xi, xr), packed half
+                        const float xr = __uint_as_float(r[cc][2 * c3]), xi = __uint_as_float(r[cc][2 * c3 + 1]);
+                        const __half2 x = __floats2half2_rn(xr, xi), xs = __floats2half2_rn(-xi, xr);
+                        const __half2 kk = u2h(kw[c3]);
+                        h8[c3] = h2u(__hfma2(__low2half2(kk), x, __hmul2(__high2half2(kk), xs)));
                     }
                     tmem_st8(tbase + lq + c2 * 8, h8);
                 }
@@ -654,9 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         for (int e = 0; e < 4; ++e) {
                             // j3 = 2e, 2e + 1 live in chunk cc = e / 2 at j3l = 2(e % 2), +1
                             const int cc = e >> 1, j3l = 2 * (e & 1);
-                            float a0 = __uint_as_float(r[cc][j3l][2 * jj]), a1 = __uint_as_float(r[cc][j3l + 1][2 * jj]);
-                            float b0 = __uint_as_float(r[cc][j3l][2 * jj + 1]);
-                            float b1 = __uint_as_float(r[cc][j3l + 1][2 * jj + 1]);
+                            float a0 = __uint_as_float(r[cc][j3l][2 * jj]) * kscale;
+                            float a1 = __uint_as_float(r[cc][j3l + 1][2 * jj]) * kscale;
+                            float b0 = __uint_as_float(r[cc][j3l][2 * jj + 1]) * kscale;
+                            float b1 = __uint_as_float(r[cc][j3l + 1][2 * jj + 1]) * kscale;
                             if (a.v) {
                                 const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
                                 a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
