@@ -71,18 +71,22 @@ constexpr int kChunksPerUnit = 44;   // 8 chunks in each of S1..S2', 4 in S1'
 // chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
 __host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
 __host__ __device__ __forceinline__ int chunk_index(int c) { return c < 40 ? (c & 7) : c - 40; }
-// Besides its buffer (chunk g waits for epilogue g - 4), a chunk reads data
-// that whole earlier epilogues wrote.  Every S3 chunk needs all of E2 (chunk
-// 15), every S2' chunk all of E3' (chunk 31), and S1''s second chunk E2' for
-// j3 = 4..7 (chunk 39); other chunks are covered by the buffer rule.  Returns
-// how many chunks back that epilogue is (0 = none).  With several MMA
-// issuers this must be explicit: chunks of one stage are issued
-// independently.
-__host__ __device__ __forceinline__ int chunk_extra_lag(int c) {
-    if (c >= 16 && c < 20) return c - 15;
-    if (c >= 32 && c < 36) return c - 31;
-    if (c == 41) return 2;
-    return 0;
+// Ordering.  An epilogue warp releases an accumulator buffer as soon as its
+// TMEM loads have landed in registers, before the math and the stores, so
+// the MMA for chunk c + 4 can start early.  Because every epilogue warp works
+// through its chunks in order, "buffer of chunk c released" still implies
+// that all the work of the chunks before c's pair is done (stores fenced),
+// which covers most data dependencies.  The chunks that regroup the data
+// need whole stages instead, signalled by per-tile stage barriers: the first
+// S3 chunks (16..19) need all of E2, the first S2' chunks (32..35) all of
+// E3', and the S1' chunks for j3 = 4..7 (41, 43) the last E2' pair.  Returns
+// the stage barrier chunk c waits for, or -1.  With several MMA issuers this
+// must be explicit: chunks of one stage are issued independently.
+__host__ __device__ __forceinline__ int chunk_stage_barrier(int c) {
+    if (c >= 16 && c < 20) return 0;
+    if (c >= 32 && c < 36) return 1;
+    if (c == 41 || c == 43) return 2;
+    return -1;
 }
 constexpr uint32_t kWaitLimit = 1u << 20;
 
@@ -158,7 +162,6 @@ __device__ __forceinline__ uint32_t pack_h2(float re, float im) {
     __half2 h = __floats2half2_rn(re, im);
     return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
 // Twiddle products in packed half precision.  A twiddle t = (tr, ti) is held
 // as the two half2 values tp = (tr, ti) and tq = (-ti, tr); then
@@ -218,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
     uint64_t* dfree = bar + 5;     // [kDBuf] accumulator buffer drained (16 epilogue warps)
     uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
     uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
+    uint64_t* bar_stage = bar + 11;   // [3] E2, E3', E2' done for the tile (16 epilogue warps)
     uint32_t* tmem_base_sh = (uint32_t*)(smem + kOffMisc);
     volatile int* abort_flag = (volatile int*)(smem + kOffMisc + 4);
 
@@ -234,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         }
         mbar_init(bar_fin, kMmaWarps);
         mbar_init(bar_k, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar_stage[i], kEpiWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -305,12 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const uint32_t b = g % kDBuf;
                 // the buffer's previous contents must have been drained ...
                 if (g >= kDBuf && !wait(&dfree[b], ((g - kDBuf) / kDBuf) & 1)) { ok = false; fail(); break; }
-                // ... and chunks that regroup the data need more recent
-                // epilogues (each warp finishes its epilogues in order)
-                const int lag = chunk_extra_lag(c);
-                if (lag && !wait(&dfree[(g - lag) % kDBuf], ((g - lag) / kDBuf) & 1)) {
-                    ok = false; fail(); break;
-                }
+                // ... and chunks that regroup the data need whole stages
+                const int sb = chunk_stage_barrier(c);
+                if (sb >= 0 && !wait(&bar_stage[sb], iter & 1)) { ok = false; fail(); break; }
                 tc_fence_after();
                 if (lane == 0) {
                     // descriptors are loop-invariant bases plus an offset in
@@ -476,13 +478,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 tc_fence_after();
                 return true;
             };
-            auto end_pair = [&](int c) {
+            // the pair's accumulators are in registers: hand the buffers back
+            auto release = [&](int c) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&dfree[c & 3]);
                     mbar_arrive(&dfree[(c & 3) + 1]);
                 }
+            };
+            // this warp's part of a whole stage is written (TMEM stores waited
+            // for, shared-memory stores fenced for the async proxy)
+            auto stage_done = [&](int i) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_stage[i]);
             };
             auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (c & 3); };
 
@@ -496,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
                 tc_wait_ld();
+                release(c);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     uint8_t* tile = smem + kOffData + (k + cc) * kTile + (4 * q + s) * 1024;
@@ -511,7 +522,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             for (int k = 0; k < 8; k += 2) {
                 if (!(ok = begin_pair(k))) break;
                 e_transpose(k, k);
-                end_pair(k);
             }
             // E2: lane = c1; columns c2 = 8s + i of j3 = k, k+1; twiddle
             // wM^(c1 j3); A3 (TMEM) cols c2*8 + j3 (two adjacent columns)
@@ -524,13 +534,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
                 const Tw16 t0 = stwM[lane * k], t1 = stwM[lane * (k + 1)];
                 tc_wait_ld();
+                release(c);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     tmem_st2(tbase + lq + (8 * s + i) * 8 + k, cmul_h(r[0][2 * i], r[0][2 * i + 1], t0),
                              cmul_h(r[1][2 * i], r[1][2 * i + 1], t1));
                 tc_wait_st();
-                end_pair(c);
             }
+            if (ok) stage_done(0);
             // EK: lane = c1; columns c3 of c2 = 4(k+cc) + s; times the filter
             // spectrum row in its fp16 form K/scale (|K/scale| <= 1, so the
             // inverse stages see values no larger than the forward output);
@@ -545,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
                 tc_wait_ld();
+                release(c);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c2 = 4 * (k + cc) + s;
@@ -574,7 +586,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     tmem_st8(tbase + lq + c2 * 8, h8);
                 }
                 tc_wait_st();
-                end_pair(c);
             }
             // E3': lane = c1; columns (c2 = 4(k+cc) + cl, j3 = 2s + jj);
             // twiddle conj wM^(c1 j3); A5 tile j3, row 32q + c1, K pairs of
@@ -590,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     for (int cl = 0; cl < 4; ++cl) tmem_ld4(dcol(c + cc) + cl * 16 + 4 * s, r[cc][cl]);
                 const Tw16 t0 = tw16_conj(stwM[lane * (2 * s)]), t1 = tw16_conj(stwM[lane * (2 * s + 1)]);
                 tc_wait_ld();
+                release(c);
                 const uint32_t m = 32 * q + lane;
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
@@ -604,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     }
                 }
                 fence_proxy_async_smem();
-                end_pair(c);
             }
+            if (ok) stage_done(1);
 #pragma unroll
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
 #pragma unroll 1
@@ -613,8 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const int c = 32 + k;
                 if (!(ok = begin_pair(c))) break;
                 e_transpose(c, k);
-                end_pair(c);
             }
+            if (ok) stage_done(2);
 #pragma unroll
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
             // EO: lane = l; the pair (h, jh = 0, 1) holds j1 in [8h, 8h+8) for
@@ -625,25 +637,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             for (int h = 0; h < 2 && ok; ++h) {
                 const int c = 40 + 2 * h;
                 if (!(ok = begin_pair(c))) break;
-                if (P.valid) {
-                    // output gate values: rows j1 = 8h + 2s + jj, eight
-                    // consecutive t each, requested before the TMEM loads
-                    uint4 va[2], vb[2];
-                    {
-                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+                // output gate values: rows j1 = 8h + 2s + jj, eight consecutive
+                // t each, requested before the TMEM loads (an empty pair reads
+                // row 0 of the channel and discards it)
+                uint4 va[2], vb[2];
+                {
+                    const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane;
-                            va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
-                            vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
-                        }
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane;
+                        va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
+                        vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
                     }
-                    uint32_t r[2][4][4];
+                }
+                uint32_t r[2][4][4];
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
+                for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-                        for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dcol(c + cc) + j3l * 16 + 4 * s, r[cc][j3l]);
-                    tc_wait_ld();
+                    for (int j3l = 0; j3l < 4; ++j3l) tmem_ld4(dcol(c + cc) + j3l * 16 + 4 * s, r[cc][j3l]);
+                tc_wait_ld();
+                release(c);
+                if (P.valid) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const int64_t t0 = 256 * (8 * h + 2 * s + jj) + 8 * lane;
@@ -669,7 +683,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
                     }
                 }
-                end_pair(c);
             }
         }
     }
