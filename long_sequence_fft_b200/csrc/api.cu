@@ -159,7 +159,7 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         e = upload(&p->tw, host_twiddles(p->M, p->M, 1));
         p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
     } else if (p->path == kPathSimtStaged) {
-        p->logC = p->logM - 1 < 14 ? p->logM - 1 : 14;
+        p->logC = staged_log_cols(p->logM);
         p->logR = p->logM - p->logC;
         p->logTab = p->logC;
         const int64_t C = int64_t(1) << p->logC;

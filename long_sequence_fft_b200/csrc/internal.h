@@ -11,6 +11,20 @@ namespace fftconv {
 enum Path : int { kPathSimtFused = 1, kPathSimtStaged = 2, kPathTcFused = 3 };
 enum DType : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
 
+// Staged path factorization M = R * C (log2 of C for log2(M) = logM): rows
+// of C = 1024 points, or longer where that keeps R <= 256, and C <= 2^14
+// (the row kernel's limit).  Measured on B200 this balances the column and
+// row passes far better than the longest rows: N = 32768 runs 1.8x faster as
+// 64 x 1024 than as 4 x 16384, N = 2^20 5% faster as 256 x 8192 than as
+// 128 x 16384.  Every staged plan and the static-scratch entry point use it,
+// so they share the K_f layout [H][R][C].
+inline int staged_log_cols(int logM) {
+    int lc = logM - 8 > 10 ? logM - 8 : 10;
+    if (lc > logM - 1) lc = logM - 1;
+    if (lc > 14) lc = 14;
+    return lc;
+}
+
 struct Plan {
     int64_t N = 0, H = 0, L = 0, M = 0;
     int logM = 0;

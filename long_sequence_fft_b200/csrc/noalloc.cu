@@ -154,7 +154,7 @@ extern "C" int fftconv_forward_noalloc(const void* u, const void* K_f, void* y, 
     p.logM = logM;
     p.dtype = (int)dtype;
     p.path = kPathSimtStaged;
-    p.logC = logM - 1 < kMaxLogC ? logM - 1 : kMaxLogC;
+    p.logC = staged_log_cols(logM);     // the K_f layout of every staged plan
     p.logR = logM - p.logC;
     p.logTab = p.logC;
     p.twSplit = (logM + 1) / 2;
