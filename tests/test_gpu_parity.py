@@ -102,7 +102,7 @@ def _sampled_ref(w, inp, seq, ts):
 
 @pytest.mark.parametrize("name", sorted(W.WORKLOADS))
 def test_workload_full_size_sampled(name):
-    """Full BASELINE shapes, the benchmark's launch configuration (order 0),
+    """Full workload shapes, the benchmark's launch configuration (order 0),
     compared at seeded sample points against direct sums."""
     w = W.WORKLOADS[name]
     inp = W.make_all(w)
