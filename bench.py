@@ -55,6 +55,9 @@ def read_peaks():
 
 
 def read_traffic(kernel_key: str):
+    """DRAM bytes per launch of the workload's dominant kernel from a committed
+    ncu capture, or None.  The entry names the kernel's source file and its
+    SHA-256 at capture time; a kernel changed since then reads as None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
@@ -63,6 +66,13 @@ def read_traffic(kernel_key: str):
     ent = d.get(kernel_key)
     if not ent:
         return None
+    import hashlib
+    src = os.path.join(ROOT, ent.get("source", ""))
+    if not os.path.isfile(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != ent.get("source_sha256"):
+            return None
     return ent
 
 
