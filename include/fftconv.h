@@ -84,7 +84,15 @@ FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
                         fftconv_dtype_t dtype, int order);
 
 /* As fftconv_plan_create with a filter of length L (1 <= L <= N): the
- * partial convolution, defined as the convolution with k zero-padded to N. */
+ * partial convolution, defined as the convolution with k zero-padded to N
+ * (FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
+ * summary and "Approach": partial convolutions).
+ * With a 16-bit dtype, N > 4096 and L <= 2049, orders 0, 2 and 3 choose the
+ * tensor-core path as overlap-save: windows of 4096 inputs with hop 2048, each
+ * one 8192-point transform, N/2048 - 1 windows per sequence.  Such a plan
+ * stores the 8192-point filter spectrum, so fftconv_forward rejects a
+ * block_mask and fftconv_filter_to_rfft is unsupported on it
+ * (FFTCONV_ERR_UNSUPPORTED); orders 1 and 4 keep the 2N-point spectrum. */
 FFTCONV_API int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H,
                            fftconv_dtype_t dtype, int order, int64_t L);
 
@@ -118,7 +126,8 @@ FFTCONV_API int fftconv_filter_precompute(fftconv_plan_t plan, const void* k, vo
  *                also holds the Nyquist bin N); 0 zeroes those bins (and their
  *                Hermitian mirrors), anything else keeps them.
  *   mask_h     : 1 (one mask row for all channels) or H; ignored when
- *                block_mask is NULL.
+ *                block_mask is NULL.  A block_mask on an overlap-save plan
+ *                (see fftconv_plan_create_ex) is FFTCONV_ERR_UNSUPPORTED.
  * Asynchronous on `stream`; allocates nothing.  Calls on the staged path
  * share the plan's workspace and must be serialised on one stream. */
 FFTCONV_API int fftconv_forward(fftconv_plan_t plan, const void* u, const void* K_f, void* y,
@@ -171,7 +180,8 @@ FFTCONV_API int fftconv_forward_noalloc(const void* u, const void* K_f, void* y,
                                         fftconv_stream_t stream);
 
 /* Test hook: export K_f in natural order as out[h, f, 0..1] = (Re, Im) of
- * rfft(k)[f] for f in [0, N] (normalisation undone), fp32, device. */
+ * rfft(k)[f] for f in [0, N] (normalisation undone), fp32, device.
+ * FFTCONV_ERR_UNSUPPORTED on an overlap-save plan (see fftconv_plan_create_ex). */
 FFTCONV_API int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out,
                            fftconv_stream_t stream);
 

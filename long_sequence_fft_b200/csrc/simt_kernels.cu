@@ -548,7 +548,7 @@ cudaError_t simt_fused_forward(const Plan& p, const ForwardArgs& a, cudaStream_t
 }
 
 cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
-    if (p.logM != 13) return cudaErrorInvalidValue;
+    if (p.L > 4096) return cudaErrorInvalidValue;     // the 8192-point spectrum of k (<= 4096 taps)
     const size_t smem = sizeof(float2) * smem_elems<1>(1 << 13);
     FFTCONV_DISPATCH_T(p.dtype, {
         auto kern = simt_precompute_tc8192_kernel<T>;

@@ -60,8 +60,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int kN = 4096;
-constexpr int kM = 8192;
+constexpr int kN = 4096;          // window length (inputs and outputs per transform)
+constexpr int kM = 8192;          // transform length
+constexpr int kHop = 2048;        // overlap-save hop for longer sequences
 constexpr int kEpiWarps = 16;
 constexpr int kMmaWarps = 4;     // one MMA issuer per SMSP; issuer i owns accumulator buffer i
 constexpr int kThreads = (kEpiWarps + kMmaWarps) * 32;
@@ -125,9 +126,11 @@ struct TcArgs {
     const uint8_t* mask;
     int64_t mask_h;
     int64_t B, H;
+    int64_t N;                 // sequence length (row stride of u, w, v, y)
+    int64_t nwin;              // windows per sequence (1 for N = 4096)
     int64_t pb;                // pairs per channel, ceil(B/2)
-    int64_t tpc;               // tiles per channel, ceil(pb/4)
-    int64_t nunits;            // H * tpc
+    int64_t tpc;               // tiles per window, ceil(pb/4)
+    int64_t nunits;            // H * nwin * tpc
     const uint4* bimg;         // DFT factors, image of the shared-memory region
     const float2* tw1024;      // exp(-2 pi i e/1024), e < 1024
     const float2* twM;         // exp(-2 pi i e/8192), e < 256
@@ -186,21 +189,50 @@ __device__ __forceinline__ uint32_t cmul_h(uint32_t xr, uint32_t xi, Tw16 t) {
 __device__ __forceinline__ uint32_t swz(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
 
 struct PairInfo {
-    int64_t o0, o1;      // element offsets of rows b0 and b1 (o1 < 0: absent)
+    int64_t o0, o1;      // element offsets of the window in rows b0 and b1 (o1 < 0: absent)
     int64_t h;
     bool valid;
+    bool tail_only;      // only window positions t >= kHop are outputs
 };
 
-// A tile holds 4 pairs of batch rows of ONE channel: tile u covers channel
-// u / tpc and pairs 4*(u % tpc) + q, q < 4 (pairs past ceil(B/2) are empty).
+// A tile holds 4 pairs of batch rows of ONE channel and one window: unit u
+// covers channel u / (nwin*tpc), window j = (u / tpc) % nwin and pairs
+// 4*(u % tpc) + q, q < 4 (pairs past ceil(B/2) are empty).
+//
+// Overlap-save (sequences longer than 4096, filters of L <= 2049 taps): the
+// kernel's transform gives the first 4096 outputs of the linear convolution
+// of a 4096-sample window with the filter, exact wherever the filter's whole
+// history lies inside the window, i.e. from window position L - 1 on.
+// Window j starts at 2048 j; window 0 keeps all 4096 outputs (there is no
+// history before t = 0), window j > 0 keeps positions [2048, 4096), i.e.
+// y[2048 (j+1), 2048 (j+2)).  N / 2048 - 1 windows cover the sequence.
+// Tile indices fit in 32 bits (the host rejects launches of 2^31 tiles or
+// more), so the decomposition uses 32-bit division.  WIN = false is the
+// single-window case (N = 4096), with the row stride and the window fixed.
+template <bool WIN>
 __device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t unit, int q) {
     PairInfo p;
-    p.h = unit / a.tpc;
-    const int64_t bp = 4 * (unit % a.tpc) + q;
+    if constexpr (!WIN) {
+        p.h = unit / a.tpc;
+        const int64_t bp = 4 * (unit % a.tpc) + q;
+        p.valid = bp < a.pb;
+        p.tail_only = false;
+        const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
+        p.o0 = (b0 * a.H + p.h) * kN;
+        p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * kN : -1;
+        return p;
+    }
+    const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
+    const uint32_t h = un / per_ch;
+    const uint32_t rem = un - h * per_ch;
+    const uint32_t j = rem / tpc;
+    p.h = h;
+    const int64_t bp = 4 * (int64_t)(rem - j * tpc) + q;
     p.valid = bp < a.pb;
+    p.tail_only = j > 0;
     const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
-    p.o0 = (b0 * a.H + p.h) * kN;
-    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * kN : -1;
+    p.o0 = (b0 * a.H + p.h) * a.N + kHop * j;
+    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * a.N + kHop * j : -1;
     return p;
 }
 
@@ -211,7 +243,7 @@ __host__ __device__ __forceinline__ int k16_index(int c1, int c2, int c3) {
     return ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + (c3 & 3);
 }
 
-template <typename T>
+template <typename T, bool WIN>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -300,7 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     // the previous tile is finished with the filter buffer (its
                     // epilogue warps arrived on bar_in after all their reads)
                     mbar_expect_tx(bar_k, kKBytes);
-                    bulk_copy_g2s(smem + kOffK, a.Kh16 + (unit / a.tpc) * (int64_t)kM, kKBytes, bar_k);
+                    bulk_copy_g2s(smem + kOffK,
+                                  a.Kh16 + (WIN ? (int64_t)((uint32_t)unit / ((uint32_t)a.nwin * (uint32_t)a.tpc))
+                                                : unit / a.tpc) * kM,
+                                  kKBytes, bar_k);
                 }
                 ++k_issued;
                 __syncwarp();
@@ -352,23 +387,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     // their last S2 chunk; measured against one warp at the
                     // tile start, 3.5% faster overall (and 7% faster than no
                     // prefetch).
+                    const void* pf_src = nullptr;
+                    uint32_t pf_bytes = kN * sizeof(T);
                     const int64_t nu = unit + gridDim.x;
                     if (nu < a.nunits && (lane >> 3) == issuer) {
-                        const PairInfo Q = pair_info(a, nu, lane >> 3);
+                        const PairInfo Q = pair_info<WIN>(a, nu, issuer);
                         const int which = lane & 7;
-                        const void* src = nullptr;
-                        uint32_t bytes = kN * sizeof(T);
                         if (Q.valid) {
-                            if (which == 0) src = (const T*)a.u + Q.o0;
-                            else if (which == 1 && a.w) src = (const T*)a.w + Q.o0;
-                            else if (which == 2 && a.v) src = (const T*)a.v + Q.o0;
-                            else if (which == 3 && Q.o1 >= 0) src = (const T*)a.u + Q.o1;
-                            else if (which == 4 && Q.o1 >= 0 && a.w) src = (const T*)a.w + Q.o1;
-                            else if (which == 5 && Q.o1 >= 0 && a.v) src = (const T*)a.v + Q.o1;
-                            else if (which == 6 && (lane >> 3) == 0) { src = a.Kh16 + Q.h * (int64_t)kM; bytes = kKBytes; }
+                            if (which == 0) pf_src = (const T*)a.u + Q.o0;
+                            else if (which == 1 && a.w) pf_src = (const T*)a.w + Q.o0;
+                            else if (which == 2 && a.v) pf_src = (const T*)a.v + Q.o0;
+                            else if (which == 3 && Q.o1 >= 0) pf_src = (const T*)a.u + Q.o1;
+                            else if (which == 4 && Q.o1 >= 0 && a.w) pf_src = (const T*)a.w + Q.o1;
+                            else if (which == 5 && Q.o1 >= 0 && a.v) pf_src = (const T*)a.v + Q.o1;
+                            else if (which == 6 && issuer == 0) { pf_src = a.Kh16 + Q.h * (int64_t)kM; pf_bytes = kKBytes; }
                         }
-                        if (src) prefetch_l2(src, bytes);
                     }
+                    if (pf_src) prefetch_l2(pf_src, pf_bytes);
                     __syncwarp();
                 }
             }
@@ -404,14 +439,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         int iter = 0;
         bool ok = true;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
-            const PairInfo P = pair_info(a, unit, q);
-            // row pointers are formed from the kernel parameters on use (they
-            // live in constant memory), keeping registers for the stages
-            const bool has1 = P.o1 >= 0;
+            const int64_t hch = WIN ? (int64_t)((uint32_t)unit / ((uint32_t)a.nwin * (uint32_t)a.tpc))
+                                    : unit / a.tpc;   // the tile's channel
 
             // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [4s, 4s+4).
             // Loads are issued in batches before any use (absent rows or gates
-            // read a present row and are masked afterwards).
+            // read a present row and are masked afterwards).  Row offsets are
+            // formed here and again for the output stage instead of being
+            // kept, which keeps registers for the stages.
+            const PairInfo P = pair_info<WIN>(a, unit, q);
+            const bool has1 = P.o1 >= 0;
             {
                 const int64_t oo1 = has1 ? P.o1 : P.o0;
                 const T* pu0 = (const T*)a.u + P.o0;
@@ -463,9 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             const __half2* Ks = (const __half2*)(smem + kOffK);
             // loaded once per tile and pinned in a register (an opaque move
             // keeps the compiler from re-issuing the global load at each use)
-            float kscale = __ldg(&a.Kscale[P.h]);
+            float kscale = __ldg(&a.Kscale[hch]);
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
-            const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : P.h) * nblk : nullptr;
+            const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : hch) * nblk : nullptr;
 
             // Accumulator chunks are handled in pairs (c, c+1) of one stage:
             // both are waited for and loaded before one TMEM-load wait, and
@@ -638,6 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // 41 + 2h) covers j3 in [4h, 4h+4); this warp takes j1 = 4s + jj
             // and writes y = s_h * v * z for the four consecutive
             // t = 256 j1 + 8 l + 4h + (0..3) of each row as one 8-byte store.
+            // In a window after the first, positions t < 2048 (j1 < 8: warps
+            // with s < 2) are not outputs; their gate loads still read inside
+            // the sequence and are discarded.
+            const bool emit = P.valid && !(P.tail_only && s < 2);
 #pragma unroll 1
             for (int h = 0; h < 2 && ok; ++h) {
                 const int c = 40 + 2 * h;
@@ -662,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     for (int jl = 0; jl < 2; ++jl) tmem_ld8(dcol(c + cc) + jl * 32 + 8 * s, r[cc][jl]);
                 tc_wait_ld();
                 release(c);
-                if (P.valid) {
+                if (emit) {
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const int64_t t0 = 256 * (4 * s + jj) + 8 * lane + 4 * h;
@@ -795,9 +836,13 @@ __global__ void tc_export_kernel(const __half2* __restrict__ Kh, const float* __
 
 }  // namespace
 
-bool tc_supported(int64_t N, int64_t /*L*/, int dtype) {
-    return N == kN && (dtype == kF16 || dtype == kBF16);
+bool tc_supported(int64_t N, int64_t L, int dtype) {
+    if (dtype != kF16 && dtype != kBF16) return false;
+    if (N == kN) return true;
+    return N > kN && L <= kHop + 1;      // overlap-save windows (N a power of two)
 }
+
+int64_t tc_windows(int64_t N) { return N == kN ? 1 : N / kHop - 1; }
 
 cudaError_t tc_plan_init(Plan& p) {
     TcResources* r = new TcResources();
@@ -811,24 +856,25 @@ cudaError_t tc_plan_init(Plan& p) {
     if (e == cudaSuccess) e = cudaMalloc((void**)&r->twM, t2.size() * sizeof(float2));
     if (e == cudaSuccess) e = cudaMemcpy(r->twM, t2.data(), t2.size() * sizeof(float2), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
-    // the SIMT engine computes the filter spectrum (any length), so the plan
-    // also carries its twiddle table
-    p.logTab = p.logM;
+    // the SIMT engine computes the filter's 8192-point spectrum, so the plan
+    // also carries that twiddle table
+    p.logTab = 13;
     if (e == cudaSuccess) {
-        std::vector<float2> tw(p.M);
-        for (int64_t i = 0; i < p.M; ++i) {
-            const std::complex<double> z = wpow(i, p.M, -1);
+        std::vector<float2> tw(kM);
+        for (int64_t i = 0; i < kM; ++i) {
+            const std::complex<double> z = wpow(i, kM, -1);
             tw[i] = make_float2((float)z.real(), (float)z.imag());
         }
         e = cudaMalloc((void**)&p.tw, tw.size() * sizeof(float2));
         if (e == cudaSuccess) e = cudaMemcpy(p.tw, tw.data(), tw.size() * sizeof(float2), cudaMemcpyHostToDevice);
     }
     if (e == cudaSuccess) {
-        e = cudaFuncSetAttribute(tc_fftconv_n4096_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(tc_fftconv_n4096_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSmemBytes);
+        const void* kernels[4] = {(const void*)tc_fftconv_n4096_kernel<__nv_bfloat16, false>,
+                                  (const void*)tc_fftconv_n4096_kernel<__nv_bfloat16, true>,
+                                  (const void*)tc_fftconv_n4096_kernel<__half, false>,
+                                  (const void*)tc_fftconv_n4096_kernel<__half, true>};
+        for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+            e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     }
     return e;
 }
@@ -859,18 +905,22 @@ cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H;
+    a.N = p.N;
+    a.nwin = tc_windows(p.N);
     a.pb = (fa.B + 1) / 2;
     a.tpc = (a.pb + 3) / 4;
-    a.nunits = p.H * a.tpc;
+    a.nunits = p.H * a.nwin * a.tpc;
     a.bimg = (const uint4*)r->bimg;
     a.tw1024 = r->tw1024;
     a.twM = r->twM;
     a.status = p.status;
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
     if (p.dtype == kBF16)
-        tc_fftconv_n4096_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
+        a.nwin > 1 ? tc_fftconv_n4096_kernel<__nv_bfloat16, true><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a)
+                   : tc_fftconv_n4096_kernel<__nv_bfloat16, false><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
     else
-        tc_fftconv_n4096_kernel<__half><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
+        a.nwin > 1 ? tc_fftconv_n4096_kernel<__half, true><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a)
+                   : tc_fftconv_n4096_kernel<__half, false><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -215,3 +215,36 @@ def test_bad_arguments_are_rejected_without_launch():
     with pytest.raises(lsf.FFTConvError) as e:
         lsf.Plan(1000, 2, "f32")
     assert e.value.status == lsf.ERR_UNSUPPORTED
+
+
+# ------------------------------------------------- overlap-save windows ---
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("N,L,B", [(8192, 2048, 3), (8192, 2049, 2), (8192, 1, 1), (16384, 300, 3),
+                                   (32768, 1024, 1)])
+def test_overlap_save_windows(dtype, N, L, B):
+    """Sequences longer than 4096 with filters of L <= 2049 taps run as
+    overlapping 4096-sample windows on the tensor-core kernel."""
+    inp = _rand_inputs(B, 2, N, L, dtype, gated=(B != 1), seed=N + L + B)
+    y, plan = run_cuda(inp, dtype, order=0)
+    assert plan.path_name == "tc_fused"
+    assert_close(y, _oracle(inp), dtype, f"overlap-save {dtype} N={N} L={L} B={B}")
+
+
+def test_overlap_save_limits():
+    import long_sequence_fft_b200 as lsf
+    import torch
+    # one tap too many for the windows: the SIMT path serves it
+    assert lsf.Plan(8192, 2, "bf16", L=2050).path_name != "tc_fused"
+    plan = lsf.Plan(8192, 2, "bf16", L=2048)
+    assert plan.path_name == "tc_fused"
+    k = torch.zeros((2, 2048), dtype=torch.bfloat16, device="cuda")
+    Kf = plan.precompute(k)
+    u = torch.zeros((2, 2, 8192), dtype=torch.bfloat16, device="cuda")
+    mask = torch.ones((1, 8192 // 32), dtype=torch.uint8, device="cuda")
+    with pytest.raises(lsf.FFTConvError) as e:
+        plan.forward(u, Kf, mask=mask)
+    assert e.value.status == lsf.ERR_UNSUPPORTED
+    with pytest.raises(lsf.FFTConvError) as e:
+        plan.export_rfft(Kf)
+    assert e.value.status == lsf.ERR_UNSUPPORTED
