@@ -190,6 +190,17 @@ FFTCONV_API int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, flo
  * since the last call (the word is reset to OK by this call). */
 FFTCONV_API int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream);
 
+/* Self-test of the device-side failure path (the pages describe none; this
+ * exists so the bounded waits can be tested without faulting a GPU).  Launches
+ * one warp on `stream` that waits on an on-chip barrier with the convolution
+ * kernels' bounded wait, giving up after `polls` (1 <= polls <= 2^20) blocking
+ * polls.  arrive != 0: the barrier is signalled first and the wait succeeds;
+ * arrive == 0: nothing signals it, the wait gives up and the plan's status
+ * word becomes FFTCONV_ERR_TIMEOUT (read and reset by fftconv_device_status).
+ * Asynchronous; allocates nothing; the context stays usable. */
+FFTCONV_API int fftconv_selftest_bounded_wait(fftconv_plan_t plan, int64_t polls, int arrive,
+                                  fftconv_stream_t stream);
+
 /* Static description of a status code. */
 FFTCONV_API const char* fftconv_status_string(int status);
 

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libfftconv.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m long_sequence_fft_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python long_sequence_fft_b200/build.py` "
         "(nvcc, sm_100a). There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -51,6 +51,7 @@ _SIGNATURES = {
                                             _sz, _vp]),
     "fftconv_filter_to_rfft": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
     "fftconv_device_status": (ctypes.c_int, [_vp, _vp]),
+    "fftconv_selftest_bounded_wait": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp]),
     "fftconv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fftconv_last_error": (ctypes.c_char_p, []),
     "fftconv_version": (ctypes.c_char_p, []),

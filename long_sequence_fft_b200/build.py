@@ -1,6 +1,9 @@
 """Build the CUDA library (libfftconv.so) in-tree for sm_100a with nvcc.
 
-Usage: python -m long_sequence_fft_b200.build [--force]
+Usage: python long_sequence_fft_b200/build.py [--force]
+
+(Run it by path: importing the package loads the library it builds, which
+fails while the library is missing or older than the C ABI.)
 """
 from __future__ import annotations
 

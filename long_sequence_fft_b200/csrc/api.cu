@@ -361,6 +361,16 @@ int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fft
     return FFTCONV_OK;
 }
 
+int fftconv_selftest_bounded_wait(fftconv_plan_t plan, int64_t polls, int arrive, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    if (polls < 1 || polls > (int64_t(1) << 20))
+        return fail(FFTCONV_ERR_INVALID_ARG, "polls=%lld outside [1, 2^20]", (long long)polls);
+    cudaError_t e = selftest_bounded_wait(plan->p, (uint32_t)polls, arrive ? 1 : 0, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return FFTCONV_OK;
+}
+
 int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream) {
     g_last_error.clear();
     if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");

@@ -85,5 +85,6 @@ size_t tc_filter_bytes(const Plan& p);
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s);
+cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s);
 
 }  // namespace fftconv

@@ -924,6 +924,33 @@ cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Self-test of the bounded-wait path: one warp initialises an mbarrier that
+// expects one arrival and waits for its first phase with the same bounded
+// wait the convolution kernels use (at most `polls` blocking polls).  With
+// `arrive` set, lane 0 arrives first and the wait succeeds; otherwise nothing
+// arrives, the wait gives up and the kernel records FFTCONV_ERR_TIMEOUT in the
+// status word, exactly as a convolution kernel would.  Nothing is faulted and
+// the context stays usable.
+__global__ void bounded_wait_selftest_kernel(int* status, uint32_t polls, int arrive) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (arrive && threadIdx.x == 0) mbar_arrive(&bar);
+    __syncwarp();
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar, 0, &abort_flag, polls));
+    if (!ok && threadIdx.x == 0) atomicExch(status, kStatusTimeout);
+}
+
+cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(p.status, polls, arrive);
+    return cudaGetLastError();
+}
+
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
     const int64_t total = p.H * (kN + 1);
     int blocks = (int)((total + 255) / 256);

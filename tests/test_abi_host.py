@@ -42,6 +42,7 @@ def test_status_strings_and_null_handles():
     assert lib.fftconv_plan_path(None) == lsf.ERR_INVALID_ARG
     assert lib.fftconv_forward(None, None, None, None, 1, 1, 1, None, None, None, 0, None) == lsf.ERR_INVALID_ARG
     assert b"plan" in lib.fftconv_last_error()
+    assert lib.fftconv_selftest_bounded_wait(None, 16, 0, None) == lsf.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("N,H,dtype,order,L,status", [
