@@ -142,9 +142,15 @@ FFTCONV_API size_t fftconv_forward_host_staging_bytes(fftconv_plan_t plan, int64
 
 /* fftconv_forward on HOST buffers: copies u_host (and w_host, v_host,
  * mask_host) into the caller's device staging buffer, runs the forward pass
- * and copies y back into y_host, all asynchronously on `stream` (page-locked
- * host memory makes the copies asynchronous; pageable memory works but
- * blocks).  K_f stays a device pointer.  staging: device, at least
+ * and copies y back into y_host.  The work is pipelined over up to 8 chunks of
+ * batch rows: uploads run on a plan-owned copy stream, each chunk's forward
+ * pass on `stream`, downloads on a second plan-owned copy stream, so the two
+ * copy directions and the compute overlap.  The call as a whole is ordered on
+ * `stream` (it starts after the stream's earlier work; later work on the
+ * stream sees y_host written) and returns without waiting (page-locked host
+ * memory keeps the copies asynchronous; pageable memory works but blocks).
+ * Calls on one plan share its copy streams and must be issued from one host
+ * thread in order.  K_f stays a device pointer.  staging: device, at least
  * fftconv_forward_host_staging_bytes(...) bytes, 256-byte aligned. */
 FFTCONV_API int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, const void* K_f,
                          void* y_host, int64_t B, int64_t H, int64_t N,

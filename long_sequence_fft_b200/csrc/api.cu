@@ -73,6 +73,14 @@ void free_plan(Plan* p) {
     cudaFree(p->twHi);
     cudaFree(p->work);
     cudaFree(p->status);
+    if (p->copy_in) cudaStreamDestroy(p->copy_in);
+    if (p->copy_out) cudaStreamDestroy(p->copy_out);
+    if (p->ev_start) cudaEventDestroy(p->ev_start);
+    if (p->ev_out) cudaEventDestroy(p->ev_out);
+    for (int i = 0; i < Plan::kHostChunks; ++i) {
+        if (p->ev_in[i]) cudaEventDestroy(p->ev_in[i]);
+        if (p->ev_comp[i]) cudaEventDestroy(p->ev_comp[i]);
+    }
     cudaSetDevice(cur);
     delete p;
 }
@@ -292,6 +300,30 @@ int fftconv_forward(fftconv_plan_t plan, const void* u, const void* K_f, void* y
 
 static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+}  // extern "C"
+
+// Copy streams and events of the host-buffer entry point, created once per
+// plan on the plan's device (non-blocking streams, events without timing).
+static int host_resources(Plan& p) {
+    if (p.copy_in) return FFTCONV_OK;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(p.device);
+    cudaError_t e = cudaStreamCreateWithFlags(&p.copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.ev_start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.ev_out, cudaEventDisableTiming);
+    for (int i = 0; i < Plan::kHostChunks && e == cudaSuccess; ++i) {
+        e = cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.ev_comp[i], cudaEventDisableTiming);
+    }
+    cudaSetDevice(cur);
+    if (e != cudaSuccess) return cuda_fail(e, "host-buffer streams");
+    return FFTCONV_OK;
+}
+
+extern "C" {
+
 size_t fftconv_forward_host_staging_bytes(fftconv_plan_t plan, int64_t B, int has_w, int has_v, int has_mask,
                                           int64_t mask_h) {
     if (!plan || B < 0) return 0;
@@ -334,16 +366,47 @@ int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, const void* K_
     cudaStream_t s = (cudaStream_t)stream;
     int rc = validate_forward(p, du, K_f, dy, B, H, N, dw, dv, dm, mask_h);
     if (rc != FFTCONV_OK) return rc;
-    cudaError_t e = cudaMemcpyAsync(du, u_host, bytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && w_host) e = cudaMemcpyAsync(dw, w_host, bytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && v_host) e = cudaMemcpyAsync(dv, v_host, bytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && mask_host) e = cudaMemcpyAsync(dm, mask_host, mbytes, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-    ForwardArgs a{du, dw, dv, dy, K_f, dm, mask_host ? mask_h : 0, B};
-    rc = run_forward(p, a, s);
+    rc = host_resources(plan->p);
     if (rc != FFTCONV_OK) return rc;
-    e = cudaMemcpyAsync(y_host, dy, bytes, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+
+    // Pipelined over chunks of batch rows: chunk i's uploads run on the copy-in
+    // stream, its forward pass on `stream`, its download on the copy-out
+    // stream, so uploads, compute and downloads of different chunks overlap
+    // (the two copy directions use separate engines).  `stream` orders the
+    // whole call: the copies start after its earlier work, and its later work
+    // waits for the last download.
+    const size_t row = (size_t)p.H * (size_t)p.N * dtype_size(p.dtype);
+    int64_t rows = (B + Plan::kHostChunks - 1) / Plan::kHostChunks;
+    rows += rows & 1;                                // whole pairs of rows
+    const int nchunks = (int)((B + rows - 1) / rows);
+    Plan& q = plan->p;
+    cudaError_t e = cudaEventRecord(q.ev_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(q.copy_in, q.ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(q.copy_out, q.ev_start, 0);
+    if (e == cudaSuccess && mask_host) e = cudaMemcpyAsync(dm, mask_host, mbytes, cudaMemcpyHostToDevice, q.copy_in);
+    for (int i = 0; i < nchunks && e == cudaSuccess; ++i) {
+        const int64_t r0 = i * rows, nr = (B - r0 < rows) ? B - r0 : rows;
+        const size_t off = (size_t)r0 * row, nb = (size_t)nr * row;
+        e = cudaMemcpyAsync((char*)du + off, (const char*)u_host + off, nb, cudaMemcpyHostToDevice, q.copy_in);
+        if (e == cudaSuccess && w_host)
+            e = cudaMemcpyAsync((char*)dw + off, (const char*)w_host + off, nb, cudaMemcpyHostToDevice, q.copy_in);
+        if (e == cudaSuccess && v_host)
+            e = cudaMemcpyAsync((char*)dv + off, (const char*)v_host + off, nb, cudaMemcpyHostToDevice, q.copy_in);
+        if (e == cudaSuccess) e = cudaEventRecord(q.ev_in[i], q.copy_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, q.ev_in[i], 0);
+        if (e != cudaSuccess) break;
+        ForwardArgs a{(const char*)du + off, dw ? (const char*)dw + off : nullptr,
+                      dv ? (const char*)dv + off : nullptr, (char*)dy + off, K_f, dm, mask_host ? mask_h : 0, nr};
+        rc = run_forward(p, a, s);
+        if (rc != FFTCONV_OK) return rc;
+        e = cudaEventRecord(q.ev_comp[i], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(q.copy_out, q.ev_comp[i], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync((char*)y_host + off, (const char*)dy + off, nb, cudaMemcpyDeviceToHost, q.copy_out);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(q.ev_out, q.copy_out);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, q.ev_out, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline");
     return FFTCONV_OK;
 }
 

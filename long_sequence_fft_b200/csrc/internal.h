@@ -52,6 +52,13 @@ struct Plan {
     void* tc = nullptr;
 
     int* status = nullptr;      // device status word (timeouts)
+
+    // host-buffer entry point: copy streams and chunk events, created on
+    // first use (fftconv_forward_host)
+    static constexpr int kHostChunks = 8;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_out = nullptr;
+    cudaEvent_t ev_in[kHostChunks] = {}, ev_comp[kHostChunks] = {};
 };
 
 struct ForwardArgs {
