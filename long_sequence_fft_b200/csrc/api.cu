@@ -256,9 +256,9 @@ static int validate_forward(const Plan& p, const void* u, const void* K_f, void*
         return fail(FFTCONV_ERR_INVALID_ARG, "mask_h=%lld must be 1 or H=%lld", (long long)mask_h, (long long)H);
     if (mask && N < 32) return fail(FFTCONV_ERR_UNSUPPORTED, "block mask needs N >= 32");
     if (p.path == kPathTcFused &&
-        (double)H * (double)tc_windows(p.N) * (double)(((B + 1) / 2 + 3) / 4) >= 2147483648.0)
+        (double)H * (double)tc_tiles_per_pair_group(p.N, p.L) * (double)(((B + 1) / 2 + 3) / 4) >= 2147483648.0)
         return fail(FFTCONV_ERR_UNSUPPORTED, "too many tiles for one launch");
-    if (mask && p.path == kPathTcFused && tc_windows(p.N) > 1)
+    if (mask && p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "block masks act on the 2N-point spectrum; this overlap-save plan (N=%lld, L=%lld) "
                     "has none: create the plan with order 1 or 4",
@@ -415,7 +415,7 @@ int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fft
     if (!plan || !K_f || !out) return fail(FFTCONV_ERR_INVALID_ARG, "plan, K_f and out must be non-NULL");
     if (!aligned16(K_f) || ((uintptr_t)out & 7u)) return fail(FFTCONV_ERR_ALIGNMENT, "K_f/out misaligned");
     const Plan& p = plan->p;
-    if (p.path == kPathTcFused && tc_windows(p.N) > 1)
+    if (p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "this overlap-save plan stores the 8192-point spectrum of k, not the 2N-point one");
     cudaError_t e = (p.path == kPathTcFused) ? tc_export_rfft(p, K_f, out, (cudaStream_t)stream)

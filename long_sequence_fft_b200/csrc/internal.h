@@ -86,6 +86,8 @@ bool simt_fused_supported(int logM);
 // tensor-core path (tc_kernels.cu)
 bool tc_supported(int64_t N, int64_t L, int dtype);
 int64_t tc_windows(int64_t N);   // overlap-save windows per sequence (1: one transform)
+bool tc_overlap_save(int64_t N, int64_t L);   // the plan runs overlap-save windows
+int64_t tc_tiles_per_pair_group(int64_t N, int64_t L);   // tiles per (channel, 4 pairs)
 cudaError_t tc_plan_init(Plan& p);
 void tc_plan_free(Plan& p);
 size_t tc_filter_bytes(const Plan& p);

@@ -55,6 +55,7 @@
 namespace fftconv {
 
 cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t simt_precompute_to_tc_split(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 
 namespace {
 
@@ -67,7 +68,14 @@ constexpr int kEpiWarps = 16;
 constexpr int kMmaWarps = 4;     // one MMA issuer per SMSP; issuer i owns accumulator buffer i
 constexpr int kThreads = (kEpiWarps + kMmaWarps) * 32;
 constexpr int kDBuf = 4;             // accumulator ring: 4 buffers of 64 TMEM columns
-constexpr int kChunksPerUnit = 44;   // 8 chunks in each of S1..S2', 4 in S1'
+
+// Kernel modes.  0: sequences of 4096 (one zero-padded 8192-point transform
+// per sequence, first 4096 outputs).  1: overlap-save windows of 4096 for
+// longer sequences with short filters.  2: sequences of 8192 with full-length
+// filters through the 16384-point spectrum split by bin parity (see
+// pair_info): the 8192-point transform then takes all 8192 inputs and returns
+// all 8192 outputs.
+constexpr int kModePlain = 0, kModeWindows = 1, kModeSplit = 2;
 
 // chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
 __host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
@@ -91,23 +99,34 @@ __host__ __device__ __forceinline__ int chunk_stage_barrier(int c) {
 }
 constexpr uint32_t kWaitLimit = 1u << 20;
 
-// shared-memory map (bytes from a 1024-aligned base)
+// shared-memory map (bytes from a 1024-aligned base) and per-mode sizes
 constexpr int kTile = 16384;                 // 128 rows x 128 B, 128-byte swizzle
-constexpr int kOffData = 0;                  // 8 tiles (one per j3)
-constexpr int kOffBS1 = 8 * kTile;           // K=32 N=64   4 KB
-constexpr int kOffBS2 = kOffBS1 + 4096;      // K=64 N=64   8 KB
-constexpr int kOffBS3 = kOffBS2 + 8192;      // 32 x (K=16 N=16)  16 KB
-constexpr int kOffBS3i = kOffBS3 + 16384;    // 32 x (K=16 N=16)  16 KB
-constexpr int kOffBS2i = kOffBS3i + 16384;   // K=64 N=64   8 KB
-constexpr int kOffBS1i = kOffBS2i + 8192;    // K=64 N=32   4 KB
-constexpr int kOffBEnd = kOffBS1i + 4096;
-constexpr int kBImageBytes = kOffBEnd - kOffBS1;   // 57344
-constexpr int kOffK = kOffBEnd;              // the tile's filter spectrum, 8192 x half2
-constexpr int kKBytes = kM * 4;
-constexpr int kOffTwM = kOffK + kKBytes;     // exp(-2 pi i e/8192), 256 x float2
-constexpr int kOffBars = kOffTwM + 2048;     // 16 mbarrier slots
-constexpr int kOffMisc = kOffBars + 128;     // tmem base, abort flag
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;    // + alignment slack
+constexpr int kKBytes = kM * 4;              // one filter spectrum row, 8192 x half2
+template <int MODE>
+struct Lay {
+    static constexpr bool kFull = MODE == kModeSplit;   // all 8192 inputs and outputs
+    static constexpr int kJ1 = kFull ? 32 : 16;         // nonzero inputs / kept outputs per j3
+    static constexpr int OffData = 0;                   // 8 tiles (one per j3)
+    static constexpr int OffBS1 = 8 * kTile;            // K=2*kJ1 N=64        4 / 8 KB
+    static constexpr int OffBS2 = OffBS1 + kJ1 * 256;   // K=64 N=64           8 KB
+    static constexpr int OffBS3 = OffBS2 + 8192;        // 32 x (K=16 N=16)    16 KB
+    static constexpr int OffBS3i = OffBS3 + 16384;      // 32 x (K=16 N=16)    16 KB
+    static constexpr int OffBS2i = OffBS3i + 16384;     // K=64 N=64           8 KB
+    static constexpr int OffBS1i = OffBS2i + 8192;      // K=64 N=2*kJ1        4 / 8 KB
+    static constexpr int OffBEnd = OffBS1i + kJ1 * 256;
+    static constexpr int BImageBytes = OffBEnd - OffBS1;
+    static constexpr int OffK = OffBEnd;                // the tile's filter spectrum row
+    // the 256-entry w8192 twiddle table lives in shared memory except in the
+    // split mode, whose larger factors leave no room (it is read through L1)
+    static constexpr bool kTwShared = !kFull;
+    static constexpr int OffTwM = OffK + kKBytes;
+    static constexpr int OffBars = OffTwM + (kTwShared ? 2048 : 0);   // 16 mbarrier slots
+    static constexpr int OffMisc = OffBars + 128;       // tmem base, abort flag
+    static constexpr int SmemBytes = OffMisc + 64 + 1024;              // + alignment slack
+    static constexpr int Chunks = kFull ? 48 : 44;      // 8 per stage S1..S2', S1' 4 or 8
+};
+static_assert(Lay<kModeSplit>::SmemBytes <= 232448, "shared memory");
+static_assert(Lay<kModePlain>::SmemBytes <= 232448, "shared memory");
 
 // byte offset of element (n, k) of a K x N B operand in the no-swizzle
 // K-major layout used for every DFT factor: 8x8 core matrices, K-halves
@@ -115,6 +134,11 @@ constexpr int kSmemBytes = kOffMisc + 64 + 1024;    // + alignment slack
 inline size_t bimg_offset(int n, int k, int N) {
     return (size_t)(k / 8) * (N / 8) * 128 + (size_t)(n / 8) * 128 + (n % 8) * 16 + (k % 8) * 2;
 }
+
+// A twiddle in packed half precision (see cmul_h).
+struct Tw16 {
+    uint32_t p, q;
+};
 
 struct TcArgs {
     const void* u;
@@ -133,7 +157,10 @@ struct TcArgs {
     int64_t nunits;            // H * nwin * tpc
     const uint4* bimg;         // DFT factors, image of the shared-memory region
     const float2* tw1024;      // exp(-2 pi i e/1024), e < 1024
-    const float2* twM;         // exp(-2 pi i e/8192), e < 256
+    const Tw16* twM16;         // exp(-2 pi i e/8192), e < 256, as half2 pairs
+    const float2* tw16k;       // split mode: exp(-2 pi i t/16384), t < 8192
+    float2 w16k_j3[8];         // split mode: exp(-2 pi i j/16384), j < 8
+    uint4* scratch;            // split mode: [CTAs][4 pairs][8192] half2, z_even of the group
     int* status;
 };
 
@@ -170,9 +197,6 @@ __device__ __forceinline__ uint32_t pack_h2(float re, float im) {
 // as the two half2 values tp = (tr, ti) and tq = (-ti, tr); then
 //   x t = re(x) tp + im(x) tq,   x conj(t) = re(x) tp* + im(x) tq*
 // with tp* = (tr, -ti) and tq* = (ti, tr), each a sign flip of one half.
-struct Tw16 {
-    uint32_t p, q;
-};
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 __device__ __forceinline__ Tw16 tw16(float2 t) {
@@ -193,6 +217,7 @@ struct PairInfo {
     int64_t h;
     bool valid;
     bool tail_only;      // only window positions t >= kHop are outputs
+    bool odd;            // split mode: the tile of odd spectrum bins
 };
 
 // A tile holds 4 pairs of batch rows of ONE channel and one window: unit u
@@ -207,19 +232,40 @@ struct PairInfo {
 // history before t = 0), window j > 0 keeps positions [2048, 4096), i.e.
 // y[2048 (j+1), 2048 (j+2)).  N / 2048 - 1 windows cover the sequence.
 // Tile indices fit in 32 bits (the host rejects launches of 2^31 tiles or
-// more), so the decomposition uses 32-bit division.  WIN = false is the
-// single-window case (N = 4096), with the row stride and the window fixed.
-template <bool WIN>
+// more), so the decomposition uses 32-bit division.  In the plain mode the
+// row stride and the window are fixed.
+template <int MODE>
 __device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t unit, int q) {
     PairInfo p;
-    if constexpr (!WIN) {
+    if constexpr (MODE == kModePlain) {
         p.h = unit / a.tpc;
         const int64_t bp = 4 * (unit % a.tpc) + q;
         p.valid = bp < a.pb;
         p.tail_only = false;
+        p.odd = false;
         const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
         p.o0 = (b0 * a.H + p.h) * kN;
         p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * kN : -1;
+        return p;
+    }
+    if constexpr (MODE == kModeSplit) {
+        // Split mode (N = 8192, full-length filter).  With M = 16384 and x zero
+        // for t >= 8192, X(2f) is the 8192-point transform of x and X(2f+1)
+        // that of x[t] w16384^t; the output is
+        //   y[t] = (z_even[t] + w16384^-t z_odd[t]) / 2,
+        // z_e the inverse 8192-point transform of X(2f+e) K(2f+e) (unitary
+        // factors, unnormalised K).  Unit u is group u / 2 (4 pairs of one
+        // channel) and parity u % 2; a CTA takes both parities of a group
+        // back to back, parking z_even in its scratch slot for the odd tile.
+        const int64_t g = unit >> 1;
+        p.h = g / a.tpc;
+        const int64_t bp = 4 * (g % a.tpc) + q;
+        p.valid = bp < a.pb;
+        p.tail_only = false;
+        p.odd = unit & 1;
+        const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
+        p.o0 = (b0 * a.H + p.h) * a.N;
+        p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * a.N : -1;
         return p;
     }
     const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
@@ -230,10 +276,35 @@ __device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t unit, int
     const int64_t bp = 4 * (int64_t)(rem - j * tpc) + q;
     p.valid = bp < a.pb;
     p.tail_only = j > 0;
+    p.odd = false;
     const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
     p.o0 = (b0 * a.H + p.h) * a.N + kHop * j;
     p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * a.N + kHop * j : -1;
     return p;
+}
+
+// A CTA's first unit and the one after `u` (the split mode takes the two
+// parity tiles of a group back to back).
+template <int MODE>
+__device__ __forceinline__ int64_t first_unit() {
+    return MODE == kModeSplit ? 2 * (int64_t)blockIdx.x : (int64_t)blockIdx.x;
+}
+template <int MODE>
+__device__ __forceinline__ int64_t next_unit(int64_t u) {
+    if constexpr (MODE == kModeSplit) return (u & 1) ? u + 2 * (int64_t)gridDim.x - 1 : u + 1;
+    return u + gridDim.x;
+}
+// The tile's channel, and its filter row in K_f (the split mode stores the
+// even and the odd bins of each channel as two rows).
+template <int MODE>
+__device__ __forceinline__ int64_t unit_channel(const TcArgs& a, int64_t u) {
+    if constexpr (MODE == kModeWindows) return (int64_t)((uint32_t)u / ((uint32_t)a.nwin * (uint32_t)a.tpc));
+    if constexpr (MODE == kModeSplit) return (u >> 1) / a.tpc;
+    return u / a.tpc;
+}
+template <int MODE>
+__device__ __forceinline__ int64_t unit_filter_row(const TcArgs& a, int64_t u) {
+    return MODE == kModeSplit ? 2 * unit_channel<MODE>(a, u) + (u & 1) : unit_channel<MODE>(a, u);
 }
 
 // position of spectrum value f = c1 + 32 c2 + 1024 c3 in a channel's fp16 row:
@@ -243,19 +314,20 @@ __host__ __device__ __forceinline__ int k16_index(int c1, int c2, int c3) {
     return ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + (c3 & 3);
 }
 
-template <typename T, bool WIN>
+template <typename T, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a) {
+    using LY = Lay<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* bar = (uint64_t*)(smem + kOffBars);
+    uint64_t* bar = (uint64_t*)(smem + LY::OffBars);
     uint64_t* bar_in = bar + 0;    // the tile's input is in TMEM (16 epilogue warps)
     uint64_t* dfull = bar + 1;     // [kDBuf] accumulator buffer written (tcgen05.commit)
     uint64_t* dfree = bar + 5;     // [kDBuf] accumulator buffer drained (16 epilogue warps)
     uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
     uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
     uint64_t* bar_stage = bar + 11;   // [3] E2, E3', E2' done for the tile (16 epilogue warps)
-    uint32_t* tmem_base_sh = (uint32_t*)(smem + kOffMisc);
-    volatile int* abort_flag = (volatile int*)(smem + kOffMisc + 4);
+    uint32_t* tmem_base_sh = (uint32_t*)(smem + LY::OffMisc);
+    volatile int* abort_flag = (volatile int*)(smem + LY::OffMisc + 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -277,12 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
     if (warp == kEpiWarps) tmem_alloc(tmem_base_sh, 512);   // the first MMA warp owns TMEM
     // DFT factors and the w8192 twiddle table into shared memory
     {
-        uint4* dst = (uint4*)(smem + kOffBS1);
-        for (int i = tid; i < kBImageBytes / 16; i += kThreads) dst[i] = __ldg(&a.bimg[i]);
-        Tw16* t2 = (Tw16*)(smem + kOffTwM);
-        for (int i = tid; i < 256; i += kThreads) t2[i] = tw16(__ldg(&a.twM[i]));
+        uint4* dst = (uint4*)(smem + LY::OffBS1);
+        for (int i = tid; i < LY::BImageBytes / 16; i += kThreads) dst[i] = __ldg(&a.bimg[i]);
+        if constexpr (LY::kTwShared) {
+            Tw16* t2 = (Tw16*)(smem + LY::OffTwM);
+            for (int i = tid; i < 256; i += kThreads) t2[i] = a.twM16[i];
+        }
     }
-    const Tw16* stwM = (const Tw16*)(smem + kOffTwM);
+    const Tw16* stwM = LY::kTwShared ? (const Tw16*)(smem + LY::OffTwM) : a.twM16;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -312,19 +386,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         const uint32_t id16 = idesc_f16_f32(128, 16);
         const uint32_t id32 = idesc_f16_f32(128, 32);
         // descriptor bases (start address in 16-byte units in the low bits)
-        const uint64_t dS1 = make_desc(sbase + kOffBS1, 1024, 128, 0);    // K-step: +2048 B
-        const uint64_t dS2 = make_desc(sbase + kOffBS2, 1024, 128, 0);    // K-step: +2048 B
-        const uint64_t dS2i = make_desc(sbase + kOffBS2i, 1024, 128, 0);
-        const uint64_t dS3 = make_desc(sbase + kOffBS3, 256, 128, 0);     // per c2: +512 B
-        const uint64_t dS3i = make_desc(sbase + kOffBS3i, 256, 128, 0);
-        const uint64_t dS1i = make_desc(sbase + kOffBS1i, 512, 128, 0);   // N half: +256 B, K-step: +1024 B
-        const uint64_t dA = make_desc(sbase + kOffData, 16, 1024, 2);     // tile: +16384 B, K-step: +32 B
+        const uint64_t dS1 = make_desc(sbase + LY::OffBS1, 1024, 128, 0);    // K-step: +2048 B
+        const uint64_t dS2 = make_desc(sbase + LY::OffBS2, 1024, 128, 0);    // K-step: +2048 B
+        const uint64_t dS2i = make_desc(sbase + LY::OffBS2i, 1024, 128, 0);
+        const uint64_t dS3 = make_desc(sbase + LY::OffBS3, 256, 128, 0);     // per c2: +512 B
+        const uint64_t dS3i = make_desc(sbase + LY::OffBS3i, 256, 128, 0);
+        // S1' factor: N = 2 kJ1 columns (LBO = kJ1 * 32 B); a 32-column half
+        // is +512 B, a K step +kJ1 * 64 B
+        const uint64_t dS1i = make_desc(sbase + LY::OffBS1i, LY::kJ1 * 32, 128, 0);
+        const uint64_t dA = make_desc(sbase + LY::OffData, 16, 1024, 2);     // tile: +16384 B, K-step: +32 B
         uint32_t g = 0;          // global chunk counter (accumulator buffer g % kDBuf)
         int iter = 0;
         int k_issued = 0;        // filter-row copies issued
         bool ok = true;
         g = issuer;
-        for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
+        for (int64_t unit = first_unit<MODE>(); unit < a.nunits && ok; unit = next_unit<MODE>(unit), ++iter) {
             if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
             tc_fence_after();
             if (issuer == 0) {
@@ -332,16 +408,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     // the previous tile is finished with the filter buffer (its
                     // epilogue warps arrived on bar_in after all their reads)
                     mbar_expect_tx(bar_k, kKBytes);
-                    bulk_copy_g2s(smem + kOffK,
-                                  a.Kh16 + (WIN ? (int64_t)((uint32_t)unit / ((uint32_t)a.nwin * (uint32_t)a.tpc))
-                                                : unit / a.tpc) * kM,
-                                  kKBytes, bar_k);
+                    bulk_copy_g2s(smem + LY::OffK, a.Kh16 + unit_filter_row<MODE>(a, unit) * kM, kKBytes, bar_k);
                 }
                 ++k_issued;
                 __syncwarp();
             }
 #pragma unroll 1
-            for (int c = issuer; c < kChunksPerUnit && ok; c += kMmaWarps, g += kMmaWarps) {
+            for (int c = issuer; c < LY::Chunks && ok; c += kMmaWarps, g += kMmaWarps) {
                 const int stage = chunk_stage(c), k = chunk_index(c);
                 const uint32_t b = g % kDBuf;
                 // the buffer's previous contents must have been drained ...
@@ -354,9 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     // descriptors are loop-invariant bases plus an offset in
                     // 16-byte units added to the start-address field
                     const uint32_t d = tbase + 256 + 64 * b;
-                    if (stage == 0) {            // S1: A1 (TMEM) cols j3*16 + j1, j3 = k
-                        mma_ts(d, tbase + k * 16, dS1, id64, 0);
-                        mma_ts(d, tbase + k * 16 + 8, dS1 + 128, id64, 1);
+                    if (stage == 0) {            // S1: A1 (TMEM) cols j3*kJ1 + j1, j3 = k
+#pragma unroll
+                        for (int ks = 0; ks < LY::kJ1 / 8; ++ks)
+                            mma_ts(d, tbase + k * LY::kJ1 + 8 * ks, dS1 + 128 * ks, id64, ks);
                     } else if (stage == 1 || stage == 4) {   // S2 / S2': smem tile j3 = k
                         const uint64_t db = stage == 1 ? dS2 : dS2i;
                         const uint64_t da = dA + (uint64_t)(k * (kTile >> 4));
@@ -366,13 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         const uint64_t db = (stage == 2 ? dS3 : dS3i) + (uint64_t)(4 * k * 32);
 #pragma unroll
                         for (int cl = 0; cl < 4; ++cl) mma_ts(d + cl * 16, tbase + (4 * k + cl) * 8, db + 32 * cl, id16, 0);
-                    } else {                     // S1': j3 = 2k + jl, all j1 < 16 (N = 32)
-                        const uint64_t da = dA + (uint64_t)(2 * k * (kTile >> 4));
+                    } else {                     // S1': j3 = 2(k%4) + jl, j1 in [16h, 16h+16), h = k/4 (N = 32)
+                        const uint64_t da = dA + (uint64_t)(2 * (k & 3) * (kTile >> 4));
+                        const uint64_t db = dS1i + (uint64_t)(32 * (k >> 2));
 #pragma unroll
                         for (int jl = 0; jl < 2; ++jl) {
 #pragma unroll
                             for (int s = 0; s < 4; ++s)
-                                mma_ss(d + jl * 32, da + jl * (kTile >> 4) + 2 * s, dS1i + 64 * s, id32, s);
+                                mma_ss(d + jl * 32, da + jl * (kTile >> 4) + 2 * s, db + LY::kJ1 * 4 * s, id32, s);
                         }
                     }
                     tc_commit(&dfull[b]);
@@ -388,10 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     // tile start, 3.5% faster overall (and 7% faster than no
                     // prefetch).
                     const void* pf_src = nullptr;
-                    uint32_t pf_bytes = kN * sizeof(T);
-                    const int64_t nu = unit + gridDim.x;
+                    uint32_t pf_bytes = (MODE == kModeSplit ? 2 * kN : kN) * sizeof(T);
+                    const int64_t nu = next_unit<MODE>(unit);
                     if (nu < a.nunits && (lane >> 3) == issuer) {
-                        const PairInfo Q = pair_info<WIN>(a, nu, issuer);
+                        const PairInfo Q = pair_info<MODE>(a, nu, issuer);
                         const int which = lane & 7;
                         if (Q.valid) {
                             if (which == 0) pf_src = (const T*)a.u + Q.o0;
@@ -400,7 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             else if (which == 3 && Q.o1 >= 0) pf_src = (const T*)a.u + Q.o1;
                             else if (which == 4 && Q.o1 >= 0 && a.w) pf_src = (const T*)a.w + Q.o1;
                             else if (which == 5 && Q.o1 >= 0 && a.v) pf_src = (const T*)a.v + Q.o1;
-                            else if (which == 6 && issuer == 0) { pf_src = a.Kh16 + Q.h * (int64_t)kM; pf_bytes = kKBytes; }
+                            else if (which == 6 && issuer == 0) {
+                                pf_src = a.Kh16 + unit_filter_row<MODE>(a, nu) * kM;
+                                pf_bytes = kKBytes;
+                            }
                         }
                     }
                     if (pf_src) prefetch_l2(pf_src, pf_bytes);
@@ -427,7 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         const int q = warp & 3;          // lane quarter = pair within the tile
         const int s = warp >> 2;         // column slice
         const uint32_t lq = (uint32_t)(32 * q) << 16;
-        const int64_t nblk = kN / 32;
+        // the convolution's length and transform length (mask bins)
+        constexpr int kSeqN = LY::kFull ? 2 * kN : kN, kSeqM = 2 * kSeqN;
+        const int64_t nblk = kSeqN / 32;
 
         // w1024^(c1 l) with (c1, l) = (8s + i, lane) in E1 and (lane, 8s + i)
         // in E2' -- the same eight values, kept in registers; wM^(c1 j3) with
@@ -438,16 +518,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 
         int iter = 0;
         bool ok = true;
-        for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
-            const int64_t hch = WIN ? (int64_t)((uint32_t)unit / ((uint32_t)a.nwin * (uint32_t)a.tpc))
-                                    : unit / a.tpc;   // the tile's channel
+        for (int64_t unit = first_unit<MODE>(); unit < a.nunits && ok; unit = next_unit<MODE>(unit), ++iter) {
+            const int64_t hch = unit_channel<MODE>(a, unit);
 
-            // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [4s, 4s+4).
+            // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [J s, J s + J)
+            // with J = kJ1 / 4 (split mode: times w16384^t in the odd tile).
             // Loads are issued in batches before any use (absent rows or gates
             // read a present row and are masked afterwards).  Row offsets are
             // formed here and again for the output stage instead of being
             // kept, which keeps registers for the stages.
-            const PairInfo P = pair_info<WIN>(a, unit, q);
+            const PairInfo P = pair_info<MODE>(a, unit, q);
             const bool has1 = P.o1 >= 0;
             {
                 const int64_t oo1 = has1 ? P.o1 : P.o0;
@@ -457,12 +537,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
                 const bool has_w = a.w != nullptr;
                 const bool keep0 = P.valid, keep1 = has1;
+                constexpr int J = LY::kJ1 / 4;
 #pragma unroll
-                for (int jp = 0; jp < 2; ++jp) {
+                for (int jp = 0; jp < J / 2; ++jp) {
                     uint4 ld[2][4];
 #pragma unroll
                     for (int jh = 0; jh < 2; ++jh) {
-                        const int64_t t0 = 256 * (4 * s + 2 * jp + jh) + 8 * lane;
+                        const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
                         ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
                         ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
                         ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
@@ -471,6 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     uint32_t pk[8][2];
 #pragma unroll
                     for (int jh = 0; jh < 2; ++jh) {
+                        float2 w0 = make_float2(1.f, 0.f);     // w16384^t0 (odd split tile)
+                        if constexpr (LY::kFull) {
+                            if (P.odd) w0 = __ldg(&a.tw16k[256 * (J * s + 2 * jp + jh) + 8 * lane]);
+                        }
                         const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
                         const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
                         const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
@@ -484,12 +569,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             }
                             if (!keep0) xa = make_float2(0.f, 0.f);
                             if (!keep1) xb = make_float2(0.f, 0.f);
+                            if constexpr (LY::kFull) {
+                                if (P.odd) {
+                                    // (a + i b)[t] times w16384^t, t = t0 + 2e (+1)
+                                    const float2 wa0 = cmul(w0, a.w16k_j3[2 * e]), wa1 = cmul(w0, a.w16k_j3[2 * e + 1]);
+                                    const float2 z0 = cmul(make_float2(xa.x, xb.x), wa0);
+                                    const float2 z1 = cmul(make_float2(xa.y, xb.y), wa1);
+                                    xa = make_float2(z0.x, z1.x);
+                                    xb = make_float2(z0.y, z1.y);
+                                }
+                            }
                             pk[2 * e][jh] = pack_h2(xa.x, xb.x);
                             pk[2 * e + 1][jh] = pack_h2(xa.y, xb.y);
                         }
                     }
 #pragma unroll
-                    for (int j3 = 0; j3 < 8; ++j3) tmem_st2(tbase + lq + j3 * 16 + 4 * s + 2 * jp, pk[j3][0], pk[j3][1]);
+                    for (int j3 = 0; j3 < 8; ++j3)
+                        tmem_st2(tbase + lq + j3 * LY::kJ1 + J * s + 2 * jp, pk[j3][0], pk[j3][1]);
                 }
                 tc_wait_st();
                 tc_fence_before();
@@ -497,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 if (lane == 0) mbar_arrive(bar_in);
             }
 
-            const __half2* Ks = (const __half2*)(smem + kOffK);
+            const __half2* Ks = (const __half2*)(smem + LY::OffK);
             // loaded once per tile and pinned in a register (an opaque move
             // keeps the compiler from re-issuing the global load at each use)
             float kscale = __ldg(&a.Kscale[hch]);
@@ -511,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // buffer c % 4; 44 chunks per tile) and the store patterns are
             // fixed at compile time.
             auto begin_pair = [&](int c) -> bool {
-                const uint32_t par = (uint32_t)(iter ^ (c >> 2)) & 1u;   // use number 11*iter + c/4 of the buffer
+                // use number (Chunks/4)*iter + c/4 of the buffer
+                const uint32_t par = (uint32_t)(iter * (LY::Chunks / 4) + (c >> 2)) & 1u;
                 if (!wait(&dfull[c & 3], par) || !wait(&dfull[(c & 3) + 1], par)) {
                     fail();
                     return false;
@@ -550,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 release(c);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    uint8_t* tile = smem + kOffData + (k + cc) * kTile + (4 * q + s) * 1024;
+                    uint8_t* tile = smem + LY::OffData + (k + cc) * kTile + (4 * q + s) * 1024;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         *(uint32_t*)(tile + i * 128 + ((4 * lane) ^ (i << 4))) = cmul_h(r[cc][2 * i], r[cc][2 * i + 1], tw[i]);
@@ -609,8 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         // its mirror M - f share one rfft bin)
 #pragma unroll
                         for (int c3 = 0; c3 < 8; ++c3) {
-                            const int f = lane + 32 * c2 + 1024 * c3;
-                            int blk = (f <= kN ? f : kM - f) >> 5;
+                            const int f8 = lane + 32 * c2 + 1024 * c3;
+                            const int f = LY::kFull ? 2 * f8 + (P.odd ? 1 : 0) : f8;   // bin of the full spectrum
+                            int blk = (f <= kSeqN ? f : kSeqM - f) >> 5;
                             blk = blk < (int)nblk ? blk : (int)nblk - 1;
                             if (__ldg(&mrow[blk]) == 0) kw[c3] = 0u;
                         }
@@ -646,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const uint32_t m = 32 * q + lane;
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
-                    uint8_t* tile = smem + kOffData + (2 * s + jj) * kTile;
+                    uint8_t* tile = smem + LY::OffData + (2 * s + jj) * kTile;
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         uint32_t hq[4];
@@ -670,27 +768,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             if (ok) stage_done(2);
 #pragma unroll
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
-            // EO: lane = l; chunk 40 + k holds j3 = 2k + jl (jl = 0, 1) for all
-            // j1 < 16 at columns jl*32 + 2*j1.  Output pair h (chunks 40 + 2h,
-            // 41 + 2h) covers j3 in [4h, 4h+4); this warp takes j1 = 4s + jj
-            // and writes y = s_h * v * z for the four consecutive
-            // t = 256 j1 + 8 l + 4h + (0..3) of each row as one 8-byte store.
+            // EO: lane = l; chunk 40 + k holds j3 = 2(k%4) + jl (jl = 0, 1) for
+            // j1 in [16 (k/4), 16 (k/4) + 16) at columns jl*32 + 2*(j1 % 16).
+            // Output pair hp (chunks 40 + 2hp, 41 + 2hp) covers j3 in
+            // [4 (hp%2), 4 (hp%2) + 4) of that j1 half; this warp takes
+            // j1 = 16 (hp/2) + 4s + jj and the four consecutive
+            // t = 256 j1 + 8 l + 4 (hp%2) + (0..3) of each row.  Plain and window
+            // modes: y = s_h v z, one 8-byte store per row.  Split mode: the
+            // even tile parks z in the CTA's scratch slot (16 bytes per four t),
+            // the odd tile writes y = s_h v (z_even + w16384^-t z_odd) / 2.
             // In a window after the first, positions t < 2048 (j1 < 8: warps
             // with s < 2) are not outputs; their gate loads still read inside
             // the sequence and are discarded.
-            const bool emit = P.valid && !(P.tail_only && s < 2);
+            const bool emit = P.valid && !(P.tail_only && s < 2) && (!LY::kFull || P.odd);
+            const bool park = LY::kFull && P.valid && !P.odd;
+            uint4* slot = LY::kFull ? a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4) : nullptr;
 #pragma unroll 1
-            for (int h = 0; h < 2 && ok; ++h) {
-                const int c = 40 + 2 * h;
+            for (int hp = 0; hp < (LY::Chunks - 40) / 2 && ok; ++hp) {
+                const int c = 40 + 2 * hp;
+                const int jb = 16 * (hp >> 1) + 4 * s;       // this warp's first j1
+                const int tb = 8 * lane + 4 * (hp & 1);
                 // output gate values, requested before the accumulator wait so
                 // that their latency overlaps it (an empty pair reads row 0 of
                 // the channel and discards it)
                 uint2 va[4], vb[4];
-                {
+                if (!LY::kFull || P.odd) {
                     const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        const int64_t t0 = 256 * (4 * s + jj) + 8 * lane + 4 * h;
+                        const int64_t t0 = 256 * (jb + jj) + tb;
                         va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
                         vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
                     }
@@ -703,20 +809,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     for (int jl = 0; jl < 2; ++jl) tmem_ld8(dcol(c + cc) + jl * 32 + 8 * s, r[cc][jl]);
                 tc_wait_ld();
                 release(c);
+                if (park) {
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        // j3 = 4 (hp%2) + 2 cc + jl, in t order
+                        slot[(256 * (jb + jj) + tb) >> 2] =
+                            make_uint4(pack_h2(__uint_as_float(r[0][0][2 * jj]), __uint_as_float(r[0][0][2 * jj + 1])),
+                                       pack_h2(__uint_as_float(r[0][1][2 * jj]), __uint_as_float(r[0][1][2 * jj + 1])),
+                                       pack_h2(__uint_as_float(r[1][0][2 * jj]), __uint_as_float(r[1][0][2 * jj + 1])),
+                                       pack_h2(__uint_as_float(r[1][1][2 * jj]), __uint_as_float(r[1][1][2 * jj + 1])));
+                    }
+                }
                 if (emit) {
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        const int64_t t0 = 256 * (4 * s + jj) + 8 * lane + 4 * h;
+                        const int64_t t0 = 256 * (jb + jj) + tb;
                         const uint32_t vaw[2] = {va[jj].x, va[jj].y};
                         const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
+                        uint4 zev = make_uint4(0, 0, 0, 0);
+                        float2 w0 = make_float2(1.f, 0.f);
+                        if constexpr (LY::kFull) {
+                            zev = slot[t0 >> 2];
+                            w0 = __ldg(&a.tw16k[t0]);
+                        }
+                        const uint32_t zw[4] = {zev.x, zev.y, zev.z, zev.w};
                         uint32_t oa[2], ob[2];
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            // j3 = 4h + 2e + (0, 1): chunk cc = e, jl = 0, 1
-                            float a0 = __uint_as_float(r[e][0][2 * jj]) * kscale;
-                            float a1 = __uint_as_float(r[e][1][2 * jj]) * kscale;
-                            float b0 = __uint_as_float(r[e][0][2 * jj + 1]) * kscale;
-                            float b1 = __uint_as_float(r[e][1][2 * jj + 1]) * kscale;
+                            // j3 = 4 (hp%2) + 2e + (0, 1): chunk cc = e, jl = 0, 1
+                            float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
+                            float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
+                            float sc = kscale;
+                            if constexpr (LY::kFull) {
+                                // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
+                                const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
+                                const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
+                                const float2 ze0 = __half22float2(u2h(zw[2 * e])), ze1 = __half22float2(u2h(zw[2 * e + 1]));
+                                a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
+                                a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
+                                sc *= 0.5f;
+                            }
+                            a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
                             if (a.v) {
                                 const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
                                 a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
@@ -744,9 +877,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 // ----------------------------------------------------------- host side ---
 
 struct TcResources {
+    int mode = kModePlain;
     uint8_t* bimg = nullptr;
     float2* tw1024 = nullptr;
-    float2* twM = nullptr;
+    Tw16* twM16 = nullptr;
+    float2* tw16k = nullptr;      // split mode
+    uint4* scratch = nullptr;     // split mode: num_sms x 4 x 8192 half2
     int num_sms = 0;
 };
 
@@ -777,19 +913,22 @@ void put_complex_matrix(std::vector<uint8_t>& img, size_t base, int n_out, int n
         }
 }
 
+template <int MODE>
 std::vector<uint8_t> build_bimage() {
-    std::vector<uint8_t> img(kBImageBytes, 0);
+    using LY = Lay<MODE>;
+    constexpr int J = LY::kJ1;
+    std::vector<uint8_t> img(LY::BImageBytes, 0);
     const double r32 = 1.0 / std::sqrt(32.0), r8 = 1.0 / std::sqrt(8.0);
-    auto off = [](int o) { return (size_t)(o - kOffBS1); };
+    auto off = [](int o) { return (size_t)(o - LY::OffBS1); };
     std::vector<std::complex<double>> F;
-    // S1: c1 <- j1 (j1 < 16)
-    F.assign(32 * 16, 0);
-    for (int c = 0; c < 32; ++c) for (int j = 0; j < 16; ++j) F[c * 16 + j] = wpow((long long)c * j, 32, -1) * r32;
-    put_complex_matrix(img, off(kOffBS1), 32, 16, F);
+    // S1: c1 <- j1 (j1 < J: the nonzero inputs)
+    F.assign(32 * J, 0);
+    for (int c = 0; c < 32; ++c) for (int j = 0; j < J; ++j) F[c * J + j] = wpow((long long)c * j, 32, -1) * r32;
+    put_complex_matrix(img, off(LY::OffBS1), 32, J, F);
     // S2: c2 <- l
     F.assign(32 * 32, 0);
     for (int c = 0; c < 32; ++c) for (int j = 0; j < 32; ++j) F[c * 32 + j] = wpow((long long)c * j, 32, -1) * r32;
-    put_complex_matrix(img, off(kOffBS2), 32, 32, F);
+    put_complex_matrix(img, off(LY::OffBS2), 32, 32, F);
     // S3 (per c2): c3 <- j3 with w8^(c3 j3) w256^(c2 j3);  S3': j3 <- c3, conjugate
     for (int c2 = 0; c2 < 32; ++c2) {
         std::vector<std::complex<double>> G(64), Gi(64);
@@ -799,18 +938,36 @@ std::vector<uint8_t> build_bimage() {
                 G[c3 * 8 + j3] = gv;
                 Gi[j3 * 8 + c3] = std::conj(gv);
             }
-        put_complex_matrix(img, off(kOffBS3) + c2 * 512, 8, 8, G);
-        put_complex_matrix(img, off(kOffBS3i) + c2 * 512, 8, 8, Gi);
+        put_complex_matrix(img, off(LY::OffBS3) + c2 * 512, 8, 8, G);
+        put_complex_matrix(img, off(LY::OffBS3i) + c2 * 512, 8, 8, Gi);
     }
     // S2': l <- c2
     F.assign(32 * 32, 0);
     for (int l = 0; l < 32; ++l) for (int c = 0; c < 32; ++c) F[l * 32 + c] = wpow((long long)c * l, 32, +1) * r32;
-    put_complex_matrix(img, off(kOffBS2i), 32, 32, F);
-    // S1': j1 <- c1 (j1 < 16)
-    F.assign(16 * 32, 0);
-    for (int j = 0; j < 16; ++j) for (int c = 0; c < 32; ++c) F[j * 32 + c] = wpow((long long)c * j, 32, +1) * r32;
-    put_complex_matrix(img, off(kOffBS1i), 16, 32, F);
+    put_complex_matrix(img, off(LY::OffBS2i), 32, 32, F);
+    // S1': j1 <- c1 (j1 < J: the kept outputs)
+    F.assign(J * 32, 0);
+    for (int j = 0; j < J; ++j) for (int c = 0; c < 32; ++c) F[j * 32 + c] = wpow((long long)c * j, 32, +1) * r32;
+    put_complex_matrix(img, off(LY::OffBS1i), J, 32, F);
     return img;
+}
+
+uint16_t half_bits(float x) {
+    const __half h = __float2half_rn(x);
+    uint16_t b;
+    std::memcpy(&b, &h, 2);
+    return b;
+}
+// exp(-2 pi i e / 8192), e < 256, as the packed-half pair (tr, ti), (-ti, tr)
+std::vector<Tw16> twiddle_table16() {
+    std::vector<Tw16> t(256);
+    for (int e = 0; e < 256; ++e) {
+        const std::complex<double> z = wpow(e, kM, -1);
+        const float tr = (float)z.real(), ti = (float)z.imag();
+        t[e].p = (uint32_t)half_bits(tr) | ((uint32_t)half_bits(ti) << 16);
+        t[e].q = (uint32_t)half_bits(-ti) | ((uint32_t)half_bits(tr) << 16);
+    }
+    return t;
 }
 
 std::vector<float2> twiddle_table(int n, int count) {
@@ -822,60 +979,99 @@ std::vector<float2> twiddle_table(int n, int count) {
     return t;
 }
 
+// K_f -> rfft bins [0, N] of each channel.  split = 0: one row of the
+// 8192-point spectrum per channel; split = 1: the 16384-point spectrum as
+// two rows per channel (even bins, odd bins).
 __global__ void tc_export_kernel(const __half2* __restrict__ Kh, const float* __restrict__ scale,
-                                 float* __restrict__ out, int64_t H) {
-    const int64_t total = H * (kN + 1);
+                                 float* __restrict__ out, int64_t H, int split) {
+    const int64_t nb = split ? 2 * kN + 1 : kN + 1;
+    const int64_t total = H * nb;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t h = i / (kN + 1), f = i % (kN + 1);
-        const int c1 = (int)(f & 31), c2 = (int)((f >> 5) & 31), c3 = (int)(f >> 10);
-        const float2 z = __half22float2(Kh[h * kM + k16_index(c1, c2, c3)]);
+        const int64_t h = i / nb, f = i % nb;
+        const int64_t row = split ? 2 * h + (f & 1) : h;
+        const int64_t f8 = split ? f >> 1 : f;
+        const int c1 = (int)(f8 & 31), c2 = (int)((f8 >> 5) & 31), c3 = (int)(f8 >> 10);
+        const float2 z = __half22float2(Kh[row * kM + k16_index(c1, c2, c3)]);
         out[2 * i] = z.x * scale[h];
         out[2 * i + 1] = z.y * scale[h];
     }
+}
+
+// Kernel mode of a plan: sequences of 4096 run plain; sequences of 8192 run
+// the parity split unless the filter is short enough for windows; longer
+// sequences need windows (filters of at most 2049 taps).
+int tc_mode(int64_t N, int64_t L) {
+    if (N == kN) return kModePlain;
+    if (N == 2 * kN && L > kHop + 1) return kModeSplit;
+    return kModeWindows;
 }
 
 }  // namespace
 
 bool tc_supported(int64_t N, int64_t L, int dtype) {
     if (dtype != kF16 && dtype != kBF16) return false;
-    if (N == kN) return true;
+    if (N == kN || N == 2 * kN) return true;
     return N > kN && L <= kHop + 1;      // overlap-save windows (N a power of two)
 }
 
 int64_t tc_windows(int64_t N) { return N == kN ? 1 : N / kHop - 1; }
+bool tc_overlap_save(int64_t N, int64_t L) { return tc_mode(N, L) == kModeWindows; }
+int64_t tc_tiles_per_pair_group(int64_t N, int64_t L) {
+    const int m = tc_mode(N, L);
+    return m == kModeWindows ? tc_windows(N) : (m == kModeSplit ? 2 : 1);
+}
+
+namespace {
+
+template <int MODE>
+cudaError_t set_smem_attributes() {
+    cudaError_t e = cudaFuncSetAttribute(tc_fftconv_n4096_kernel<__nv_bfloat16, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<MODE>::SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_n4096_kernel<__half, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Lay<MODE>::SmemBytes);
+    return e;
+}
+
+template <typename V>
+cudaError_t upload_vec(V** dst, const std::vector<V>& v) {
+    cudaError_t e = cudaMalloc((void**)dst, v.size() * sizeof(V));
+    if (e == cudaSuccess) e = cudaMemcpy(*dst, v.data(), v.size() * sizeof(V), cudaMemcpyHostToDevice);
+    return e;
+}
+
+template <int MODE>
+void launch_mode(const Plan& p, const TcArgs& a, int64_t grid, cudaStream_t s) {
+    if (p.dtype == kBF16)
+        tc_fftconv_n4096_kernel<__nv_bfloat16, MODE><<<(unsigned)grid, kThreads, Lay<MODE>::SmemBytes, s>>>(a);
+    else
+        tc_fftconv_n4096_kernel<__half, MODE><<<(unsigned)grid, kThreads, Lay<MODE>::SmemBytes, s>>>(a);
+}
+
+}  // namespace
 
 cudaError_t tc_plan_init(Plan& p) {
     TcResources* r = new TcResources();
     p.tc = r;
-    const std::vector<uint8_t> img = build_bimage();
+    r->mode = tc_mode(p.N, p.L);
+    const std::vector<uint8_t> img = r->mode == kModeSplit ? build_bimage<kModeSplit>() : build_bimage<kModePlain>();
     cudaError_t e = cudaMalloc((void**)&r->bimg, img.size());
     if (e == cudaSuccess) e = cudaMemcpy(r->bimg, img.data(), img.size(), cudaMemcpyHostToDevice);
-    const std::vector<float2> t1 = twiddle_table(1024, 1024), t2 = twiddle_table(kM, 256);
-    if (e == cudaSuccess) e = cudaMalloc((void**)&r->tw1024, t1.size() * sizeof(float2));
-    if (e == cudaSuccess) e = cudaMemcpy(r->tw1024, t1.data(), t1.size() * sizeof(float2), cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMalloc((void**)&r->twM, t2.size() * sizeof(float2));
-    if (e == cudaSuccess) e = cudaMemcpy(r->twM, t2.data(), t2.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddle_table(1024, 1024));
+    if (e == cudaSuccess) e = upload_vec(&r->twM16, twiddle_table16());
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
-    // the SIMT engine computes the filter's 8192-point spectrum, so the plan
-    // also carries that twiddle table
-    p.logTab = 13;
-    if (e == cudaSuccess) {
-        std::vector<float2> tw(kM);
-        for (int64_t i = 0; i < kM; ++i) {
-            const std::complex<double> z = wpow(i, kM, -1);
-            tw[i] = make_float2((float)z.real(), (float)z.imag());
-        }
-        e = cudaMalloc((void**)&p.tw, tw.size() * sizeof(float2));
-        if (e == cudaSuccess) e = cudaMemcpy(p.tw, tw.data(), tw.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && r->mode == kModeSplit) {
+        e = upload_vec(&r->tw16k, twiddle_table(2 * kM, kM));
+        if (e == cudaSuccess) e = cudaMalloc((void**)&r->scratch, (size_t)r->num_sms * 4 * kM * sizeof(uint32_t));
     }
-    if (e == cudaSuccess) {
-        const void* kernels[4] = {(const void*)tc_fftconv_n4096_kernel<__nv_bfloat16, false>,
-                                  (const void*)tc_fftconv_n4096_kernel<__nv_bfloat16, true>,
-                                  (const void*)tc_fftconv_n4096_kernel<__half, false>,
-                                  (const void*)tc_fftconv_n4096_kernel<__half, true>};
-        for (int i = 0; i < 4 && e == cudaSuccess; ++i)
-            e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    }
+    // the SIMT engine computes the filter spectrum (8192 points, or 16384 in
+    // the split mode), so the plan also carries that twiddle table
+    const int64_t mf = r->mode == kModeSplit ? 2 * kM : kM;
+    p.logTab = r->mode == kModeSplit ? 14 : 13;
+    if (e == cudaSuccess) e = upload_vec(&p.tw, twiddle_table((int)mf, (int)mf));
+    if (e == cudaSuccess) e = set_smem_attributes<kModePlain>();
+    if (e == cudaSuccess) e = set_smem_attributes<kModeWindows>();
+    if (e == cudaSuccess) e = set_smem_attributes<kModeSplit>();
     return e;
 }
 
@@ -884,17 +1080,25 @@ void tc_plan_free(Plan& p) {
     if (!r) return;
     cudaFree(r->bimg);
     cudaFree(r->tw1024);
-    cudaFree(r->twM);
+    cudaFree(r->twM16);
+    cudaFree(r->tw16k);
+    cudaFree(r->scratch);
     delete r;
     p.tc = nullptr;
 }
 
-// K_f: [H] rows of 8192 complex fp16 (scaled so the largest component is 1),
-// then [H] fp32 scales.
-size_t tc_filter_bytes(const Plan& p) { return (size_t)p.H * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15)); }
+static int64_t tc_filter_rows(const Plan& p) { return tc_mode(p.N, p.L) == kModeSplit ? 2 * p.H : p.H; }
+
+// K_f: rows of 8192 complex fp16 (scaled so each channel's largest component
+// is 1; the split mode has two rows per channel, even and odd bins), then [H]
+// fp32 scales.
+size_t tc_filter_bytes(const Plan& p) {
+    return (size_t)tc_filter_rows(p) * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
+}
 
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
-    return simt_precompute_to_tc_layout(p, k, Kf, s);
+    return tc_mode(p.N, p.L) == kModeSplit ? simt_precompute_to_tc_split(p, k, Kf, s)
+                                           : simt_precompute_to_tc_layout(p, k, Kf, s);
 }
 
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
@@ -902,25 +1106,29 @@ cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     TcArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.Kh16 = (const __half2*)fa.Kf;
-    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)tc_filter_rows(p) * kKBytes);
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H;
     a.N = p.N;
-    a.nwin = tc_windows(p.N);
+    a.nwin = r->mode == kModeWindows ? tc_windows(p.N) : 1;
     a.pb = (fa.B + 1) / 2;
     a.tpc = (a.pb + 3) / 4;
-    a.nunits = p.H * a.nwin * a.tpc;
+    const int64_t groups = p.H * a.nwin * a.tpc;       // CTA-sized work items
+    a.nunits = r->mode == kModeSplit ? 2 * groups : groups;
     a.bimg = (const uint4*)r->bimg;
     a.tw1024 = r->tw1024;
-    a.twM = r->twM;
+    a.twM16 = r->twM16;
+    a.tw16k = r->tw16k;
+    a.scratch = r->scratch;
+    for (int j = 0; j < 8; ++j) {
+        const std::complex<double> z = wpow(j, 2 * kM, -1);
+        a.w16k_j3[j] = make_float2((float)z.real(), (float)z.imag());
+    }
     a.status = p.status;
-    const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
-    if (p.dtype == kBF16)
-        a.nwin > 1 ? tc_fftconv_n4096_kernel<__nv_bfloat16, true><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a)
-                   : tc_fftconv_n4096_kernel<__nv_bfloat16, false><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
-    else
-        a.nwin > 1 ? tc_fftconv_n4096_kernel<__half, true><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a)
-                   : tc_fftconv_n4096_kernel<__half, false><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a);
+    const int64_t grid = groups < r->num_sms ? groups : r->num_sms;
+    if (r->mode == kModeSplit) launch_mode<kModeSplit>(p, a, grid, s);
+    else if (r->mode == kModeWindows) launch_mode<kModeWindows>(p, a, grid, s);
+    else launch_mode<kModePlain>(p, a, grid, s);
     return cudaGetLastError();
 }
 
@@ -952,11 +1160,13 @@ cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cud
 }
 
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
-    const int64_t total = p.H * (kN + 1);
+    const int split = tc_mode(p.N, p.L) == kModeSplit ? 1 : 0;
+    const int64_t total = p.H * (p.N + 1);
     int blocks = (int)((total + 255) / 256);
     if (blocks > 65535) blocks = 65535;
     tc_export_kernel<<<blocks, 256, 0, s>>>((const __half2*)Kf,
-                                            (const float*)((const uint8_t*)Kf + (size_t)p.H * kKBytes), out, p.H);
+                                            (const float*)((const uint8_t*)Kf + (size_t)tc_filter_rows(p) * kKBytes),
+                                            out, p.H, split);
     return cudaGetLastError();
 }
 

@@ -234,14 +234,16 @@ def test_overlap_save_windows(dtype, N, L, B):
 def test_overlap_save_limits():
     import long_sequence_fft_b200 as lsf
     import torch
-    # one tap too many for the windows: the SIMT path serves it
-    assert lsf.Plan(8192, 2, "bf16", L=2050).path_name != "tc_fused"
-    plan = lsf.Plan(8192, 2, "bf16", L=2048)
+    # one tap too many for the windows: at N = 8192 the parity split serves
+    # it, longer sequences go to the SIMT path
+    assert lsf.Plan(8192, 2, "bf16", L=2050).path_name == "tc_fused"
+    assert lsf.Plan(16384, 2, "bf16", L=2050).path_name != "tc_fused"
+    plan = lsf.Plan(16384, 2, "bf16", L=2048)
     assert plan.path_name == "tc_fused"
     k = torch.zeros((2, 2048), dtype=torch.bfloat16, device="cuda")
     Kf = plan.precompute(k)
-    u = torch.zeros((2, 2, 8192), dtype=torch.bfloat16, device="cuda")
-    mask = torch.ones((1, 8192 // 32), dtype=torch.uint8, device="cuda")
+    u = torch.zeros((2, 2, 16384), dtype=torch.bfloat16, device="cuda")
+    mask = torch.ones((1, 16384 // 32), dtype=torch.uint8, device="cuda")
     with pytest.raises(lsf.FFTConvError) as e:
         plan.forward(u, Kf, mask=mask)
     assert e.value.status == lsf.ERR_UNSUPPORTED
@@ -271,3 +273,31 @@ def test_forward_host_pipelined_chunks_match_device_path():
         plan.forward_host(uh, Kf, yh, staging, w_host=wh, v_host=vh, mask_host=mh)
         torch.cuda.synchronize()
         assert torch.equal(yh, yd.cpu())
+
+
+# ---------------------------------------------- N = 8192 parity split ---
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("B,L,gated,mask_frac", [(3, 8192, True, 0.0), (2, 8192, False, 0.75), (1, 5000, True, 0.5),
+                                                 (5, 2050, True, 0.0), (4, 8192, True, 0.3)])
+def test_split_n8192_full_filters(dtype, B, L, gated, mask_frac):
+    """N = 8192 with filters longer than the windows allow: the 16384-point
+    spectrum split by bin parity, masks included."""
+    inp = _rand_inputs(B, 3, 8192, L, dtype, gated=gated, mask_frac=mask_frac, seed=B * 7 + L)
+    y, plan = run_cuda(inp, dtype, order=0)
+    assert plan.path_name == "tc_fused"
+    assert_close(y, _oracle(inp), dtype, f"split {dtype} B={B} L={L} mask={mask_frac}")
+
+
+def test_split_n8192_export_and_shared_mask():
+    import long_sequence_fft_b200 as lsf
+    k = W.round_to(RNG.standard_normal((3, 8192), dtype=np.float32) / 90.0, "bf16")
+    plan = lsf.Plan(8192, 3, "bf16")
+    Kf = plan.precompute(to_dev(k, "bf16"))
+    got = plan.export_rfft(Kf).cpu().numpy().astype(np.complex128)
+    ref = oracle.filter_rfft(k, 8192)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-3
+    inp = _rand_inputs(3, 3, 8192, 8192, "bf16", gated=True, mask_frac=0.75, seed=21)
+    inp["mask"] = inp["mask"][:1]
+    y, _ = run_cuda(inp, "bf16")
+    assert_close(y, _oracle(inp), "bf16", "split, one mask row for all channels")
