@@ -46,6 +46,7 @@
 #include <cmath>
 #include <complex>
 #include <cstring>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
@@ -707,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
                         for (int c3 = 0; c3 < 8; ++c3) {
                             const int f8 = lane + 32 * c2 + 1024 * c3;
-                            const int f = LY::kFull ? 2 * f8 + (P.odd ? 1 : 0) : f8;   // bin of the full spectrum
+                            const int f = LY::kFull ? 2 * f8 + (int)(unit & 1) : f8;   // bin of the full spectrum
                             int blk = (f <= kSeqN ? f : kSeqM - f) >> 5;
                             blk = blk < (int)nblk ? blk : (int)nblk - 1;
                             if (__ldg(&mrow[blk]) == 0) kw[c3] = 0u;
@@ -780,87 +781,102 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // In a window after the first, positions t < 2048 (j1 < 8: warps
             // with s < 2) are not outputs; their gate loads still read inside
             // the sequence and are discarded.
-            const bool emit = P.valid && !(P.tail_only && s < 2) && (!LY::kFull || P.odd);
-            const bool park = LY::kFull && P.valid && !P.odd;
-            uint4* slot = LY::kFull ? a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4) : nullptr;
+            // (the split parity is re-derived from the unit where it is used:
+            // a flag kept across the stages costs a register they need)
+            const bool odd = LY::kFull && (unit & 1);
+            // One output pass per tile, specialised for parking z_even (split
+            // mode, even tile) or writing y: a single loop doing either keeps
+            // both paths' state live and spills.
+            auto output_pass = [&](auto park_tag) {
+                constexpr bool PARK = decltype(park_tag)::value;
+                const bool emit = !PARK && P.valid && !(P.tail_only && s < 2);
+                const bool park = PARK && P.valid;
 #pragma unroll 1
-            for (int hp = 0; hp < (LY::Chunks - 40) / 2 && ok; ++hp) {
-                const int c = 40 + 2 * hp;
-                const int jb = 16 * (hp >> 1) + 4 * s;       // this warp's first j1
-                const int tb = 8 * lane + 4 * (hp & 1);
-                // output gate values, requested before the accumulator wait so
-                // that their latency overlaps it (an empty pair reads row 0 of
-                // the channel and discards it)
-                uint2 va[4], vb[4];
-                if (!LY::kFull || P.odd) {
-                    const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+                for (int hp = 0; hp < (LY::Chunks - 40) / 2 && ok; ++hp) {
+                    const int c = 40 + 2 * hp;
+                    const int jb = 16 * (hp >> 1) + 4 * s;       // this warp's first j1
+                    const int tb = 8 * lane + 4 * (hp & 1);
+                    // output gate values, requested before the accumulator wait so
+                    // that their latency overlaps it (an empty pair reads row 0 of
+                    // the channel and discards it)
+                    uint2 va[4], vb[4];
+                    if (!PARK) {
+                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int64_t t0 = 256 * (jb + jj) + tb;
-                        va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
-                        vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
-                    }
-                }
-                if (!(ok = begin_pair(c))) break;
-                uint32_t r[2][2][8];
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                    for (int jl = 0; jl < 2; ++jl) tmem_ld8(dcol(c + cc) + jl * 32 + 8 * s, r[cc][jl]);
-                tc_wait_ld();
-                release(c);
-                if (park) {
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        // j3 = 4 (hp%2) + 2 cc + jl, in t order
-                        slot[(256 * (jb + jj) + tb) >> 2] =
-                            make_uint4(pack_h2(__uint_as_float(r[0][0][2 * jj]), __uint_as_float(r[0][0][2 * jj + 1])),
-                                       pack_h2(__uint_as_float(r[0][1][2 * jj]), __uint_as_float(r[0][1][2 * jj + 1])),
-                                       pack_h2(__uint_as_float(r[1][0][2 * jj]), __uint_as_float(r[1][0][2 * jj + 1])),
-                                       pack_h2(__uint_as_float(r[1][1][2 * jj]), __uint_as_float(r[1][1][2 * jj + 1])));
-                    }
-                }
-                if (emit) {
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int64_t t0 = 256 * (jb + jj) + tb;
-                        const uint32_t vaw[2] = {va[jj].x, va[jj].y};
-                        const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
-                        uint4 zev = make_uint4(0, 0, 0, 0);
-                        float2 w0 = make_float2(1.f, 0.f);
-                        if constexpr (LY::kFull) {
-                            zev = slot[t0 >> 2];
-                            w0 = __ldg(&a.tw16k[t0]);
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int64_t t0 = 256 * (jb + jj) + tb;
+                            va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
+                            vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
                         }
-                        const uint32_t zw[4] = {zev.x, zev.y, zev.z, zev.w};
-                        uint32_t oa[2], ob[2];
+                    }
+                    if (!(ok = begin_pair(c))) break;
+                    uint32_t r[2][2][8];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            // j3 = 4 (hp%2) + 2e + (0, 1): chunk cc = e, jl = 0, 1
-                            float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
-                            float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
-                            float sc = kscale;
+                    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                        for (int jl = 0; jl < 2; ++jl) tmem_ld8(dcol(c + cc) + jl * 32 + 8 * s, r[cc][jl]);
+                    tc_wait_ld();
+                    release(c);
+                    if (park) {
+                        uint4* slot = a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4);
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            // j3 = 4 (hp%2) + 2 cc + jl, in t order
+                            slot[(256 * (jb + jj) + tb) >> 2] =
+                                make_uint4(pack_h2(__uint_as_float(r[0][0][2 * jj]), __uint_as_float(r[0][0][2 * jj + 1])),
+                                           pack_h2(__uint_as_float(r[0][1][2 * jj]), __uint_as_float(r[0][1][2 * jj + 1])),
+                                           pack_h2(__uint_as_float(r[1][0][2 * jj]), __uint_as_float(r[1][0][2 * jj + 1])),
+                                           pack_h2(__uint_as_float(r[1][1][2 * jj]), __uint_as_float(r[1][1][2 * jj + 1])));
+                        }
+                    }
+                    if (emit) {
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int64_t t0 = 256 * (jb + jj) + tb;
+                            const uint32_t vaw[2] = {va[jj].x, va[jj].y};
+                            const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
+                            uint4 zev = make_uint4(0, 0, 0, 0);
+                            float2 w0 = make_float2(1.f, 0.f);
                             if constexpr (LY::kFull) {
-                                // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
-                                const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
-                                const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
-                                const float2 ze0 = __half22float2(u2h(zw[2 * e])), ze1 = __half22float2(u2h(zw[2 * e + 1]));
-                                a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
-                                a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
-                                sc *= 0.5f;
+                                zev = a.scratch[((int64_t)blockIdx.x * 4 + q) * (kM / 4) + (t0 >> 2)];
+                                w0 = __ldg(&a.tw16k[t0]);
                             }
-                            a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
-                            if (a.v) {
-                                const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
-                                a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
+                            const uint32_t zw[4] = {zev.x, zev.y, zev.z, zev.w};
+                            uint32_t oa[2], ob[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                // j3 = 4 (hp%2) + 2e + (0, 1): chunk cc = e, jl = 0, 1
+                                float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
+                                float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
+                                float sc = kscale;
+                                if constexpr (LY::kFull) {
+                                    // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
+                                    const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
+                                    const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
+                                    const float2 ze0 = __half22float2(u2h(zw[2 * e])), ze1 = __half22float2(u2h(zw[2 * e + 1]));
+                                    a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
+                                    a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
+                                    sc *= 0.5f;
+                                }
+                                a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
+                                if (a.v) {
+                                    const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
+                                    a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
+                                }
+                                oa[e] = IO<T>::pack2(a0, a1);
+                                ob[e] = IO<T>::pack2(b0, b1);
                             }
-                            oa[e] = IO<T>::pack2(a0, a1);
-                            ob[e] = IO<T>::pack2(b0, b1);
+                            *(uint2*)((T*)a.y + P.o0 + t0) = make_uint2(oa[0], oa[1]);
+                            if (has1) *(uint2*)((T*)a.y + P.o1 + t0) = make_uint2(ob[0], ob[1]);
                         }
-                        *(uint2*)((T*)a.y + P.o0 + t0) = make_uint2(oa[0], oa[1]);
-                        if (has1) *(uint2*)((T*)a.y + P.o1 + t0) = make_uint2(ob[0], ob[1]);
                     }
                 }
+            };
+            if constexpr (LY::kFull) {
+                if (odd) output_pass(std::false_type{});
+                else output_pass(std::true_type{});
+            } else {
+                output_pass(std::false_type{});
             }
         }
     }
