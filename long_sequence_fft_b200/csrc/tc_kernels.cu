@@ -771,18 +771,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
             // EO: lane = l; chunk 40 + k holds j3 = 2(k%4) + jl (jl = 0, 1) for
             // j1 in [16 (k/4), 16 (k/4) + 16) at columns jl*32 + 2*(j1 % 16).
-            // Output pair hp (chunks 40 + 2hp, 41 + 2hp) covers j3 in
-            // [4 (hp%2), 4 (hp%2) + 4) of that j1 half; this warp takes
-            // j1 = 16 (hp/2) + 4s + jj and the four consecutive
-            // t = 256 j1 + 8 l + 4 (hp%2) + (0..3) of each row.  Plain and window
-            // modes: y = s_h v z, one 8-byte store per row.  Split mode: the
-            // even tile parks z in the CTA's scratch slot (16 bytes per four t),
-            // the odd tile writes y = s_h v (z_even + w16384^-t z_odd) / 2.
-            // In a window after the first, positions t < 2048 (j1 < 8: warps
-            // with s < 2) are not outputs; their gate loads still read inside
-            // the sequence and are discarded.
-            // (the split parity is re-derived from the unit where it is used:
-            // a flag kept across the stages costs a register they need)
+            // The four chunks of quad Q (40 + 4Q .. 43 + 4Q) hold all eight j3
+            // of that j1 half, so a thread gets the eight consecutive
+            // t = 256 j1 + 8 l + j3 of each row: one 16-byte store (512
+            // contiguous bytes per warp store).  This warp takes
+            // j1 = 16Q + 4s + 2 hf + jj in two halves hf (two j1 each, the
+            // register budget of one pass).  Plain and window modes:
+            // y = s_h v z.  Split mode: the even tile parks z in the CTA's
+            // scratch slot, the odd tile writes y = s_h v (z_even + w16384^-t
+            // z_odd) / 2.  In a window after the first, positions t < 2048
+            // (j1 < 8: warps with s < 2) are not outputs; their gate loads still
+            // read inside the sequence and are discarded.
+            // (The split parity is re-derived from the unit where it is used:
+            // a flag kept across the stages costs a register they need.)
             const bool odd = LY::kFull && (unit & 1);
             // One output pass per tile, specialised for parking z_even (split
             // mode, even tile) or writing y: a single loop doing either keeps
@@ -792,82 +793,92 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const bool emit = !PARK && P.valid && !(P.tail_only && s < 2);
                 const bool park = PARK && P.valid;
 #pragma unroll 1
-                for (int hp = 0; hp < (LY::Chunks - 40) / 2 && ok; ++hp) {
-                    const int c = 40 + 2 * hp;
-                    const int jb = 16 * (hp >> 1) + 4 * s;       // this warp's first j1
-                    const int tb = 8 * lane + 4 * (hp & 1);
-                    // output gate values, requested before the accumulator wait so
-                    // that their latency overlaps it (an empty pair reads row 0 of
-                    // the channel and discards it)
-                    uint2 va[4], vb[4];
-                    if (!PARK) {
-                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+                for (int Q = 0; Q < (LY::Chunks - 40) / 4 && ok; ++Q) {
+                    const int c0 = 40 + 4 * Q;
+#pragma unroll 1
+                    for (int hf = 0; hf < 2 && ok; ++hf) {
+                        const int jb = 16 * Q + 4 * s + 2 * hf;      // this pass's first j1
+                        // output gate values, requested before the accumulator
+                        // wait so that their latency overlaps it (an empty pair
+                        // reads row 0 of the channel and discards it)
+                        uint4 va[2], vb[2];
+                        if (!PARK) {
+                            const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const int64_t t0 = 256 * (jb + jj) + tb;
-                            va[jj] = __ldg((const uint2*)(vr + P.o0 + t0));
-                            vb[jj] = __ldg((const uint2*)(vr + (has1 ? P.o1 : P.o0) + t0));
-                        }
-                    }
-                    if (!(ok = begin_pair(c))) break;
-                    uint32_t r[2][2][8];
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                        for (int jl = 0; jl < 2; ++jl) tmem_ld8(dcol(c + cc) + jl * 32 + 8 * s, r[cc][jl]);
-                    tc_wait_ld();
-                    release(c);
-                    if (park) {
-                        uint4* slot = a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4);
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            // j3 = 4 (hp%2) + 2 cc + jl, in t order
-                            slot[(256 * (jb + jj) + tb) >> 2] =
-                                make_uint4(pack_h2(__uint_as_float(r[0][0][2 * jj]), __uint_as_float(r[0][0][2 * jj + 1])),
-                                           pack_h2(__uint_as_float(r[0][1][2 * jj]), __uint_as_float(r[0][1][2 * jj + 1])),
-                                           pack_h2(__uint_as_float(r[1][0][2 * jj]), __uint_as_float(r[1][0][2 * jj + 1])),
-                                           pack_h2(__uint_as_float(r[1][1][2 * jj]), __uint_as_float(r[1][1][2 * jj + 1])));
-                        }
-                    }
-                    if (emit) {
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const int64_t t0 = 256 * (jb + jj) + tb;
-                            const uint32_t vaw[2] = {va[jj].x, va[jj].y};
-                            const uint32_t vbw[2] = {vb[jj].x, vb[jj].y};
-                            uint4 zev = make_uint4(0, 0, 0, 0);
-                            float2 w0 = make_float2(1.f, 0.f);
-                            if constexpr (LY::kFull) {
-                                zev = a.scratch[((int64_t)blockIdx.x * 4 + q) * (kM / 4) + (t0 >> 2)];
-                                w0 = __ldg(&a.tw16k[t0]);
+                            for (int jj = 0; jj < 2; ++jj) {
+                                const int64_t t0 = 256 * (jb + jj) + 8 * lane;
+                                va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
+                                vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
                             }
-                            const uint32_t zw[4] = {zev.x, zev.y, zev.z, zev.w};
-                            uint32_t oa[2], ob[2];
+                        }
+                        if (hf == 0 && (!(ok = begin_pair(c0)) || !(ok = begin_pair(c0 + 2)))) break;
+                        // r[cc][jl][2 jj + (re, im)]: chunk c0 + cc, j3 = 2 cc + jl, j1 = jb + jj
+                        uint32_t r[4][2][4];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                // j3 = 4 (hp%2) + 2e + (0, 1): chunk cc = e, jl = 0, 1
-                                float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
-                                float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
-                                float sc = kscale;
+                        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                            for (int jl = 0; jl < 2; ++jl)
+                                tmem_ld4(dcol(c0 + cc) + jl * 32 + 8 * s + 4 * hf, r[cc][jl]);
+                        tc_wait_ld();
+                        if (hf == 1) {
+                            release(c0);
+                            release(c0 + 2);
+                        }
+                        if (park) {
+                            uint4* slot = a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4);
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                uint32_t hz[8];
+#pragma unroll
+                                for (int j3 = 0; j3 < 8; ++j3)
+                                    hz[j3] = pack_h2(__uint_as_float(r[j3 >> 1][j3 & 1][2 * jj]),
+                                                     __uint_as_float(r[j3 >> 1][j3 & 1][2 * jj + 1]));
+                                const int64_t t0 = 256 * (jb + jj) + 8 * lane;
+                                slot[t0 >> 2] = make_uint4(hz[0], hz[1], hz[2], hz[3]);
+                                slot[(t0 >> 2) + 1] = make_uint4(hz[4], hz[5], hz[6], hz[7]);
+                            }
+                        }
+                        if (emit) {
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                const int64_t t0 = 256 * (jb + jj) + 8 * lane;
+                                const uint32_t vaw[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
+                                const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
+                                float2 w0 = make_float2(1.f, 0.f);
+                                [[maybe_unused]] const uint4* zslot = nullptr;   // z_even of these t (split, odd tile)
                                 if constexpr (LY::kFull) {
-                                    // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
-                                    const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
-                                    const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
-                                    const float2 ze0 = __half22float2(u2h(zw[2 * e])), ze1 = __half22float2(u2h(zw[2 * e + 1]));
-                                    a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
-                                    a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
-                                    sc *= 0.5f;
+                                    zslot = a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4) + (t0 >> 2);
+                                    w0 = __ldg(&a.tw16k[t0]);
                                 }
-                                a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
-                                if (a.v) {
-                                    const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
-                                    a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
+                                uint32_t oa[4], ob[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    // j3 = 2e (chunk c0 + e, jl 0) and 2e + 1 (jl 1)
+                                    float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
+                                    float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
+                                    float sc = kscale;
+                                    if constexpr (LY::kFull) {
+                                        // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
+                                        const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
+                                        const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
+                                        // z_even of t0 + 2e (+1), loaded where used
+                                        const uint2 zp = reinterpret_cast<const uint2*>(zslot)[e];
+                                        const float2 ze0 = __half22float2(u2h(zp.x)), ze1 = __half22float2(u2h(zp.y));
+                                        a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
+                                        a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
+                                        sc *= 0.5f;
+                                    }
+                                    a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
+                                    if (a.v) {
+                                        const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
+                                        a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
+                                    }
+                                    oa[e] = IO<T>::pack2(a0, a1);
+                                    ob[e] = IO<T>::pack2(b0, b1);
                                 }
-                                oa[e] = IO<T>::pack2(a0, a1);
-                                ob[e] = IO<T>::pack2(b0, b1);
+                                *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                                if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
                             }
-                            *(uint2*)((T*)a.y + P.o0 + t0) = make_uint2(oa[0], oa[1]);
-                            if (has1) *(uint2*)((T*)a.y + P.o1 + t0) = make_uint2(ob[0], ob[1]);
                         }
                     }
                 }
