@@ -517,82 +517,89 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i) tw[i] = tw16(__ldg(&a.tw1024[((8 * s + i) * lane) & 1023]));
 
+        // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [J s, J s + J)
+        // with J = kJ1 / 4 (split mode: times w16384^t in the odd tile), into
+        // the TMEM A1 columns; then arrive on bar_in.  Loads are issued in
+        // batches before any use (absent rows or gates read a present row and
+        // are masked afterwards).  A tile's input is loaded while the previous
+        // tile's last stage runs (the A columns are free once S3' is done), so
+        // its first MMAs can start as soon as the accumulator ring drains.
+        auto load_tile = [&](int64_t lu) {
+            const PairInfo LP = pair_info<MODE>(a, lu, q);
+            const bool hasL = LP.o1 >= 0;
+            const int64_t oo1 = hasL ? LP.o1 : LP.o0;
+            const T* pu0 = (const T*)a.u + LP.o0;
+            const T* pw0 = a.w ? (const T*)a.w + LP.o0 : pu0;
+            const T* pu1 = (const T*)a.u + oo1;
+            const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
+            const bool has_w = a.w != nullptr;
+            const bool keep0 = LP.valid, keep1 = hasL;
+            constexpr int J = LY::kJ1 / 4;
+#pragma unroll
+            for (int jp = 0; jp < J / 2; ++jp) {
+                uint4 ld[2][4];
+#pragma unroll
+                for (int jh = 0; jh < 2; ++jh) {
+                    const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
+                    ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
+                    ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
+                    ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
+                    ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+                }
+                uint32_t pk[8][2];
+#pragma unroll
+                for (int jh = 0; jh < 2; ++jh) {
+                    float2 w0 = make_float2(1.f, 0.f);     // w16384^t0 (odd split tile)
+                    if constexpr (LY::kFull) {
+                        if (LP.odd) w0 = __ldg(&a.tw16k[256 * (J * s + 2 * jp + jh) + 8 * lane]);
+                    }
+                    const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
+                    const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
+                    const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
+                    const uint32_t wb[4] = {ld[jh][3].x, ld[jh][3].y, ld[jh][3].z, ld[jh][3].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float2 xa = IO<T>::unpack2(ua[e]), xb = IO<T>::unpack2(ub[e]);
+                        if (has_w) {
+                            const float2 g0 = IO<T>::unpack2(wa[e]), g1 = IO<T>::unpack2(wb[e]);
+                            xa.x *= g0.x; xa.y *= g0.y; xb.x *= g1.x; xb.y *= g1.y;
+                        }
+                        if (!keep0) xa = make_float2(0.f, 0.f);
+                        if (!keep1) xb = make_float2(0.f, 0.f);
+                        if constexpr (LY::kFull) {
+                            if (LP.odd) {
+                                // (a + i b)[t] times w16384^t, t = t0 + 2e (+1)
+                                const float2 wa0 = cmul(w0, a.w16k_j3[2 * e]), wa1 = cmul(w0, a.w16k_j3[2 * e + 1]);
+                                const float2 z0 = cmul(make_float2(xa.x, xb.x), wa0);
+                                const float2 z1 = cmul(make_float2(xa.y, xb.y), wa1);
+                                xa = make_float2(z0.x, z1.x);
+                                xb = make_float2(z0.y, z1.y);
+                            }
+                        }
+                        pk[2 * e][jh] = pack_h2(xa.x, xb.x);
+                        pk[2 * e + 1][jh] = pack_h2(xa.y, xb.y);
+                    }
+                }
+#pragma unroll
+                for (int j3 = 0; j3 < 8; ++j3)
+                    tmem_st2(tbase + lq + j3 * LY::kJ1 + J * s + 2 * jp, pk[j3][0], pk[j3][1]);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_in);
+        };
+
         int iter = 0;
         bool ok = true;
+        if (first_unit<MODE>() < a.nunits) load_tile(first_unit<MODE>());
         for (int64_t unit = first_unit<MODE>(); unit < a.nunits && ok; unit = next_unit<MODE>(unit), ++iter) {
             const int64_t hch = unit_channel<MODE>(a, unit);
 
-            // ---- load: x = u*w for t = 256*j1 + 8*l + j3, j1 in [J s, J s + J)
-            // with J = kJ1 / 4 (split mode: times w16384^t in the odd tile).
-            // Loads are issued in batches before any use (absent rows or gates
-            // read a present row and are masked afterwards).  Row offsets are
-            // formed here and again for the output stage instead of being
-            // kept, which keeps registers for the stages.
+            // (this tile's input was loaded before the loop or during the
+            // previous tile's last stage: see load_tile)
             const PairInfo P = pair_info<MODE>(a, unit, q);
             const bool has1 = P.o1 >= 0;
-            {
-                const int64_t oo1 = has1 ? P.o1 : P.o0;
-                const T* pu0 = (const T*)a.u + P.o0;
-                const T* pw0 = a.w ? (const T*)a.w + P.o0 : pu0;
-                const T* pu1 = (const T*)a.u + oo1;
-                const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
-                const bool has_w = a.w != nullptr;
-                const bool keep0 = P.valid, keep1 = has1;
-                constexpr int J = LY::kJ1 / 4;
-#pragma unroll
-                for (int jp = 0; jp < J / 2; ++jp) {
-                    uint4 ld[2][4];
-#pragma unroll
-                    for (int jh = 0; jh < 2; ++jh) {
-                        const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
-                        ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
-                        ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
-                        ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
-                        ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
-                    }
-                    uint32_t pk[8][2];
-#pragma unroll
-                    for (int jh = 0; jh < 2; ++jh) {
-                        float2 w0 = make_float2(1.f, 0.f);     // w16384^t0 (odd split tile)
-                        if constexpr (LY::kFull) {
-                            if (P.odd) w0 = __ldg(&a.tw16k[256 * (J * s + 2 * jp + jh) + 8 * lane]);
-                        }
-                        const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
-                        const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
-                        const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
-                        const uint32_t wb[4] = {ld[jh][3].x, ld[jh][3].y, ld[jh][3].z, ld[jh][3].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float2 xa = IO<T>::unpack2(ua[e]), xb = IO<T>::unpack2(ub[e]);
-                            if (has_w) {
-                                const float2 g0 = IO<T>::unpack2(wa[e]), g1 = IO<T>::unpack2(wb[e]);
-                                xa.x *= g0.x; xa.y *= g0.y; xb.x *= g1.x; xb.y *= g1.y;
-                            }
-                            if (!keep0) xa = make_float2(0.f, 0.f);
-                            if (!keep1) xb = make_float2(0.f, 0.f);
-                            if constexpr (LY::kFull) {
-                                if (P.odd) {
-                                    // (a + i b)[t] times w16384^t, t = t0 + 2e (+1)
-                                    const float2 wa0 = cmul(w0, a.w16k_j3[2 * e]), wa1 = cmul(w0, a.w16k_j3[2 * e + 1]);
-                                    const float2 z0 = cmul(make_float2(xa.x, xb.x), wa0);
-                                    const float2 z1 = cmul(make_float2(xa.y, xb.y), wa1);
-                                    xa = make_float2(z0.x, z1.x);
-                                    xb = make_float2(z0.y, z1.y);
-                                }
-                            }
-                            pk[2 * e][jh] = pack_h2(xa.x, xb.x);
-                            pk[2 * e + 1][jh] = pack_h2(xa.y, xb.y);
-                        }
-                    }
-#pragma unroll
-                    for (int j3 = 0; j3 < 8; ++j3)
-                        tmem_st2(tbase + lq + j3 * LY::kJ1 + J * s + 2 * jp, pk[j3][0], pk[j3][1]);
-                }
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_in);
-            }
 
             const __half2* Ks = (const __half2*)(smem + LY::OffK);
             // loaded once per tile and pinned in a register (an opaque move
@@ -769,6 +776,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             if (ok) stage_done(2);
 #pragma unroll
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
+            {
+                const int64_t nu = next_unit<MODE>(unit);
+                if (ok && nu < a.nunits) load_tile(nu);
+            }
             // EO: lane = l; chunk 40 + k holds j3 = 2(k%4) + jl (jl = 0, 1) for
             // j1 in [16 (k/4), 16 (k/4) + 16) at columns jl*32 + 2*(j1 % 16).
             // The four chunks of quad Q (40 + 4Q .. 43 + 4Q) hold all eight j3
