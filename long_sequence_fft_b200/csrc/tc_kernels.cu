@@ -524,7 +524,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         // are masked afterwards).  A tile's input is loaded while the previous
         // tile's last stage runs (the A columns are free once S3' is done), so
         // its first MMAs can start as soon as the accumulator ring drains.
-        auto load_tile = [&](int64_t lu) {
+        // part 0 loads the first half of the j1 batches, part 1 the second
+        // half and then signals bar_in; the two halves fill the waits before
+        // S2' and before S1' of the previous tile.
+        auto load_tile = [&](int64_t lu, int part) {
             const PairInfo LP = pair_info<MODE>(a, lu, q);
             const bool hasL = LP.o1 >= 0;
             const int64_t oo1 = hasL ? LP.o1 : LP.o0;
@@ -535,8 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             const bool has_w = a.w != nullptr;
             const bool keep0 = LP.valid, keep1 = hasL;
             constexpr int J = LY::kJ1 / 4;
+            constexpr int kHalf = J / 4;      // batches of two j1 per part
 #pragma unroll
-            for (int jp = 0; jp < J / 2; ++jp) {
+            for (int jq = 0; jq < kHalf; ++jq) {
+                const int jp = part * kHalf + jq;
                 uint4 ld[2][4];
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
@@ -584,15 +589,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 for (int j3 = 0; j3 < 8; ++j3)
                     tmem_st2(tbase + lq + j3 * LY::kJ1 + J * s + 2 * jp, pk[j3][0], pk[j3][1]);
             }
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_in);
+            if (part == 1) {
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_in);
+            }
         };
 
         int iter = 0;
         bool ok = true;
-        if (first_unit<MODE>() < a.nunits) load_tile(first_unit<MODE>());
+        if (first_unit<MODE>() < a.nunits) {
+            load_tile(first_unit<MODE>(), 0);
+            load_tile(first_unit<MODE>(), 1);
+        }
         for (int64_t unit = first_unit<MODE>(); unit < a.nunits && ok; unit = next_unit<MODE>(unit), ++iter) {
             const int64_t hch = unit_channel<MODE>(a, unit);
 
@@ -765,6 +775,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 fence_proxy_async_smem();
             }
             if (ok) stage_done(1);
+            {
+                // first half of the next tile's input (the A columns are free
+                // now that S3' is done)
+                const int64_t nu = next_unit<MODE>(unit);
+                if (ok && nu < a.nunits) load_tile(nu, 0);
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
 #pragma unroll 1
@@ -778,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             for (int i = 0; i < 8; ++i) tw[i] = tw16_conj(tw[i]);
             {
                 const int64_t nu = next_unit<MODE>(unit);
-                if (ok && nu < a.nunits) load_tile(nu);
+                if (ok && nu < a.nunits) load_tile(nu, 1);
             }
             // EO: lane = l; chunk 40 + k holds j3 = 2(k%4) + jl (jl = 0, 1) for
             // j1 in [16 (k/4), 16 (k/4) + 16) at columns jl*32 + 2*(j1 % 16).
