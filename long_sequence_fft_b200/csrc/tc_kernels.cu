@@ -7,15 +7,23 @@
 // cores, permutations become on-chip transposes, and the whole convolution
 // (gates included, "Key results") is one kernel.
 //
-// This kernel: sequence length N = 4096, transform length M = 8192.
-//   t = 256*j1 + 8*l + j3   (j1 < 32, zero for j1 >= 16;  l < 32;  j3 < 8)
+// The transform engine: 8192-point transforms of 4-pair tiles.
+//   t = 256*j1 + 8*l + j3   (j1 < 32, l < 32, j3 < 8)
 //   f = c1 + 32*c2 + 1024*c3
-//   exp(-2 pi i f t / M) = w32^(c1 j1) w1024^(c1 l) wM^(c1 j3) w32^(c2 l) w256^(c2 j3) w8^(c3 j3)
-// Forward: S1 contracts j1 (DFT-32 on 16 nonzero inputs), twiddle w1024^(c1 l),
-// S2 contracts l (DFT-32), twiddle wM^(c1 j3), S3 contracts j3 with the
-// per-c2 factor w8^(c3 j3) w256^(c2 j3) (the second twiddle folded into the
-// matrix).  Product with the filter spectrum, then the mirror image with
-// conjugate factors; the last inverse stage emits only t < N.
+//   exp(-2 pi i f t / 8192) = w32^(c1 j1) w1024^(c1 l) w8192^(c1 j3) w32^(c2 l) w256^(c2 j3) w8^(c3 j3)
+// Forward: S1 contracts j1 (DFT-32), twiddle w1024^(c1 l), S2 contracts l
+// (DFT-32), twiddle w8192^(c1 j3), S3 contracts j3 with the per-c2 factor
+// w8^(c3 j3) w256^(c2 j3) (the second twiddle folded into the matrix).
+// Product with the filter spectrum, then the mirror image with conjugate
+// factors (S3', S2', S1').
+//
+// Three modes use it (see Lay and pair_info):
+//   plain    N = 4096: x zero for t >= 4096 (S1 sees 16 nonzero j1), S1' emits
+//            only t < 4096;
+//   windows  N > 4096 with filters of at most 2049 taps: overlap-save windows
+//            of 4096 inputs, hop 2048;
+//   split    N = 8192 with longer filters: the 16384-point spectrum split by
+//            bin parity into two 8192-point transforms of all 8192 inputs.
 //
 // Data layout.  One CTA tile = 4 pairs of batch rows (the two real sequences
 // of a pair are the real and imaginary parts of one complex sequence; the
@@ -28,18 +36,22 @@
 // contract the lane digit (S2, S2') and the last inverse stage take A from
 // shared memory, written by the previous epilogue in the transposed order
 // (the "on-chip transpose").  Accumulators are fp32 in TMEM.  The epilogue
-// warps round them to fp16 and apply the twiddles in packed half precision
-// (the rounding the next stage's operands take anyway, plus one product
-// rounding); the filter product is taken in fp32 before rounding.  Each
-// DFT factor carries 1/sqrt(n), so the forward and inverse transforms are
-// unitary and the filter spectrum is used unnormalised.
+// warps round them to fp16 and apply the twiddles and the filter product
+// (K / s_h, |K / s_h| <= 1) in packed half precision; the channel scale s_h
+// is applied to y in fp32.  Each DFT factor carries 1/sqrt(n), so the forward
+// and inverse transforms are unitary and the filter spectrum is used
+// unnormalised.
 //
 // Warp roles: warps 0..15 are epilogue warps (warp w serves lane quarter
-// w % 4 and the column slice w / 4), warp 16 issues the MMAs.  Accumulators
-// are double-buffered (two 128-column TMEM buffers); mbarriers hand chunks
-// between the MMA warp and the epilogue warps.  Every wait is bounded: on
-// timeout the kernel records FFTCONV_ERR_TIMEOUT in the plan's status word,
-// drains, frees its TMEM and returns.
+// w % 4 and the column slice w / 4); warps 16..19 issue the MMAs, one per SM
+// sub-partition.  A tile's work is a sequence of 64-column accumulator
+// chunks (44, or 48 in the split mode) cycled through a ring of four TMEM
+// buffers; mbarriers hand chunks between the MMA warps and the epilogue
+// warps, and the epilogue hands a buffer back as soon as its TMEM loads have
+// landed.  The next tile's input is loaded while the current tile's last
+// stages run.  Every wait is bounded: on timeout the kernel records
+// FFTCONV_ERR_TIMEOUT in the plan's status word, drains, frees its TMEM and
+// returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -380,8 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         // ============================ MMA issuers ===========================
         // A single thread can issue a tcgen05.mma only every ~100 cycles, far
         // slower than the tensor core retires these small MMAs, so four warps
-        // issue: issuer i handles the chunks g = i (mod 4), which all use
-        // accumulator buffer i (44 chunks per tile keeps the assignment fixed).
+        // issue: issuer i handles the chunks c = i (mod 4) of every tile, which
+        // all use ring buffer i.
         const int issuer = warp - kEpiWarps;
         const uint32_t id64 = idesc_f16_f32(128, 64);
         const uint32_t id16 = idesc_f16_f32(128, 16);
@@ -622,8 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // both are waited for and loaded before one TMEM-load wait, and
             // the fences and barrier arrivals are shared.  Each stage has its
             // own loop, so the stage, the ring slots (chunk c of a tile uses
-            // buffer c % 4; 44 chunks per tile) and the store patterns are
-            // fixed at compile time.
+            // buffer c % 4) and the store patterns are fixed at compile time.
             auto begin_pair = [&](int c) -> bool {
                 // use number (Chunks/4)*iter + c/4 of the buffer
                 const uint32_t par = (uint32_t)(iter * (LY::Chunks / 4) + (c >> 2)) & 1u;
