@@ -32,6 +32,7 @@ struct PairRows {
     const T* v0 = nullptr; const T* v1 = nullptr;
     T* y0 = nullptr; T* y1 = nullptr;
     int nvalid = 0;   // inputs at t >= nvalid read as zero (filter length)
+    bool vec4 = false;  // rows aligned for 4-element vector accesses (load4 / store4)
 
     __device__ __forceinline__ float2 load(int t) const {
         if (t >= nvalid) return make_float2(0.f, 0.f);
@@ -43,6 +44,56 @@ struct PairRows {
             if (w1) b *= to_f32(w1[t]);
         }
         return make_float2(a, b);
+    }
+    // Four consecutive positions t .. t+3 (t a multiple of 4) with one vector
+    // access per row where the rows allow it; positions at or past nvalid
+    // read as zero.
+    __device__ __forceinline__ void load4(int t, float2 (&x)[4]) const {
+        if (vec4 && t + 4 <= nvalid) {
+            float a[4], b[4] = {0.f, 0.f, 0.f, 0.f}, g[4];
+            ld4(u0 + t, a);
+            if (w0) { ld4(w0 + t, g); for (int e = 0; e < 4; ++e) a[e] *= g[e]; }
+            if (u1) {
+                ld4(u1 + t, b);
+                if (w1) { ld4(w1 + t, g); for (int e = 0; e < 4; ++e) b[e] *= g[e]; }
+            }
+            for (int e = 0; e < 4; ++e) x[e] = make_float2(a[e], b[e]);
+        } else {
+            for (int e = 0; e < 4; ++e) x[e] = load(t + e);
+        }
+    }
+    __device__ __forceinline__ void store4(int t, const float2 (&z)[4]) const {
+        if (!vec4) {
+            for (int e = 0; e < 4; ++e) store(t + e, z[e]);
+            return;
+        }
+        float a[4], b[4], g[4];
+        for (int e = 0; e < 4; ++e) { a[e] = z[e].x; b[e] = z[e].y; }
+        if (v0) { ld4(v0 + t, g); for (int e = 0; e < 4; ++e) a[e] *= g[e]; }
+        st4(y0 + t, a);
+        if (y1) {
+            if (v1) { ld4(v1 + t, g); for (int e = 0; e < 4; ++e) b[e] *= g[e]; }
+            st4(y1 + t, b);
+        }
+    }
+    static __device__ __forceinline__ void ld4(const T* p, float (&o)[4]) {
+        if constexpr (sizeof(T) == 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(p));
+            o[0] = q.x; o[1] = q.y; o[2] = q.z; o[3] = q.w;
+        } else {
+            const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+            const T* h = reinterpret_cast<const T*>(&q);
+            for (int e = 0; e < 4; ++e) o[e] = to_f32(h[e]);
+        }
+    }
+    static __device__ __forceinline__ void st4(T* p, const float (&v)[4]) {
+        if constexpr (sizeof(T) == 4) {
+            *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+            T h[4];
+            for (int e = 0; e < 4; ++e) h[e] = from_f32<T>(v[e]);
+            *reinterpret_cast<uint2*>(p) = *reinterpret_cast<const uint2*>(h);
+        }
     }
     __device__ __forceinline__ void store(int t, float2 z) const {
         float a = z.x, b = z.y;
@@ -73,6 +124,7 @@ __device__ __forceinline__ PairRows<T> pair_rows(const ForwardArgs& a, int64_t H
     r.y0 = (T*)a.y + o0;
     r.y1 = has1 ? (T*)a.y + o1 : nullptr;
     r.nvalid = (int)N;
+    r.vec4 = (N % 4) == 0;      // rows start at multiples of N; buffers are 16-byte aligned
     *h_out = (int)h;
     return r;
 }
@@ -376,10 +428,16 @@ staged_col_fwd_kernel(StagedArgs A) {
     const int64_t col0 = (int64_t)blockIdx.x * TC;
     int h;
     const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
-    for (int idx = tid; idx < R * TC; idx += kColThreads) {
-        const int j = idx / TC, col = idx % TC;
-        s[sidx<TC>(j, col)] = (j < R / 2) ? io.load((int)(j * C + col0 + col)) : make_float2(0.f, 0.f);
+    // the nonzero half (j < R/2), four consecutive columns per thread
+    for (int idx = tid; idx < (R / 2) * (TC / 4); idx += kColThreads) {
+        const int j = idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
+        float2 x[4];
+        io.load4((int)(j * C + col0 + c4), x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[sidx<TC>(j, c4 + e)] = x[e];
     }
+    for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads)
+        s[sidx<TC>(R / 2 + idx / TC, idx % TC)] = make_float2(0.f, 0.f);
     __syncthreads();
     fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
     float2* W = A.work + pl * (R * C);
@@ -451,9 +509,12 @@ staged_col_inv_kernel(StagedArgs A) {
     }
     __syncthreads();
     inv_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
-    for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads) {
-        const int j = idx / TC, col = idx % TC;
-        io.store((int)(j * C + col0 + col), s[sidx<TC>(j, col)]);
+    for (int idx = tid; idx < (R / 2) * (TC / 4); idx += kColThreads) {
+        const int j = idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
+        float2 z[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) z[e] = s[sidx<TC>(j, c4 + e)];
+        io.store4((int)(j * C + col0 + c4), z);
     }
 }
 
