@@ -70,13 +70,16 @@ typedef enum {
 typedef enum {
     FFTCONV_PATH_SIMT_FUSED = 1,    /* fp32 FFT in shared memory, one kernel  */
     FFTCONV_PATH_SIMT_STAGED = 2,   /* fp32, column/row passes via workspace  */
-    FFTCONV_PATH_TC_FUSED = 3       /* tcgen05 tensor-core Monarch, one kernel */
+    FFTCONV_PATH_TC_FUSED = 3,      /* tcgen05 tensor-core Monarch, one kernel */
+    FFTCONV_PATH_TC_STAGED = 4      /* staged, tensor-core row pass of 8192    */
 } fftconv_path_t;
 
 /* Create a plan for sequences of length N (a power of two, 256 <= N <= 2^22)
  * and H channels with full-length filters (L = N).  `order` selects the
  * decomposition: 0 = automatic; 2 or 3 = fused on-chip kernel (N <= 8192);
- * 4 = the staged path with one workspace round trip (any N); other values are
+ * 4 = the staged path with one workspace round trip (any N); 5 = the staged
+ * path whose row pass runs on the tensor cores (fp16/bf16, 16384 <= N <= 2^21,
+ * L > 2049; order 0 chooses it for those plans); other values are
  * FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
  * (a few hundred KB) and its workspace (staged path only) on the current
  * device.  *out receives the plan, or NULL on failure. */

@@ -30,8 +30,9 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 F32, F16, BF16 = 0, 1, 2
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_OOM, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
-PATH_SIMT_FUSED, PATH_SIMT_STAGED, PATH_TC_FUSED = 1, 2, 3
-PATH_NAMES = {PATH_SIMT_FUSED: "simt_fused", PATH_SIMT_STAGED: "simt_staged", PATH_TC_FUSED: "tc_fused"}
+PATH_SIMT_FUSED, PATH_SIMT_STAGED, PATH_TC_FUSED, PATH_TC_STAGED = 1, 2, 3, 4
+PATH_NAMES = {PATH_SIMT_FUSED: "simt_fused", PATH_SIMT_STAGED: "simt_staged", PATH_TC_FUSED: "tc_fused",
+              PATH_TC_STAGED: "tc_staged"}
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -116,7 +117,9 @@ class Plan:
 
     order: 0 automatic, 1 fp32 shared-memory FFT in one kernel (N <= 8192),
     2/3 fused on-chip kernel (tensor cores where available), 4 staged passes
-    through a workspace (any N).  L < N gives the partial convolution."""
+    through a workspace (any N), 5 staged passes with the row pass on the
+    tensor cores (fp16/bf16, 16384 <= N <= 2^21, L > 2049).  L < N gives the
+    partial convolution."""
 
     def __init__(self, N: int, H: int, dtype="bf16", order: int = 0, L: Optional[int] = None):
         self.N, self.H = int(N), int(H)

@@ -133,7 +133,7 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
     if ((N & (N - 1)) != 0) return fail(FFTCONV_ERR_UNSUPPORTED, "N=%lld is not a power of two", (long long)N);
     if (N < 256 || N > (int64_t(1) << 22))
         return fail(FFTCONV_ERR_UNSUPPORTED, "N=%lld outside [256, 2^22]", (long long)N);
-    if (order < 0 || order > 4) return fail(FFTCONV_ERR_UNSUPPORTED, "order %d not in {0,1,2,3,4}", order);
+    if (order < 0 || order > 5) return fail(FFTCONV_ERR_UNSUPPORTED, "order %d not in {0,1,2,3,4,5}", order);
     if (H > (int64_t(1) << 24)) return fail(FFTCONV_ERR_UNSUPPORTED, "H=%lld too large", (long long)H);
 
     Plan* p = new (std::nothrow) Plan();
@@ -143,7 +143,18 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
     cudaGetDevice(&p->device);
 
     const bool tc_ok = tc_supported(N, L, (int)dtype);
-    if (order == 4 || (order == 0 && !tc_ok && !simt_fused_supported(p->logM))) {
+    const bool tc_staged_ok = tc_staged_supported(N, L, (int)dtype);
+    if (order == 5) {
+        if (!tc_staged_ok) {
+            delete p;
+            return fail(FFTCONV_ERR_UNSUPPORTED,
+                        "order 5 needs fp16/bf16, 16384 <= N <= 2^21 and L > 2049 (N=%lld, L=%lld)",
+                        (long long)N, (long long)L);
+        }
+        p->path = kPathTcStaged;
+    } else if (order == 0 && !tc_ok && tc_staged_ok) {
+        p->path = kPathTcStaged;
+    } else if (order == 4 || (order == 0 && !tc_ok && !simt_fused_supported(p->logM))) {
         p->path = kPathSimtStaged;
     } else if (order == 1) {
         if (!simt_fused_supported(p->logM)) { delete p; return fail(FFTCONV_ERR_UNSUPPORTED, "order 1 needs N <= 8192"); }
@@ -166,8 +177,9 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         p->logTab = p->logM;
         e = upload(&p->tw, host_twiddles(p->M, p->M, 1));
         p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
-    } else if (p->path == kPathSimtStaged) {
-        p->logC = staged_log_cols(p->logM);
+    } else if (p->path == kPathSimtStaged || p->path == kPathTcStaged) {
+        // (the tensor-core row pass takes rows of 8192)
+        p->logC = p->path == kPathTcStaged ? kTcRowLogC : staged_log_cols(p->logM);
         p->logR = p->logM - p->logC;
         p->logTab = p->logC;
         const int64_t C = int64_t(1) << p->logC;
@@ -183,6 +195,10 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         p->workBytes = per_pair * (size_t)p->chunkPairs;
         if (e == cudaSuccess) e = cudaMalloc((void**)&p->work, p->workBytes);
         p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
+        if (p->path == kPathTcStaged) {
+            if (e == cudaSuccess) e = tc_rows_init(*p);
+            p->filter_bytes = tc_staged_filter_bytes(*p);
+        }
     } else {
         e = tc_plan_init(*p);
         p->filter_bytes = tc_filter_bytes(*p);
@@ -235,6 +251,7 @@ int fftconv_filter_precompute(fftconv_plan_t plan, const void* k, void* K_f, fft
     switch (p.path) {
         case kPathSimtFused: e = simt_fused_precompute(p, k, K_f, s); break;
         case kPathSimtStaged: e = simt_staged_precompute(p, k, K_f, s); break;
+        case kPathTcStaged: e = tc_staged_precompute(p, k, K_f, s); break;
         default: e = tc_precompute(p, k, K_f, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "filter precompute launch");
@@ -280,6 +297,7 @@ static int run_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s) {
     switch (p.path) {
         case kPathSimtFused: e = simt_fused_forward(p, a, s); break;
         case kPathSimtStaged: e = simt_staged_forward(p, a, s); break;
+        case kPathTcStaged: e = tc_staged_forward(p, a, s); break;
         default: e = tc_forward(p, a, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
@@ -418,8 +436,9 @@ int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fft
     if (p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "this overlap-save plan stores the 8192-point spectrum of k, not the 2N-point one");
-    cudaError_t e = (p.path == kPathTcFused) ? tc_export_rfft(p, K_f, out, (cudaStream_t)stream)
-                                             : simt_export_rfft(p, K_f, out, (cudaStream_t)stream);
+    cudaError_t e = p.path == kPathTcFused    ? tc_export_rfft(p, K_f, out, (cudaStream_t)stream)
+                    : p.path == kPathTcStaged ? tc_rows_export(p, K_f, out, (cudaStream_t)stream)
+                                              : simt_export_rfft(p, K_f, out, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "export launch");
     return FFTCONV_OK;
 }

@@ -8,7 +8,7 @@
 
 namespace fftconv {
 
-enum Path : int { kPathSimtFused = 1, kPathSimtStaged = 2, kPathTcFused = 3 };
+enum Path : int { kPathSimtFused = 1, kPathSimtStaged = 2, kPathTcFused = 3, kPathTcStaged = 4 };
 enum DType : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
 
 // Staged path factorization M = R * C (log2 of C for log2(M) = logM): rows
@@ -95,5 +95,18 @@ cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s);
 cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s);
+
+// staged path with the tensor-core row pass (rows of C = 8192): the column
+// passes are the SIMT ones (simt_kernels.cu), the row pass and the filter
+// layout are the tensor-core kernel's (tc_kernels.cu)
+constexpr int kTcRowLogC = 13;
+bool tc_staged_supported(int64_t N, int64_t L, int dtype);
+size_t tc_staged_filter_bytes(const Plan& p);
+cudaError_t tc_rows_init(Plan& p);
+cudaError_t tc_rows_forward(const Plan& p, const ForwardArgs& fa, int64_t pair0, int64_t npairs, cudaStream_t s);
+cudaError_t tc_rows_convert(const Plan& p, int64_t h0, int64_t nch, void* Kf, cudaStream_t s);
+cudaError_t tc_rows_export(const Plan& p, const void* Kf, float* out, cudaStream_t s);
+cudaError_t tc_staged_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
+cudaError_t tc_staged_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 
 }  // namespace fftconv

@@ -380,8 +380,12 @@ cudaError_t launch_fused_pre(const Plan& p, const void* k, void* Kf, cudaStream_
 
 // ------------------------------------------------------ staged kernels ---
 
-constexpr int kColTile = 32;    // columns per CTA in the column passes
 constexpr int kColThreads = 256;
+// columns per CTA in the column passes: 32, or more for short columns so that
+// a CTA holds at least 2048 values (R = 8: 256 columns, one radix-8 DFT per
+// thread); at most 256, which divides every staged C (C >= 256)
+template <int LOGR>
+constexpr int col_tile() { return (2048 >> LOGR) > 256 ? 256 : ((2048 >> LOGR) < 32 ? 32 : (2048 >> LOGR)); }
 
 template <int LOGC>
 constexpr int row_threads() { return (1 << LOGC) / 32 < 128 ? 128 : ((1 << LOGC) / 32 > 512 ? 512 : (1 << LOGC) / 32); }
@@ -400,6 +404,7 @@ struct StagedArgs {
     // precompute mode: input k [H, L] instead of u/w; pair == channel
     const void* k;
     int64_t L;
+    int64_t kf_pair0;       // precompute mode: channel of the first K_f row written
 };
 
 template <typename T>
@@ -420,7 +425,7 @@ template <int LOGR, typename T>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_fwd_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
-    constexpr int TC = kColTile;
+    constexpr int TC = col_tile<LOGR>();
     extern __shared__ float2 s[];
     const int tid = threadIdx.x;
     const int64_t C = (int64_t)1 << A.logC;
@@ -480,7 +485,7 @@ staged_row_kernel(StagedArgs A) {
     } else {
         fwd_stages<LOGC, 0, K, 1, NT>(s, A.tw, 0, tid);
         const float inv = 1.0f / (float)A.M;
-        const int64_t h = A.pair0 + pl;
+        const int64_t h = A.pair0 + pl - A.kf_pair0;
         float2* out = (float2*)A.fa.y + (h * R + c) * C;   // fa.y carries K_f here
         for (int i = tid; i < C; i += NT) out[i] = cscale(s[sidx<1>(i, 0)], inv);
     }
@@ -492,7 +497,7 @@ template <int LOGR, typename T>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_inv_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
-    constexpr int TC = kColTile;
+    constexpr int TC = col_tile<LOGR>();
     extern __shared__ float2 s[];
     const int tid = threadIdx.x;
     const int64_t C = (int64_t)1 << A.logC;
@@ -520,8 +525,8 @@ staged_col_inv_kernel(StagedArgs A) {
 
 template <int LOGR, typename T>
 cudaError_t launch_cols(const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
-    const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * kColTile;
-    dim3 grid((unsigned)(C / kColTile), (unsigned)A.npairs);
+    const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * col_tile<LOGR>();
+    dim3 grid((unsigned)(C / col_tile<LOGR>()), (unsigned)A.npairs);
     if (!inverse) {
         auto kern = staged_col_fwd_kernel<LOGR, T>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -601,6 +606,55 @@ cudaError_t staged_forward_t(const Plan& p, const ForwardArgs& fa, const void* k
             e = cols_dispatch<T>(p.logR, A, C, true, st);
             if (e != cudaSuccess) return e;
         }
+    }
+    return cudaSuccess;
+}
+
+// Staged path with the tensor-core row pass: per chunk of pairs the forward
+// column pass, the tensor-core kernel over the chunk's rows (forward 8192-point
+// transform, filter product, inverse, in place) and the inverse column pass.
+template <typename T>
+cudaError_t tc_staged_forward_t(const Plan& p, const ForwardArgs& fa, cudaStream_t st) {
+    StagedArgs A{};
+    A.fa = fa;
+    A.H = p.H; A.N = p.N; A.M = p.M;
+    A.logC = p.logC;
+    A.work = p.work;
+    A.tw = p.tw; A.twLo = p.twLo; A.twHi = p.twHi; A.twSplit = p.twSplit;
+    const int64_t C = (int64_t)1 << p.logC;
+    const int64_t total = p.H * ((fa.B + 1) / 2);
+    for (int64_t first = 0; first < total; first += p.chunkPairs) {
+        A.pair0 = first;
+        A.npairs = total - first < p.chunkPairs ? total - first : p.chunkPairs;
+        cudaError_t e = cols_dispatch<T>(p.logR, A, C, false, st);
+        if (e == cudaSuccess) e = tc_rows_forward(p, fa, first, A.npairs, st);
+        if (e == cudaSuccess) e = cols_dispatch<T>(p.logR, A, C, true, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// Its filter precompute: the staged forward transform of k (column pass, then
+// the fp32 row pass scaled by 1/M) into the workspace, chunk by chunk, and the
+// conversion of each chunk's rows to the tensor-core layout.
+template <typename T>
+cudaError_t tc_staged_precompute_t(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    StagedArgs A{};
+    A.fa.y = p.work;        // the row pass writes the chunk's spectra in place
+    A.H = p.H; A.N = p.N; A.M = p.M;
+    A.logC = p.logC;
+    A.work = p.work;
+    A.tw = p.tw; A.twLo = p.twLo; A.twHi = p.twHi; A.twSplit = p.twSplit;
+    A.k = k; A.L = p.L;
+    const int64_t C = (int64_t)1 << p.logC, R = (int64_t)1 << p.logR;
+    for (int64_t first = 0; first < p.H; first += p.chunkPairs) {
+        A.pair0 = first;
+        A.kf_pair0 = first;
+        A.npairs = p.H - first < p.chunkPairs ? p.H - first : p.chunkPairs;
+        cudaError_t e = cols_dispatch<T>(p.logR, A, C, false, st);
+        if (e == cudaSuccess) e = rows_dispatch<1>(p.logC, A, R, st);
+        if (e == cudaSuccess) e = tc_rows_convert(p, first, A.npairs, Kf, st);
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
@@ -698,6 +752,22 @@ cudaError_t simt_staged_precompute(const Plan& p, const void* k, void* Kf, cudaS
     ForwardArgs fa{};
     fa.y = Kf;      // the row pass in precompute mode writes K_f through fa.y
     FFTCONV_DISPATCH_T(p.dtype, return staged_forward_t<T>(p, fa, k, st))
+}
+
+cudaError_t tc_staged_forward(const Plan& p, const ForwardArgs& a, cudaStream_t st) {
+    switch (p.dtype) {
+        case kF16: return tc_staged_forward_t<__half>(p, a, st);
+        case kBF16: return tc_staged_forward_t<__nv_bfloat16>(p, a, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t tc_staged_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    switch (p.dtype) {
+        case kF16: return tc_staged_precompute_t<__half>(p, k, Kf, st);
+        case kBF16: return tc_staged_precompute_t<__nv_bfloat16>(p, k, Kf, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t simt_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t st) {

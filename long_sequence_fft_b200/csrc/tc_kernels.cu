@@ -63,6 +63,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "simt_fft.cuh"   // perm_to_freq: the order of the staged row pass
 #include "tc_ptx.cuh"
 
 namespace fftconv {
@@ -88,7 +89,10 @@ constexpr int kDBuf = 4;             // accumulator ring: 4 buffers of 64 TMEM c
 // filters through the 16384-point spectrum split by bin parity (see
 // pair_info): the 8192-point transform then takes all 8192 inputs and returns
 // all 8192 outputs.
-constexpr int kModePlain = 0, kModeWindows = 1, kModeSplit = 2;
+// 3 (rows): the row pass of the staged path, M = R x 8192: full-length
+// 8192-point transforms of complex workspace rows, product with that row's
+// part of the spectrum, inverse, written back in place.
+constexpr int kModePlain = 0, kModeWindows = 1, kModeSplit = 2, kModeRows = 3;
 
 // chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
 __host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
@@ -117,7 +121,8 @@ constexpr int kTile = 16384;                 // 128 rows x 128 B, 128-byte swizz
 constexpr int kKBytes = kM * 4;              // one filter spectrum row, 8192 x half2
 template <int MODE>
 struct Lay {
-    static constexpr bool kFull = MODE == kModeSplit;   // all 8192 inputs and outputs
+    static constexpr bool kFull = MODE == kModeSplit || MODE == kModeRows;   // all 8192 inputs and outputs
+    static constexpr bool kSplit = MODE == kModeSplit;  // even/odd bin tiles
     static constexpr int kJ1 = kFull ? 32 : 16;         // nonzero inputs / kept outputs per j3
     static constexpr int OffData = 0;                   // 8 tiles (one per j3)
     static constexpr int OffBS1 = 8 * kTile;            // K=2*kJ1 N=64        4 / 8 KB
@@ -129,16 +134,19 @@ struct Lay {
     static constexpr int OffBEnd = OffBS1i + kJ1 * 256;
     static constexpr int BImageBytes = OffBEnd - OffBS1;
     static constexpr int OffK = OffBEnd;                // the tile's filter spectrum row
+    // (the rows mode has four filter rows per tile, read through L2)
+    static constexpr bool kKShared = MODE != kModeRows;
     // the 256-entry w8192 twiddle table lives in shared memory except in the
     // split mode, whose larger factors leave no room (it is read through L1)
-    static constexpr bool kTwShared = !kFull;
-    static constexpr int OffTwM = OffK + kKBytes;
+    static constexpr bool kTwShared = !kSplit;
+    static constexpr int OffTwM = OffK + (kKShared ? kKBytes : 0);
     static constexpr int OffBars = OffTwM + (kTwShared ? 2048 : 0);   // 16 mbarrier slots
     static constexpr int OffMisc = OffBars + 128;       // tmem base, abort flag
     static constexpr int SmemBytes = OffMisc + 64 + 1024;              // + alignment slack
     static constexpr int Chunks = kFull ? 48 : 44;      // 8 per stage S1..S2', S1' 4 or 8
 };
 static_assert(Lay<kModeSplit>::SmemBytes <= 232448, "shared memory");
+static_assert(Lay<kModeRows>::SmemBytes <= 232448, "shared memory");
 static_assert(Lay<kModePlain>::SmemBytes <= 232448, "shared memory");
 
 // byte offset of element (n, k) of a K x N B operand in the no-swizzle
@@ -174,6 +182,10 @@ struct TcArgs {
     const float2* tw16k;       // split mode: exp(-2 pi i t/16384), t < 8192
     float2 w16k_j3[8];         // split mode: exp(-2 pi i j/16384), j < 8
     uint4* scratch;            // split mode: [CTAs][4 pairs][8192] half2, z_even of the group
+    float2* work;              // rows mode: the staged workspace [pairs][R][8192] complex fp32
+    int64_t R;                 // rows mode: rows per pair
+    int64_t pair0;             // rows mode: first pair of this chunk
+    float rin, rout;           // rows mode: input scale (keeps fp16 in range), output scale
     int* status;
 };
 
@@ -231,6 +243,7 @@ struct PairInfo {
     bool valid;
     bool tail_only;      // only window positions t >= kHop are outputs
     bool odd;            // split mode: the tile of odd spectrum bins
+    int64_t krow;        // rows mode: this quarter's filter row (channel * R + row)
 };
 
 // A tile holds 4 pairs of batch rows of ONE channel and one window: unit u
@@ -259,6 +272,20 @@ __device__ __forceinline__ PairInfo pair_info(const TcArgs& a, int64_t unit, int
         const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
         p.o0 = (b0 * a.H + p.h) * kN;
         p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + p.h) * kN : -1;
+        return p;
+    }
+    if constexpr (MODE == kModeRows) {
+        // Rows mode: unit u is pair u / (R/4) of the chunk and rows
+        // c = 4 (u % (R/4)) + q; o0 indexes the workspace row (complex).
+        const int64_t qpr = a.R / 4;
+        const int64_t pl = unit / qpr, c = 4 * (unit - pl * qpr) + q;
+        p.h = (a.pair0 + pl) / a.pb;
+        p.valid = true;
+        p.tail_only = false;
+        p.odd = false;
+        p.o0 = (pl * a.R + c) * (int64_t)kM;
+        p.o1 = -1;
+        p.krow = p.h * a.R + c;
         return p;
     }
     if constexpr (MODE == kModeSplit) {
@@ -311,6 +338,7 @@ __device__ __forceinline__ int64_t next_unit(int64_t u) {
 // even and the odd bins of each channel as two rows).
 template <int MODE>
 __device__ __forceinline__ int64_t unit_channel(const TcArgs& a, int64_t u) {
+    if constexpr (MODE == kModeRows) return (a.pair0 + u / (a.R / 4)) / a.pb;
     if constexpr (MODE == kModeWindows) return (int64_t)((uint32_t)u / ((uint32_t)a.nwin * (uint32_t)a.tpc));
     if constexpr (MODE == kModeSplit) return (u >> 1) / a.tpc;
     return u / a.tpc;
@@ -416,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         for (int64_t unit = first_unit<MODE>(); unit < a.nunits && ok; unit = next_unit<MODE>(unit), ++iter) {
             if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
             tc_fence_after();
-            if (issuer == 0) {
+            if (issuer == 0 && MODE != kModeRows) {      // (rows mode reads its filter rows through L2)
                 if (lane == 0) {
                     // the previous tile is finished with the filter buffer (its
                     // epilogue warps arrived on bar_in after all their reads)
@@ -478,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     const void* pf_src = nullptr;
                     uint32_t pf_bytes = (MODE == kModeSplit ? 2 * kN : kN) * sizeof(T);
                     const int64_t nu = next_unit<MODE>(unit);
-                    if (nu < a.nunits && (lane >> 3) == issuer) {
+                    if (MODE != kModeRows && nu < a.nunits && (lane >> 3) == issuer) {
                         const PairInfo Q = pair_info<MODE>(a, nu, issuer);
                         const int which = lane & 7;
                         if (Q.valid) {
@@ -519,8 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
         const int s = warp >> 2;         // column slice
         const uint32_t lq = (uint32_t)(32 * q) << 16;
         // the convolution's length and transform length (mask bins)
+        // (rows mode: the plan's N, M = R x 8192)
         constexpr int kSeqN = LY::kFull ? 2 * kN : kN, kSeqM = 2 * kSeqN;
-        const int64_t nblk = kSeqN / 32;
+        const int64_t nblk = (MODE == kModeRows ? a.N : kSeqN) / 32;
 
         // w1024^(c1 l) with (c1, l) = (8s + i, lane) in E1 and (lane, 8s + i)
         // in E2' -- the same eight values, kept in registers; wM^(c1 j3) with
@@ -554,6 +583,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
             for (int jq = 0; jq < kHalf; ++jq) {
                 const int jp = part * kHalf + jq;
+                uint32_t pk[8][2];
+                if constexpr (MODE == kModeRows) {
+                    // complex fp32 workspace row: eight consecutive t per j1
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const float4* src = reinterpret_cast<const float4*>(
+                            a.work + LP.o0 + 256 * (J * s + 2 * jp + jh) + 8 * lane);
+                        float4 f[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) f[i] = __ldg(src + i);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            pk[2 * i][jh] = pack_h2(f[i].x * a.rin, f[i].y * a.rin);
+                            pk[2 * i + 1][jh] = pack_h2(f[i].z * a.rin, f[i].w * a.rin);
+                        }
+                    }
+                } else {
                 uint4 ld[2][4];
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
@@ -563,11 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
                     ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
                 }
-                uint32_t pk[8][2];
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
                     float2 w0 = make_float2(1.f, 0.f);     // w16384^t0 (odd split tile)
-                    if constexpr (LY::kFull) {
+                    if constexpr (LY::kSplit) {
                         if (LP.odd) w0 = __ldg(&a.tw16k[256 * (J * s + 2 * jp + jh) + 8 * lane]);
                     }
                     const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
@@ -583,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         }
                         if (!keep0) xa = make_float2(0.f, 0.f);
                         if (!keep1) xb = make_float2(0.f, 0.f);
-                        if constexpr (LY::kFull) {
+                        if constexpr (LY::kSplit) {
                             if (LP.odd) {
                                 // (a + i b)[t] times w16384^t, t = t0 + 2e (+1)
                                 const float2 wa0 = cmul(w0, a.w16k_j3[2 * e]), wa1 = cmul(w0, a.w16k_j3[2 * e + 1]);
@@ -596,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         pk[2 * e][jh] = pack_h2(xa.x, xb.x);
                         pk[2 * e + 1][jh] = pack_h2(xa.y, xb.y);
                     }
+                }
                 }
 #pragma unroll
                 for (int j3 = 0; j3 < 8; ++j3)
@@ -626,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             const __half2* Ks = (const __half2*)(smem + LY::OffK);
             // loaded once per tile and pinned in a register (an opaque move
             // keeps the compiler from re-issuing the global load at each use)
-            float kscale = __ldg(&a.Kscale[hch]);
+            float kscale = __ldg(&a.Kscale[MODE == kModeRows ? P.krow : hch]);
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : hch) * nblk : nullptr;
 
@@ -714,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // inverse stages see values no larger than the forward output);
             // the channel scale is applied to y in fp32.  A4 (TMEM) cols
             // c2*8 + c3 (in place)
-            if (ok && !(ok = wait(bar_k, iter & 1))) fail();
+            if (MODE != kModeRows && ok && !(ok = wait(bar_k, iter & 1))) fail();
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 16 + k;
@@ -727,8 +773,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c2 = 4 * (k + cc) + s;
-                    const uint4 k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
-                    const uint4 k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
+                    uint4 k0, k1;
+                    if constexpr (MODE == kModeRows) {   // this quarter's row, through L2
+                        const __half2* Kq = a.Kh16 + P.krow * (int64_t)kM;
+                        k0 = __ldg((const uint4*)(Kq + k16_index(lane, c2, 0)));
+                        k1 = __ldg((const uint4*)(Kq + k16_index(lane, c2, 4)));
+                    } else {
+                        k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
+                        k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
+                    }
                     uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
                     if (mrow) {
                         // frequency-sparse filter: zero the masked bins (f and
@@ -736,8 +789,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
                         for (int c3 = 0; c3 < 8; ++c3) {
                             const int f8 = lane + 32 * c2 + 1024 * c3;
-                            const int f = LY::kFull ? 2 * f8 + (int)(unit & 1) : f8;   // bin of the full spectrum
-                            int blk = (f <= kSeqN ? f : kSeqM - f) >> 5;
+                            int blk;
+                            if constexpr (MODE == kModeRows) {
+                                // bin c + R f8 of the 2N-point spectrum, c = this
+                                // row (krow mod R, R a power of two; 2N <= 2^22)
+                                const int f = (int)((uint32_t)P.krow & (uint32_t)(a.R - 1)) + (int)a.R * f8;
+                                blk = (f <= (int)a.N ? f : 2 * (int)a.N - f) >> 5;
+                            } else {
+                                const int f = LY::kSplit ? 2 * f8 + (int)(unit & 1) : f8;   // bin of the full spectrum
+                                blk = (f <= kSeqN ? f : kSeqM - f) >> 5;
+                            }
                             blk = blk < (int)nblk ? blk : (int)nblk - 1;
                             if (__ldg(&mrow[blk]) == 0) kw[c3] = 0u;
                         }
@@ -822,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             // read inside the sequence and are discarded.
             // (The split parity is re-derived from the unit where it is used:
             // a flag kept across the stages costs a register they need.)
-            const bool odd = LY::kFull && (unit & 1);
+            const bool odd = LY::kSplit && (unit & 1);
             // One output pass per tile, specialised for parking z_even (split
             // mode, even tile) or writing y: a single loop doing either keeps
             // both paths' state live and spills.
@@ -840,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                         // wait so that their latency overlaps it (an empty pair
                         // reads row 0 of the channel and discards it)
                         uint4 va[2], vb[2];
-                        if (!PARK) {
+                        if (!PARK && MODE != kModeRows) {
                             const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
@@ -876,7 +937,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                 slot[(t0 >> 2) + 1] = make_uint4(hz[4], hz[5], hz[6], hz[7]);
                             }
                         }
-                        if (emit) {
+                        if (MODE == kModeRows && emit) {
+                            // z s_h back into the workspace row, times the output
+                            // scale: the filter rows hold rfft(k)/M (the column
+                            // passes expect the 1/M in the product), so it undoes
+                            // the unitary pair's 1/8192 and the input scale
+                            const float sc = kscale * a.rout;
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                float4* dst = reinterpret_cast<float4*>(a.work + P.o0 + 256 * (jb + jj) + 8 * lane);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    dst[e] = make_float4(__uint_as_float(r[e][0][2 * jj]) * sc,
+                                                         __uint_as_float(r[e][0][2 * jj + 1]) * sc,
+                                                         __uint_as_float(r[e][1][2 * jj]) * sc,
+                                                         __uint_as_float(r[e][1][2 * jj + 1]) * sc);
+                            }
+                        }
+                        if (MODE != kModeRows && emit) {
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
                                 const int64_t t0 = 256 * (jb + jj) + 8 * lane;
@@ -884,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                 const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
                                 float2 w0 = make_float2(1.f, 0.f);
                                 [[maybe_unused]] const uint4* zslot = nullptr;   // z_even of these t (split, odd tile)
-                                if constexpr (LY::kFull) {
+                                if constexpr (LY::kSplit) {
                                     zslot = a.scratch + ((int64_t)blockIdx.x * 4 + q) * (kM / 4) + (t0 >> 2);
                                     w0 = __ldg(&a.tw16k[t0]);
                                 }
@@ -895,7 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                     float a0 = __uint_as_float(r[e][0][2 * jj]), a1 = __uint_as_float(r[e][1][2 * jj]);
                                     float b0 = __uint_as_float(r[e][0][2 * jj + 1]), b1 = __uint_as_float(r[e][1][2 * jj + 1]);
                                     float sc = kscale;
-                                    if constexpr (LY::kFull) {
+                                    if constexpr (LY::kSplit) {
                                         // (z_even + conj(w16384^t) z_odd) / 2, t = t0 + 2e (+1)
                                         const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
                                         const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
@@ -921,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     }
                 }
             };
-            if constexpr (LY::kFull) {
+            if constexpr (LY::kSplit) {
                 if (odd) output_pass(std::false_type{});
                 else output_pass(std::true_type{});
             } else {
@@ -1221,6 +1299,126 @@ __global__ void bounded_wait_selftest_kernel(int* status, uint32_t polls, int ar
 
 cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s) {
     bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(p.status, polls, arrive);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------ staged row engine ---
+
+namespace {
+
+// workspace row (h0 + ch, c) of the staged forward transform of k (permuted
+// positions, rfft(k)/M) -> K_f row h * R + c in the tensor-core layout with
+// its own scale (one CTA per row)
+__global__ void tc_rows_convert_kernel(const float2* __restrict__ work, __half2* __restrict__ Kh,
+                                       float* __restrict__ scales, int64_t h0, int64_t R) {
+    constexpr int NT = 256;
+    __shared__ float red[NT / 32];
+    const int64_t row = blockIdx.x;                    // (ch, c) within the chunk
+    const int64_t ch = row / R, c = row - ch * R;
+    const float2* src = work + row * (int64_t)kM;
+    float m = 0.f;
+    for (int p = threadIdx.x; p < kM; p += NT) {
+        const float2 z = src[p];
+        m = fmaxf(m, fmaxf(fabsf(z.x), fabsf(z.y)));
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int i = 0; i < NT / 32; ++i) m = fmaxf(m, red[i]);
+    const float sc = m > 0.f ? m : 1.f, inv = 1.f / sc;
+    const int64_t krow = (h0 + ch) * R + c;
+    for (int p = threadIdx.x; p < kM; p += NT) {
+        const int k = (int)perm_to_freq(p, 13);       // the row transform's output order
+        const float2 z = src[p];
+        Kh[krow * kM + k16_index(k & 31, (k >> 5) & 31, k >> 10)] = __floats2half2_rn(z.x * inv, z.y * inv);
+    }
+    if (threadIdx.x == 0) scales[krow] = sc;
+}
+
+// K_f of a staged tensor-core plan -> rfft bins [0, N]: bin f is row c = f % R,
+// position k = f / R; the 1/M is undone
+__global__ void tc_rows_export_kernel(const __half2* __restrict__ Kh, const float* __restrict__ scales,
+                                      float* __restrict__ out, int64_t H, int64_t N, int64_t R) {
+    const int64_t nb = N + 1, total = H * nb;
+    const float m = (float)(2 * N);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t h = i / nb, f = i - h * nb;
+        const int64_t c = f % R, k = f / R, krow = h * R + c;
+        const float2 z = __half22float2(Kh[krow * kM + k16_index((int)(k & 31), (int)((k >> 5) & 31), (int)(k >> 10))]);
+        out[2 * i] = z.x * scales[krow] * m;
+        out[2 * i + 1] = z.y * scales[krow] * m;
+    }
+}
+
+}  // namespace
+
+bool tc_staged_supported(int64_t N, int64_t L, int dtype) {
+    return (dtype == kF16 || dtype == kBF16) && N >= 4 * kN && N <= (int64_t(1) << 21) && L > kHop + 1;
+}
+
+size_t tc_staged_filter_bytes(const Plan& p) {
+    const int64_t rows = p.H * (p.M / kM);
+    return (size_t)rows * kKBytes + (((size_t)rows * 4 + 15) & ~size_t(15));
+}
+
+cudaError_t tc_rows_init(Plan& p) {
+    TcResources* r = new TcResources();
+    p.tc = r;
+    r->mode = kModeRows;
+    const std::vector<uint8_t> img = build_bimage<kModeRows>();
+    cudaError_t e = cudaMalloc((void**)&r->bimg, img.size());
+    if (e == cudaSuccess) e = cudaMemcpy(r->bimg, img.data(), img.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddle_table(1024, 1024));
+    if (e == cudaSuccess) e = upload_vec(&r->twM16, twiddle_table16());
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
+    if (e == cudaSuccess) e = set_smem_attributes<kModeRows>();
+    return e;
+}
+
+cudaError_t tc_rows_forward(const Plan& p, const ForwardArgs& fa, int64_t pair0, int64_t npairs, cudaStream_t s) {
+    const TcResources* r = (const TcResources*)p.tc;
+    const int64_t R = p.M / kM;
+    TcArgs a{};
+    a.Kh16 = (const __half2*)fa.Kf;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)(p.H * R) * kKBytes);
+    a.mask = fa.mask; a.mask_h = fa.mask_h;
+    a.B = fa.B; a.H = p.H; a.N = p.N;
+    a.nwin = 1;
+    a.pb = (fa.B + 1) / 2;
+    a.tpc = 1;
+    a.work = p.work; a.R = R; a.pair0 = pair0;
+    // the column pass sums R/2 inputs per workspace value: scale by a power
+    // of two near 1/sqrt(R) (exact) so that the fp16 operands keep the
+    // inputs' range
+    int lr = 0;
+    while ((int64_t(1) << (lr + 1)) <= R) ++lr;
+    a.rin = std::ldexp(1.0f, -(lr / 2));
+    a.rout = std::ldexp((float)kM, lr / 2);
+    a.nunits = npairs * (R / 4);
+    a.bimg = (const uint4*)r->bimg;
+    a.tw1024 = r->tw1024;
+    a.twM16 = r->twM16;
+    a.status = p.status;
+    const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
+    launch_mode<kModeRows>(p, a, grid, s);
+    return cudaGetLastError();
+}
+
+cudaError_t tc_rows_convert(const Plan& p, int64_t h0, int64_t nch, void* Kf, cudaStream_t s) {
+    const int64_t R = p.M / kM;
+    tc_rows_convert_kernel<<<(unsigned)(nch * R), 256, 0, s>>>(
+        p.work, (__half2*)Kf, (float*)((uint8_t*)Kf + (size_t)(p.H * R) * kKBytes), h0, R);
+    return cudaGetLastError();
+}
+
+cudaError_t tc_rows_export(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
+    const int64_t R = p.M / kM, total = p.H * (p.N + 1);
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 65535) blocks = 65535;
+    tc_rows_export_kernel<<<blocks, 256, 0, s>>>((const __half2*)Kf,
+                                                 (const float*)((const uint8_t*)Kf + (size_t)(p.H * R) * kKBytes), out,
+                                                 p.H, p.N, R);
     return cudaGetLastError();
 }
 

@@ -52,6 +52,10 @@ def test_status_strings_and_null_handles():
     (1024, 0, 0, 0, 1024, -1),     # no channels
     (1024, 2, 7, 0, 1024, -1),     # unknown dtype
     (1024, 2, 0, 9, 1024, -2),     # unknown order
+    (1024, 2, 0, 6, 1024, -2),
+    (32768, 2, 0, 5, 32768, -2),   # tensor-core staged rows: fp16/bf16 only,
+    (8192, 2, 1, 5, 8192, -2),     # N >= 16384,
+    (32768, 2, 2, 5, 2049, -2),    # and filters longer than the windows take
     (1024, 2, 0, 0, 2048, -1),     # filter longer than the sequence
     (1024, 2, 0, 0, 0, -1),
 ])

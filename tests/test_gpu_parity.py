@@ -301,3 +301,57 @@ def test_split_n8192_export_and_shared_mask():
     inp["mask"] = inp["mask"][:1]
     y, _ = run_cuda(inp, "bf16")
     assert_close(y, _oracle(inp), "bf16", "split, one mask row for all channels")
+
+
+# ------------------------------------- staged path, tensor-core row pass ---
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("N,L,B,H,gated,mask_frac", [
+    (16384, 16384, 3, 2, True, 0.0),        # R = 4: one tile per pair, an unpaired row
+    (16384, 2050, 4, 3, False, 0.5),        # shortest filter the staged tiles take
+    (32768, 4096, 2, 3, True, 0.3),
+    (65536, 65536, 1, 2, True, 0.0),        # R = 16: four tiles per pair
+    (1 << 20, 1 << 20, 1, 5, False, 0.0),   # R = 256, 4 pairs per workspace chunk: 2 chunks
+])
+def test_tc_staged_rows(dtype, N, L, B, H, gated, mask_frac):
+    """Long sequences on the staged path whose row pass (rows of 8192) runs
+    on the tensor cores, against the oracle element by element."""
+    inp = _rand_inputs(B, H, N, L, dtype, gated=gated, mask_frac=mask_frac, seed=N // 1024 + L + B)
+    y, plan = run_cuda(inp, dtype, order=5)
+    assert plan.path_name == "tc_staged"
+    assert_close(y, _oracle(inp), dtype, f"tc_staged {dtype} N={N} L={L} B={B} H={H} mask={mask_frac}")
+
+
+def test_tc_staged_is_the_automatic_choice_and_exports():
+    import long_sequence_fft_b200 as lsf
+    k = W.round_to(RNG.standard_normal((3, 32768), dtype=np.float32) / 180.0, "f16")
+    plan = lsf.Plan(32768, 3, "f16")
+    assert plan.path_name == "tc_staged"
+    Kf = plan.precompute(to_dev(k, "f16"))
+    got = plan.export_rfft(Kf).cpu().numpy().astype(np.complex128)
+    ref = oracle.filter_rfft(k, 32768)
+    # fp16 spectrum rows, each with its own scale: half-precision storage bound
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-3
+    # the short-filter plan of the same length keeps the overlap-save windows
+    assert lsf.Plan(32768, 3, "f16", L=2049).path_name == "tc_fused"
+    # the SIMT staged path stays available as order 4
+    assert lsf.Plan(32768, 3, "f16", order=4).path_name == "simt_staged"
+
+
+def test_tc_staged_forward_host_chunks():
+    """The pipelined host-buffer call splits the batch into chunks; each
+    chunk's launches start at its own pair offset."""
+    import torch
+    import long_sequence_fft_b200 as lsf
+    B, H, N = 9, 2, 16384
+    inp = _rand_inputs(B, H, N, N, "bf16", gated=True, seed=99)
+    plan = lsf.Plan(N, H, "bf16", order=5)
+    Kf = plan.precompute(to_dev(inp["k"], "bf16"))
+    tdt = W.torch_dtype("bf16")
+    host = {n: torch.from_numpy(inp[n]).to(tdt).pin_memory() for n in ("u", "w", "v")}
+    y_host = torch.empty((B, H, N), dtype=tdt).pin_memory()
+    staging = torch.empty(plan.staging_bytes(B, True, True), dtype=torch.uint8, device="cuda")
+    plan.forward_host(host["u"], Kf, y_host, staging, w_host=host["w"], v_host=host["v"])
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    assert_close(y_host.float().numpy().astype(np.float64), _oracle(inp), "bf16", "tc_staged forward_host")
