@@ -188,10 +188,16 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         if (e == cudaSuccess) e = upload(&p->twLo, host_twiddles(p->M, int64_t(1) << p->twSplit, 1));
         if (e == cudaSuccess)
             e = upload(&p->twHi, host_twiddles(p->M, p->M >> p->twSplit, int64_t(1) << p->twSplit));
-        // workspace: a chunk of pairs of about 64 MB (L2-sized), at least one
-        const size_t per_pair = (size_t)p->M * sizeof(float2);
-        p->chunkPairs = (int64_t)((size_t(64) << 20) / per_pair);
-        if (p->chunkPairs < 1) p->chunkPairs = 1;
+        // workspace: the SIMT passes take a chunk of pairs of about 64 MB
+        // (L2-sized), at least one.  The tensor-core row pass keeps the
+        // workspace in fp16 and takes chunks of 512 MB (at least two pairs, so
+        // that the fp32 filter precompute fits one channel): its launches then
+        // run many tiles per SM, which measured faster on B200 than L2-sized
+        // chunks (N = 32768: 0.84 against 0.99 ms per call in fp32).
+        const bool ws16 = p->path == kPathTcStaged;
+        const size_t per_pair = (size_t)p->M * (ws16 ? 2 * sizeof(uint16_t) : sizeof(float2));
+        p->chunkPairs = (int64_t)((size_t(ws16 ? 512 : 64) << 20) / per_pair);
+        if (p->chunkPairs < (ws16 ? 2 : 1)) p->chunkPairs = ws16 ? 2 : 1;
         p->workBytes = per_pair * (size_t)p->chunkPairs;
         if (e == cudaSuccess) e = cudaMalloc((void**)&p->work, p->workBytes);
         p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);

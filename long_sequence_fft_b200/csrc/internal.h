@@ -44,7 +44,7 @@ struct Plan {
     int twSplit = 0;            // bits of the low table
     float2* twLo = nullptr;     // exp(-2 pi i e / M), e < 2^twSplit
     float2* twHi = nullptr;     // exp(-2 pi i (e << twSplit) / M)
-    float2* work = nullptr;     // [chunkPairs][R][C] complex fp32
+    float2* work = nullptr;     // [chunkPairs][R][C] complex fp32 (fp16 on the tensor-core staged path)
     int64_t chunkPairs = 0;
     size_t workBytes = 0;
 
@@ -102,6 +102,7 @@ cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cud
 constexpr int kTcRowLogC = 13;
 bool tc_staged_supported(int64_t N, int64_t L, int dtype);
 size_t tc_staged_filter_bytes(const Plan& p);
+size_t tc_staged_spectrum_bytes(const Plan& p);   // the fp16 rows; the [H * R] fp32 scales follow
 cudaError_t tc_rows_init(Plan& p);
 cudaError_t tc_rows_forward(const Plan& p, const ForwardArgs& fa, int64_t pair0, int64_t npairs, cudaStream_t s);
 cudaError_t tc_rows_convert(const Plan& p, int64_t h0, int64_t nch, void* Kf, cudaStream_t s);

@@ -14,6 +14,8 @@
 // twiddle), a row pass (length-C forward DFT, product with K_f, inverse) and
 // an inverse column pass, through a plan-owned workspace.  This is the
 // "I/O between memory levels" regime of the FlashFFTConv page (Limitations).
+#include <cmath>
+
 #include "internal.h"
 #include "simt_fft.cuh"
 
@@ -381,11 +383,13 @@ cudaError_t launch_fused_pre(const Plan& p, const void* k, void* Kf, cudaStream_
 // ------------------------------------------------------ staged kernels ---
 
 constexpr int kColThreads = 256;
-// columns per CTA in the column passes: 32, or more for short columns so that
-// a CTA holds at least 2048 values (R = 8: 256 columns, one radix-8 DFT per
-// thread); at most 256, which divides every staged C (C >= 256)
+// columns per CTA in the shared-memory column passes: 2048 / R, within
+// [16, 256] (256 divides every staged C >= 256).  Long columns take 16: for
+// R = 256 measured on B200 (N = 2^20), 16 columns per CTA (32 KB of shared
+// memory, more CTAs resident) ran the call 5% faster than 32 and 1.5x faster
+// than 64.
 template <int LOGR>
-constexpr int col_tile() { return (2048 >> LOGR) > 256 ? 256 : ((2048 >> LOGR) < 32 ? 32 : (2048 >> LOGR)); }
+constexpr int col_tile() { return (2048 >> LOGR) > 256 ? 256 : ((2048 >> LOGR) < 16 ? 16 : (2048 >> LOGR)); }
 
 template <int LOGC>
 constexpr int row_threads() { return (1 << LOGC) / 32 < 128 ? 128 : ((1 << LOGC) / 32 > 512 ? 512 : (1 << LOGC) / 32); }
@@ -405,6 +409,12 @@ struct StagedArgs {
     const void* k;
     int64_t L;
     int64_t kf_pair0;       // precompute mode: channel of the first K_f row written
+    // half-precision workspace (the tensor-core row pass): the forward column
+    // pass stores its values times rin as fp16; the row pass leaves its
+    // results unscaled; the inverse column pass multiplies row c of channel h
+    // by kscale[h * R + c] * rout
+    const float* kscale;
+    float rin, rout;
 };
 
 template <typename T>
@@ -421,7 +431,7 @@ __device__ __forceinline__ PairRows<T> staged_rows(const StagedArgs& A, int64_t 
 
 // Column pass: length-R DFT over j of x[j*C + r] (upper half zero), twiddle
 // exp(-2 pi i c r / M), stored at work[pair][c][r] in natural c order.
-template <int LOGR, typename T>
+template <int LOGR, typename T, bool WS16>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_fwd_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
@@ -445,13 +455,29 @@ staged_col_fwd_kernel(StagedArgs A) {
         s[sidx<TC>(R / 2 + idx / TC, idx % TC)] = make_float2(0.f, 0.f);
     __syncthreads();
     fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
-    float2* W = A.work + pl * (R * C);
-    for (int idx = tid; idx < R * TC; idx += kColThreads) {
-        const int p = idx / TC, col = idx % TC;
-        const int64_t c = perm_to_freq(p, LOGR);
-        const int64_t r = col0 + col;
-        const float2 z = cmul(s[sidx<TC>(p, col)], tw_M(A.twLo, A.twHi, A.twSplit, c * r));
-        W[c * C + r] = z;
+    // twiddle w_M^(c r) and store: each thread keeps one column r and walks
+    // CPG consecutive c (a warp writes 32 consecutive r of one c).  The
+    // twiddle comes from the table at every eighth c and as a product with
+    // w_M^r in between (at most seven fp32 products, a few ulps): a table
+    // read per element at stride c would touch up to 32 cache lines per warp.
+    constexpr int NG = kColThreads / TC, CPG = R / NG;
+    static_assert(CPG % 8 == 0, "column groups walk whole runs of 8");
+    const int col = tid % TC, g = tid / TC;
+    const int64_t r = col0 + col;
+    const float2 step = tw_M(A.twLo, A.twHi, A.twSplit, r);
+    for (int i0 = 0; i0 < CPG; i0 += 8) {
+        const int64_t cb = (int64_t)g * CPG + i0;
+        float2 w = tw_M(A.twLo, A.twHi, A.twSplit, cb * r);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i) w = cmul(w, step);
+            const int64_t c = cb + i;
+            const float2 z = cmul(s[sidx<TC>((int)freq_to_perm(c, LOGR), col)], w);
+            if constexpr (WS16)
+                reinterpret_cast<__half2*>(A.work)[pl * (R * C) + c * C + r] = __floats2half2_rn(z.x * A.rin, z.y * A.rin);
+            else
+                A.work[pl * (R * C) + c * C + r] = z;
+        }
     }
 }
 
@@ -493,7 +519,7 @@ staged_row_kernel(StagedArgs A) {
 
 // Inverse column pass: conjugate twiddle, inverse length-R DFT over c, and
 // y = v * z for t = j*C + r < N.
-template <int LOGR, typename T>
+template <int LOGR, typename T, bool WS16>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_inv_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
@@ -505,12 +531,30 @@ staged_col_inv_kernel(StagedArgs A) {
     const int64_t col0 = (int64_t)blockIdx.x * TC;
     int h;
     const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
-    const float2* W = A.work + pl * (R * C);
-    for (int idx = tid; idx < R * TC; idx += kColThreads) {
-        const int p = idx / TC, col = idx % TC;
-        const int64_t c = perm_to_freq(p, LOGR);
+    {
+        // the forward pass's walk in reverse roles: load, conjugate twiddle
+        constexpr int NG = kColThreads / TC, CPG = R / NG;
+        static_assert(CPG % 8 == 0, "column groups walk whole runs of 8");
+        const int col = tid % TC, g = tid / TC;
         const int64_t r = col0 + col;
-        s[sidx<TC>(p, col)] = cmulc(W[c * C + r], tw_M(A.twLo, A.twHi, A.twSplit, c * r));
+        const float2 step = tw_M(A.twLo, A.twHi, A.twSplit, r);
+        for (int i0 = 0; i0 < CPG; i0 += 8) {
+            const int64_t cb = (int64_t)g * CPG + i0;
+            float2 w = tw_M(A.twLo, A.twHi, A.twSplit, cb * r);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (i) w = cmul(w, step);
+                const int64_t c = cb + i;
+                float2 z;
+                if constexpr (WS16) {
+                    z = __half22float2(reinterpret_cast<const __half2*>(A.work)[pl * (R * C) + c * C + r]);
+                    z = cscale(z, __ldg(&A.kscale[(int64_t)h * R + c]) * A.rout);
+                } else {
+                    z = A.work[pl * (R * C) + c * C + r];
+                }
+                s[sidx<TC>((int)freq_to_perm(c, LOGR), col)] = cmulc(z, w);
+            }
+        }
     }
     __syncthreads();
     inv_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
@@ -523,22 +567,134 @@ staged_col_inv_kernel(StagedArgs A) {
     }
 }
 
-template <int LOGR, typename T>
-cudaError_t launch_cols(const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
-    const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * col_tile<LOGR>();
-    dim3 grid((unsigned)(C / col_tile<LOGR>()), (unsigned)A.npairs);
-    if (!inverse) {
-        auto kern = staged_col_fwd_kernel<LOGR, T>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kColThreads, smem, st>>>(A);
-    } else {
-        auto kern = staged_col_inv_kernel<LOGR, T>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kColThreads, smem, st>>>(A);
+// Column passes for short columns (R <= 8) without shared memory: a thread
+// takes four consecutive columns r .. r+3 of one pair, holds their R values in
+// registers and does the whole length-R DFT there.  Loads and stores are
+// 8- and 16-byte vectors, coalesced across the warp (consecutive threads,
+// consecutive columns); measured on B200 the shared-memory kernels run these
+// short columns at about a third of the memory bandwidth.
+constexpr int kRegColThreads = 256;
+
+template <int LOGR, typename T, bool WS16>
+__global__ void __launch_bounds__(kRegColThreads)
+staged_col_fwd_reg_kernel(StagedArgs A) {
+    constexpr int R = 1 << LOGR;
+    const int64_t C = (int64_t)1 << A.logC;
+    const int64_t pl = blockIdx.y;
+    const int64_t r0 = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    int h;
+    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    float2 x[4][R];
+#pragma unroll
+    for (int j = 0; j < R / 2; ++j) {
+        float2 q[4];
+        io.load4((int)(j * C + r0), q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e][j] = q[e];
     }
-    return cudaGetLastError();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Dft<R, -1>::run_half_input(x[e]);
+    // w_M^(c r) as powers of w_M^r (at most seven products)
+    float2 step[4], w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        step[e] = tw_M(A.twLo, A.twHi, A.twSplit, r0 + e);
+        w[e] = make_float2(1.f, 0.f);
+    }
+#pragma unroll
+    for (int c = 0; c < R; ++c) {
+        float2 z[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (c) w[e] = cmul(w[e], step[e]);
+            z[e] = cmul(x[e][c], w[e]);
+        }
+        const int64_t o = pl * (R * C) + c * C + r0;
+        if constexpr (WS16) {
+            __half2 hz[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hz[e] = __floats2half2_rn(z[e].x * A.rin, z[e].y * A.rin);
+            *reinterpret_cast<uint4*>(reinterpret_cast<__half2*>(A.work) + o) = *reinterpret_cast<const uint4*>(hz);
+        } else {
+            reinterpret_cast<float4*>(A.work + o)[0] = make_float4(z[0].x, z[0].y, z[1].x, z[1].y);
+            reinterpret_cast<float4*>(A.work + o)[1] = make_float4(z[2].x, z[2].y, z[3].x, z[3].y);
+        }
+    }
+}
+
+template <int LOGR, typename T, bool WS16>
+__global__ void __launch_bounds__(kRegColThreads)
+staged_col_inv_reg_kernel(StagedArgs A) {
+    constexpr int R = 1 << LOGR;
+    const int64_t C = (int64_t)1 << A.logC;
+    const int64_t pl = blockIdx.y;
+    const int64_t r0 = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    int h;
+    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    float2 x[4][R];
+    float2 step[4], w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        step[e] = tw_M(A.twLo, A.twHi, A.twSplit, r0 + e);
+        w[e] = make_float2(1.f, 0.f);
+    }
+#pragma unroll
+    for (int c = 0; c < R; ++c) {
+        const int64_t o = pl * (R * C) + c * C + r0;
+        float2 z[4];
+        if constexpr (WS16) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __half2*>(A.work) + o));
+            const __half2* hz = reinterpret_cast<const __half2*>(&q);
+            const float sc = __ldg(&A.kscale[(int64_t)h * R + c]) * A.rout;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) z[e] = cscale(__half22float2(hz[e]), sc);
+        } else {
+            const float4 a = reinterpret_cast<const float4*>(A.work + o)[0];
+            const float4 b = reinterpret_cast<const float4*>(A.work + o)[1];
+            z[0] = make_float2(a.x, a.y); z[1] = make_float2(a.z, a.w);
+            z[2] = make_float2(b.x, b.y); z[3] = make_float2(b.z, b.w);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (c) w[e] = cmul(w[e], step[e]);
+            x[e][c] = cmulc(z[e], w[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Dft<R, +1>::run(x[e]);
+#pragma unroll
+    for (int j = 0; j < R / 2; ++j) {
+        const float2 q[4] = {x[0][j], x[1][j], x[2][j], x[3][j]};
+        io.store4((int)(j * C + r0), q);
+    }
+}
+
+template <int LOGR, typename T, bool WS16>
+cudaError_t launch_cols(const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
+    if constexpr (LOGR <= 3) {
+        // one thread per four columns: C / 4 threads per pair (C >= 256 a
+        // power of two, so blocks of min(C / 4, 256) threads tile it exactly)
+        const unsigned threads = C / 4 < kRegColThreads ? (unsigned)(C / 4) : kRegColThreads;
+        dim3 grid((unsigned)(C / 4 / threads), (unsigned)A.npairs);
+        if (!inverse) staged_col_fwd_reg_kernel<LOGR, T, WS16><<<grid, threads, 0, st>>>(A);
+        else staged_col_inv_reg_kernel<LOGR, T, WS16><<<grid, threads, 0, st>>>(A);
+        return cudaGetLastError();
+    } else {
+        const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * col_tile<LOGR>();
+        dim3 grid((unsigned)(C / col_tile<LOGR>()), (unsigned)A.npairs);
+        if (!inverse) {
+            auto kern = staged_col_fwd_kernel<LOGR, T, WS16>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<grid, kColThreads, smem, st>>>(A);
+        } else {
+            auto kern = staged_col_inv_kernel<LOGR, T, WS16>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<grid, kColThreads, smem, st>>>(A);
+        }
+        return cudaGetLastError();
+    }
 }
 
 template <int LOGC, int MODE>
@@ -554,18 +710,18 @@ cudaError_t launch_rows(const StagedArgs& A, int64_t R, cudaStream_t st) {
 }
 
 // Runtime -> compile-time dispatch helpers.
-template <typename T>
+template <typename T, bool WS16 = false>
 cudaError_t cols_dispatch(int logR, const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
     switch (logR) {
-        case 1: return launch_cols<1, T>(A, C, inverse, st);
-        case 2: return launch_cols<2, T>(A, C, inverse, st);
-        case 3: return launch_cols<3, T>(A, C, inverse, st);
-        case 4: return launch_cols<4, T>(A, C, inverse, st);
-        case 5: return launch_cols<5, T>(A, C, inverse, st);
-        case 6: return launch_cols<6, T>(A, C, inverse, st);
-        case 7: return launch_cols<7, T>(A, C, inverse, st);
-        case 8: return launch_cols<8, T>(A, C, inverse, st);
-        case 9: return launch_cols<9, T>(A, C, inverse, st);
+        case 1: return launch_cols<1, T, WS16>(A, C, inverse, st);
+        case 2: return launch_cols<2, T, WS16>(A, C, inverse, st);
+        case 3: return launch_cols<3, T, WS16>(A, C, inverse, st);
+        case 4: return launch_cols<4, T, WS16>(A, C, inverse, st);
+        case 5: return launch_cols<5, T, WS16>(A, C, inverse, st);
+        case 6: return launch_cols<6, T, WS16>(A, C, inverse, st);
+        case 7: return launch_cols<7, T, WS16>(A, C, inverse, st);
+        case 8: return launch_cols<8, T, WS16>(A, C, inverse, st);
+        case 9: return launch_cols<9, T, WS16>(A, C, inverse, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -622,13 +778,20 @@ cudaError_t tc_staged_forward_t(const Plan& p, const ForwardArgs& fa, cudaStream
     A.work = p.work;
     A.tw = p.tw; A.twLo = p.twLo; A.twHi = p.twHi; A.twSplit = p.twSplit;
     const int64_t C = (int64_t)1 << p.logC;
+    // fp16 workspace scaled by a power of two near 1/sqrt(R) (exact): the
+    // column pass sums R/2 inputs per value, the scale keeps the operands in
+    // the inputs' range; the unitary 8192-point pair of the row pass leaves
+    // 1/8192, undone with the scale by rout
+    A.kscale = (const float*)((const uint8_t*)fa.Kf + tc_staged_spectrum_bytes(p));
+    A.rin = std::ldexp(1.0f, -(p.logR / 2));
+    A.rout = (float)C * std::ldexp(1.0f, p.logR / 2);
     const int64_t total = p.H * ((fa.B + 1) / 2);
     for (int64_t first = 0; first < total; first += p.chunkPairs) {
         A.pair0 = first;
         A.npairs = total - first < p.chunkPairs ? total - first : p.chunkPairs;
-        cudaError_t e = cols_dispatch<T>(p.logR, A, C, false, st);
+        cudaError_t e = cols_dispatch<T, true>(p.logR, A, C, false, st);
         if (e == cudaSuccess) e = tc_rows_forward(p, fa, first, A.npairs, st);
-        if (e == cudaSuccess) e = cols_dispatch<T>(p.logR, A, C, true, st);
+        if (e == cudaSuccess) e = cols_dispatch<T, true>(p.logR, A, C, true, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -647,10 +810,13 @@ cudaError_t tc_staged_precompute_t(const Plan& p, const void* k, void* Kf, cudaS
     A.tw = p.tw; A.twLo = p.twLo; A.twHi = p.twHi; A.twSplit = p.twSplit;
     A.k = k; A.L = p.L;
     const int64_t C = (int64_t)1 << p.logC, R = (int64_t)1 << p.logR;
-    for (int64_t first = 0; first < p.H; first += p.chunkPairs) {
+    // (fp32 spectra: a chunk holds half as many channels as fp16 pairs)
+    int64_t per = (int64_t)(p.workBytes / ((size_t)p.M * sizeof(float2)));
+    if (per < 1) return cudaErrorInvalidValue;
+    for (int64_t first = 0; first < p.H; first += per) {
         A.pair0 = first;
         A.kf_pair0 = first;
-        A.npairs = p.H - first < p.chunkPairs ? p.H - first : p.chunkPairs;
+        A.npairs = p.H - first < per ? p.H - first : per;
         cudaError_t e = cols_dispatch<T>(p.logR, A, C, false, st);
         if (e == cudaSuccess) e = rows_dispatch<1>(p.logC, A, R, st);
         if (e == cudaSuccess) e = tc_rows_convert(p, first, A.npairs, Kf, st);

@@ -182,10 +182,9 @@ struct TcArgs {
     const float2* tw16k;       // split mode: exp(-2 pi i t/16384), t < 8192
     float2 w16k_j3[8];         // split mode: exp(-2 pi i j/16384), j < 8
     uint4* scratch;            // split mode: [CTAs][4 pairs][8192] half2, z_even of the group
-    float2* work;              // rows mode: the staged workspace [pairs][R][8192] complex fp32
+    uint4* work;               // rows mode: the staged workspace [pairs][R][8192] complex fp16
     int64_t R;                 // rows mode: rows per pair
     int64_t pair0;             // rows mode: first pair of this chunk
-    float rin, rout;           // rows mode: input scale (keeps fp16 in range), output scale
     int* status;
 };
 
@@ -585,19 +584,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 const int jp = part * kHalf + jq;
                 uint32_t pk[8][2];
                 if constexpr (MODE == kModeRows) {
-                    // complex fp32 workspace row: eight consecutive t per j1
+                    // complex fp16 workspace row, already scaled: eight
+                    // consecutive t per j1 (two 16-byte loads)
 #pragma unroll
                     for (int jh = 0; jh < 2; ++jh) {
-                        const float4* src = reinterpret_cast<const float4*>(
-                            a.work + LP.o0 + 256 * (J * s + 2 * jp + jh) + 8 * lane);
-                        float4 f[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) f[i] = __ldg(src + i);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            pk[2 * i][jh] = pack_h2(f[i].x * a.rin, f[i].y * a.rin);
-                            pk[2 * i + 1][jh] = pack_h2(f[i].z * a.rin, f[i].w * a.rin);
-                        }
+                        const uint4* src = a.work + (LP.o0 + 256 * (J * s + 2 * jp + jh) + 8 * lane) / 4;
+                        const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
+                        pk[0][jh] = x0.x; pk[1][jh] = x0.y; pk[2][jh] = x0.z; pk[3][jh] = x0.w;
+                        pk[4][jh] = x1.x; pk[5][jh] = x1.y; pk[6][jh] = x1.z; pk[7][jh] = x1.w;
                     }
                 } else {
                 uint4 ld[2][4];
@@ -672,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
             const __half2* Ks = (const __half2*)(smem + LY::OffK);
             // loaded once per tile and pinned in a register (an opaque move
             // keeps the compiler from re-issuing the global load at each use)
-            float kscale = __ldg(&a.Kscale[MODE == kModeRows ? P.krow : hch]);
+            float kscale = MODE == kModeRows ? 1.f : __ldg(&a.Kscale[hch]);   // (rows: applied by the column pass)
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : hch) * nblk : nullptr;
 
@@ -764,6 +758,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 16 + k;
+                // rows mode: this quarter's filter row comes through L2 (or
+                // HBM); the loads are issued before the accumulator wait so
+                // that their latency overlaps it
+                [[maybe_unused]] uint4 kpre[2][2];
+                if constexpr (MODE == kModeRows) {
+                    const __half2* Kq = a.Kh16 + P.krow * (int64_t)kM;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        kpre[cc][0] = __ldg((const uint4*)(Kq + k16_index(lane, 4 * (k + cc) + s, 0)));
+                        kpre[cc][1] = __ldg((const uint4*)(Kq + k16_index(lane, 4 * (k + cc) + s, 4)));
+                    }
+                }
                 if (!(ok = begin_pair(c))) break;
                 uint32_t r[2][16];
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
@@ -774,10 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c2 = 4 * (k + cc) + s;
                     uint4 k0, k1;
-                    if constexpr (MODE == kModeRows) {   // this quarter's row, through L2
-                        const __half2* Kq = a.Kh16 + P.krow * (int64_t)kM;
-                        k0 = __ldg((const uint4*)(Kq + k16_index(lane, c2, 0)));
-                        k1 = __ldg((const uint4*)(Kq + k16_index(lane, c2, 4)));
+                    if constexpr (MODE == kModeRows) {
+                        k0 = kpre[cc][0];
+                        k1 = kpre[cc][1];
                     } else {
                         k0 = *(const uint4*)(Ks + k16_index(lane, c2, 0));
                         k1 = *(const uint4*)(Ks + k16_index(lane, c2, 4));
@@ -938,20 +943,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             }
                         }
                         if (MODE == kModeRows && emit) {
-                            // z s_h back into the workspace row, times the output
-                            // scale: the filter rows hold rfft(k)/M (the column
-                            // passes expect the 1/M in the product), so it undoes
-                            // the unitary pair's 1/8192 and the input scale
-                            const float sc = kscale * a.rout;
+                            // z back into the workspace row as fp16, unscaled
+                            // (the inverse column pass applies the row's filter
+                            // scale and undoes the unitary pair's 1/8192)
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
-                                float4* dst = reinterpret_cast<float4*>(a.work + P.o0 + 256 * (jb + jj) + 8 * lane);
+                                uint32_t hz[8];
 #pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    dst[e] = make_float4(__uint_as_float(r[e][0][2 * jj]) * sc,
-                                                         __uint_as_float(r[e][0][2 * jj + 1]) * sc,
-                                                         __uint_as_float(r[e][1][2 * jj]) * sc,
-                                                         __uint_as_float(r[e][1][2 * jj + 1]) * sc);
+                                for (int j3 = 0; j3 < 8; ++j3)
+                                    hz[j3] = pack_h2(__uint_as_float(r[j3 >> 1][j3 & 1][2 * jj]),
+                                                     __uint_as_float(r[j3 >> 1][j3 & 1][2 * jj + 1]));
+                                uint4* dst = a.work + (P.o0 + 256 * (jb + jj) + 8 * lane) / 4;
+                                dst[0] = make_uint4(hz[0], hz[1], hz[2], hz[3]);
+                                dst[1] = make_uint4(hz[4], hz[5], hz[6], hz[7]);
                             }
                         }
                         if (MODE != kModeRows && emit) {
@@ -1357,6 +1361,8 @@ bool tc_staged_supported(int64_t N, int64_t L, int dtype) {
     return (dtype == kF16 || dtype == kBF16) && N >= 4 * kN && N <= (int64_t(1) << 21) && L > kHop + 1;
 }
 
+size_t tc_staged_spectrum_bytes(const Plan& p) { return (size_t)(p.H * (p.M / kM)) * kKBytes; }
+
 size_t tc_staged_filter_bytes(const Plan& p) {
     const int64_t rows = p.H * (p.M / kM);
     return (size_t)rows * kKBytes + (((size_t)rows * 4 + 15) & ~size_t(15));
@@ -1387,14 +1393,7 @@ cudaError_t tc_rows_forward(const Plan& p, const ForwardArgs& fa, int64_t pair0,
     a.nwin = 1;
     a.pb = (fa.B + 1) / 2;
     a.tpc = 1;
-    a.work = p.work; a.R = R; a.pair0 = pair0;
-    // the column pass sums R/2 inputs per workspace value: scale by a power
-    // of two near 1/sqrt(R) (exact) so that the fp16 operands keep the
-    // inputs' range
-    int lr = 0;
-    while ((int64_t(1) << (lr + 1)) <= R) ++lr;
-    a.rin = std::ldexp(1.0f, -(lr / 2));
-    a.rout = std::ldexp((float)kM, lr / 2);
+    a.work = (uint4*)p.work; a.R = R; a.pair0 = pair0;
     a.nunits = npairs * (R / 4);
     a.bimg = (const uint4*)r->bimg;
     a.tw1024 = r->tw1024;
