@@ -277,8 +277,11 @@ def main():
     value = mg.job_throughput(w.elems, ctx, ms_per_step)
 
     launches_per_step = 1
-    if plan.path == lsf.PATH_SIMT_STAGED:
-        chunk = max(1, plan.workspace_bytes // (2 * w.N * 8))
+    if plan.path in (lsf.PATH_SIMT_STAGED, lsf.PATH_TC_STAGED):
+        # column pass, row pass, inverse column pass per workspace chunk
+        # (fp32 workspace: 2N x 8 bytes per pair; fp16 on the tensor-core path)
+        per_pair = 2 * w.N * (8 if plan.path == lsf.PATH_SIMT_STAGED else 4)
+        chunk = max(1, plan.workspace_bytes // per_pair)
         pairs = w.H * ((w.B + 1) // 2)
         launches_per_step = 3 * ((pairs + chunk - 1) // chunk)
 
@@ -322,7 +325,9 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16" if plan.path == lsf.PATH_TC_FUSED else "f32",
+        # arithmetic of the path: fp16 tensor-core operands (fp32 accumulate);
+        # the tensor-core staged path runs its column passes in fp32
+        "dtype": "f16" if plan.path in (lsf.PATH_TC_FUSED, lsf.PATH_TC_STAGED) else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated,
                    "io_dtype": w.dtype, "path": plan.path_name, "parallelism": f"channel shards x{world}",

@@ -355,3 +355,18 @@ def test_tc_staged_forward_host_chunks():
     torch.cuda.synchronize()
     assert plan.device_status() == 0
     assert_close(y_host.float().numpy().astype(np.float64), _oracle(inp), "bf16", "tc_staged forward_host")
+
+
+@pytest.mark.parametrize("dtype,order,N,L,B,H,gated,mask_frac", [
+    ("f32", 4, 1 << 17, 1 << 17, 1, 2, False, 0.0),     # fp32 staged, 256 x 1024
+    ("bf16", 4, 1 << 18, 5000, 3, 1, True, 0.5),        # 256 x 1024, partial filter, mask
+    ("f16", 5, 1 << 21, 1 << 21, 1, 1, True, 0.0),      # tensor-core rows, 512 x 8192
+    ("bf16", 5, 1 << 18, 1 << 18, 2, 2, False, 0.25),   # tensor-core rows, 64 x 8192
+])
+def test_staged_long_columns(dtype, order, N, L, B, H, gated, mask_frac):
+    """Long columns (64 to 512 values: the shared-memory column passes) with
+    fp32 and tensor-core row passes, against the oracle element by element."""
+    inp = _rand_inputs(B, H, N, L, dtype, gated=gated, mask_frac=mask_frac, seed=N // 4096 + order)
+    y, plan = run_cuda(inp, dtype, order=order)
+    assert plan.path_name == ("simt_staged" if order == 4 else "tc_staged")
+    assert_close(y, _oracle(inp), dtype, f"staged {dtype} order={order} N={N} L={L}")
