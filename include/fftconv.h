@@ -78,7 +78,7 @@ typedef enum {
  * and H channels with full-length filters (L = N).  `order` selects the
  * decomposition: 0 = automatic; 2 or 3 = fused on-chip kernel (N <= 8192);
  * 4 = the staged path with one workspace round trip (any N); 5 = the staged
- * path whose row pass runs on the tensor cores (fp16/bf16, 16384 <= N <= 2^21,
+ * path whose row pass runs on the tensor cores (fp16/bf16, 16384 <= N <= 2^22,
  * L > 2049; order 0 chooses it for those plans); other values are
  * FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
  * (a few hundred KB) and its workspace (staged path only) on the current

@@ -118,7 +118,7 @@ class Plan:
     order: 0 automatic, 1 fp32 shared-memory FFT in one kernel (N <= 8192),
     2/3 fused on-chip kernel (tensor cores where available), 4 staged passes
     through a workspace (any N), 5 staged passes with the row pass on the
-    tensor cores (fp16/bf16, 16384 <= N <= 2^21, L > 2049).  L < N gives the
+    tensor cores (fp16/bf16, 16384 <= N <= 2^22, L > 2049).  L < N gives the
     partial convolution."""
 
     def __init__(self, N: int, H: int, dtype="bf16", order: int = 0, L: Optional[int] = None):

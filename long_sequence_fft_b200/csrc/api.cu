@@ -148,7 +148,7 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         if (!tc_staged_ok) {
             delete p;
             return fail(FFTCONV_ERR_UNSUPPORTED,
-                        "order 5 needs fp16/bf16, 16384 <= N <= 2^21 and L > 2049 (N=%lld, L=%lld)",
+                        "order 5 needs fp16/bf16, 16384 <= N <= 2^22 and L > 2049 (N=%lld, L=%lld)",
                         (long long)N, (long long)L);
         }
         p->path = kPathTcStaged;

@@ -722,6 +722,7 @@ cudaError_t cols_dispatch(int logR, const StagedArgs& A, int64_t C, bool inverse
         case 7: return launch_cols<7, T, WS16>(A, C, inverse, st);
         case 8: return launch_cols<8, T, WS16>(A, C, inverse, st);
         case 9: return launch_cols<9, T, WS16>(A, C, inverse, st);
+        case 10: return launch_cols<10, T, WS16>(A, C, inverse, st);   // rows of 8192 at N = 2^22
         default: return cudaErrorInvalidValue;
     }
 }

@@ -797,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                             int blk;
                             if constexpr (MODE == kModeRows) {
                                 // bin c + R f8 of the 2N-point spectrum, c = this
-                                // row (krow mod R, R a power of two; 2N <= 2^22)
+                                // row (krow mod R, R a power of two; 2N <= 2^23)
                                 const int f = (int)((uint32_t)P.krow & (uint32_t)(a.R - 1)) + (int)a.R * f8;
                                 blk = (f <= (int)a.N ? f : 2 * (int)a.N - f) >> 5;
                             } else {
@@ -1358,7 +1358,7 @@ __global__ void tc_rows_export_kernel(const __half2* __restrict__ Kh, const floa
 }  // namespace
 
 bool tc_staged_supported(int64_t N, int64_t L, int dtype) {
-    return (dtype == kF16 || dtype == kBF16) && N >= 4 * kN && N <= (int64_t(1) << 21) && L > kHop + 1;
+    return (dtype == kF16 || dtype == kBF16) && N >= 4 * kN && N <= (int64_t(1) << 22) && L > kHop + 1;
 }
 
 size_t tc_staged_spectrum_bytes(const Plan& p) { return (size_t)(p.H * (p.M / kM)) * kKBytes; }

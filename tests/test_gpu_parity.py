@@ -77,6 +77,7 @@ REDUCED = {
     "dna_bf16_n1m": dict(H=2),
     "partial_bf16_n8k": dict(B=3, H=3),
     "sparse_bf16_n8k": dict(B=3, H=3),
+    "dna_bf16_n4m_l1m": dict(H=2),
 }
 
 
@@ -362,6 +363,8 @@ def test_tc_staged_forward_host_chunks():
     ("bf16", 4, 1 << 18, 5000, 3, 1, True, 0.5),        # 256 x 1024, partial filter, mask
     ("f16", 5, 1 << 21, 1 << 21, 1, 1, True, 0.0),      # tensor-core rows, 512 x 8192
     ("bf16", 5, 1 << 18, 1 << 18, 2, 2, False, 0.25),   # tensor-core rows, 64 x 8192
+    ("bf16", 0, 1 << 22, 1 << 20, 1, 1, True, 0.5),     # 4M with a 1M filter: 1024 x 8192
+    ("f32", 4, 1 << 22, 1 << 20, 1, 1, False, 0.0),     # the same on fp32 lanes, 512 x 16384
 ])
 def test_staged_long_columns(dtype, order, N, L, B, H, gated, mask_frac):
     """Long columns (64 to 512 values: the shared-memory column passes) with

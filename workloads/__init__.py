@@ -10,10 +10,11 @@ Recipe: seed = 1000 + workload index; tensor ``t`` of a workload draws from
 ``np.random.default_rng([seed, TENSOR_IDS[t]])``.  Values are drawn in float32
 and rounded to the dtype with round-to-nearest-even (torch ``.to``).
 
-The five workloads mirror the sequence lengths the FlashFFTConv page measures
+The workloads mirror the sequence lengths the FlashFFTConv page measures
 (1K forward latency, 8K Hyena filters with 2K partial filters, the 1M-token
-HyenaDNA setting, 75% frequency sparsity); there is no dataset here, and the
-DNA-like workload is a synthetic stand-in for genome data.
+HyenaDNA setting and its extension to 4M tokens with partial filters, 75%
+frequency sparsity); there is no dataset here, and the DNA-like workloads are
+a synthetic stand-in for genome data.
 """
 from __future__ import annotations
 
@@ -82,6 +83,11 @@ WORKLOADS = {
     "sparse_bf16_n8k": Workload("sparse_bf16_n8k", 6, 16, 768, 8192, 8192, "bf16", True,
                                 "plain", sparsity=0.75,
                                 description="gated bf16 B=16 H=768 N=8192, 75% block-sparse rfft(k)"),
+    # the sequence extension with partial filters (1M-token filters on 4M
+    # sequences), the same element count as the 1M DNA workload
+    "dna_bf16_n4m_l1m": Workload("dna_bf16_n4m_l1m", 7, 1, 32, 1 << 22, 1 << 20, "bf16", False,
+                                 "decay:1e-5", u_kind="dna",
+                                 description="bf16 conv B=1 H=32 N=4M, filter length 1M, DNA-like input"),
 }
 
 # The workload the benchmark times at one GPU.
