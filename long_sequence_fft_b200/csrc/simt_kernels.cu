@@ -384,12 +384,16 @@ cudaError_t launch_fused_pre(const Plan& p, const void* k, void* Kf, cudaStream_
 
 constexpr int kColThreads = 256;
 // columns per CTA in the shared-memory column passes: 2048 / R, within
-// [16, 256] (256 divides every staged C >= 256).  Long columns take 16: for
-// R = 256 measured on B200 (N = 2^20), 16 columns per CTA (32 KB of shared
-// memory, more CTAs resident) ran the call 5% faster than 32 and 1.5x faster
-// than 64.
+// [16, 256] (256 divides every staged C >= 256), and 8 for R >= 512.  Long
+// columns need narrow tiles so that several CTAs stay resident: measured on
+// B200, R = 256 (N = 2^20) ran the call 5% faster with 16 columns per CTA
+// (32 KB of shared memory) than with 32 and 1.5x faster than with 64;
+// R = 1024 (N = 2^22) 1.34x faster with 8 (64 KB) than with 16 (128 KB, one
+// CTA per SM), and 1.30x faster than with 4 (16-byte row segments).
 template <int LOGR>
-constexpr int col_tile() { return (2048 >> LOGR) > 256 ? 256 : ((2048 >> LOGR) < 16 ? 16 : (2048 >> LOGR)); }
+constexpr int col_tile() {
+    return LOGR >= 9 ? 8 : ((2048 >> LOGR) > 256 ? 256 : ((2048 >> LOGR) < 16 ? 16 : (2048 >> LOGR)));
+}
 
 template <int LOGC>
 constexpr int row_threads() { return (1 << LOGC) / 32 < 128 ? 128 : ((1 << LOGC) / 32 > 512 ? 512 : (1 << LOGC) / 32); }
