@@ -79,8 +79,11 @@ typedef enum {
  * decomposition: 0 = automatic; 2 or 3 = fused on-chip kernel (N <= 8192);
  * 4 = the staged path with one workspace round trip (any N); 5 = the staged
  * path whose row pass runs on the tensor cores (fp16/bf16, 16384 <= N <= 2^22,
- * L > 2049; order 0 chooses it for those plans); other values are
- * FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
+ * L > 2049; order 0 chooses it for those plans, as overlap-save windows of
+ * 2 x hop points when the filter is at most half the sequence: hop = the
+ * power of two >= max(L, 16384); such a windowed plan rejects block masks
+ * and fftconv_filter_to_rfft with FFTCONV_ERR_UNSUPPORTED, order 5 keeps the
+ * full transform); other values are FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
  * (a few hundred KB) and its workspace (staged path only) on the current
  * device.  *out receives the plan, or NULL on failure. */
 FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,

@@ -178,6 +178,23 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         e = upload(&p->tw, host_twiddles(p->M, p->M, 1));
         p->filter_bytes = (size_t)H * (size_t)p->M * sizeof(float2);
     } else if (p->path == kPathSimtStaged || p->path == kPathTcStaged) {
+        // Automatic tensor-core staged plans with a filter much shorter than
+        // the sequence run overlap-save windows: hop Lw = the smallest power
+        // of two >= max(L, 16384), one 2 Lw-point transform per window,
+        // N / Lw windows per sequence (the same number of transform points as
+        // one 2N-point transform, in shorter columns).  The filter spectrum
+        // then has 2 Lw points, so such plans take no block mask and export
+        // no 2N-point spectrum; order 5 keeps the full transform.
+        if (p->path == kPathTcStaged && order == 0) {
+            int64_t lw = 16384;
+            while (lw < L) lw *= 2;
+            if (2 * lw <= N) {
+                p->winHop = lw;
+                p->nwin = N / lw;
+                p->M = 2 * lw;
+                p->logM = ilog2(p->M);
+            }
+        }
         // (the tensor-core row pass takes rows of 8192)
         p->logC = p->path == kPathTcStaged ? kTcRowLogC : staged_log_cols(p->logM);
         p->logR = p->logM - p->logC;
@@ -281,10 +298,10 @@ static int validate_forward(const Plan& p, const void* u, const void* K_f, void*
     if (p.path == kPathTcFused &&
         (double)H * (double)tc_tiles_per_pair_group(p.N, p.L) * (double)(((B + 1) / 2 + 3) / 4) >= 2147483648.0)
         return fail(FFTCONV_ERR_UNSUPPORTED, "too many tiles for one launch");
-    if (mask && p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
+    if (mask && ((p.path == kPathTcFused && tc_overlap_save(p.N, p.L)) || p.nwin > 1))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "block masks act on the 2N-point spectrum; this overlap-save plan (N=%lld, L=%lld) "
-                    "has none: create the plan with order 1 or 4",
+                    "has none: create the plan with order 1 or 4 (or 5 for N >= 16384, L > 2049)",
                     (long long)p.N, (long long)p.L);
     if (B > (int64_t(1) << 30) / 1) {
         if ((double)B * (double)H > 4.0e9) return fail(FFTCONV_ERR_UNSUPPORTED, "B*H too large");
@@ -442,6 +459,10 @@ int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fft
     if (p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "this overlap-save plan stores the 8192-point spectrum of k, not the 2N-point one");
+    if (p.nwin > 1)
+        return fail(FFTCONV_ERR_UNSUPPORTED,
+                    "this overlap-save plan stores the %lld-point spectrum of k, not the 2N-point one",
+                    (long long)p.M);
     cudaError_t e = p.path == kPathTcFused    ? tc_export_rfft(p, K_f, out, (cudaStream_t)stream)
                     : p.path == kPathTcStaged ? tc_rows_export(p, K_f, out, (cudaStream_t)stream)
                                               : simt_export_rfft(p, K_f, out, (cudaStream_t)stream);

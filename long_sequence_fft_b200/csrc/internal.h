@@ -45,6 +45,11 @@ struct Plan {
     float2* twLo = nullptr;     // exp(-2 pi i e / M), e < 2^twSplit
     float2* twHi = nullptr;     // exp(-2 pi i (e << twSplit) / M)
     float2* work = nullptr;     // [chunkPairs][R][C] complex fp32 (fp16 on the tensor-core staged path)
+    // tensor-core staged path, overlap-save windows (nwin > 1): transforms of
+    // M = 2 winHop points, window w of a sequence reads inputs
+    // [(w-1) winHop, (w+1) winHop) (zero before 0) and writes outputs
+    // [w winHop, (w+1) winHop); the workspace units are (pair, window)
+    int64_t winHop = 0, nwin = 1;
     int64_t chunkPairs = 0;
     size_t workBytes = 0;
 

@@ -419,7 +419,27 @@ struct StagedArgs {
     // by kscale[h * R + c] * rout
     const float* kscale;
     float rin, rout;
+    // overlap-save windows (column kernels with WIN): unit u of the chunk is
+    // window u % nwin of pair u / nwin; the window's position t is sequence
+    // position (w - 1) winHop + t, inputs before 0 read as zero, and only its
+    // second half t >= winHop is output
+    int64_t nwin, winHop;
 };
+
+// pair, window and the sequence position of window position 0 of unit u
+struct UnitPos {
+    int64_t pair, win, base;
+};
+template <bool WIN>
+__device__ __forceinline__ UnitPos unit_pos(const StagedArgs& A, int64_t u) {
+    UnitPos p{u, 0, 0};
+    if constexpr (WIN) {
+        p.pair = u / A.nwin;
+        p.win = u - p.pair * A.nwin;
+        p.base = (p.win - 1) * A.winHop;
+    }
+    return p;
+}
 
 template <typename T>
 __device__ __forceinline__ PairRows<T> staged_rows(const StagedArgs& A, int64_t pair, int* h) {
@@ -435,7 +455,7 @@ __device__ __forceinline__ PairRows<T> staged_rows(const StagedArgs& A, int64_t 
 
 // Column pass: length-R DFT over j of x[j*C + r] (upper half zero), twiddle
 // exp(-2 pi i c r / M), stored at work[pair][c][r] in natural c order.
-template <int LOGR, typename T, bool WS16>
+template <int LOGR, typename T, bool WS16, bool WIN>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_fwd_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
@@ -445,18 +465,28 @@ staged_col_fwd_kernel(StagedArgs A) {
     const int64_t C = (int64_t)1 << A.logC;
     const int64_t pl = blockIdx.y;
     const int64_t col0 = (int64_t)blockIdx.x * TC;
+    const UnitPos U = unit_pos<WIN>(A, A.pair0 + pl);
     int h;
-    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
-    // the nonzero half (j < R/2), four consecutive columns per thread
-    for (int idx = tid; idx < (R / 2) * (TC / 4); idx += kColThreads) {
+    const PairRows<T> io = staged_rows<T>(A, U.pair, &h);
+    // the nonzero rows (j < R/2; a window: all R, the first window's first
+    // half zero), four consecutive columns per thread
+    constexpr int JN = WIN ? R : R / 2;
+    for (int idx = tid; idx < JN * (TC / 4); idx += kColThreads) {
         const int j = idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
         float2 x[4];
-        io.load4((int)(j * C + col0 + c4), x);
+        if (WIN && U.win == 0 && j < R / 2) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = make_float2(0.f, 0.f);
+        } else {
+            io.load4((int)(U.base + j * C + col0 + c4), x);
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[sidx<TC>(j, c4 + e)] = x[e];
     }
-    for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads)
-        s[sidx<TC>(R / 2 + idx / TC, idx % TC)] = make_float2(0.f, 0.f);
+    if constexpr (!WIN) {
+        for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads)
+            s[sidx<TC>(R / 2 + idx / TC, idx % TC)] = make_float2(0.f, 0.f);
+    }
     __syncthreads();
     fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
     // twiddle w_M^(c r) and store: each thread keeps one column r and walks
@@ -523,7 +553,7 @@ staged_row_kernel(StagedArgs A) {
 
 // Inverse column pass: conjugate twiddle, inverse length-R DFT over c, and
 // y = v * z for t = j*C + r < N.
-template <int LOGR, typename T, bool WS16>
+template <int LOGR, typename T, bool WS16, bool WIN>
 __global__ void __launch_bounds__(kColThreads)
 staged_col_inv_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
@@ -533,8 +563,9 @@ staged_col_inv_kernel(StagedArgs A) {
     const int64_t C = (int64_t)1 << A.logC;
     const int64_t pl = blockIdx.y;
     const int64_t col0 = (int64_t)blockIdx.x * TC;
+    const UnitPos U = unit_pos<WIN>(A, A.pair0 + pl);
     int h;
-    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    const PairRows<T> io = staged_rows<T>(A, U.pair, &h);
     {
         // the forward pass's walk in reverse roles: load, conjugate twiddle
         constexpr int NG = kColThreads / TC, CPG = R / NG;
@@ -562,12 +593,14 @@ staged_col_inv_kernel(StagedArgs A) {
     }
     __syncthreads();
     inv_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    // outputs: the first half (t < N), or a window's second half
+    constexpr int J0 = WIN ? R / 2 : 0;
     for (int idx = tid; idx < (R / 2) * (TC / 4); idx += kColThreads) {
-        const int j = idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
+        const int j = J0 + idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
         float2 z[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) z[e] = s[sidx<TC>(j, c4 + e)];
-        io.store4((int)(j * C + col0 + c4), z);
+        io.store4((int)(U.base + j * C + col0 + c4), z);
     }
 }
 
@@ -579,25 +612,36 @@ staged_col_inv_kernel(StagedArgs A) {
 // short columns at about a third of the memory bandwidth.
 constexpr int kRegColThreads = 256;
 
-template <int LOGR, typename T, bool WS16>
+template <int LOGR, typename T, bool WS16, bool WIN>
 __global__ void __launch_bounds__(kRegColThreads)
 staged_col_fwd_reg_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
     const int64_t C = (int64_t)1 << A.logC;
     const int64_t pl = blockIdx.y;
     const int64_t r0 = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    const UnitPos U = unit_pos<WIN>(A, A.pair0 + pl);
     int h;
-    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    const PairRows<T> io = staged_rows<T>(A, U.pair, &h);
     float2 x[4][R];
+    // the nonzero rows (j < R/2; a window: all R, the first window's first
+    // half zero)
 #pragma unroll
-    for (int j = 0; j < R / 2; ++j) {
+    for (int j = 0; j < (WIN ? R : R / 2); ++j) {
         float2 q[4];
-        io.load4((int)(j * C + r0), q);
+        if (WIN && U.win == 0 && j < R / 2) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q[e] = make_float2(0.f, 0.f);
+        } else {
+            io.load4((int)(U.base + j * C + r0), q);
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) x[e][j] = q[e];
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) Dft<R, -1>::run_half_input(x[e]);
+    for (int e = 0; e < 4; ++e) {
+        if constexpr (WIN) Dft<R, -1>::run(x[e]);
+        else Dft<R, -1>::run_half_input(x[e]);
+    }
     // w_M^(c r) as powers of w_M^r (at most seven products)
     float2 step[4], w[4];
 #pragma unroll
@@ -626,15 +670,16 @@ staged_col_fwd_reg_kernel(StagedArgs A) {
     }
 }
 
-template <int LOGR, typename T, bool WS16>
+template <int LOGR, typename T, bool WS16, bool WIN>
 __global__ void __launch_bounds__(kRegColThreads)
 staged_col_inv_reg_kernel(StagedArgs A) {
     constexpr int R = 1 << LOGR;
     const int64_t C = (int64_t)1 << A.logC;
     const int64_t pl = blockIdx.y;
     const int64_t r0 = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    const UnitPos U = unit_pos<WIN>(A, A.pair0 + pl);
     int h;
-    const PairRows<T> io = staged_rows<T>(A, A.pair0 + pl, &h);
+    const PairRows<T> io = staged_rows<T>(A, U.pair, &h);
     float2 x[4][R];
     float2 step[4], w[4];
 #pragma unroll
@@ -666,33 +711,35 @@ staged_col_inv_reg_kernel(StagedArgs A) {
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) Dft<R, +1>::run(x[e]);
+    // outputs: the first half (t < N), or a window's second half
 #pragma unroll
-    for (int j = 0; j < R / 2; ++j) {
+    for (int jj = 0; jj < R / 2; ++jj) {
+        const int j = (WIN ? R / 2 : 0) + jj;
         const float2 q[4] = {x[0][j], x[1][j], x[2][j], x[3][j]};
-        io.store4((int)(j * C + r0), q);
+        io.store4((int)(U.base + j * C + r0), q);
     }
 }
 
-template <int LOGR, typename T, bool WS16>
+template <int LOGR, typename T, bool WS16, bool WIN>
 cudaError_t launch_cols(const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
     if constexpr (LOGR <= 3) {
         // one thread per four columns: C / 4 threads per pair (C >= 256 a
         // power of two, so blocks of min(C / 4, 256) threads tile it exactly)
         const unsigned threads = C / 4 < kRegColThreads ? (unsigned)(C / 4) : kRegColThreads;
         dim3 grid((unsigned)(C / 4 / threads), (unsigned)A.npairs);
-        if (!inverse) staged_col_fwd_reg_kernel<LOGR, T, WS16><<<grid, threads, 0, st>>>(A);
-        else staged_col_inv_reg_kernel<LOGR, T, WS16><<<grid, threads, 0, st>>>(A);
+        if (!inverse) staged_col_fwd_reg_kernel<LOGR, T, WS16, WIN><<<grid, threads, 0, st>>>(A);
+        else staged_col_inv_reg_kernel<LOGR, T, WS16, WIN><<<grid, threads, 0, st>>>(A);
         return cudaGetLastError();
     } else {
         const size_t smem = sizeof(float2) * (size_t)(1 << LOGR) * col_tile<LOGR>();
         dim3 grid((unsigned)(C / col_tile<LOGR>()), (unsigned)A.npairs);
         if (!inverse) {
-            auto kern = staged_col_fwd_kernel<LOGR, T, WS16>;
+            auto kern = staged_col_fwd_kernel<LOGR, T, WS16, WIN>;
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             kern<<<grid, kColThreads, smem, st>>>(A);
         } else {
-            auto kern = staged_col_inv_kernel<LOGR, T, WS16>;
+            auto kern = staged_col_inv_kernel<LOGR, T, WS16, WIN>;
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             kern<<<grid, kColThreads, smem, st>>>(A);
@@ -714,19 +761,19 @@ cudaError_t launch_rows(const StagedArgs& A, int64_t R, cudaStream_t st) {
 }
 
 // Runtime -> compile-time dispatch helpers.
-template <typename T, bool WS16 = false>
+template <typename T, bool WS16 = false, bool WIN = false>
 cudaError_t cols_dispatch(int logR, const StagedArgs& A, int64_t C, bool inverse, cudaStream_t st) {
     switch (logR) {
-        case 1: return launch_cols<1, T, WS16>(A, C, inverse, st);
-        case 2: return launch_cols<2, T, WS16>(A, C, inverse, st);
-        case 3: return launch_cols<3, T, WS16>(A, C, inverse, st);
-        case 4: return launch_cols<4, T, WS16>(A, C, inverse, st);
-        case 5: return launch_cols<5, T, WS16>(A, C, inverse, st);
-        case 6: return launch_cols<6, T, WS16>(A, C, inverse, st);
-        case 7: return launch_cols<7, T, WS16>(A, C, inverse, st);
-        case 8: return launch_cols<8, T, WS16>(A, C, inverse, st);
-        case 9: return launch_cols<9, T, WS16>(A, C, inverse, st);
-        case 10: return launch_cols<10, T, WS16>(A, C, inverse, st);   // rows of 8192 at N = 2^22
+        case 1: return launch_cols<1, T, WS16, WIN>(A, C, inverse, st);
+        case 2: return launch_cols<2, T, WS16, WIN>(A, C, inverse, st);
+        case 3: return launch_cols<3, T, WS16, WIN>(A, C, inverse, st);
+        case 4: return launch_cols<4, T, WS16, WIN>(A, C, inverse, st);
+        case 5: return launch_cols<5, T, WS16, WIN>(A, C, inverse, st);
+        case 6: return launch_cols<6, T, WS16, WIN>(A, C, inverse, st);
+        case 7: return launch_cols<7, T, WS16, WIN>(A, C, inverse, st);
+        case 8: return launch_cols<8, T, WS16, WIN>(A, C, inverse, st);
+        case 9: return launch_cols<9, T, WS16, WIN>(A, C, inverse, st);
+        case 10: return launch_cols<10, T, WS16, WIN>(A, C, inverse, st);   // rows of 8192 at N = 2^22
         default: return cudaErrorInvalidValue;
     }
 }
@@ -790,13 +837,20 @@ cudaError_t tc_staged_forward_t(const Plan& p, const ForwardArgs& fa, cudaStream
     A.kscale = (const float*)((const uint8_t*)fa.Kf + tc_staged_spectrum_bytes(p));
     A.rin = std::ldexp(1.0f, -(p.logR / 2));
     A.rout = (float)C * std::ldexp(1.0f, p.logR / 2);
-    const int64_t total = p.H * ((fa.B + 1) / 2);
+    // workspace units: pairs, or (pair, window) with overlap-save windows
+    const bool win = p.nwin > 1;
+    A.nwin = p.nwin;
+    A.winHop = p.winHop;
+    const int64_t total = p.H * ((fa.B + 1) / 2) * p.nwin;
     for (int64_t first = 0; first < total; first += p.chunkPairs) {
         A.pair0 = first;
         A.npairs = total - first < p.chunkPairs ? total - first : p.chunkPairs;
-        cudaError_t e = cols_dispatch<T, true>(p.logR, A, C, false, st);
+        cudaError_t e = win ? cols_dispatch<T, true, true>(p.logR, A, C, false, st)
+                            : cols_dispatch<T, true, false>(p.logR, A, C, false, st);
         if (e == cudaSuccess) e = tc_rows_forward(p, fa, first, A.npairs, st);
-        if (e == cudaSuccess) e = cols_dispatch<T, true>(p.logR, A, C, true, st);
+        if (e == cudaSuccess)
+            e = win ? cols_dispatch<T, true, true>(p.logR, A, C, true, st)
+                    : cols_dispatch<T, true, false>(p.logR, A, C, true, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

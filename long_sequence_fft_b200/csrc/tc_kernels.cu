@@ -1391,7 +1391,9 @@ cudaError_t tc_rows_forward(const Plan& p, const ForwardArgs& fa, int64_t pair0,
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H; a.N = p.N;
     a.nwin = 1;
-    a.pb = (fa.B + 1) / 2;
+    // workspace units per channel (rows mode divides by it for the channel):
+    // the pairs, times the overlap-save windows of each
+    a.pb = (fa.B + 1) / 2 * p.nwin;
     a.tpc = 1;
     a.work = (uint4*)p.work; a.R = R; a.pair0 = pair0;
     a.nunits = npairs * (R / 4);

@@ -363,7 +363,7 @@ def test_tc_staged_forward_host_chunks():
     ("bf16", 4, 1 << 18, 5000, 3, 1, True, 0.5),        # 256 x 1024, partial filter, mask
     ("f16", 5, 1 << 21, 1 << 21, 1, 1, True, 0.0),      # tensor-core rows, 512 x 8192
     ("bf16", 5, 1 << 18, 1 << 18, 2, 2, False, 0.25),   # tensor-core rows, 64 x 8192
-    ("bf16", 0, 1 << 22, 1 << 20, 1, 1, True, 0.5),     # 4M with a 1M filter: 1024 x 8192
+    ("bf16", 5, 1 << 22, 1 << 20, 1, 1, True, 0.5),     # 4M with a 1M filter: 1024 x 8192
     ("f32", 4, 1 << 22, 1 << 20, 1, 1, False, 0.0),     # the same on fp32 lanes, 512 x 16384
 ])
 def test_staged_long_columns(dtype, order, N, L, B, H, gated, mask_frac):
@@ -373,3 +373,39 @@ def test_staged_long_columns(dtype, order, N, L, B, H, gated, mask_frac):
     y, plan = run_cuda(inp, dtype, order=order)
     assert plan.path_name == ("simt_staged" if order == 4 else "tc_staged")
     assert_close(y, _oracle(inp), dtype, f"staged {dtype} order={order} N={N} L={L}")
+
+
+@pytest.mark.parametrize("dtype,N,L,B,H,nwin", [
+    ("bf16", 32768, 4096, 3, 2, 2),          # hop 16384: 32768-point windows, 4 x 8192
+    ("f16", 65536, 16384, 2, 1, 4),          # L equal to the hop
+    ("bf16", 1 << 20, 20000, 1, 2, 32),      # hop 32768: 8 x 8192 columns in registers
+    ("f16", 1 << 21, 300000, 1, 1, 4),       # hop 2^19: 128 x 8192 columns in shared memory
+])
+def test_tc_staged_overlap_save_windows(dtype, N, L, B, H, nwin):
+    """Automatic plans with a filter much shorter than the sequence run the
+    staged tensor-core path over overlap-save windows (2 x hop points, the
+    first window's first half zero, each window's second half output)."""
+    inp = _rand_inputs(B, H, N, L, dtype, gated=True, seed=N // 1024 + L % 977)
+    y, plan = run_cuda(inp, dtype, order=0)
+    assert plan.path_name == "tc_staged"
+    assert_close(y, _oracle(inp), dtype, f"tc_staged windows {dtype} N={N} L={L} B={B} (nwin={nwin})")
+    # the same filter without windows (order 5) agrees with the oracle too
+    y5, plan5 = run_cuda(inp, dtype, order=5)
+    assert_close(y5, _oracle(inp), dtype, f"tc_staged full {dtype} N={N} L={L}")
+
+
+def test_tc_staged_windows_reject_mask_and_export():
+    import torch
+    import long_sequence_fft_b200 as lsf
+    N, H, L = 32768, 2, 4096
+    inp = _rand_inputs(1, H, N, L, "bf16", gated=False, mask_frac=0.5, seed=5)
+    plan = lsf.Plan(N, H, "bf16", L=L)
+    Kf = plan.precompute(to_dev(inp["k"], "bf16"))
+    u = to_dev(inp["u"], "bf16")
+    with pytest.raises(lsf.FFTConvError) as ei:
+        plan.forward(u, Kf, mask=torch.from_numpy(inp["mask"]).cuda())
+    assert ei.value.status == lsf.ERR_UNSUPPORTED
+    with pytest.raises(lsf.FFTConvError) as ei:
+        plan.export_rfft(Kf)
+    assert ei.value.status == lsf.ERR_UNSUPPORTED
+    assert plan.device_status() == 0
