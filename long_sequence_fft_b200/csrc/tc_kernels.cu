@@ -17,13 +17,17 @@
 // Product with the filter spectrum, then the mirror image with conjugate
 // factors (S3', S2', S1').
 //
-// Three modes use it (see Lay and pair_info):
+// Four modes use it (see Lay and pair_info):
 //   plain    N = 4096: x zero for t >= 4096 (S1 sees 16 nonzero j1), S1' emits
 //            only t < 4096;
 //   windows  N > 4096 with filters of at most 2049 taps: overlap-save windows
 //            of 4096 inputs, hop 2048;
 //   split    N = 8192 with longer filters: the 16384-point spectrum split by
-//            bin parity into two 8192-point transforms of all 8192 inputs.
+//            bin parity into two 8192-point transforms of all 8192 inputs;
+//   rows     the row pass of the staged path for longer sequences (M = R x
+//            8192): a tile is four complex fp16 workspace rows of one pair,
+//            each transformed, multiplied by its own filter row and
+//            transformed back in place (the column passes are SIMT kernels).
 //
 // Data layout.  One CTA tile = 4 pairs of batch rows (the two real sequences
 // of a pair are the real and imaginary parts of one complex sequence; the
@@ -45,7 +49,7 @@
 // Warp roles: warps 0..15 are epilogue warps (warp w serves lane quarter
 // w % 4 and the column slice w / 4); warps 16..19 issue the MMAs, one per SM
 // sub-partition.  A tile's work is a sequence of 64-column accumulator
-// chunks (44, or 48 in the split mode) cycled through a ring of four TMEM
+// chunks (44, or 48 in the split and rows modes) cycled through a ring of four TMEM
 // buffers; mbarriers hand chunks between the MMA warps and the epilogue
 // warps, and the epilogue hands a buffer back as soon as its TMEM loads have
 // landed.  The next tile's input is loaded while the current tile's last
@@ -166,8 +170,9 @@ struct TcArgs {
     const void* w;
     const void* v;
     void* y;
-    const __half2* Kh16;       // [H] rows of 8192 complex fp16 (see k16_index), unnormalised / scale
-    const float* Kscale;       // [H] per-channel scale of the fp16 rows
+    const __half2* Kh16;       // rows of 8192 complex fp16 (see k16_index): [H] unnormalised / scale;
+                               // split mode [2H] (even, odd bins); rows mode [H * R], spectrum / M / scale
+    const float* Kscale;       // the rows' scales: [H] per channel ([H * R] per row in rows mode)
     const uint8_t* mask;
     int64_t mask_h;
     int64_t B, H;
