@@ -83,9 +83,11 @@ typedef enum {
  * 2 x hop points when the filter is at most half the sequence: hop = the
  * power of two >= max(L, 16384); such a windowed plan rejects block masks
  * and fftconv_filter_to_rfft with FFTCONV_ERR_UNSUPPORTED, order 5 keeps the
- * full transform); other values are FFTCONV_ERR_UNSUPPORTED.  Synchronous: allocates the plan's device tables
- * (a few hundred KB) and its workspace (staged path only) on the current
- * device.  *out receives the plan, or NULL on failure. */
+ * full transform); other values are FFTCONV_ERR_UNSUPPORTED.  Synchronous:
+ * allocates the plan's device tables (a few hundred KB) and, on the staged
+ * paths, its workspace (about 64 MB for order 4, 512 MB for the tensor-core
+ * staged path; fftconv_workspace_bytes) on the current device.  *out receives
+ * the plan, or NULL on failure. */
 FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
                         fftconv_dtype_t dtype, int order);
 
