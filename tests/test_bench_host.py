@@ -1,0 +1,59 @@
+"""Host-side logic of the benchmark, on the CPU: the compulsory-byte formula
+behind `roofline.achieved` and the source-hash guard on the committed DRAM
+traffic figures behind `roofline.traffic`."""
+import hashlib
+import json
+import os
+
+import pytest
+
+import bench
+import workloads as W
+
+
+# Compulsory HBM bytes per call: E (s_u + s_y + gated (s_w + s_v)) + H bins 8,
+# bins = N + 1 (L + 1 for a partial filter, the kept bins when masked).  The
+# values are that formula evaluated by hand for each workload's shape.
+@pytest.mark.parametrize("name,expected", [
+    ("fp32_n1k", 8 * 1024 * 8 + 8 * 1025 * 8),                        # 131,136
+    ("gated_bf16_n4k", 64 * 768 * 4096 * 8 + 768 * 4097 * 8),         # 1,635,784,704
+    ("fp16_n32k", 8 * 256 * 32768 * 4 + 256 * 32769 * 8),             # 335,546,368
+    ("dna_bf16_n1m", (1 << 27) * 4 + 128 * ((1 << 20) + 1) * 8),      # 1,610,613,760
+    ("partial_bf16_n8k", 16 * 768 * 8192 * 8 + 768 * 2049 * 8),       # 817,895,424
+    ("sparse_bf16_n8k", 16 * 768 * 8192 * 8 + 768 * 2048 * 8),        # 817,889,280: round(0.25 * 8193) bins
+    ("dna_bf16_n4m_l1m", (1 << 27) * 4 + 32 * ((1 << 20) + 1) * 8),   # 805,306,624
+])
+def test_algorithmic_bytes(name, expected):
+    assert bench.algorithmic_bytes(W.WORKLOADS[name]) == expected
+
+
+def _fake_root(tmp_path, src_text, recorded_hash):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text(src_text)
+    entry = {"bytes_per_launch": 123, "source": "k.cu", "source_sha256": recorded_hash}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps({"w:path": entry}))
+    return str(tmp_path)
+
+
+def test_traffic_is_read_while_the_source_is_unchanged(tmp_path, monkeypatch):
+    src = "kernel source\n"
+    root = _fake_root(tmp_path, src, hashlib.sha256(src.encode()).hexdigest())
+    monkeypatch.setattr(bench, "ROOT", root)
+    assert bench.read_traffic("w:path")["bytes_per_launch"] == 123
+    assert bench.read_traffic("other:path") is None
+
+
+def test_traffic_is_dropped_once_the_source_changes(tmp_path, monkeypatch):
+    root = _fake_root(tmp_path, "kernel source, edited\n", hashlib.sha256(b"kernel source\n").hexdigest())
+    monkeypatch.setattr(bench, "ROOT", root)
+    assert bench.read_traffic("w:path") is None
+
+
+def test_committed_traffic_entries_name_existing_sources():
+    with open(os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as f:
+        d = json.load(f)
+    assert d
+    for key, ent in d.items():
+        assert os.path.isfile(os.path.join(bench.ROOT, ent["source"])), key
+        assert ent["bytes_per_launch"] == ent["dram_bytes_read"] + ent["dram_bytes_write"], key
+        assert "--clock-control none" in ent["command"], key
