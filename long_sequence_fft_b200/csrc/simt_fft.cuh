@@ -147,6 +147,33 @@ __device__ __forceinline__ void fwd_stage(float2* s, const float2* __restrict__ 
     }
 }
 
+// Forward stage 0 of a transform whose upper half is zero (x[p] = 0 for
+// p >= L/2, i.e. for the slowest digit j_0 >= R_0/2): reads only the nonzero
+// half of each butterfly's inputs and skips the first butterfly level
+// (Dft::run_half_input).  The zero half need not be stored.
+template <int LOGL, int TC, int NT>
+__device__ __forceinline__ void fwd_stage0_half_input(float2* s, const float2* __restrict__ tw, int twshift,
+                                                      int tid) {
+    constexpr int LB = Sched<LOGL>::bits(0);
+    constexpr int R = 1 << LB;
+    constexpr int SB = Sched<LOGL>::stride_bits(0);
+    constexpr int S = 1 << SB;
+    constexpr int G = S * TC;                    // stage 0: one butterfly per (r < S, column)
+    for (int g = tid; g < G; g += NT) {
+        const int col = (TC == 1) ? 0 : (g % TC);
+        const int r = (TC == 1) ? g : (g / TC);
+        float2 x[R];
+#pragma unroll
+        for (int j = 0; j < R / 2; ++j) x[j] = s[sidx<TC>(r + j * S, col)];
+#pragma unroll
+        for (int j = R / 2; j < R; ++j) x[j] = make_float2(0.f, 0.f);
+        Dft<R, -1>::run_half_input(x);
+        if constexpr (S > 1) twiddle_powers<R, false>(x, tw, r << (twshift + (LOGL - SB - LB)));
+#pragma unroll
+        for (int c = 0; c < R; ++c) s[sidx<TC>(r + c * S, col)] = x[c];
+    }
+}
+
 // Inverse of fwd_stage (conjugate twiddle, then inverse DFT).  Unnormalised.
 template <int LOGL, int I, int TC, int NT>
 __device__ __forceinline__ void inv_stage(float2* s, const float2* __restrict__ tw, int twshift, int tid) {

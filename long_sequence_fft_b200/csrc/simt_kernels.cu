@@ -491,12 +491,16 @@ staged_col_fwd_kernel(StagedArgs A) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[sidx<TC>(j, c4 + e)] = x[e];
     }
-    if constexpr (!WIN) {
-        for (int idx = tid; idx < (R / 2) * TC; idx += kColThreads)
-            s[sidx<TC>(R / 2 + idx / TC, idx % TC)] = make_float2(0.f, 0.f);
-    }
     __syncthreads();
-    fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    if constexpr (WIN) {
+        fwd_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    } else {
+        // the upper half (j >= R/2) is zero: the first stage reads only the
+        // lower half, so that half is never stored
+        fwd_stage0_half_input<LOGR, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+        __syncthreads();
+        fwd_stages<LOGR, 1, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
+    }
     // twiddle w_M^(c r) and store: each thread keeps one column r and walks
     // CPG consecutive c (a warp writes 32 consecutive r of one c).  The
     // twiddle comes from the table at every eighth c and as a product with
