@@ -52,7 +52,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
-// 1-D bulk copy global -> shared (TMA engine, no tensor map, no multicast);
+// 1-D bulk copy global -> shared (TMA engine, no tensor map, this CTA only);
 // completion is reported to the mbarrier as transaction bytes.  Addresses
 // 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
