@@ -63,8 +63,30 @@ typedef enum {
     FFTCONV_ERR_ALIGNMENT = -3,     /* pointer not 16-byte aligned            */
     FFTCONV_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed   */
     FFTCONV_ERR_OOM = -5,           /* plan allocation failed                 */
-    FFTCONV_ERR_TIMEOUT = -6        /* a bounded device wait gave up          */
+    FFTCONV_ERR_TIMEOUT = -6,       /* a bounded device wait gave up          */
+    FFTCONV_ERR_RANGE = -7          /* non-finite result: an fp16 intermediate
+                                       of a 16-bit tensor-core plan overflowed
+                                       (or an input held inf/NaN); see below  */
 } fftconv_status_t;
+
+/* Range of the 16-bit tensor-core paths (FFTCONV_PATH_TC_FUSED and
+ * FFTCONV_PATH_TC_STAGED).  Their transform intermediates are fp16 (largest
+ * finite value 65504); the fp32 paths (orders 1 and 4) keep fp32 throughout.
+ *   - Fused kernel (N = 4096, the N = 8192 parity split, overlap-save
+ *     windows): each unitary stage can grow a value by at most the number of
+ *     its inputs over the square root of its length, so with max|u*w| <= 90
+ *     no intermediate can overflow whatever the data and the filter.  Above
+ *     that it depends on the data: a constant (DC) input overflows the forward
+ *     transform near max|u*w| = 1450, zero-mean random data stays finite far
+ *     beyond.
+ *   - Staged tensor-core path (N >= 16384): no data-independent bound is
+ *     useful; inputs with a large mean overflow near max|u*w| = 10^3 for
+ *     R = 2N/8192 = 256 rows per column.
+ * An overflow is never silent: the kernels that write y check every
+ * convolution value (before the output gate v) and, if one is inf or NaN,
+ * set the plan's status word to FFTCONV_ERR_RANGE, which
+ * fftconv_device_status returns (and resets).  y then holds the non-finite
+ * values; rerun such inputs with an fp32 plan (order 4) or rescale u. */
 
 /* Kernel family a plan uses (fftconv_plan_path). */
 typedef enum {
@@ -178,16 +200,22 @@ FFTCONV_API int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, co
  *     16-byte aligned; w, v, block_mask may be NULL).
  *   K_f : the filter transform that fftconv_filter_precompute wrote for an
  *     order-4 plan with the same N, H and dtype (made once, by code that may
- *     allocate, e.g. when the filter is loaded).
+ *     allocate, e.g. when the filter is loaded).  It is read as that layout,
+ *     H x 2N complex fp32 values: a K_f from a plan of any other order is both
+ *     the wrong layout and too short, so the call would read past its end.
  *   N   : power of two, 256 <= N <= 2^20 (2N complex fp32 values must fit the
  *     scratch); larger N returns FFTCONV_ERR_UNSUPPORTED with the limit in
  *     fftconv_last_error().
- * Calls no cudaMalloc/cudaFree and allocates nothing else.  The first call on
- * a device resolves the device addresses of the static arrays
- * (cudaGetSymbolAddress), so that first call should come before any stream
- * capture.  All calls share the scratch arrays and each call overwrites them,
+ * Calls no cudaMalloc/cudaFree and allocates nothing else.  Every call looks up
+ * the device addresses of the static arrays in the calling thread's current
+ * context (cudaGetSymbolAddress); the first call on a device may load the
+ * library's device code there, so make that first call before any stream
+ * capture.  The passes' twiddle tables live in the static arrays too and are
+ * refilled only when N or the context differs from the previous call on that
+ * device.  All calls share these arrays and each call overwrites the scratch,
  * so calls whose execution overlaps on the GPU (other streams, other host
- * threads) race; serialise them. */
+ * threads) race; serialise them (a call also relies on the tables an earlier
+ * call of the same N filled having been written). */
 FFTCONV_API int fftconv_forward_noalloc(const void* u, const void* K_f, void* y, int64_t B, int64_t H,
                                         int64_t N, fftconv_dtype_t dtype, const void* w, const void* v,
                                         const uint8_t* block_mask, int64_t mask_h,
@@ -200,8 +228,10 @@ FFTCONV_API int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, flo
                            fftconv_stream_t stream);
 
 /* Synchronise `stream` and return the plan's device status word:
- * FFTCONV_OK, or FFTCONV_ERR_TIMEOUT if a bounded device-side wait gave up
- * since the last call (the word is reset to OK by this call). */
+ * FFTCONV_OK, FFTCONV_ERR_TIMEOUT if a bounded device-side wait gave up, or
+ * FFTCONV_ERR_RANGE if a 16-bit tensor-core forward produced non-finite
+ * values (see the range note above), since the last call (the word is reset
+ * to OK by this call). */
 FFTCONV_API int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream);
 
 /* Self-test of the device-side failure path (the pages describe none; this

@@ -29,7 +29,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 F32, F16, BF16 = 0, 1, 2
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_OOM, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_OOM, ERR_TIMEOUT, ERR_RANGE = 0, -1, -2, -3, -4, -5, -6, -7
 PATH_SIMT_FUSED, PATH_SIMT_STAGED, PATH_TC_FUSED, PATH_TC_STAGED = 1, 2, 3, 4
 PATH_NAMES = {PATH_SIMT_FUSED: "simt_fused", PATH_SIMT_STAGED: "simt_staged", PATH_TC_FUSED: "tc_fused",
               PATH_TC_STAGED: "tc_staged"}

@@ -114,6 +114,7 @@ const char* fftconv_status_string(int status) {
         case FFTCONV_ERR_CUDA: return "CUDA error";
         case FFTCONV_ERR_OOM: return "out of device memory";
         case FFTCONV_ERR_TIMEOUT: return "device wait timed out";
+        case FFTCONV_ERR_RANGE: return "non-finite result (fp16 intermediate out of range)";
         default: return "unknown status";
     }
 }
@@ -491,7 +492,10 @@ int fftconv_device_status(fftconv_plan_t plan, fftconv_stream_t stream) {
     if (host != 0) {
         int zero = 0;
         cudaMemcpy(plan->p.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
-        return fail(host, "a bounded device wait timed out");
+        return fail(host, host == FFTCONV_ERR_RANGE
+                              ? "a forward call produced non-finite values: an fp16 intermediate overflowed "
+                                "(or an input held inf/NaN)"
+                              : "a bounded device wait timed out");
     }
     return FFTCONV_OK;
 }

@@ -157,6 +157,19 @@ struct Dft<1, DIR> {
 
 // ------------------------------------------------------- status word ---
 
-enum : int { kStatusOk = 0, kStatusTimeout = -6 };
+enum : int { kStatusOk = 0, kStatusTimeout = -6, kStatusRange = -7 };
+
+// Non-finite detector for the 16-bit tensor-core paths, whose intermediates
+// are fp16: acc stays 0 while every value folded in is finite and becomes NaN
+// once one is inf or NaN (0 * inf and 0 * NaN are NaN).  Inline PTX keeps the
+// compiler from folding x * 0 away.
+__device__ __forceinline__ void nonfinite_fold(float& acc, float x) {
+    asm("fma.rn.f32 %0, %1, 0f00000000, %0;" : "+f"(acc) : "f"(x));
+}
+// Record FFTCONV_ERR_RANGE in the status word if acc saw a non-finite value
+// (an earlier timeout is not overwritten).
+__device__ __forceinline__ void nonfinite_report(float acc, int* status) {
+    if (acc != acc) atomicCAS(status, 0, kStatusRange);
+}
 
 }  // namespace fftconv

@@ -42,15 +42,29 @@ static __device__ __align__(256) float2 g_twC[int64_t(1) << kMaxLogC];
 static __device__ __align__(256) float2 g_twLo[int64_t(1) << ((kMaxLogM + 1) / 2)];
 static __device__ __align__(256) float2 g_twHi[int64_t(1) << ((kMaxLogM + 1) / 2)];
 
+// Device addresses of the static arrays in the calling thread's current
+// context.  They are looked up on every call (a host-side query that
+// allocates nothing once the module is loaded): a cached address would go
+// stale after cudaDeviceReset or under a context other than the one it was
+// taken in, and the passes would then write through it.
 struct DeviceSymbols {
-    bool ready = false;
     float2* scratch = nullptr;
     float2* twC = nullptr;
     float2* twLo = nullptr;
     float2* twHi = nullptr;
 };
-DeviceSymbols g_symbols[kMaxDevices];
-std::mutex g_symbols_mutex;
+
+// Which twiddle tables the static arrays hold, per device: the transform
+// length they were filled for and the context that filled them (a context id
+// from the driver is unique for the life of the process).  A call refills
+// them only when either differs.
+struct ResidentTables {
+    unsigned long long ctx_id = 0;
+    int logM = 0;
+    float2* twC = nullptr;
+};
+ResidentTables g_resident[kMaxDevices];
+std::mutex g_resident_mutex;
 
 int noalloc_fail(int status, const char* fmt, ...) {
     char buf[400];
@@ -83,26 +97,45 @@ __global__ void fill_twiddles(float2* twC, int64_t C, float2* lo, int64_t nlo, f
     }
 }
 
-// Resolve the device addresses of the static arrays for the current device
+// Resolve the device addresses of the static arrays for the current context
 // (host code cannot use the array names as device pointers).
-int device_symbols(DeviceSymbols** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+int device_symbols(DeviceSymbols* s, int* dev) {
+    cudaError_t e = cudaGetDevice(dev);
     if (e != cudaSuccess) return noalloc_fail(FFTCONV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return noalloc_fail(FFTCONV_ERR_UNSUPPORTED, "device index %d", dev);
-    std::lock_guard<std::mutex> lock(g_symbols_mutex);
-    DeviceSymbols& s = g_symbols[dev];
-    if (!s.ready) {
-        e = cudaGetSymbolAddress((void**)&s.scratch, g_scratch);
-        if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s.twC, g_twC);
-        if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s.twLo, g_twLo);
-        if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s.twHi, g_twHi);
-        if (e != cudaSuccess)
-            return noalloc_fail(FFTCONV_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-        s.ready = true;
-    }
-    *out = &s;
+    if (*dev < 0 || *dev >= kMaxDevices) return noalloc_fail(FFTCONV_ERR_UNSUPPORTED, "device index %d", *dev);
+    e = cudaGetSymbolAddress((void**)&s->scratch, g_scratch);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s->twC, g_twC);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s->twLo, g_twLo);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&s->twHi, g_twHi);
+    if (e != cudaSuccess) return noalloc_fail(FFTCONV_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     return FFTCONV_OK;
+}
+
+// Unique id of the calling thread's current context, through the driver
+// entry points the runtime exposes (no link-time dependency on the driver
+// library).  Returns false if the driver cannot say: the tables are then
+// refilled on every call.
+bool current_context_id(unsigned long long* id) {
+    using GetCurrent = int (*)(void**);
+    using GetId = int (*)(void*, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1) == cudaSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess && q2 == cudaDriverEntryPointSuccess) {
+            get_current = (GetCurrent)f1;
+            get_id = (GetId)f2;
+        }
+    });
+    if (!get_current || !get_id) return false;
+    void* ctx = nullptr;
+    if (get_current(&ctx) != 0 || !ctx) return false;
+    return get_id(ctx, id) == 0 && *id != 0;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -138,11 +171,15 @@ extern "C" int fftconv_forward_noalloc(const void* u, const void* K_f, void* y, 
     if (block_mask && mask_h != 1 && mask_h != H)
         return noalloc_fail(FFTCONV_ERR_INVALID_ARG, "mask_h must be 1 or H");
     const size_t bytes = (size_t)B * (size_t)H * (size_t)N * (dtype == FFTCONV_F32 ? 4 : 2);
-    if (overlap(y, bytes, u, bytes) || overlap(y, bytes, w, bytes) || overlap(y, bytes, v, bytes))
+    // K_f is the order-4 layout: H rows of 2N complex fp32 values
+    const size_t kf_bytes = (size_t)H * (size_t)(2 * N) * sizeof(float2);
+    if (overlap(y, bytes, u, bytes) || overlap(y, bytes, w, bytes) || overlap(y, bytes, v, bytes) ||
+        overlap(y, bytes, K_f, kf_bytes))
         return noalloc_fail(FFTCONV_ERR_INVALID_ARG, "y overlaps an input");
 
-    DeviceSymbols* sym = nullptr;
-    int rc = device_symbols(&sym);
+    DeviceSymbols sym;
+    int dev = 0;
+    int rc = device_symbols(&sym, &dev);
     if (rc != FFTCONV_OK) return rc;
 
     // A plan-shaped description on the stack pointing at the static arrays;
@@ -158,19 +195,37 @@ extern "C" int fftconv_forward_noalloc(const void* u, const void* K_f, void* y, 
     p.logR = logM - p.logC;
     p.logTab = p.logC;
     p.twSplit = (logM + 1) / 2;
-    p.tw = sym->twC;
-    p.twLo = sym->twLo;
-    p.twHi = sym->twHi;
-    p.work = sym->scratch;
+    p.tw = sym.twC;
+    p.twLo = sym.twLo;
+    p.twHi = sym.twHi;
+    p.work = sym.scratch;
     p.chunkPairs = kScratchElems / p.M;
     p.workBytes = (size_t)kScratchElems * sizeof(float2);
 
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t C = int64_t(1) << p.logC;
     const int64_t nlo = int64_t(1) << p.twSplit, nhi = p.M >> p.twSplit;
-    fill_twiddles<<<64, 256, 0, s>>>(p.tw, C, p.twLo, nlo, p.twHi, nhi, p.M, p.twSplit);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return noalloc_fail(FFTCONV_ERR_CUDA, "twiddle fill: %s", cudaGetErrorString(e));
+    {
+        // refill the twiddle tables only when N or the context changed since
+        // the last fill on this device (the fill is ordered on `s` before the
+        // passes; earlier calls' passes read tables of the same N)
+        unsigned long long ctx = 0;
+        const bool known = current_context_id(&ctx);
+        std::lock_guard<std::mutex> lock(g_resident_mutex);
+        ResidentTables& r = g_resident[dev];
+        if (!known || r.ctx_id != ctx || r.logM != logM || r.twC != p.tw) {
+            fill_twiddles<<<64, 256, 0, s>>>(p.tw, C, p.twLo, nlo, p.twHi, nhi, p.M, p.twSplit);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) {
+                r = ResidentTables{};
+                return noalloc_fail(FFTCONV_ERR_CUDA, "twiddle fill: %s", cudaGetErrorString(e));
+            }
+            r.ctx_id = known ? ctx : 0;
+            r.logM = known ? logM : 0;
+            r.twC = p.tw;
+        }
+    }
+    cudaError_t e;
     ForwardArgs a{u, w, v, y, K_f, block_mask, block_mask ? mask_h : 0, B};
     e = simt_staged_forward(p, a, s);
     if (e != cudaSuccess) return noalloc_fail(FFTCONV_ERR_CUDA, "staged passes: %s", cudaGetErrorString(e));

@@ -419,6 +419,10 @@ struct StagedArgs {
     // by kscale[h * R + c] * rout
     const float* kscale;
     float rin, rout;
+    // the plan's status word; the inverse column passes of the half-precision
+    // workspace record FFTCONV_ERR_RANGE there when the convolution came out
+    // non-finite (an fp16 intermediate overflowed)
+    int* status;
     // overlap-save windows (column kernels with WIN): unit u of the chunk is
     // window u % nwin of pair u / nwin; the window's position t is sequence
     // position (w - 1) winHop + t, inputs before 0 read as zero, and only its
@@ -607,13 +611,18 @@ staged_col_inv_kernel(StagedArgs A) {
     inv_stages<LOGR, 0, Sched<LOGR>::K, TC, kColThreads>(s, A.tw, A.logC - LOGR, tid);
     // outputs: the first half (t < N), or a window's second half
     constexpr int J0 = WIN ? R / 2 : 0;
+    float nf = 0.f;
     for (int idx = tid; idx < (R / 2) * (TC / 4); idx += kColThreads) {
         const int j = J0 + idx / (TC / 4), c4 = 4 * (idx % (TC / 4));
         float2 z[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) z[e] = s[sidx<TC>(j, c4 + e)];
+        for (int e = 0; e < 4; ++e) {
+            z[e] = s[sidx<TC>(j, c4 + e)];
+            if constexpr (WS16) { nonfinite_fold(nf, z[e].x); nonfinite_fold(nf, z[e].y); }
+        }
         io.store4((int)(U.base + j * C + col0 + c4), z);
     }
+    if constexpr (WS16) nonfinite_report(nf, A.status);
 }
 
 // Column passes for short columns (R <= 8) without shared memory: a thread
@@ -728,12 +737,18 @@ staged_col_inv_reg_kernel(StagedArgs A) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) Dft<R, +1>::run(x[e]);
     // outputs: the first half (t < N), or a window's second half
+    float nf = 0.f;
 #pragma unroll
     for (int jj = 0; jj < R / 2; ++jj) {
         const int j = (WIN ? R / 2 : 0) + jj;
         const float2 q[4] = {x[0][j], x[1][j], x[2][j], x[3][j]};
+        if constexpr (WS16) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { nonfinite_fold(nf, q[e].x); nonfinite_fold(nf, q[e].y); }
+        }
         io.store4((int)(U.base + j * C + r0), q);
     }
+    if constexpr (WS16) nonfinite_report(nf, A.status);
 }
 
 template <int LOGR, typename T, bool WS16, bool WIN>
@@ -851,6 +866,7 @@ cudaError_t tc_staged_forward_t(const Plan& p, const ForwardArgs& fa, cudaStream
     // the inputs' range; the unitary 8192-point pair of the row pass leaves
     // 1/8192, undone with the scale by rout
     A.kscale = (const float*)((const uint8_t*)fa.Kf + tc_staged_spectrum_bytes(p));
+    A.status = p.status;
     A.rin = std::ldexp(1.0f, -(p.logR / 2));
     A.rout = (float)C * std::ldexp(1.0f, p.logR / 2);
     // workspace units: pairs, or (pair, window) with overlap-save windows

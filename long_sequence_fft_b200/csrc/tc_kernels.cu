@@ -656,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 
         int iter = 0;
         bool ok = true;
+        float nf = 0.f;          // non-finite detector over the outputs (fp16 range)
         if (first_unit<MODE>() < a.nunits) {
             load_tile(first_unit<MODE>(), 0);
             load_tile(first_unit<MODE>(), 1);
@@ -994,6 +995,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                         sc *= 0.5f;
                                     }
                                     a0 *= sc; a1 *= sc; b0 *= sc; b1 *= sc;
+                                    nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
+                                    nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
                                     if (a.v) {
                                         const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
                                         a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
@@ -1015,6 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                 output_pass(std::false_type{});
             }
         }
+        if constexpr (MODE != kModeRows) nonfinite_report(nf, a.status);
     }
 
     tc_fence_before();

@@ -1,0 +1,214 @@
+"""GPU parity of the tensor-core paths beyond the basic cases.
+
+1. Element-wise comparison with the fp64 oracle at sizes that give every CTA
+   of the persistent tensor-core kernel at least three tiles (148 CTAs at
+   most: the "next tile loaded during the current tile's last stages" path and
+   the split mode's parked z_even are exercised many times per CTA), in every
+   mode the kernel has: plain (N = 4096), overlap-save windows (partial
+   filters), the N = 8192 parity split (masked) and the staged path's row
+   pass.  The launch configuration is the plan's own, as in the benchmark.
+2. Closed forms the convolution must reproduce on every tensor-core mode
+   (exact results of the definition "FlashFFTConv: Efficient Convolutions for
+   Long Sequences with Tensor Cores", summary and "Approach", with the
+   dtype-rounded inputs): delta and shifted-delta filters give the (gated,
+   shifted) input back; u = 1 gives the running sum of the filter (t + 1 for
+   k = 1, a geometric sum for k = r^s); an all-zero block mask gives exactly
+   zero and an all-ones mask reproduces the unmasked call bit for bit.
+3. The fp16 range guard: inputs at the documented bound stay finite with
+   status OK, inputs beyond it set FFTCONV_ERR_RANGE instead of returning
+   inf/NaN silently.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from parity_util import assert_close, run_cuda
+
+pytestmark = pytest.mark.gpu
+
+SMS = 148         # CTAs of the persistent tensor-core kernel (B200)
+
+
+def _inputs(B, H, N, L, dtype, gated, mask_frac=0.0, seed=0, shared_mask=False):
+    rng = np.random.default_rng(seed)
+    out = {"u": W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype),
+           "k": W.round_to(rng.standard_normal((H, L), dtype=np.float32) / np.float32(np.sqrt(L)), dtype),
+           "w": None, "v": None, "mask": None}
+    if gated:
+        out["w"] = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+        out["v"] = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    if mask_frac > 0:
+        out["mask"] = (rng.random((1 if shared_mask else H, N // 32)) >= mask_frac).astype(np.uint8)
+    return out
+
+
+def _compare(inp, dtype, what, order=0, path="tc_fused"):
+    y, plan = run_cuda(inp, dtype, order=order)
+    assert plan.path_name == path, (what, plan.path_name)
+    ref = oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"], mask=inp["mask"])
+    e = assert_close(y, ref, dtype, what)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    # the literal max-abs error beside the bound it is held to
+    print(f"{what}: rel_l2={e:.2e} max_abs={np.max(np.abs(y - ref)):.3e} (2e-2*rms={2e-2 * rms:.3e})")
+    return y
+
+
+# ------------------------------------------------- many tiles per CTA ---
+
+def test_plain_mode_three_tiles_per_cta():
+    B, H, N = 16, 256, 4096
+    tiles = H * ((B // 2 + 3) // 4)                     # 4 pairs of one channel per tile
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, N, "bf16", gated=True, seed=1), "bf16", f"plain {tiles} tiles")
+
+
+def test_plain_mode_ragged_batch_many_tiles():
+    # B = 13: six full pairs and an unpaired row per channel, two tiles per
+    # channel, the second one ragged
+    B, H, N = 13, 240, 4096
+    tiles = H * (((B + 1) // 2 + 3) // 4)
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, N, "f16", gated=False, seed=2), "f16", f"plain ragged {tiles} tiles")
+
+
+def test_windows_mode_three_tiles_per_cta():
+    B, H, N, L = 16, 80, 8192, 2048
+    tiles = H * (N // 2048 - 1) * ((B // 2 + 3) // 4)
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, L, "bf16", gated=True, seed=3), "bf16", f"windows {tiles} tiles")
+
+
+def test_split_mode_three_tiles_per_cta():
+    B, H, N = 16, 128, 8192
+    groups = H * ((B // 2 + 3) // 4)
+    assert 2 * groups >= 3 * SMS                        # even and odd tile per group
+    _compare(_inputs(B, H, N, N, "bf16", gated=True, mask_frac=0.75, seed=4, shared_mask=True), "bf16",
+             f"split {2 * groups} tiles")
+
+
+def test_rows_mode_three_tiles_per_cta():
+    B, H, N = 8, 64, 32768
+    units = H * (B // 2) * ((2 * N // 8192) // 4)       # rows mode: 4 rows of one pair per tile
+    assert units >= 3 * SMS
+    _compare(_inputs(B, H, N, N, "f16", gated=True, seed=5), "f16", f"rows {units} tiles", order=0,
+             path="tc_staged")
+
+
+# ------------------------------------------------------- closed forms ---
+
+MODES = [  # (name, N, L, order, path)
+    ("plain", 4096, 4096, 0, "tc_fused"),
+    ("windows", 8192, 2048, 0, "tc_fused"),
+    ("split", 8192, 8192, 0, "tc_fused"),
+    ("rows", 16384, 16384, 5, "tc_staged"),
+]
+
+
+def _run(u, k, dtype, order, path, w=None, v=None, mask=None):
+    inp = {"u": u, "k": k, "w": w, "v": v, "mask": mask}
+    y, plan = run_cuda(inp, dtype, order=order)
+    assert plan.path_name == path
+    return y
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("name,N,L,order,path", MODES)
+def test_delta_filters_return_the_input(name, N, L, order, path, dtype):
+    rng = np.random.default_rng(N + L)
+    B, H = 3, 2
+    u = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    w = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    v = W.round_to(rng.standard_normal((B, H, N), dtype=np.float32), dtype)
+    x = u.astype(np.float64) * w * v
+    k = np.zeros((H, L), np.float32)
+    k[:, 0] = 1.0
+    y = _run(u, k, dtype, order, path, w=w, v=v)
+    assert_close(y, x, dtype, f"{name}: delta filter")
+    # shifted delta (a different shift per channel): y[t] = (u w)[t - d] v[t]
+    d = [min(5, L - 1), min(L - 1, 1500)]
+    k = np.zeros((H, L), np.float32)
+    ref = np.zeros((B, H, N))
+    for h in range(H):
+        k[h, d[h]] = 1.0
+        ref[:, h, d[h]:] = (u[:, h, :N - d[h]].astype(np.float64) * w[:, h, :N - d[h]]) * v[:, h, d[h]:]
+    y = _run(u, k, dtype, order, path, w=w, v=v)
+    assert_close(y, ref, dtype, f"{name}: shifted delta")
+
+
+@pytest.mark.parametrize("name,N,L,order,path", MODES)
+def test_running_sums_of_the_filter(name, N, L, order, path):
+    """u = 1: y[t] = sum_{s <= min(t, L-1)} k[s]; k = 1 gives t + 1 (capped at
+    L for a partial filter) and k = r^s the geometric sum."""
+    dtype = "f16" if N > 4096 else "bf16"
+    B, H = 2, 2
+    u = np.ones((B, H, N), np.float32)
+    t = np.arange(N)
+    k1 = np.ones((H, L), np.float32)
+    y = _run(u, k1, dtype, order, path)
+    ref = np.broadcast_to(np.minimum(t, L - 1) + 1.0, (B, H, N))
+    assert_close(y, ref, dtype, f"{name}: u = k = 1")
+    r = np.array([0.999, 0.99], np.float64)
+    kg = W.round_to((r[:, None] ** np.arange(L)[None, :]).astype(np.float32), dtype)
+    y = _run(u, kg, dtype, order, path)
+    cs = np.cumsum(kg.astype(np.float64), axis=1)        # the rounded taps' running sums
+    ref = np.broadcast_to(cs[:, np.minimum(t, L - 1)][None], (B, H, N))
+    assert_close(y, ref, dtype, f"{name}: geometric filter")
+    # and the geometric closed form itself, within the rounding of the taps
+    closed = (1 - r[:, None] ** (np.minimum(t, L - 1)[None, :] + 1)) / (1 - r[:, None])
+    assert np.max(np.abs(cs[:, np.minimum(t, L - 1)] - closed) / closed) < 5e-3
+
+
+@pytest.mark.parametrize("name,N,order,path", [("split", 8192, 0, "tc_fused"), ("rows", 16384, 5, "tc_staged")])
+def test_zero_and_full_masks_on_tensor_cores(name, N, order, path):
+    inp = _inputs(3, 2, N, N, "bf16", gated=True, seed=N)
+    inp["mask"] = np.zeros((1, N // 32), np.uint8)
+    y, plan = run_cuda(inp, "bf16", order=order)
+    assert plan.path_name == path
+    assert np.max(np.abs(y)) == 0.0, f"{name}: all-zero mask must give exact zeros"
+    inp["mask"] = np.full((2, N // 32), 9, np.uint8)     # any nonzero byte keeps the block
+    y1, _ = run_cuda(inp, "bf16", order=order)
+    inp["mask"] = None
+    y2, _ = run_cuda(inp, "bf16", order=order)
+    assert np.array_equal(y1, y2), f"{name}: all-ones mask must equal the unmasked call"
+
+
+# --------------------------------------------------------- fp16 range ---
+
+def _status_after(u, k, dtype, order, N, L):
+    import long_sequence_fft_b200 as lsf
+    import torch
+    from parity_util import to_dev
+    plan = lsf.Plan(N, u.shape[1], dtype, order=order, L=L)
+    Kf = plan.precompute(to_dev(k, dtype))
+    y = plan.forward(to_dev(u, dtype), Kf)
+    torch.cuda.synchronize()
+    status = lsf.library().fftconv_device_status(plan.handle, None)
+    again = lsf.library().fftconv_device_status(plan.handle, None)
+    return y.float().cpu().numpy().astype(np.float64), status, again, plan
+
+
+@pytest.mark.parametrize("name,N,L,order,path,edge,beyond", [
+    ("plain", 4096, 4096, 0, "tc_fused", 90.0, 1500.0),
+    ("windows", 8192, 2048, 0, "tc_fused", 90.0, 1500.0),
+    ("split", 8192, 8192, 0, "tc_fused", 90.0, 3000.0),
+    ("rows", 16384, 16384, 5, "tc_staged", 90.0, 2000.0),
+])
+def test_fp16_range_guard(name, N, L, order, path, edge, beyond):
+    import long_sequence_fft_b200 as lsf
+    B, H = 2, 1
+    k = np.zeros((H, L), np.float32)
+    k[:, 0] = 1.0                                        # delta: y = u, flat spectrum
+    # at the documented data-independent bound: finite, status OK, exact result
+    u = np.full((B, H, N), edge, np.float32)
+    y, status, again, plan = _status_after(u, k, "bf16", order, N, L)
+    assert plan.path_name == path
+    assert status == lsf.OK and np.isfinite(y).all()
+    assert_close(y, u.astype(np.float64), "bf16", f"{name}: constant {edge} at the bound")
+    # a constant input far beyond it overflows the fp16 forward transform: the
+    # call reports FFTCONV_ERR_RANGE (and the status word resets on read)
+    u = np.full((B, H, N), beyond, np.float32)
+    y, status, again, _ = _status_after(u, k, "bf16", order, N, L)
+    assert status == lsf.ERR_RANGE, (name, status)
+    assert again == lsf.OK
+    assert not np.isfinite(y).all()
