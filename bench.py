@@ -19,7 +19,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -34,15 +33,46 @@ METRIC = "FFT-conv B*H*N elems/s and achieved % of roofline (1xB200)"
 UNIT = "elems/s"
 
 
-def algorithmic_bytes(w: W.Workload) -> int:
+TC_PATHS = ("tc_fused", "tc_staged")
+
+
+def kf_bytes_per_bin(path: str) -> int:
+    """Stored width of one filter-spectrum bin: complex fp16 (4 B) on the
+    tensor-core paths, complex fp32 (8 B) on the fp32-lane paths."""
+    return 4 if path in TC_PATHS else 8
+
+
+def algorithmic_bytes(w: W.Workload, path: str = "simt_fused") -> int:
     """Compulsory HBM bytes of one forward call: read u (and w, v), write y,
-    read the filter spectrum once (N+1 complex fp32 bins per channel)."""
+    read the filter spectrum once at its stored width (N+1 bins per channel;
+    L+1 for a partial filter; the kept bins for a block-sparse one)."""
     esz = 4 if w.dtype == "f32" else 2
     per_elem = 2 * esz + (2 * esz if w.gated else 0)
     bins = (w.L + 1) if w.L < w.N else (w.N + 1)
     if w.sparsity > 0:
         bins = int(round((1 - w.sparsity) * (w.N + 1)))
-    return w.elems * per_elem + w.H * bins * 8
+    return w.elems * per_elem + w.H * bins * kf_bytes_per_bin(path)
+
+
+def mma_flops_per_elem(w: W.Workload, path: str):
+    """(schedule, flops per output element) of the tensor-core contractions the
+    path issues, counted from the instruction shapes (complex values as real
+    pairs: 2 flops per real multiply-add).  The 8192-point engine is
+    32 x 32 x 8.  A zero-padded transform of 4096 inputs whose first 4096
+    outputs are kept (N = 4096, and each overlap-save window) issues
+    8*32 + 16*(32 + 8) = 896 per point of its window; a transform of all 8192
+    inputs and outputs (the N = 8192 parity split, the staged row pass)
+    16*(32 + 32 + 8) = 1152 per point.  fp32-lane paths issue none."""
+    if path == "tc_fused":
+        if w.N == 4096:
+            return "32x32x8", 896.0
+        if w.N == 8192 and w.L > 2049:
+            return "32x32x8 (x2 parity halves)", 1152.0
+        nwin = w.N // 2048 - 1
+        return "32x32x8 windows", 896.0 * nwin * 4096 / w.N
+    if path == "tc_staged":
+        return "columns on fp32 lanes x rows 32x32x8", 1152.0
+    return "fp32 lanes", 0.0
 
 
 def read_peaks():
@@ -77,75 +107,89 @@ def read_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 20 ms while running."""
+    """SM clock, power and clock-event reasons of the benchmark's GPU, sampled
+    through NVML every `interval` seconds on a background thread while the
+    timed region runs (the timed work runs in ctypes calls and CUDA
+    synchronisation, which release the interpreter lock)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"bench_clocks_{os.getpid()}.csv")
+    def __init__(self, torch_device: int, interval: float = 0.001):
+        self.dev = torch_device
+        self.interval = interval
+        self.samples = []
+        self.max_mhz = None
+        self.thread = None
+        self.error = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self, h, stop):
+        import pynvml
+        while not stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, rs, pw))
+            except Exception as e:  # pragma: no cover - driver-side failure
+                self.error = repr(e)
+                return
+            stop.wait(self.interval)
 
     def __enter__(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "20"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._run, args=(h, self.stop), daemon=True)
+            self.thread.start()
+        except Exception as e:
+            self.error = repr(e)
+            self.thread = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         return False
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return None
-        sm, smmax, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smmax = max(smmax, float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() in ("active", "1"):
-                        reasons.add(n)
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smmax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return None if self.error is None else {"error": self.error}
+        reasons = set()
+        for _, rs, _ in self.samples:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "power_w_max": max(x[2] for x in self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------- oracle ---
 
-def time_oracle(w: W.Workload, target_s: float = 10.0):
+def time_oracle(w: W.Workload, target_s: float = 10.0, cores: int = 0, H: int = 64):
     """The fp64 oracle on a bounded sample of the workload: a block of whole
-    sequences (b, h) of the workload's shape, convolved repeatedly on all host
-    cores until about `target_s` seconds have passed.  Returns (elems/s,
-    cores, description)."""
+    sequences (b, h) of the workload's shape, convolved repeatedly on `cores`
+    host threads (0: all) until about `target_s` seconds have passed.  Returns
+    (elems/s, threads, description)."""
     import oracle
-    cores = os.cpu_count() or 1
-    sub = w.with_shape(B=min(w.B, 16), H=min(w.H, 64))
+    cores = cores or (os.cpu_count() or 1)
+    sub = w.with_shape(B=min(w.B, 16), H=min(w.H, H))
     inp = W.make_all(sub)
     done, t0 = 0, time.perf_counter()
     while True:
@@ -195,6 +239,71 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- main ---
 
+# Workloads timed beside the headline (one GPU): every other configuration
+# of the hot path, each for at least about a second of steps.
+SIDE_WORKLOADS = ("fp32_n1k", "fp16_n32k", "dna_bf16_n1m", "partial_bf16_n8k", "sparse_bf16_n8k",
+                  "gated_bf16_n1k", "bf16_n1k", "dna_bf16_n4m_l1m")
+
+
+def roofline_entry(w: W.Workload, path: str, ms_per_step: float, hbm_peak: float, tc_peak: float):
+    """Roofline of one workload: T_roof = max(compulsory bytes at the measured
+    HBM bandwidth, issued MMA flops at the measured dense bf16/fp16 peak);
+    frac = T_roof / T_measured, and the HBM-only fraction beside it."""
+    abytes = algorithmic_bytes(w, path)
+    sched, fpe = mma_flops_per_elem(w, path)
+    t_hbm = abytes / (hbm_peak * 1e9)
+    t_mma = fpe * w.elems / (tc_peak * 1e12)
+    t = ms_per_step * 1e-3
+    return {"algorithmic_bytes": abytes, "achieved_gbs": abytes / t / 1e9, "hbm_frac": t_hbm / t,
+            "mma_schedule": sched, "mma_flops_per_elem": fpe, "t_hbm_us": t_hbm * 1e6, "t_mma_us": t_mma * 1e6,
+            "frac": max(t_hbm, t_mma) / t, "bound": "hbm" if t_hbm >= t_mma else "tensor"}
+
+
+def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: float = 1.0):
+    """One configuration end to end on the device: seeded inputs copied to HBM,
+    plan, filter precompute, 3 warm-up calls, then enough calls for about
+    `min_seconds`, timed with CUDA events on the launching stream while NVML
+    samples the clocks."""
+    import torch
+    import long_sequence_fft_b200 as lsf
+    w = W.WORKLOADS[name]
+    inp = W.make_all(w)
+    dt = W.torch_dtype(w.dtype)
+    dev = lambda a: None if a is None else torch.from_numpy(a).to(dt).cuda()
+    u, k, g, v = dev(inp["u"]), dev(inp["k"]), dev(inp["w"]), dev(inp["v"])
+    del inp["u"], inp["w"], inp["v"]
+    mask = torch.from_numpy(inp["mask"]).cuda() if inp["mask"] is not None else None
+    plan = lsf.Plan(w.N, w.H, w.dtype, L=w.L)
+    Kf = plan.precompute(k)
+    y = torch.empty_like(u)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    steps = int(min(20000, max(10, min_seconds / max(e0.elapsed_time(e1) * 1e-3, 1e-6))))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    status = plan.device_status()
+    entry = {"B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated, "io_dtype": w.dtype,
+             "sparsity": w.sparsity, "path": plan.path_name, "steps": steps, "ms_per_step": ms,
+             "value": w.elems / (ms * 1e-3), "unit": UNIT, "device_status": status,
+             "clocks": clk.summary()}
+    entry.update(roofline_entry(w, plan.path_name, ms, hbm_peak, tc_peak))
+    del u, k, g, v, y, Kf, plan
+    torch.cuda.empty_cache()
+    return entry
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -204,11 +313,13 @@ def main():
     ap.add_argument("--workload", default=W.BENCH_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--order", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip timing the other configurations beside the headline")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--B", type=int, default=None,
                     help="override the batch size (small cases for profiling; not a bench number)")
     ap.add_argument("--profile", action="store_true",
-                    help="profiling run: skip the host-buffer and CPU-baseline legs")
+                    help="profiling run: skip the host-buffer, CPU-baseline and side-workload legs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -313,11 +424,10 @@ def main():
     esz = uh.element_size()
     h2d = w.elems * esz * (1 + (gh is not None) + (vh is not None)) + (0 if mh is None else mh.numel())
     d2h = w.elems * esz
-    del staging, uh, gh, vh, yh
+    del staging, uh, gh, vh, yh, inp
 
     hbm_peak, tc_peak, peak_kind = read_peaks()
-    abytes = algorithmic_bytes(w)
-    achieved = abytes / (ms_per_step * 1e-3) / 1e9          # per launch-group (one forward)
+    roof = roofline_entry(w, plan.path_name, ms_per_step, hbm_peak, tc_peak)
     kernel_key = f"{w.name}:{plan.path_name}"
     traffic = read_traffic(kernel_key)
 
@@ -332,20 +442,29 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated,
                    "io_dtype": w.dtype, "path": plan.path_name, "parallelism": f"channel shards x{world}",
                    "l2": "inputs exceed L2 (1.2 GB resident), no flush"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+        "roofline": {"bound": "hbm", "achieved": roof["achieved_gbs"], "peak": hbm_peak, "unit": "GB/s",
+                     "frac": roof["hbm_frac"], "peak_kind": peak_kind,
                      "traffic": None if traffic is None else traffic.get("bytes_per_launch"),
-                     "algorithmic_bytes": abytes,
-                     "kernel": kernel_key},
+                     "algorithmic_bytes": roof["algorithmic_bytes"], "kernel": kernel_key,
+                     "mma_schedule": roof["mma_schedule"], "mma_flops_per_elem": roof["mma_flops_per_elem"],
+                     "mma_peak_tflops": tc_peak, "t_hbm_us": roof["t_hbm_us"], "t_mma_us": roof["t_mma_us"],
+                     "frac_max_of_hbm_and_mma": roof["frac"]},
         "e2e": {"value": mg.job_throughput(w.elems, ctx, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "filter_precompute_ms": precompute_ms,
         "clocks": clk.summary(),
     }
+    del u, k, g, v, y, Kf, plan, mask
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_workloads:
+        line["workloads"] = {name: time_side_workload(name, hbm_peak, tc_peak) for name in SIDE_WORKLOADS
+                             if name != w.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, cores, sample = time_oracle(w)
-        line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        v_one, _, sample_one = time_oracle(w, target_s=8.0, cores=1, H=4)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                "single_core": {"value": v_one, "unit": UNIT, "cores": 1, "sample": sample_one}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     mg.shutdown(ctx)

@@ -53,8 +53,11 @@ struct Plan {
     int64_t chunkPairs = 0;
     size_t workBytes = 0;
 
-    // tensor-core path resources (owned by the tc translation unit)
+    // tensor-core path resources (owned by the tc translation units:
+    // tc_kernels.cu for the parity split and the staged row pass,
+    // tc_planar.cu for sequences of 4096 and overlap-save windows)
     void* tc = nullptr;
+    void* tcp = nullptr;
 
     int* status = nullptr;      // device status word (timeouts)
 
@@ -100,6 +103,14 @@ cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& a, cudaStream_t s);
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s);
 cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s);
+
+// tensor-core fused kernel with planar complex data (tc_planar.cu): plain
+// sequences of 4096 and overlap-save windows
+cudaError_t tc_planar_init(Plan& p);
+void tc_planar_free(Plan& p);
+cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& a, bool windows, cudaStream_t s);
+cudaError_t tc_planar_export(const Plan& p, const void* Kf, float* out, cudaStream_t s);
 
 // staged path with the tensor-core row pass (rows of C = 8192): the column
 // passes are the SIMT ones (simt_kernels.cu), the row pass and the filter

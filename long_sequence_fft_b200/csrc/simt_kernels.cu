@@ -313,6 +313,53 @@ simt_precompute_tc8192_kernel(const T* __restrict__ k, int64_t L, __half2* __res
     if (tid == 0) scales[h] = sc;
 }
 
+// The same 8192-point spectrum in the planar tensor-core format
+// (tc_planar.cu): per channel 8192 complex fp16 values K[f] / s_h, f = c1 +
+// 32 c2 + 1024 c3, the real part in half (c3 & 1) of 32-bit word
+// ((c2*2 + c3/4)*32 + c1)*4 + 2*((c3 & 3)/2) and the imaginary part in the
+// same half of the next word; s_h = max |Re|, |Im| over the channel, stored
+// after the H rows.
+template <typename T>
+__global__ void __launch_bounds__(fused_threads<13>())
+simt_precompute_tc_pp_kernel(const T* __restrict__ k, int64_t L, __half* __restrict__ Kh,
+                             float* __restrict__ scales, const float2* __restrict__ tw) {
+    constexpr int LOGM = 13;
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    extern __shared__ float2 s[];
+    __shared__ float red[NT / 32];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x;
+    PairRows<T> io;
+    io.u0 = k + (int64_t)h * L;
+    io.nvalid = (int)L;
+    first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
+    float m = 0.f;
+    for (int p = tid; p < (1 << LOGM); p += NT) {
+        const float2 z = s[sidx<1>(p, 0)];
+        m = fmaxf(m, fmaxf(fabsf(z.x), fabsf(z.y)));
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int i = 0; i < NT / 32; ++i) m = fmaxf(m, red[i]);
+    const float sc = m > 0.f ? m : 1.f;
+    const float inv = 1.f / sc;
+    __half* out = Kh + (int64_t)h * (2 << LOGM);
+    for (int p = tid; p < (1 << LOGM); p += NT) {
+        const int f = (int)perm_to_freq(p, LOGM);
+        const int c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
+        const int word = ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + 2 * ((c3 & 3) >> 1);
+        const float2 z = s[sidx<1>(p, 0)];
+        out[2 * word + (c3 & 1)] = __float2half_rn(z.x * inv);
+        out[2 * word + 2 + (c3 & 1)] = __float2half_rn(z.y * inv);
+    }
+    if (tid == 0) scales[h] = sc;
+}
+
 // The 16384-point spectrum in the split tensor-core format: per channel two
 // rows of 8192 complex fp16, row e holding K[2f + e] / s_h at position
 // ((c2*2 + c3/4)*32 + c1)*4 + c3%4 of f = c1 + 32 c2 + 1024 c3, with
@@ -984,6 +1031,19 @@ cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf,
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (__half2*)Kf,
+                                                               (float*)((uint8_t*)Kf + (size_t)p.H * (8192 * 4)), p.tw);
+        return cudaGetLastError();
+    })
+}
+
+cudaError_t simt_precompute_to_tc_pp(const Plan& p, const void* k, void* Kf, cudaStream_t st) {
+    if (p.L > 4096) return cudaErrorInvalidValue;     // the 8192-point spectrum of k (<= 4096 taps)
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << 13);
+    FFTCONV_DISPATCH_T(p.dtype, {
+        auto kern = simt_precompute_tc_pp_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (__half*)Kf,
                                                                (float*)((uint8_t*)Kf + (size_t)p.H * (8192 * 4)), p.tw);
         return cudaGetLastError();
     })

@@ -1210,7 +1210,16 @@ cudaError_t tc_plan_init(Plan& p) {
     TcResources* r = new TcResources();
     p.tc = r;
     r->mode = tc_mode(p.N, p.L);
-    const std::vector<uint8_t> img = r->mode == kModeSplit ? build_bimage<kModeSplit>() : build_bimage<kModePlain>();
+    if (r->mode != kModeSplit) {
+        // sequences of 4096 and overlap-save windows run the planar kernel
+        // (tc_planar.cu); the SIMT engine computes their 8192-point filter
+        // spectrum, so the plan also carries that twiddle table
+        p.logTab = 13;
+        cudaError_t e = upload_vec(&p.tw, twiddle_table(kM, kM));
+        if (e == cudaSuccess) e = tc_planar_init(p);
+        return e;
+    }
+    const std::vector<uint8_t> img = build_bimage<kModeSplit>();
     cudaError_t e = cudaMalloc((void**)&r->bimg, img.size());
     if (e == cudaSuccess) e = cudaMemcpy(r->bimg, img.data(), img.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddle_table(1024, 1024));
@@ -1232,6 +1241,7 @@ cudaError_t tc_plan_init(Plan& p) {
 }
 
 void tc_plan_free(Plan& p) {
+    tc_planar_free(p);
     TcResources* r = (TcResources*)p.tc;
     if (!r) return;
     cudaFree(r->bimg);
@@ -1254,11 +1264,12 @@ size_t tc_filter_bytes(const Plan& p) {
 
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
     return tc_mode(p.N, p.L) == kModeSplit ? simt_precompute_to_tc_split(p, k, Kf, s)
-                                           : simt_precompute_to_tc_layout(p, k, Kf, s);
+                                           : tc_planar_precompute(p, k, Kf, s);
 }
 
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     const TcResources* r = (const TcResources*)p.tc;
+    if (r->mode != kModeSplit) return tc_planar_forward(p, fa, r->mode == kModeWindows, s);
     TcArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.Kh16 = (const __half2*)fa.Kf;
@@ -1434,6 +1445,7 @@ cudaError_t tc_rows_export(const Plan& p, const void* Kf, float* out, cudaStream
 
 cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
     const int split = tc_mode(p.N, p.L) == kModeSplit ? 1 : 0;
+    if (!split) return tc_planar_export(p, Kf, out, s);
     const int64_t total = p.H * (p.N + 1);
     int blocks = (int)((total + 255) / 256);
     if (blocks > 65535) blocks = 65535;

@@ -1,0 +1,950 @@
+// tc_planar.cu -- tensor-core (tcgen05) fused FFT convolution with planar
+// complex data, sm_100a: sequences of 4096 (one zero-padded 8192-point
+// transform per sequence) and longer sequences with filters of at most 2049
+// taps (overlap-save windows of 4096 inputs, hop 2048).
+//
+// FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
+// "Approach": the FFT convolution as an order-p Monarch decomposition --
+// matrix products with small DFT factors along one digit of the index, so
+// the transform runs on tensor cores, permutations become on-chip
+// transposes, and the whole convolution (gates included, "Key results") is
+// one kernel.
+//
+// The transform and the tiling are those of tc_kernels.cu (8192 = 32 x 32 x
+// 8, a CTA tile = 4 pairs of batch rows of one channel, pair q in TMEM lanes
+// [32q, 32q+32), six tcgen05.mma stages S1, S2, S3, S3', S2', S1' with a ring
+// of four 64-column fp32 accumulator buffers, four MMA issuer warps and
+// sixteen epilogue warps).  What differs is how complex numbers are laid out:
+//
+//   - "pair-planar" (PP): the values of a complex vector are taken two at a
+//     time; the real parts of values 2p and 2p+1 share one 32-bit word
+//     (fp16 pair) and their imaginary parts the next word.  A half2
+//     instruction then applies a twiddle or the filter to two values at
+//     once, with no shuffling of real and imaginary halves (a complex
+//     product of two values costs four half2 instructions);
+//   - "planar" (PL): all real parts, then all imaginary parts.
+//
+// The DFT factors are stored as real 2n x 2n matrices whose row (K) and
+// column (N) orders follow the operand layouts below, so the MMAs read and
+// write these layouts directly.  Every accumulator's column order is PP.
+//
+//   operand              where             K order          written by
+//   S1  A1               TMEM              PP(j1)           load (u*w)
+//   S2  A2  (MN-major)   shared, 128B sw.  PL(l)            E1: 16-byte stores
+//   S3  A3               TMEM              PP(j3)           E2
+//   S3' A4               TMEM              PP(c3)           EK (filter product)
+//   S2' A5  (K-major)    shared, 128B sw.  PP(c2)           E3': 16-byte stores
+//   S1' A6  (MN-major)   shared, 128B sw.  PL(c1)           E2': 16-byte stores
+//
+// The two stages that contract the TMEM lane digit (S2: l, S1': c1) read an
+// MN-major ("transposed") shared-memory operand: the epilogue thread that
+// holds one lane's values for consecutive output indices writes them as
+// consecutive rows of the next operand -- the on-chip transpose is a plain
+// 16-byte vector store.  Every wait is bounded: on timeout the kernel records
+// FFTCONV_ERR_TIMEOUT in the plan's status word, drains, frees its TMEM and
+// returns.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <complex>
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace fftconv {
+
+cudaError_t simt_precompute_to_tc_pp(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+
+namespace {
+
+using namespace tc;
+
+constexpr int kN = 4096;          // window length (inputs and outputs per transform)
+constexpr int kM = 8192;          // transform length
+constexpr int kHop = 2048;        // overlap-save hop for longer sequences
+constexpr int kEpiWarps = 16;
+constexpr int kMmaWarps = 4;
+constexpr int kThreads = (kEpiWarps + kMmaWarps) * 32;
+constexpr int kDBuf = 4;
+constexpr int kChunks = 44;       // 8 per stage S1..S2', 4 for S1'
+constexpr uint32_t kWaitLimit = 1u << 20;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr int kTile = 16384;                  // one data tile: 128 rows x 64 fp16
+constexpr int OffData = 0;                    // 8 tiles (one per j3)
+constexpr int OffBS1 = 8 * kTile;             // K=32  N=64   4 KB
+constexpr int OffBS2 = OffBS1 + 4096;         // K=64  N=64   8 KB
+constexpr int OffBS3 = OffBS2 + 8192;         // 32 x (K=16 N=16)  16 KB
+constexpr int OffBS3i = OffBS3 + 16384;       // 32 x (K=16 N=16)  16 KB
+constexpr int OffBS2i = OffBS3i + 16384;      // K=64  N=64   8 KB
+constexpr int OffBS1i = OffBS2i + 8192;       // K=64  N=32   4 KB
+constexpr int OffBEnd = OffBS1i + 4096;
+constexpr int BImageBytes = OffBEnd - OffBS1;
+constexpr int kKBytes = kM * 4;               // one filter spectrum row, 8192 complex fp16
+constexpr int OffK = OffBEnd;
+constexpr int OffTw = OffK + kKBytes;         // w8192^e, e < 256, as half2
+constexpr int OffBars = OffTw + 1024;
+constexpr int OffMisc = OffBars + 128;
+constexpr int SmemBytes = OffMisc + 64 + 1024;   // + alignment slack
+static_assert(SmemBytes <= 232448, "shared memory");
+
+// chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
+__host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
+__host__ __device__ __forceinline__ int chunk_index(int c) { return c < 40 ? (c & 7) : c - 40; }
+// Chunks that need a whole earlier stage (not just the chunks that the
+// accumulator ring already orders before them): the first S3 chunks need
+// all of E2, the first S2' chunks all of E3', the last S1' chunk the last E2'
+// pair.
+__host__ __device__ __forceinline__ int chunk_stage_barrier(int c) {
+    if (c >= 16 && c < 20) return 0;
+    if (c >= 32 && c < 36) return 1;
+    if (c == 43) return 2;
+    return -1;
+}
+
+// fp16 element index of the real (comp 0) or imaginary (comp 1) part of
+// value i in pair-planar and planar order (n values)
+__host__ __device__ constexpr int pp_index(int comp, int i) { return 4 * (i >> 1) + 2 * comp + (i & 1); }
+__host__ __device__ constexpr int pl_index(int comp, int i, int n) { return comp * n + i; }
+
+// byte offset of element (n, k) of a K x N B operand, K-major, no swizzle:
+// 8x8 core matrices, K-groups of 8 LBO = (N/8)*128 bytes apart
+inline size_t bimg_offset(int n, int k, int N) {
+    return (size_t)(k / 8) * (N / 8) * 128 + (size_t)(n / 8) * 128 + (n % 8) * 16 + (k % 8) * 2;
+}
+
+// 128-byte swizzle of a byte offset (1024-byte aligned atoms)
+__device__ __forceinline__ uint32_t swz(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
+// MN-major operand tile, 128-byte swizzle: element (m, k) of 128 x 64; the
+// two 64-row halves 8192 bytes apart (LBO), the K-groups of 8 1024 bytes
+// apart (SBO)
+__device__ __forceinline__ uint32_t mn_off(int m, int k) {
+    return swz((uint32_t)((m >> 6) * 8192 + (k >> 3) * 1024 + (k & 7) * 128 + (m & 63) * 2));
+}
+// K-major operand tile, 128-byte swizzle: row m holds K = 64 fp16 (128 bytes)
+__device__ __forceinline__ uint32_t k_off(int m, int kbyte) {
+    return swz((uint32_t)((m >> 3) * 1024 + (m & 7) * 128 + kbyte));
+}
+
+struct PArgs {
+    const void* u;
+    const void* w;
+    const void* v;
+    void* y;
+    const uint32_t* K;          // [H][8192] words: the spectrum / scale, PP layout (k_word)
+    const float* Kscale;        // [H]
+    const uint8_t* mask;
+    int64_t mask_h;
+    int64_t B, H, N;
+    int64_t nwin;               // windows per sequence (1 for N = 4096)
+    int64_t pb;                 // pairs per channel, ceil(B/2)
+    int64_t tpc;                // tiles per window, ceil(pb/4)
+    int64_t nunits;             // H * nwin * tpc
+    const uint4* bimg;          // DFT factor images
+    const uint32_t* tw1024;     // exp(-2 pi i e/1024) as half2, e < 1024
+    const uint32_t* tw8192;     // exp(-2 pi i e/8192) as half2, e < 256
+    int* status;
+};
+
+template <typename T>
+struct IO;
+template <>
+struct IO<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 unpack2(uint32_t v) {
+        return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+    }
+    static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+template <>
+struct IO<__half> {
+    static __device__ __forceinline__ float2 unpack2(uint32_t v) {
+        __half2 h = *reinterpret_cast<__half2*>(&v);
+        return __half22float2(h);
+    }
+    static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+// two fp32 accumulator values (as raw bits) -> one fp16 pair
+__device__ __forceinline__ uint32_t pk(uint32_t a, uint32_t b) {
+    return h2u(__floats2half2_rn(__uint_as_float(a), __uint_as_float(b)));
+}
+__device__ __forceinline__ uint32_t pkf(float a, float b) { return h2u(__floats2half2_rn(a, b)); }
+
+// (xr + i xi) (tr + i ti) for two values at once: xr, xi, tr, ti are the PP
+// words (fp16 pairs) of the real and imaginary parts
+__device__ __forceinline__ void cmul_pp(uint32_t& xr, uint32_t& xi, uint32_t tr, uint32_t ti) {
+    const __half2 a = u2h(xr), b = u2h(xi), c = u2h(tr), d = u2h(ti);
+    xr = h2u(__hfma2(__hneg2(b), d, __hmul2(a, c)));
+    xi = h2u(__hfma2(b, c, __hmul2(a, d)));
+}
+constexpr uint32_t kNegPair = 0x80008000u;   // sign bits of both halves
+
+// word index of the filter spectrum value f = c1 + 32 c2 + 1024 c3 (its real
+// part; the imaginary part is the next word), and which half: 16-byte groups
+// of four c3 values (two PP pairs), consecutive c1 in consecutive groups, so
+// a warp (c1 = lane) reads 512 contiguous bytes per (c2, c3 half)
+__host__ __device__ __forceinline__ int k_word(int c1, int c2, int c3) {
+    return ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + 2 * ((c3 & 3) >> 1);
+}
+
+struct PairInfo {
+    int64_t o0, o1;      // element offsets of the window in rows b0 and b1 (o1 < 0: absent)
+    bool valid;
+    bool tail_only;      // only window positions t >= kHop are outputs
+};
+
+// A tile holds 4 pairs of batch rows of one channel and one window: unit u
+// covers channel u / (nwin*tpc), window j = (u / tpc) % nwin and pairs
+// 4*(u % tpc) + q, q < 4 (pairs past ceil(B/2) are empty).  Window j starts
+// at 2048 j; window 0 keeps all 4096 outputs, window j > 0 keeps positions
+// [2048, 4096) (the overlap-save rule: its transform is exact from window
+// position L - 1 on, and L <= 2049).
+template <bool WIN>
+__device__ __forceinline__ PairInfo pair_info(const PArgs& a, int64_t unit, int q, int64_t* h_out) {
+    PairInfo p;
+    int64_t h, j, bp;
+    if constexpr (!WIN) {
+        h = unit / a.tpc;
+        j = 0;
+        bp = 4 * (unit % a.tpc) + q;
+    } else {
+        const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
+        const uint32_t hh = un / per_ch, rem = un - hh * per_ch, jj = rem / tpc;
+        h = hh;
+        j = jj;
+        bp = 4 * (int64_t)(rem - jj * tpc) + q;
+    }
+    p.valid = bp < a.pb;
+    p.tail_only = j > 0;
+    const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
+    const int64_t base = WIN ? kHop * j : 0;
+    p.o0 = (b0 * a.H + h) * a.N + base;
+    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + h) * a.N + base : -1;
+    *h_out = h;
+    return p;
+}
+
+template <bool WIN>
+__device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
+    if constexpr (WIN) return (int64_t)((uint32_t)u / ((uint32_t)a.nwin * (uint32_t)a.tpc));
+    return u / a.tpc;
+}
+
+template <typename T, bool WIN>
+__global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bar = (uint64_t*)(smem + OffBars);
+    uint64_t* bar_in = bar + 0;    // the tile's input is in TMEM (16 epilogue warps)
+    uint64_t* dfull = bar + 1;     // [kDBuf] accumulator buffer written (tcgen05.commit)
+    uint64_t* dfree = bar + 5;     // [kDBuf] accumulator buffer drained (16 epilogue warps)
+    uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
+    uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
+    uint64_t* bar_stage = bar + 11;   // [3] E2, E3', E2' done for the tile (16 epilogue warps)
+    uint32_t* tmem_base_sh = (uint32_t*)(smem + OffMisc);
+    volatile int* abort_flag = (volatile int*)(smem + OffMisc + 4);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (tid == 0) {
+        mbar_init(bar_in, kEpiWarps);
+        for (int i = 0; i < kDBuf; ++i) {
+            mbar_init(&dfull[i], 1);
+            mbar_init(&dfree[i], kEpiWarps);
+        }
+        mbar_init(bar_fin, kMmaWarps);
+        mbar_init(bar_k, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar_stage[i], kEpiWarps);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kEpiWarps) tmem_alloc(tmem_base_sh, 512);   // the first MMA warp owns TMEM
+    {
+        uint4* dst = (uint4*)(smem + OffBS1);
+        for (int i = tid; i < BImageBytes / 16; i += kThreads) dst[i] = __ldg(&a.bimg[i]);
+        uint32_t* t = (uint32_t*)(smem + OffTw);
+        for (int i = tid; i < 256; i += kThreads) t[i] = __ldg(&a.tw8192[i]);
+    }
+    const uint32_t* stw = (const uint32_t*)(smem + OffTw);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_base_sh;
+
+    auto wait = [&](uint64_t* b, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_bounded(b, parity, abort_flag, kWaitLimit));
+    };
+    auto fail = [&](void) {
+        if (!*abort_flag) {
+            *abort_flag = 1;
+            atomicExch(a.status, kStatusTimeout);
+        }
+    };
+
+    if (warp >= kEpiWarps) {
+        // ============================ MMA issuers ===========================
+        // issuer i handles the chunks c = i (mod 4) of every tile, which all
+        // use accumulator buffer i
+        const int issuer = warp - kEpiWarps;
+        constexpr uint32_t kTransA = 1u << 15;        // A operand MN-major
+        const uint32_t id64 = idesc_f16_f32(128, 64);
+        const uint32_t id64t = id64 | kTransA;
+        const uint32_t id16 = idesc_f16_f32(128, 16);
+        const uint32_t id32t = idesc_f16_f32(128, 32) | kTransA;
+        // B operands: K-major, no swizzle; K-groups (N/8)*128 bytes apart
+        const uint64_t dS1 = make_desc(sbase + OffBS1, 1024, 128, 0);      // K step: +2048 B
+        const uint64_t dS2 = make_desc(sbase + OffBS2, 1024, 128, 0);      // K step: +2048 B
+        const uint64_t dS2i = make_desc(sbase + OffBS2i, 1024, 128, 0);
+        const uint64_t dS3 = make_desc(sbase + OffBS3, 256, 128, 0);       // per c2: +512 B
+        const uint64_t dS3i = make_desc(sbase + OffBS3i, 256, 128, 0);
+        const uint64_t dS1i = make_desc(sbase + OffBS1i, 512, 128, 0);     // K step: +1024 B
+        // A operands in shared memory: MN-major (S2, S1') and K-major (S2')
+        const uint64_t dAmn = make_desc(sbase + OffData, 8192, 1024, 2);   // K step: +2048 B
+        const uint64_t dAk = make_desc(sbase + OffData, 16, 1024, 2);      // K step: +32 B
+        int iter = 0;
+        int k_issued = 0;
+        bool ok = true;
+        uint32_t g = issuer;
+        for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
+            if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
+            tc_fence_after();
+            if (issuer == 0) {
+                if (lane == 0) {
+                    // the previous tile is finished with the filter buffer (its
+                    // epilogue warps arrived on bar_in after all their reads)
+                    mbar_expect_tx(bar_k, kKBytes);
+                    bulk_copy_g2s(smem + OffK, a.K + unit_channel<WIN>(a, unit) * kM, kKBytes, bar_k);
+                }
+                ++k_issued;
+                __syncwarp();
+            }
+#pragma unroll 1
+            for (int c = issuer; c < kChunks && ok; c += kMmaWarps, g += kMmaWarps) {
+                const int stage = chunk_stage(c), k = chunk_index(c);
+                const uint32_t b = g % kDBuf;
+                if (g >= kDBuf && !wait(&dfree[b], ((g - kDBuf) / kDBuf) & 1)) { ok = false; fail(); break; }
+                const int sb = chunk_stage_barrier(c);
+                if (sb >= 0 && !wait(&bar_stage[sb], iter & 1)) { ok = false; fail(); break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t d = tbase + 256 + 64 * b;
+                    if (stage == 0) {            // S1: A1 cols 16 j3 + (PP j1), j3 = k
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) mma_ts(d, tbase + 16 * k + 8 * ks, dS1 + 128 * ks, id64, ks);
+                    } else if (stage == 1) {     // S2: MN-major tile j3 = k
+                        const uint64_t da = dAmn + (uint64_t)(k * (kTile >> 4));
+#pragma unroll
+                        for (int s = 0; s < 4; ++s) mma_ss(d, da + 128 * s, dS2 + 128 * s, id64t, s);
+                    } else if (stage == 2 || stage == 3) {   // S3 / S3': c2 = 4k + cl, A cols 8 c2
+                        const uint64_t db = (stage == 2 ? dS3 : dS3i) + (uint64_t)(4 * k * 32);
+#pragma unroll
+                        for (int cl = 0; cl < 4; ++cl) mma_ts(d + 16 * cl, tbase + 8 * (4 * k + cl), db + 32 * cl, id16, 0);
+                    } else if (stage == 4) {     // S2': K-major tile j3 = k
+                        const uint64_t da = dAk + (uint64_t)(k * (kTile >> 4));
+#pragma unroll
+                        for (int s = 0; s < 4; ++s) mma_ss(d, da + 2 * s, dS2i + 128 * s, id64, s);
+                    } else {                     // S1': j3 = 2k + jl, MN-major tiles, N = 32 (16 kept j1)
+#pragma unroll
+                        for (int jl = 0; jl < 2; ++jl) {
+                            const uint64_t da = dAmn + (uint64_t)((2 * k + jl) * (kTile >> 4));
+#pragma unroll
+                            for (int s = 0; s < 4; ++s) mma_ss(d + 32 * jl, da + 128 * s, dS1i + 64 * s, id32t, s);
+                        }
+                    }
+                    tc_commit(&dfull[b]);
+                }
+                __syncwarp();
+                if (c == issuer + 12) {
+                    // warm L2 with the next tile's rows (u, w, v of both
+                    // sequences of each pair, and the filter spectrum): issuer i
+                    // takes pair i
+                    const void* pf_src = nullptr;
+                    uint32_t pf_bytes = kN * sizeof(T);
+                    const int64_t nu = unit + gridDim.x;
+                    if (nu < a.nunits && (lane >> 3) == issuer) {
+                        int64_t hn;
+                        const PairInfo Q = pair_info<WIN>(a, nu, issuer, &hn);
+                        const int which = lane & 7;
+                        if (Q.valid) {
+                            if (which == 0) pf_src = (const T*)a.u + Q.o0;
+                            else if (which == 1 && a.w) pf_src = (const T*)a.w + Q.o0;
+                            else if (which == 2 && a.v) pf_src = (const T*)a.v + Q.o0;
+                            else if (which == 3 && Q.o1 >= 0) pf_src = (const T*)a.u + Q.o1;
+                            else if (which == 4 && Q.o1 >= 0 && a.w) pf_src = (const T*)a.w + Q.o1;
+                            else if (which == 5 && Q.o1 >= 0 && a.v) pf_src = (const T*)a.v + Q.o1;
+                            else if (which == 6 && issuer == 0) {
+                                pf_src = a.K + hn * kM;
+                                pf_bytes = kKBytes;
+                            }
+                        }
+                    }
+                    if (pf_src) prefetch_l2(pf_src, pf_bytes);
+                    __syncwarp();
+                }
+            }
+        }
+        // drain: every issued MMA and the last filter copy must finish before
+        // TMEM and shared memory are released -- bounded, and regardless of
+        // an abort
+        if (lane == 0) tc_commit(bar_fin);
+        __syncwarp();
+        bool drained = false;
+        for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(bar_fin, 0);
+        if (!drained) fail();
+        if (issuer == 0 && k_issued > 0) {
+            drained = false;
+            for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(bar_k, (k_issued - 1) & 1);
+            if (!drained) fail();
+        }
+        __syncwarp();
+    } else {
+        // ========================== epilogue warps ==========================
+        const int q = warp & 3;          // lane quarter = pair within the tile
+        const int s = warp >> 2;         // column slice
+        const uint32_t lq = (uint32_t)(32 * q) << 16;
+        const int64_t nblk = kN / 32;    // mask blocks (plain mode: N = 4096)
+
+        // w1024^(x (8s + i)), x = lane, i < 8, as PP pairs over i: the E1
+        // twiddle (x = l, c1 = 8s + i) and, conjugated, the E2' twiddle
+        // (x = c1, l = 8s + i)
+        uint32_t twr[4], twi[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const __half2 t0 = u2h(__ldg(&a.tw1024[(lane * (8 * s + 2 * p)) & 1023]));
+            const __half2 t1 = u2h(__ldg(&a.tw1024[(lane * (8 * s + 2 * p + 1)) & 1023]));
+            twr[p] = h2u(__lows2half2(t0, t1));
+            twi[p] = h2u(__highs2half2(t0, t1));
+        }
+
+        // ---- load: x = u*w for t = 256 j1 + 8 l + j3 (l = lane), j1 in
+        // {2P, 2P+1} with P = 2s + part, into the TMEM A1 columns 16 j3 + 2P
+        // (real pair) and 16 j3 + 2P + 1 (imaginary pair: the pair's second
+        // row); part 1 then arrives on bar_in.  A tile's input is loaded while
+        // the previous tile's last stages run (the A columns are free once S3'
+        // is done).  Absent rows or gates read a present row and are masked.
+        auto load_tile = [&](int64_t lu, int part) {
+            int64_t hl;
+            const PairInfo LP = pair_info<WIN>(a, lu, q, &hl);
+            const bool hasL = LP.o1 >= 0;
+            const int64_t oo1 = hasL ? LP.o1 : LP.o0;
+            const T* pu0 = (const T*)a.u + LP.o0;
+            const T* pw0 = a.w ? (const T*)a.w + LP.o0 : pu0;
+            const T* pu1 = (const T*)a.u + oo1;
+            const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
+            const bool has_w = a.w != nullptr;
+            const int P = 2 * s + part;
+            uint4 ld[2][4];
+#pragma unroll
+            for (int jh = 0; jh < 2; ++jh) {
+                const int64_t t0 = 256 * (2 * P + jh) + 8 * lane;
+                ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
+                ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
+                ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
+                ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+            }
+            float xa[2][8], xb[2][8];
+#pragma unroll
+            for (int jh = 0; jh < 2; ++jh) {
+                const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
+                const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
+                const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
+                const uint32_t wb[4] = {ld[jh][3].x, ld[jh][3].y, ld[jh][3].z, ld[jh][3].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 p0 = IO<T>::unpack2(ua[e]), p1 = IO<T>::unpack2(ub[e]);
+                    if (has_w) {
+                        const float2 g0 = IO<T>::unpack2(wa[e]), g1 = IO<T>::unpack2(wb[e]);
+                        p0.x *= g0.x; p0.y *= g0.y; p1.x *= g1.x; p1.y *= g1.y;
+                    }
+                    if (!LP.valid) p0 = make_float2(0.f, 0.f);
+                    if (!hasL) p1 = make_float2(0.f, 0.f);
+                    xa[jh][2 * e] = p0.x; xa[jh][2 * e + 1] = p0.y;
+                    xb[jh][2 * e] = p1.x; xb[jh][2 * e + 1] = p1.y;
+                }
+            }
+#pragma unroll
+            for (int j3 = 0; j3 < 8; ++j3)
+                tmem_st2(tbase + lq + 16 * j3 + 2 * P, pkf(xa[0][j3], xa[1][j3]), pkf(xb[0][j3], xb[1][j3]));
+            if (part == 1) {
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_in);
+            }
+        };
+
+        int iter = 0;
+        bool ok = true;
+        float nf = 0.f;          // non-finite detector over the outputs (fp16 range)
+        if ((int64_t)blockIdx.x < a.nunits) {
+            load_tile(blockIdx.x, 0);
+            load_tile(blockIdx.x, 1);
+        }
+        for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
+            int64_t hch;
+            const PairInfo P = pair_info<WIN>(a, unit, q, &hch);
+            const bool has1 = P.o1 >= 0;
+            const uint32_t* Ks = (const uint32_t*)(smem + OffK);
+            float kscale = __ldg(&a.Kscale[hch]);
+            asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
+            const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : hch) * nblk : nullptr;
+
+            auto begin_pair = [&](int c) -> bool {
+                const uint32_t par = (uint32_t)(iter * (kChunks / 4) + (c >> 2)) & 1u;
+                if (!wait(&dfull[c & 3], par) || !wait(&dfull[(c & 3) + 1], par)) {
+                    fail();
+                    return false;
+                }
+                tc_fence_after();
+                return true;
+            };
+            auto release = [&](int c) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&dfree[c & 3]);
+                    mbar_arrive(&dfree[(c & 3) + 1]);
+                }
+            };
+            auto stage_done = [&](int i) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_stage[i]);
+            };
+            auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (c & 3); };
+
+            // E1 (S1 -> S2), chunks j3 = k, k+1: lane = l; PP columns of
+            // c1 = 8s .. 8s+7; twiddle w1024^(c1 l); MN-major A2 tile j3,
+            // rows 32q + c1, K = l (real) and 32 + l (imaginary).
+            // E2' (S2' -> S1'): lane = c1; PP columns of l = 8s .. 8s+7;
+            // twiddle conj w1024^(c1 l); MN-major A6 tile j3, rows 32q + l,
+            // K = c1 and 32 + c1.  The same twiddles and the same stores.
+            auto e_transpose = [&](int c, int k, bool conj) {
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tc_wait_ld();
+                release(c);
+                const uint32_t flip = conj ? kNegPair : 0u;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t wr[4], wi[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        wr[p] = pk(r[cc][4 * p], r[cc][4 * p + 1]);
+                        wi[p] = pk(r[cc][4 * p + 2], r[cc][4 * p + 3]);
+                        cmul_pp(wr[p], wi[p], twr[p], twi[p] ^ flip);
+                    }
+                    uint8_t* tile = smem + OffData + (k + cc) * kTile;
+                    *(uint4*)(tile + mn_off(32 * q + 8 * s, lane)) = make_uint4(wr[0], wr[1], wr[2], wr[3]);
+                    *(uint4*)(tile + mn_off(32 * q + 8 * s, 32 + lane)) = make_uint4(wi[0], wi[1], wi[2], wi[3]);
+                }
+                fence_proxy_async_smem();
+            };
+
+#pragma unroll 1
+            for (int k = 0; k < 8; k += 2) {
+                if (!(ok = begin_pair(k))) break;
+                e_transpose(k, k, false);
+            }
+            // E2, chunks j3 = k, k+1: lane = c1; PP columns of c2 = 8s .. 8s+7;
+            // twiddle w8192^(c1 j3) (one PP pair over j3 = k, k+1); A3 TMEM
+            // columns 8 c2 + k (real pair), 8 c2 + k + 1 (imaginary pair)
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 8 + k;
+                if (!(ok = begin_pair(c))) break;
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                const __half2 t0 = u2h(stw[lane * k]), t1 = u2h(stw[lane * (k + 1)]);
+                const uint32_t tr = h2u(__lows2half2(t0, t1)), ti = h2u(__highs2half2(t0, t1));
+                tc_wait_ld();
+                release(c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int ire = 4 * (i >> 1) + (i & 1);
+                    uint32_t wr = pk(r[0][ire], r[1][ire]), wi = pk(r[0][ire + 2], r[1][ire + 2]);
+                    cmul_pp(wr, wi, tr, ti);
+                    tmem_st2(tbase + lq + 8 * (8 * s + i) + k, wr, wi);
+                }
+                tc_wait_st();
+            }
+            if (ok) stage_done(0);
+            // EK: lane = c1; the PP columns of c3 (all eight) of c2 = 4(k+cc) + s;
+            // times the filter spectrum K/scale (|K/scale| <= 1); A4 TMEM
+            // columns 8 c2 .. 8 c2 + 7 in place
+            if (ok && !(ok = wait(bar_k, iter & 1))) fail();
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 16 + k;
+                if (!(ok = begin_pair(c))) break;
+                uint32_t r[2][16];
+                tmem_ld16(dcol(c) + 16 * s, r[0]);
+                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tc_wait_ld();
+                release(c);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c2 = 4 * (k + cc) + s;
+                    const uint4 k0 = *(const uint4*)(Ks + k_word(lane, c2, 0));
+                    const uint4 k1 = *(const uint4*)(Ks + k_word(lane, c2, 4));
+                    uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    if (mrow) {
+                        // frequency-sparse filter: zero the masked bins (f and
+                        // its mirror 8192 - f share one rfft bin)
+#pragma unroll
+                        for (int c3 = 0; c3 < 8; ++c3) {
+                            const int f = lane + 32 * c2 + 1024 * c3;
+                            int blk = (f <= kN ? f : kM - f) >> 5;
+                            blk = blk < (int)nblk ? blk : (int)nblk - 1;
+                            if (__ldg(&mrow[blk]) == 0) {
+                                const uint32_t keep = (c3 & 1) ? 0x0000ffffu : 0xffff0000u;
+                                kw[2 * (c3 >> 1)] &= keep;
+                                kw[2 * (c3 >> 1) + 1] &= keep;
+                            }
+                        }
+                    }
+                    uint32_t h8[8];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        h8[2 * p] = pk(r[cc][4 * p], r[cc][4 * p + 1]);
+                        h8[2 * p + 1] = pk(r[cc][4 * p + 2], r[cc][4 * p + 3]);
+                        cmul_pp(h8[2 * p], h8[2 * p + 1], kw[2 * p], kw[2 * p + 1]);
+                    }
+                    tmem_st8(tbase + lq + 8 * c2, h8);
+                }
+                tc_wait_st();
+            }
+            // E3': lane = c1; chunk c + (s >> 1), its c2 = 4(k + cc) + cl for
+            // cl < 4, j3 = 4h + jj with h = s & 1 (PP columns 16 cl + 8h ..
+            // + 7); twiddle conj w8192^(c1 j3); K-major A5 tile j3, row
+            // 32q + c1, the PP K words of c2 = 4(k+cc) .. + 3 (16 bytes)
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 24 + k;
+                if (!(ok = begin_pair(c))) break;
+                const int cc = s >> 1, h = s & 1;
+                uint32_t r[4][8];
+#pragma unroll
+                for (int cl = 0; cl < 4; ++cl) tmem_ld8(dcol(c + cc) + 16 * cl + 8 * h, r[cl]);
+                tc_wait_ld();
+                release(c);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j3 = 4 * h + jj;
+                    const __half2 t = u2h(stw[lane * j3]);
+                    const uint32_t trb = h2u(__low2half2(t)), tib = h2u(__high2half2(t)) ^ kNegPair;
+                    const int ire = 4 * (jj >> 1) + (jj & 1);
+                    uint32_t w0r = pk(r[0][ire], r[1][ire]), w0i = pk(r[0][ire + 2], r[1][ire + 2]);
+                    uint32_t w1r = pk(r[2][ire], r[3][ire]), w1i = pk(r[2][ire + 2], r[3][ire + 2]);
+                    cmul_pp(w0r, w0i, trb, tib);
+                    cmul_pp(w1r, w1i, trb, tib);
+                    uint8_t* tile = smem + OffData + j3 * kTile;
+                    *(uint4*)(tile + k_off(32 * q + lane, 16 * (k + cc))) =
+                        make_uint4(w0r, w0i, w1r, w1i);
+                }
+                fence_proxy_async_smem();
+            }
+            if (ok) stage_done(1);
+            if (ok && unit + gridDim.x < a.nunits) load_tile(unit + gridDim.x, 0);
+#pragma unroll 1
+            for (int k = 0; k < 8 && ok; k += 2) {
+                const int c = 32 + k;
+                if (!(ok = begin_pair(c))) break;
+                e_transpose(c, k, true);
+            }
+            if (ok) stage_done(2);
+            if (ok && unit + gridDim.x < a.nunits) load_tile(unit + gridDim.x, 1);
+            // EO: lane = l; chunk 40 + k holds j3 = 2k + jl (jl = 0, 1) at
+            // columns 32 jl + PP(j1), j1 < 16.  This warp takes j1 = 4s + 2hf + jj
+            // in two halves hf: the PP words of j1 pair 2s + hf (columns
+            // 32 jl + 8s + 4hf .. + 3) of all four chunks give the eight
+            // consecutive t = 256 j1 + 8 l + j3 of each row: one 16-byte store.
+            // y = s_h v z; in a window after the first, positions t < 2048
+            // (j1 < 8: warps with s < 2) are not outputs.
+            {
+                const bool emit = P.valid && !(P.tail_only && s < 2);
+#pragma unroll 1
+                for (int hf = 0; hf < 2 && ok; ++hf) {
+                    const int jb = 4 * s + 2 * hf;            // this pass's first j1
+                    uint4 va[2], vb[2];
+                    {
+                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int64_t t0 = 256 * (jb + jj) + 8 * lane;
+                            va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
+                            vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                        }
+                    }
+                    if (hf == 0 && (!(ok = begin_pair(40)) || !(ok = begin_pair(42)))) break;
+                    // r[cc][jl][0..3] = re(jb), re(jb+1), im(jb), im(jb+1) of j3 = 2cc + jl
+                    uint32_t r[4][2][4];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                        for (int jl = 0; jl < 2; ++jl) tmem_ld4(dcol(40 + cc) + 32 * jl + 2 * jb, r[cc][jl]);
+                    tc_wait_ld();
+                    if (hf == 1) {
+                        release(40);
+                        release(42);
+                    }
+                    if (emit) {
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int64_t t0 = 256 * (jb + jj) + 8 * lane;
+                            const uint32_t vaw[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
+                            const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
+                            uint32_t oa[4], ob[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                // j3 = 2e (chunk 40 + e, jl 0) and 2e + 1 (jl 1)
+                                float a0 = __uint_as_float(r[e][0][jj]) * kscale;
+                                float a1 = __uint_as_float(r[e][1][jj]) * kscale;
+                                float b0 = __uint_as_float(r[e][0][2 + jj]) * kscale;
+                                float b1 = __uint_as_float(r[e][1][2 + jj]) * kscale;
+                                nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
+                                nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
+                                if (a.v) {
+                                    const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
+                                    a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
+                                }
+                                oa[e] = IO<T>::pack2(a0, a1);
+                                ob[e] = IO<T>::pack2(b0, b1);
+                            }
+                            *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                            if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                        }
+                    }
+                }
+            }
+        }
+        nonfinite_report(nf, a.status);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kEpiWarps) {     // the warp that allocated
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+        tmem_relinquish();
+    }
+}
+
+// ----------------------------------------------------------- host side ---
+
+struct Resources {
+    uint8_t* bimg = nullptr;
+    uint32_t* tw1024 = nullptr;
+    uint32_t* tw8192 = nullptr;
+    int num_sms = 0;
+};
+
+std::complex<double> wpow(long long e, long long n, int sign) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const long long r = ((e % n) + n) % n;
+    const double a = two_pi * (double)r / (double)n;
+    return std::complex<double>(std::cos(a), sign * std::sin(a));
+}
+
+void put_f16(std::vector<uint8_t>& img, size_t off, double v) {
+    const __half h = __double2half(v);
+    std::memcpy(&img[off], &h, 2);
+}
+
+// Real-pair image of the complex n_out x n_in matrix F as a K x N B operand
+// (N = Ntot columns): input value j's real and imaginary parts sit at K rows
+// kidx(0, j), kidx(1, j), output value c's at N columns nidx(0, c), nidx(1, c)
+template <class KI, class NI>
+void put_matrix(std::vector<uint8_t>& img, size_t base, int n_out, int n_in, int Ntot,
+                const std::vector<std::complex<double>>& F, KI kidx, NI nidx) {
+    for (int c = 0; c < n_out; ++c)
+        for (int j = 0; j < n_in; ++j) {
+            const std::complex<double> f = F[(size_t)c * n_in + j];
+            put_f16(img, base + bimg_offset(nidx(0, c), kidx(0, j), Ntot), f.real());
+            put_f16(img, base + bimg_offset(nidx(0, c), kidx(1, j), Ntot), -f.imag());
+            put_f16(img, base + bimg_offset(nidx(1, c), kidx(0, j), Ntot), f.imag());
+            put_f16(img, base + bimg_offset(nidx(1, c), kidx(1, j), Ntot), f.real());
+        }
+}
+
+std::vector<uint8_t> build_bimage() {
+    std::vector<uint8_t> img(BImageBytes, 0);
+    const double r32 = 1.0 / std::sqrt(32.0), r8 = 1.0 / std::sqrt(8.0);
+    auto off = [](int o) { return (size_t)(o - OffBS1); };
+    auto pp = [](int comp, int i) { return pp_index(comp, i); };
+    auto pl32 = [](int comp, int i) { return pl_index(comp, i, 32); };
+    std::vector<std::complex<double>> F;
+    // S1: c1 <- j1 (j1 < 16: the nonzero inputs)
+    F.assign(32 * 16, 0);
+    for (int c = 0; c < 32; ++c) for (int j = 0; j < 16; ++j) F[c * 16 + j] = wpow((long long)c * j, 32, -1) * r32;
+    put_matrix(img, off(OffBS1), 32, 16, 64, F, pp, pp);
+    // S2: c2 <- l
+    F.assign(32 * 32, 0);
+    for (int c = 0; c < 32; ++c) for (int j = 0; j < 32; ++j) F[c * 32 + j] = wpow((long long)c * j, 32, -1) * r32;
+    put_matrix(img, off(OffBS2), 32, 32, 64, F, pl32, pp);
+    // S3 (per c2): c3 <- j3 with w8^(c3 j3) w256^(c2 j3);  S3': j3 <- c3, conjugate
+    for (int c2 = 0; c2 < 32; ++c2) {
+        std::vector<std::complex<double>> G(64), Gi(64);
+        for (int c3 = 0; c3 < 8; ++c3)
+            for (int j3 = 0; j3 < 8; ++j3) {
+                const std::complex<double> gv = wpow((long long)c3 * j3, 8, -1) * wpow((long long)c2 * j3, 256, -1) * r8;
+                G[c3 * 8 + j3] = gv;
+                Gi[j3 * 8 + c3] = std::conj(gv);
+            }
+        put_matrix(img, off(OffBS3) + c2 * 512, 8, 8, 16, G, pp, pp);
+        put_matrix(img, off(OffBS3i) + c2 * 512, 8, 8, 16, Gi, pp, pp);
+    }
+    // S2': l <- c2
+    F.assign(32 * 32, 0);
+    for (int l = 0; l < 32; ++l) for (int c = 0; c < 32; ++c) F[l * 32 + c] = wpow((long long)c * l, 32, +1) * r32;
+    put_matrix(img, off(OffBS2i), 32, 32, 64, F, pp, pp);
+    // S1': j1 <- c1 (j1 < 16: the kept outputs)
+    F.assign(16 * 32, 0);
+    for (int j = 0; j < 16; ++j) for (int c = 0; c < 32; ++c) F[j * 32 + c] = wpow((long long)c * j, 32, +1) * r32;
+    put_matrix(img, off(OffBS1i), 16, 32, 32, F, pl32, pp);
+    return img;
+}
+
+uint32_t half2_bits(double re, double im) {
+    const __half2 h = __floats2half2_rn((float)re, (float)im);
+    uint32_t b;
+    std::memcpy(&b, &h, 4);
+    return b;
+}
+
+std::vector<uint32_t> twiddles_h2(int n, int count) {
+    std::vector<uint32_t> t(count);
+    for (int e = 0; e < count; ++e) {
+        const std::complex<double> z = wpow(e, n, -1);
+        t[e] = half2_bits(z.real(), z.imag());
+    }
+    return t;
+}
+
+template <typename V>
+cudaError_t upload_vec(V** dst, const std::vector<V>& v) {
+    cudaError_t e = cudaMalloc((void**)dst, v.size() * sizeof(V));
+    if (e == cudaSuccess) e = cudaMemcpy(*dst, v.data(), v.size() * sizeof(V), cudaMemcpyHostToDevice);
+    return e;
+}
+
+template <typename T, bool WIN>
+void launch(const PArgs& a, int64_t grid, cudaStream_t s) {
+    tc_fftconv_planar_kernel<T, WIN><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
+}
+
+// K_f (PP layout) -> rfft bins [0, N] of each channel
+__global__ void planar_export_kernel(const uint32_t* __restrict__ K, const float* __restrict__ scale,
+                                     float* __restrict__ out, int64_t H) {
+    const int64_t nb = kN + 1, total = H * nb;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t h = i / nb, f = i % nb;
+        const int c1 = (int)(f & 31), c2 = (int)((f >> 5) & 31), c3 = (int)(f >> 10);
+        const uint32_t* row = K + h * kM;
+        const int wd = k_word(c1, c2, c3), half = c3 & 1;
+        const __half re = __ushort_as_half((unsigned short)(row[wd] >> (16 * half)));
+        const __half im = __ushort_as_half((unsigned short)(row[wd + 1] >> (16 * half)));
+        out[2 * i] = __half2float(re) * scale[h];
+        out[2 * i + 1] = __half2float(im) * scale[h];
+    }
+}
+
+}  // namespace
+
+cudaError_t tc_planar_init(Plan& p) {
+    Resources* r = new Resources();
+    p.tcp = r;
+    cudaError_t e = upload_vec(&r->bimg, build_bimage());
+    if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddles_h2(1024, 1024));
+    if (e == cudaSuccess) e = upload_vec(&r->tw8192, twiddles_h2(kM, 256));
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SmemBytes);
+    return e;
+}
+
+void tc_planar_free(Plan& p) {
+    Resources* r = (Resources*)p.tcp;
+    if (!r) return;
+    cudaFree(r->bimg);
+    cudaFree(r->tw1024);
+    cudaFree(r->tw8192);
+    delete r;
+    p.tcp = nullptr;
+}
+
+// K_f: H rows of 8192 complex fp16 (the spectrum over each channel's largest
+// component, PP layout), then [H] fp32 scales
+size_t tc_planar_filter_bytes(const Plan& p) {
+    return (size_t)p.H * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
+}
+
+cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
+    return simt_precompute_to_tc_pp(p, k, Kf, s);
+}
+
+cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, bool windows, cudaStream_t s) {
+    const Resources* r = (const Resources*)p.tcp;
+    PArgs a{};
+    a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
+    a.K = (const uint32_t*)fa.Kf;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.mask = fa.mask; a.mask_h = fa.mask_h;
+    a.B = fa.B; a.H = p.H; a.N = p.N;
+    a.nwin = windows ? p.N / kHop - 1 : 1;
+    a.pb = (fa.B + 1) / 2;
+    a.tpc = (a.pb + 3) / 4;
+    a.nunits = p.H * a.nwin * a.tpc;
+    a.bimg = (const uint4*)r->bimg;
+    a.tw1024 = r->tw1024;
+    a.tw8192 = r->tw8192;
+    a.status = p.status;
+    const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
+    if (p.dtype == kBF16) {
+        if (windows) launch<__nv_bfloat16, true>(a, grid, s);
+        else launch<__nv_bfloat16, false>(a, grid, s);
+    } else {
+        if (windows) launch<__half, true>(a, grid, s);
+        else launch<__half, false>(a, grid, s);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_planar_export(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
+    const int64_t total = p.H * (kN + 1);
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 65535) blocks = 65535;
+    planar_export_kernel<<<blocks, 256, 0, s>>>((const uint32_t*)Kf,
+                                                (const float*)((const uint8_t*)Kf + (size_t)p.H * kKBytes), out, p.H);
+    return cudaGetLastError();
+}
+
+}  // namespace fftconv

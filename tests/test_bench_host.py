@@ -27,6 +27,41 @@ def test_algorithmic_bytes(name, expected):
     assert bench.algorithmic_bytes(W.WORKLOADS[name]) == expected
 
 
+# The tensor-core paths store each spectrum bin as complex fp16 (4 bytes).
+@pytest.mark.parametrize("name,path,expected", [
+    ("gated_bf16_n4k", "tc_fused", 64 * 768 * 4096 * 8 + 768 * 4097 * 4),       # 1,623,198,720
+    ("fp16_n32k", "tc_staged", 8 * 256 * 32768 * 4 + 256 * 32769 * 4),         # 301,990,912
+    ("gated_bf16_n4k", "simt_fused", 64 * 768 * 4096 * 8 + 768 * 4097 * 8),
+])
+def test_algorithmic_bytes_at_the_stored_filter_width(name, path, expected):
+    assert bench.algorithmic_bytes(W.WORKLOADS[name], path) == expected
+
+
+# Issued MMA flops per output element, from the instruction shapes of the
+# 32 x 32 x 8 engine: 8*32 + 16*(32 + 8) = 896 for a zero-padded transform
+# with half its outputs kept; 16*(32 + 32 + 8) = 1152 for a full one; three
+# overlap-save windows of 4096 points per 8192 outputs: 896 * 3 / 2.
+@pytest.mark.parametrize("name,path,expected", [
+    ("gated_bf16_n4k", "tc_fused", 896.0),
+    ("sparse_bf16_n8k", "tc_fused", 1152.0),
+    ("partial_bf16_n8k", "tc_fused", 1344.0),
+    ("fp16_n32k", "tc_staged", 1152.0),
+    ("fp32_n1k", "simt_fused", 0.0),
+])
+def test_mma_flops_per_element(name, path, expected):
+    assert bench.mma_flops_per_elem(W.WORKLOADS[name], path)[1] == expected
+
+
+def test_roofline_takes_the_slower_of_bytes_and_flops():
+    w = W.WORKLOADS["gated_bf16_n4k"]
+    r = bench.roofline_entry(w, "tc_fused", 0.5, 6531.9, 1607.7)
+    t_hbm = 1623198720 / 6531.9e9
+    t_mma = 896.0 * w.elems / 1607.7e12
+    assert abs(r["hbm_frac"] - t_hbm / 0.5e-3) < 1e-12
+    assert abs(r["frac"] - max(t_hbm, t_mma) / 0.5e-3) < 1e-12
+    assert r["bound"] == "hbm"
+
+
 def _fake_root(tmp_path, src_text, recorded_hash):
     (tmp_path / "profiles").mkdir()
     (tmp_path / "k.cu").write_text(src_text)

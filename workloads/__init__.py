@@ -88,6 +88,12 @@ WORKLOADS = {
     "dna_bf16_n4m_l1m": Workload("dna_bf16_n4m_l1m", 7, 1, 32, 1 << 22, 1 << 20, "bf16", False,
                                  "decay:1e-5", u_kind="dna",
                                  description="bf16 conv B=1 H=32 N=4M, filter length 1M, DNA-like input"),
+    # sequence length 1K at the flagship's batch x channels (64 x 768): the
+    # length of the page's kernel-level latency rows, gated and ungated
+    "gated_bf16_n1k": Workload("gated_bf16_n1k", 8, 64, 768, 1024, 1024, "bf16", True, "decay:0.001",
+                               description="gated bf16 conv B=64 H=768 N=1024"),
+    "bf16_n1k": Workload("bf16_n1k", 9, 64, 768, 1024, 1024, "bf16", False, "scaled",
+                         description="bf16 conv B=64 H=768 N=1024"),
 }
 
 # The workload the benchmark times at one GPU.
