@@ -257,7 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
     volatile int* abort_flag = (volatile int*)(smem + OffMisc + 4);
 
     const int tid = threadIdx.x;
-    const int warp = tid >> 5;
+    // the warp index through a shuffle, so the compiler knows it is the same
+    // for all lanes: everything derived from it (TMEM and shared-memory
+    // addresses, descriptors) stays in uniform registers
+    const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
     const int lane = tid & 31;
     const uint32_t sbase = smem_u32(smem);
 
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = *tmem_base_sh;
+    const uint32_t tbase = __shfl_sync(0xffffffffu, *tmem_base_sh, 0);
 
     auto wait = [&](uint64_t* b, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait_bounded(b, parity, abort_flag, kWaitLimit));

@@ -34,14 +34,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Read a shared-memory word with a volatile shared-space load.
+__device__ __forceinline__ int ld_shared_volatile(const volatile int* p) {
+    int v;
+    asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)));
+    return v;
+}
 // Wait for the phase with the given parity to complete, giving up after
 // `limit` polls (each try_wait itself blocks for a bounded, hardware-defined
-// time).  Returns false on timeout or if *abort becomes nonzero.
+// time).  Returns false on timeout or if the shared-memory word *abort has
+// become nonzero (checked every 32 polls).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                                   uint32_t limit) {
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
+        if ((i & 31u) == 31u && ld_shared_volatile(abort)) return false;
     }
     return false;
 }
