@@ -97,19 +97,37 @@ typedef enum {
 } fftconv_path_t;
 
 /* Create a plan for sequences of length N (a power of two, 256 <= N <= 2^22)
- * and H channels with full-length filters (L = N).  `order` selects the
- * decomposition: 0 = automatic; 2 or 3 = fused on-chip kernel (N <= 8192);
- * 4 = the staged path with one workspace round trip (any N); 5 = the staged
- * path whose row pass runs on the tensor cores (fp16/bf16, 16384 <= N <= 2^22,
- * L > 2049; order 0 chooses it for those plans, as overlap-save windows of
- * 2 x hop points when the filter is at most half the sequence: hop = the
- * power of two >= max(L, 16384); such a windowed plan rejects block masks
- * and fftconv_filter_to_rfft with FFTCONV_ERR_UNSUPPORTED, order 5 keeps the
- * full transform); other values are FFTCONV_ERR_UNSUPPORTED.  Synchronous:
- * allocates the plan's device tables (a few hundred KB) and, on the staged
- * paths, its workspace (about 64 MB for order 4, 512 MB for the tensor-core
- * staged path; fftconv_workspace_bytes) on the current device.  *out receives
- * the plan, or NULL on failure. */
+ * and H channels with full-length filters (L = N).
+ *
+ * `order` is the Monarch order of the decomposition, the number of DFT-factor
+ * levels the length-2N transform is split into ("Approach": order-p Monarch
+ * decomposition), read as a request for where the intermediate lives:
+ *   0     automatic (the fastest kernel this library has for the plan);
+ *   2, 3  fused: one kernel, the transform stays on chip (no intermediate in
+ *         device memory).  This library's fused kernels split every transform
+ *         they hold into three levels, so 2 and 3 are the same request.  They
+ *         exist for N <= 8192 (tensor cores for fp16/bf16 at N = 4096 and
+ *         8192; fp32 lanes otherwise) and, with filters of at most 2049 taps,
+ *         for longer N as overlap-save windows of one fused transform each.
+ *         Orders 2 and 3 at N > 8192 with L > 2049 return
+ *         FFTCONV_ERR_UNSUPPORTED: no fused kernel holds that transform on
+ *         chip; orders 0, 4 and 5 serve it;
+ *   4     staged: one intermediate pass through a plan-owned workspace in
+ *         device memory (column passes, a row pass, inverse column passes),
+ *         fp32 lanes throughout, any N.
+ * Two further values select an engine inside those families:
+ *   1     fused on fp32 lanes (N <= 8192), whatever the dtype;
+ *   5     staged, with the row pass on the tensor cores (fp16/bf16,
+ *         16384 <= N <= 2^22, L > 2049).  Order 0 chooses it for those plans,
+ *         as overlap-save windows of 2 x hop points when the filter is at most
+ *         half the sequence (hop = the power of two >= max(L, 16384)); such a
+ *         windowed plan rejects block masks and fftconv_filter_to_rfft with
+ *         FFTCONV_ERR_UNSUPPORTED, order 5 keeps the full transform.
+ * Other values are FFTCONV_ERR_UNSUPPORTED.  fftconv_plan_path reports the
+ * kernel family chosen.  Synchronous: allocates the plan's device tables (a
+ * few hundred KB) and, on the staged paths, its workspace (about 64 MB for
+ * order 4, 512 MB for the tensor-core staged path; fftconv_workspace_bytes) on
+ * the current device.  *out receives the plan, or NULL on failure. */
 FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
                         fftconv_dtype_t dtype, int order);
 
@@ -164,6 +182,32 @@ FFTCONV_API int fftconv_forward(fftconv_plan_t plan, const void* u, const void* 
                     int64_t B, int64_t H, int64_t N, const void* w, const void* v,
                     const uint8_t* block_mask, int64_t mask_h,
                     fftconv_stream_t stream);
+
+/* Gradients of y = v * conv(u * w, k) for the incoming gradient dy, for
+ * training (FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor
+ * Cores, "Key results": the convolution inside trained models; the page gives
+ * no backward, so these are the plain adjoints of the forward definition).
+ * With g = dy * v and the correlation c[t] = sum_{s<L, t+s<N} g[t+s] k[s]:
+ *     du = w * c,   dw = u * c,   dv = dy * conv(u * w, k),
+ *     dk[h, s] = sum_b sum_t g_b[t] (u*w)_b[t-s]   for s < L.
+ *   u, w, v, dy   : [B, H, N] device, plan dtype (w, v may be NULL: ones).
+ *   K_f           : from fftconv_filter_precompute on this plan.
+ *   du            : [B, H, N] device, plan dtype, required.
+ *   dw, dv        : [B, H, N] device or NULL (not computed); dw needs w and
+ *                   dv needs v.
+ *   dk            : [H, L] fp32 device or NULL; overwritten with the sum over
+ *                   the batch (the call clears it first).
+ * Outputs must not overlap each other or any input.  Supported on fp16/bf16
+ * tensor-core plans with N <= 4096 (fftconv_plan_path ==
+ * FFTCONV_PATH_TC_FUSED); other plans return FFTCONV_ERR_UNSUPPORTED.  du and
+ * dw come from one launch of the fused tensor-core kernel with the product by
+ * conj(K_f) (correlation) and two gated outputs, dv from the forward kernel
+ * with dy as the output gate, dk from fp32 transforms of dy*v and u*w per
+ * (channel, batch chunk).  Asynchronous on `stream`; allocates nothing.  The
+ * fp16 range note above applies to du, dw, dv (FFTCONV_ERR_RANGE). */
+FFTCONV_API int fftconv_backward(fftconv_plan_t plan, const void* u, const void* K_f, const void* dy,
+                                 int64_t B, int64_t H, int64_t N, const void* w, const void* v,
+                                 void* du, void* dw, void* dv, float* dk, fftconv_stream_t stream);
 
 /* Device bytes fftconv_forward_host needs as staging for B rows with the
  * given gates and mask present (nonzero = present). */

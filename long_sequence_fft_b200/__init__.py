@@ -50,6 +50,8 @@ _SIGNATURES = {
     "fftconv_forward_host_staging_bytes": (_sz, [_vp, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64]),
     "fftconv_forward_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp,
                                             _sz, _vp]),
+    "fftconv_backward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp]),
     "fftconv_filter_to_rfft": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
     "fftconv_device_status": (ctypes.c_int, [_vp, _vp]),
     "fftconv_selftest_bounded_wait": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp]),
@@ -115,11 +117,12 @@ def _stream_handle(stream) -> Optional[int]:
 class Plan:
     """A convolution plan for sequences of length N, H channels, one dtype.
 
-    order: 0 automatic, 1 fp32 shared-memory FFT in one kernel (N <= 8192),
-    2/3 fused on-chip kernel (tensor cores where available), 4 staged passes
-    through a workspace (any N), 5 staged passes with the row pass on the
-    tensor cores (fp16/bf16, 16384 <= N <= 2^22, L > 2049).  L < N gives the
-    partial convolution."""
+    order: the Monarch order requested (include/fftconv.h): 0 automatic,
+    2 or 3 fused on chip (one kernel; tensor cores where available), 4 staged
+    through a device-memory workspace on fp32 lanes (any N); and two engine
+    choices: 1 fused on fp32 lanes (N <= 8192), 5 staged with the row pass on
+    the tensor cores (fp16/bf16, 16384 <= N <= 2^22, L > 2049).  L < N gives
+    the partial convolution."""
 
     def __init__(self, N: int, H: int, dtype="bf16", order: int = 0, L: Optional[int] = None):
         self.N, self.H = int(N), int(H)
@@ -214,6 +217,23 @@ class Plan:
         _check(_lib.fftconv_forward(self._h, _ptr(u), _ptr(Kf), _ptr(out), B, self.H, self.N, _ptr(w), _ptr(v),
                                     _ptr(mask), mask_h, _stream_handle(stream)))
         return out
+
+    def backward(self, u, Kf, dy, w=None, v=None, want_dk=True, stream=None):
+        """Gradients of y = v * conv(u * w, k) for dy: dict(du, dw, dv, dk) with
+        dw only when w is given, dv only when v is given, dk an fp32 [H, L]
+        tensor (summed over the batch) when want_dk."""
+        import torch
+        B = u.shape[0]
+        shape = (B, self.H, self.N)
+        for t, name in ((u, "u"), (w, "w"), (v, "v"), (dy, "dy")):
+            self._check_tensor(t, shape, name)
+        du = torch.empty(shape, dtype=self.dtype, device=u.device)
+        dw = torch.empty_like(du) if w is not None else None
+        dv = torch.empty_like(du) if v is not None else None
+        dk = torch.empty((self.H, self.L), dtype=torch.float32, device=u.device) if want_dk else None
+        _check(_lib.fftconv_backward(self._h, _ptr(u), _ptr(Kf), _ptr(dy), B, self.H, self.N, _ptr(w), _ptr(v),
+                                     _ptr(du), _ptr(dw), _ptr(dv), _ptr(dk), _stream_handle(stream)))
+        return {"du": du, "dw": dw, "dv": dv, "dk": dk}
 
     def staging_bytes(self, B: int, has_w: bool, has_v: bool, mask_h: int = 0) -> int:
         return int(_lib.fftconv_forward_host_staging_bytes(self._h, B, int(has_w), int(has_v), int(mask_h > 0),

@@ -69,6 +69,7 @@ void free_plan(Plan* p) {
     cudaSetDevice(p->device);
     if (p->tc) tc_plan_free(*p);
     cudaFree(p->tw);
+    cudaFree(p->twgrad);
     cudaFree(p->twLo);
     cudaFree(p->twHi);
     cudaFree(p->work);
@@ -166,8 +167,10 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         p->path = kPathSimtFused;
     } else {
         delete p;
-        return fail(FFTCONV_ERR_UNSUPPORTED, "order %d: no fused kernel for N=%lld; use order 4 or 0", order,
-                    (long long)N);
+        return fail(FFTCONV_ERR_UNSUPPORTED,
+                    "order %d asks for a fused on-chip transform; none holds N=%lld with L=%lld "
+                    "(fused kernels: N <= 8192, or L <= 2049 with 16-bit data); use order 0, 4 or 5",
+                    order, (long long)N, (long long)L);
     }
 
     cudaError_t e = cudaMalloc((void**)&p->status, sizeof(int));
@@ -226,6 +229,8 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
     } else {
         e = tc_plan_init(*p);
         p->filter_bytes = tc_filter_bytes(*p);
+        // the backward pass's filter gradient transforms length 2N on fp32 lanes
+        if (e == cudaSuccess && N <= 4096) e = upload(&p->twgrad, host_twiddles(p->M, p->M, 1));
     }
     if (e != cudaSuccess) {
         free_plan(p);
@@ -299,6 +304,11 @@ static int validate_forward(const Plan& p, const void* u, const void* K_f, void*
     if (p.path == kPathTcFused &&
         (double)H * (double)tc_tiles_per_pair_group(p.N, p.L) * (double)(((B + 1) / 2 + 3) / 4) >= 2147483648.0)
         return fail(FFTCONV_ERR_UNSUPPORTED, "too many tiles for one launch");
+    if (mask && p.path == kPathTcFused && p.N < 4096)
+        return fail(FFTCONV_ERR_UNSUPPORTED,
+                    "block masks act on the 2N-point spectrum; this tensor-core plan (N=%lld) packs %lld "
+                    "sequences into one 8192-point transform: create the plan with order 1 or 4 for masks",
+                    (long long)p.N, (long long)(4096 / p.N));
     if (mask && ((p.path == kPathTcFused && tc_overlap_save(p.N, p.L)) || p.nwin > 1))
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "block masks act on the 2N-point spectrum; this overlap-save plan (N=%lld, L=%lld) "
@@ -449,6 +459,61 @@ int fftconv_forward_host(fftconv_plan_t plan, const void* u_host, const void* K_
     if (e == cudaSuccess) e = cudaEventRecord(q.ev_out, q.copy_out);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, q.ev_out, 0);
     if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline");
+    return FFTCONV_OK;
+}
+
+int fftconv_backward(fftconv_plan_t plan, const void* u, const void* K_f, const void* dy, int64_t B, int64_t H,
+                     int64_t N, const void* w, const void* v, void* du, void* dw, void* dv, float* dk,
+                     fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    const Plan& p = plan->p;
+    if (p.path != kPathTcFused || p.N > 4096)
+        return fail(FFTCONV_ERR_UNSUPPORTED,
+                    "the backward pass runs on fp16/bf16 tensor-core plans with N <= 4096 (this plan: %s, N=%lld)",
+                    p.path == kPathTcFused ? "tensor-core" : "not tensor-core", (long long)p.N);
+    int rc = validate_forward(p, u, K_f, du, B, H, N, w, v, nullptr, 0);
+    if (rc != FFTCONV_OK) return rc;
+    if (B == 0) {
+        if (dk) {
+            cudaError_t e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)(p.H * p.L), (cudaStream_t)stream);
+            if (e != cudaSuccess) return cuda_fail(e, "dk clear");
+        }
+        return FFTCONV_OK;
+    }
+    if (!dy || !du) return fail(FFTCONV_ERR_INVALID_ARG, "dy and du must be non-NULL");
+    if (dw && !w) return fail(FFTCONV_ERR_INVALID_ARG, "dw needs the gate w");
+    if (dv && !v) return fail(FFTCONV_ERR_INVALID_ARG, "dv needs the gate v");
+    if (!aligned16(dy) || !aligned16(du) || !aligned16(dw) || !aligned16(dv) || !aligned16(dk))
+        return fail(FFTCONV_ERR_ALIGNMENT, "dy, du, dw, dv and dk must be 16-byte aligned");
+    const size_t bytes = (size_t)B * (size_t)H * (size_t)N * dtype_size(p.dtype);
+    const void* ins[5] = {u, w, v, dy, K_f};
+    const size_t in_bytes[5] = {bytes, bytes, bytes, bytes, p.filter_bytes};
+    void* outs[4] = {du, dw, dv, dk};
+    const size_t out_bytes[4] = {bytes, bytes, bytes, sizeof(float) * (size_t)(p.H * p.L)};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 5; ++j)
+            if (ranges_overlap(outs[i], out_bytes[i], ins[j], in_bytes[j]))
+                return fail(FFTCONV_ERR_INVALID_ARG, "an output of the backward pass overlaps an input");
+        for (int j = i + 1; j < 4; ++j)
+            if (ranges_overlap(outs[i], out_bytes[i], outs[j], out_bytes[j]))
+                return fail(FFTCONV_ERR_INVALID_ARG, "two outputs of the backward pass overlap");
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    // dv = dy * conv(u * w, k): the forward pass with dy as the output gate
+    if (dv) {
+        ForwardArgs a{u, w, dy, dv, K_f, nullptr, 0, B};
+        e = tc_forward(p, a, s);
+    }
+    // du = w * corr(dy * v, k), dw = u * corr(dy * v, k)
+    if (e == cudaSuccess) {
+        ForwardArgs a{dy, v, w, du, K_f, nullptr, 0, B};
+        e = tc_planar_correlate(p, a, dw, u, s);
+    }
+    // dk = sum_b corr(dy * v, u * w)[:L]
+    if (e == cudaSuccess && dk) e = simt_filter_grad(p, u, w, v, dy, B, dk, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return FFTCONV_OK;
 }
 

@@ -38,6 +38,9 @@ struct Plan {
     // staged: Ltab = C).
     float2* tw = nullptr;
     int logTab = 0;
+    // exp(-2 pi i e / 2N), e < 2N: the transform table of the backward pass's
+    // filter gradient (tensor-core plans with N <= 4096)
+    float2* twgrad = nullptr;
 
     // staged path: M = R * C, two-level table for exp(-2 pi i e / M)
     int logR = 0, logC = 0;
@@ -111,6 +114,11 @@ void tc_planar_free(Plan& p);
 cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& a, bool windows, cudaStream_t s);
 cudaError_t tc_planar_export(const Plan& p, const void* Kf, float* out, cudaStream_t s);
+// backward pass (N <= 4096): the correlation launch of the planar kernel and
+// the filter gradient on fp32 lanes (simt_kernels.cu)
+cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& a, void* y2, const void* v2, cudaStream_t s);
+cudaError_t simt_filter_grad(const Plan& p, const void* u, const void* w, const void* v, const void* dy, int64_t B,
+                             float* dk, cudaStream_t s);
 
 // staged path with the tensor-core row pass (rows of C = 8192): the column
 // passes are the SIMT ones (simt_kernels.cu), the row pass and the filter

@@ -404,6 +404,61 @@ simt_precompute_tc_split_kernel(const T* __restrict__ k, int64_t L, __half2* __r
     if (tid == 0) scales[h] = sc;
 }
 
+// Filter gradient of the backward pass: dk[h, s] = sum_b sum_t g_b[t] x_b[t-s]
+// for s < L, with g = dy * v and x = u * w (gates absent: ones).  One CTA per
+// (channel, chunk of batch rows): each row's g and x ride in the real and
+// imaginary parts of one complex sequence z = g + i x, zero-padded to M; its
+// spectrum Z gives G = (Z[f] + conj Z[M-f]) / 2 and X = (Z[f] - conj Z[M-f]) / 2i
+// (g and x are real), and the CTA accumulates G conj(X) (the spectrum of the
+// correlation, exact for s < N since the padding absorbs the wrap).  One
+// inverse transform of the sum then gives the CTA's part of dk, added to the
+// (zeroed) output with atomics.  The accumulator sits in shared memory beside
+// the transform buffer, indexed by permuted position like the spectrum.
+template <int LOGM, typename T>
+__global__ void __launch_bounds__(fused_threads<LOGM>())
+simt_filter_grad_kernel(const T* __restrict__ u, const T* __restrict__ w, const T* __restrict__ v,
+                        const T* __restrict__ dy, int64_t B, int64_t H, int64_t L, int64_t rows,
+                        float* __restrict__ dk, const float2* __restrict__ tw) {
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    constexpr int M = 1 << LOGM;
+    constexpr int64_t N = M / 2;
+    extern __shared__ float2 s[];
+    float2* acc = s + smem_elems<1>(M);
+    const int tid = threadIdx.x;
+    const int64_t h = blockIdx.x;
+    const int64_t b0 = (int64_t)blockIdx.y * rows, b1 = b0 + rows < B ? b0 + rows : B;
+    for (int p = tid; p < M; p += NT) acc[p] = make_float2(0.f, 0.f);
+    for (int64_t b = b0; b < b1; ++b) {
+        const int64_t o = (b * H + h) * N;
+        PairRows<T> io;
+        io.u0 = dy + o;
+        io.w0 = v ? v + o : nullptr;
+        io.u1 = u + o;
+        io.w1 = w ? w + o : nullptr;
+        io.nvalid = (int)N;
+        __syncthreads();                       // the previous row's spectrum has been read
+        first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+        __syncthreads();
+        fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
+        for (int p = tid; p < M; p += NT) {
+            const int f = (int)perm_to_freq(p, LOGM);
+            const int pm = (int)freq_to_perm((M - f) & (M - 1), LOGM);
+            const float2 zf = s[sidx<1>(p, 0)], zm = s[sidx<1>(pm, 0)];
+            // G = (zf + conj zm) / 2, X = (zf - conj zm) / 2i
+            const float2 G = make_float2(0.5f * (zf.x + zm.x), 0.5f * (zf.y - zm.y));
+            const float2 X = make_float2(0.5f * (zf.y + zm.y), 0.5f * (zm.x - zf.x));
+            acc[p] = cadd(acc[p], cmulc(G, X));
+        }
+    }
+    __syncthreads();
+    for (int p = tid; p < M; p += NT) s[sidx<1>(p, 0)] = acc[p];
+    __syncthreads();
+    inv_stages<LOGM, 0, K, 1, NT>(s, tw, 0, tid);
+    const float inv = 1.0f / (float)M;
+    for (int t = tid; t < L; t += NT) atomicAdd(&dk[h * L + t], s[sidx<1>(t, 0)].x * inv);
+}
+
 template <int LOGM, typename T>
 cudaError_t launch_fused(const Plan& p, const ForwardArgs& a, cudaStream_t st) {
     constexpr int NT = fused_threads<LOGM>();
@@ -1047,6 +1102,54 @@ cudaError_t simt_precompute_to_tc_pp(const Plan& p, const void* k, void* Kf, cud
                                                                (float*)((uint8_t*)Kf + (size_t)p.H * (8192 * 4)), p.tw);
         return cudaGetLastError();
     })
+}
+
+template <int LOGM, typename T>
+cudaError_t launch_filter_grad(const Plan& p, const void* u, const void* w, const void* v, const void* dy,
+                               int64_t B, float* dk, const float2* tw, cudaStream_t st) {
+    constexpr int NT = fused_threads<LOGM>();
+    const size_t smem = sizeof(float2) * (smem_elems<1>(1 << LOGM) + (1 << LOGM));
+    auto kern = simt_filter_grad_kernel<LOGM, T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // rows per CTA: enough CTAs to fill the GPU several times over, each
+    // amortising its inverse transform over several rows
+    int64_t rows = (B + 7) / 8;
+    if (rows < 1) rows = 1;
+    const int64_t chunks = (B + rows - 1) / rows;
+    dim3 grid((unsigned)p.H, (unsigned)chunks);
+    kern<<<grid, NT, smem, st>>>((const T*)u, (const T*)w, (const T*)v, (const T*)dy, B, p.H, p.L, rows, dk, tw);
+    return cudaGetLastError();
+}
+
+// dk (fp32, [H, L]) <- the filter gradient over the batch; the plan's
+// transform length M = 2N (N <= 4096) and an exp(-2 pi i e / M) table
+cudaError_t simt_filter_grad(const Plan& p, const void* u, const void* w, const void* v, const void* dy, int64_t B,
+                             float* dk, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)(p.H * p.L), st);
+    if (e != cudaSuccess || B == 0) return e;
+    const float2* tw = p.twgrad;
+    switch (p.dtype) {
+        case kBF16:
+            switch (p.logM) {
+                case 9: return launch_filter_grad<9, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                case 10: return launch_filter_grad<10, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                case 11: return launch_filter_grad<11, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                case 12: return launch_filter_grad<12, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                case 13: return launch_filter_grad<13, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                default: return cudaErrorInvalidValue;
+            }
+        case kF16:
+            switch (p.logM) {
+                case 9: return launch_filter_grad<9, __half>(p, u, w, v, dy, B, dk, tw, st);
+                case 10: return launch_filter_grad<10, __half>(p, u, w, v, dy, B, dk, tw, st);
+                case 11: return launch_filter_grad<11, __half>(p, u, w, v, dy, B, dk, tw, st);
+                case 12: return launch_filter_grad<12, __half>(p, u, w, v, dy, B, dk, tw, st);
+                case 13: return launch_filter_grad<13, __half>(p, u, w, v, dy, B, dk, tw, st);
+                default: return cudaErrorInvalidValue;
+            }
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t simt_fused_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t st) {

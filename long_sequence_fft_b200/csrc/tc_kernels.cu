@@ -1157,7 +1157,7 @@ __global__ void tc_export_kernel(const __half2* __restrict__ Kh, const float* __
 // the parity split unless the filter is short enough for windows; longer
 // sequences need windows (filters of at most 2049 taps).
 int tc_mode(int64_t N, int64_t L) {
-    if (N == kN) return kModePlain;
+    if (N <= kN) return kModePlain;      // N < 4096: several sequences per transform (tc_planar.cu)
     if (N == 2 * kN && L > kHop + 1) return kModeSplit;
     return kModeWindows;
 }
@@ -1166,11 +1166,11 @@ int tc_mode(int64_t N, int64_t L) {
 
 bool tc_supported(int64_t N, int64_t L, int dtype) {
     if (dtype != kF16 && dtype != kBF16) return false;
-    if (N == kN || N == 2 * kN) return true;
+    if (N <= kN || N == 2 * kN) return true;
     return N > kN && L <= kHop + 1;      // overlap-save windows (N a power of two)
 }
 
-int64_t tc_windows(int64_t N) { return N == kN ? 1 : N / kHop - 1; }
+int64_t tc_windows(int64_t N) { return N <= kN ? 1 : N / kHop - 1; }
 bool tc_overlap_save(int64_t N, int64_t L) { return tc_mode(N, L) == kModeWindows; }
 int64_t tc_tiles_per_pair_group(int64_t N, int64_t L) {
     const int m = tc_mode(N, L);

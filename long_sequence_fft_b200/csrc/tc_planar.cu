@@ -140,7 +140,8 @@ struct PArgs {
     const uint8_t* mask;
     int64_t mask_h;
     int64_t B, H, N;
-    int64_t nwin;               // windows per sequence (1 for N = 4096)
+    int64_t nwin;               // windows per sequence (1 for N <= 4096)
+    int lseg;                   // log2(N / 256) for N <= 4096: 4096 / N sequences share a transform
     int64_t pb;                 // pairs per channel, ceil(B/2)
     int64_t tpc;                // tiles per window, ceil(pb/4)
     int64_t nunits;             // H * nwin * tpc
@@ -148,6 +149,10 @@ struct PArgs {
     const uint32_t* tw1024;     // exp(-2 pi i e/1024) as half2, e < 1024
     const uint32_t* tw8192;     // exp(-2 pi i e/8192) as half2, e < 256
     int* status;
+    // backward (correlation) launches: a second output y2 = s_h v2 z beside
+    // y = s_h v z (y2 may be NULL)
+    void* y2;
+    const void* v2;
 };
 
 template <typename T>
@@ -205,36 +210,58 @@ struct PairInfo {
     bool tail_only;      // only window positions t >= kHop are outputs
 };
 
-// A tile holds 4 pairs of batch rows of one channel and one window: unit u
-// covers channel u / (nwin*tpc), window j = (u / tpc) % nwin and pairs
-// 4*(u % tpc) + q, q < 4 (pairs past ceil(B/2) are empty).  Window j starts
-// at 2048 j; window 0 keeps all 4096 outputs, window j > 0 keeps positions
-// [2048, 4096) (the overlap-save rule: its transform is exact from window
-// position L - 1 on, and L <= 2049).
+// A tile holds 4 transform rows of one channel and one window; each row is
+// the complex sequence of a pair of batch rows (the two real sequences are its
+// real and imaginary parts).  Sequences of N = 4096: unit u covers channel
+// u / (nwin*tpc), window j = (u / tpc) % nwin and pairs 4*(u % tpc) + q,
+// q < 4 (pairs past ceil(B/2) are empty); window j starts at 2048 j; window
+// 0 keeps all 4096 outputs, window j > 0 keeps positions [2048, 4096) (the
+// overlap-save rule: its transform is exact from window position L - 1 on,
+// and L <= 2049).
+// Shorter sequences (N = 256 .. 2048) are packed: transform row q holds the
+// S = 4096 / N pairs q S + sigma (sigma < S) at positions [2N sigma,
+// 2N sigma + N), each followed by N zeros, so a tile covers 4 S pairs.  The
+// 8192-point circular convolution of such a row is the causal convolution of
+// each pair, exactly: a filter of at most N taps reaches back at most N - 1
+// positions, into that pair's own zeros (or, for sigma = 0, around the end
+// of the row into the last pair's zeros).
+struct TileBase {
+    int64_t h, bp0, j;   // channel, first pair of the tile, window
+};
 template <bool WIN>
-__device__ __forceinline__ PairInfo pair_info(const PArgs& a, int64_t unit, int q, int64_t* h_out) {
-    PairInfo p;
-    int64_t h, j, bp;
+__device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
+    TileBase t;
     if constexpr (!WIN) {
-        h = unit / a.tpc;
-        j = 0;
-        bp = 4 * (unit % a.tpc) + q;
+        t.h = unit / a.tpc;
+        t.j = 0;
+        t.bp0 = (unit - t.h * a.tpc) * (64 >> a.lseg);
     } else {
         const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
         const uint32_t hh = un / per_ch, rem = un - hh * per_ch, jj = rem / tpc;
-        h = hh;
-        j = jj;
-        bp = 4 * (int64_t)(rem - jj * tpc) + q;
+        t.h = hh;
+        t.j = jj;
+        t.bp0 = 4 * (int64_t)(rem - jj * tpc);
     }
+    return t;
+}
+// rows of transform row q, segment sigma of a tile
+template <bool WIN>
+__device__ __forceinline__ PairInfo pair_rows(const PArgs& a, const TileBase& t, int q, int sigma) {
+    PairInfo p;
+    const int64_t bp = t.bp0 + ((int64_t)q << (4 - a.lseg)) + sigma;
     p.valid = bp < a.pb;
-    p.tail_only = j > 0;
+    p.tail_only = t.j > 0;
     const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
-    const int64_t base = WIN ? kHop * j : 0;
-    p.o0 = (b0 * a.H + h) * a.N + base;
-    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + h) * a.N + base : -1;
-    *h_out = h;
+    const int64_t base = WIN ? kHop * t.j : 0;
+    p.o0 = (b0 * a.H + t.h) * a.N + base;
+    p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + t.h) * a.N + base : -1;
     return p;
 }
+// kept stage-1 index i (< 16) -> its segment and the position of its first
+// element in the segment: j1 = the i-th digit with (j1 mod 2^(lseg+1)) <
+// 2^lseg, t = 256 j1 + 8 l + j3
+__device__ __forceinline__ int seg_of(const PArgs& a, int i) { return i >> a.lseg; }
+__device__ __forceinline__ int tau_of(const PArgs& a, int i) { return 256 * (i & ((1 << a.lseg) - 1)); }
 
 template <bool WIN>
 __device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
@@ -242,7 +269,10 @@ __device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
     return u / a.tpc;
 }
 
-template <typename T, bool WIN>
+// BWD: the correlation of the backward pass -- the product with conj(K)
+// instead of K (the filter is real, so that is correlation with k) and the
+// second output y2.
+template <typename T, bool WIN, bool BWD = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -345,32 +375,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 const int sb = chunk_stage_barrier(c);
                 if (sb >= 0 && !wait(&bar_stage[sb], iter & 1)) { ok = false; fail(); break; }
                 tc_fence_after();
-                if (lane == 0) {
+                {
+                    // the whole warp evaluates the operands; one elected lane issues
                     const uint32_t d = tbase + 256 + 64 * b;
                     if (stage == 0) {            // S1: A1 cols 16 j3 + (PP j1), j3 = k
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) mma_ts(d, tbase + 16 * k + 8 * ks, dS1 + 128 * ks, id64, ks);
+                        for (int ks = 0; ks < 2; ++ks)
+                            mma_ts_warp(d, tbase + 16 * k + 8 * ks, dS1 + 128 * ks, id64, ks);
                     } else if (stage == 1) {     // S2: MN-major tile j3 = k
                         const uint64_t da = dAmn + (uint64_t)(k * (kTile >> 4));
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) mma_ss(d, da + 128 * s, dS2 + 128 * s, id64t, s);
+                        for (int s = 0; s < 4; ++s) mma_ss_warp(d, da + 128 * s, dS2 + 128 * s, id64t, s);
                     } else if (stage == 2 || stage == 3) {   // S3 / S3': c2 = 4k + cl, A cols 8 c2
                         const uint64_t db = (stage == 2 ? dS3 : dS3i) + (uint64_t)(4 * k * 32);
 #pragma unroll
-                        for (int cl = 0; cl < 4; ++cl) mma_ts(d + 16 * cl, tbase + 8 * (4 * k + cl), db + 32 * cl, id16, 0);
+                        for (int cl = 0; cl < 4; ++cl)
+                            mma_ts_warp(d + 16 * cl, tbase + 8 * (4 * k + cl), db + 32 * cl, id16, 0);
                     } else if (stage == 4) {     // S2': K-major tile j3 = k
                         const uint64_t da = dAk + (uint64_t)(k * (kTile >> 4));
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) mma_ss(d, da + 2 * s, dS2i + 128 * s, id64, s);
+                        for (int s = 0; s < 4; ++s) mma_ss_warp(d, da + 2 * s, dS2i + 128 * s, id64, s);
                     } else {                     // S1': j3 = 2k + jl, MN-major tiles, N = 32 (16 kept j1)
 #pragma unroll
                         for (int jl = 0; jl < 2; ++jl) {
                             const uint64_t da = dAmn + (uint64_t)((2 * k + jl) * (kTile >> 4));
 #pragma unroll
-                            for (int s = 0; s < 4; ++s) mma_ss(d + 32 * jl, da + 128 * s, dS1i + 64 * s, id32t, s);
+                            for (int s = 0; s < 4; ++s) mma_ss_warp(d + 32 * jl, da + 128 * s, dS1i + 64 * s, id32t, s);
                         }
                     }
-                    tc_commit(&dfull[b]);
+                    tc_commit_warp(&dfull[b]);
                 }
                 __syncwarp();
                 if (c == issuer + 12) {
@@ -378,11 +411,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     // sequences of each pair, and the filter spectrum): issuer i
                     // takes pair i
                     const void* pf_src = nullptr;
-                    uint32_t pf_bytes = kN * sizeof(T);
+                    uint32_t pf_bytes = (uint32_t)(a.N < kN ? a.N : kN) * sizeof(T);
                     const int64_t nu = unit + gridDim.x;
-                    if (nu < a.nunits && (lane >> 3) == issuer) {
-                        int64_t hn;
-                        const PairInfo Q = pair_info<WIN>(a, nu, issuer, &hn);
+                    // (packed short sequences: the row's first segments only)
+                    if (nu < a.nunits && (lane >> 3) < (16 >> a.lseg)) {
+                        const TileBase tb = tile_base<WIN>(a, nu);
+                        const int64_t hn = tb.h;
+                        const PairInfo Q = pair_rows<WIN>(a, tb, issuer, lane >> 3);
                         const int which = lane & 7;
                         if (Q.valid) {
                             if (which == 0) pf_src = (const T*)a.u + Q.o0;
@@ -391,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             else if (which == 3 && Q.o1 >= 0) pf_src = (const T*)a.u + Q.o1;
                             else if (which == 4 && Q.o1 >= 0 && a.w) pf_src = (const T*)a.w + Q.o1;
                             else if (which == 5 && Q.o1 >= 0 && a.v) pf_src = (const T*)a.v + Q.o1;
-                            else if (which == 6 && issuer == 0) {
+                            else if (which == 6 && issuer == 0 && (lane >> 3) == 0) {
                                 pf_src = a.K + hn * kM;
                                 pf_bytes = kKBytes;
                             }
@@ -441,33 +476,49 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         // row); part 1 then arrives on bar_in.  A tile's input is loaded while
         // the previous tile's last stages run (the A columns are free once S3'
         // is done).  Absent rows or gates read a present row and are masked.
-        auto load_tile = [&](int64_t lu, int part) {
-            int64_t hl;
-            const PairInfo LP = pair_info<WIN>(a, lu, q, &hl);
-            const bool hasL = LP.o1 >= 0;
-            const int64_t oo1 = hasL ? LP.o1 : LP.o0;
-            const T* pu0 = (const T*)a.u + LP.o0;
-            const T* pw0 = a.w ? (const T*)a.w + LP.o0 : pu0;
-            const T* pu1 = (const T*)a.u + oo1;
-            const T* pw1 = a.w ? (const T*)a.w + oo1 : pu1;
+        // ---- load: x = u*w for t = 256 j1 + 8 l + j3 (l = lane), j1 the kept
+        // stage-1 digits of index 2P and 2P+1 with P = 2s + part, into the TMEM
+        // A1 columns 16 j3 + 2P (real pair) and 16 j3 + 2P + 1 (imaginary
+        // pair: the pair's second row); part 1 then arrives on bar_in.  A
+        // tile's input is loaded while the previous tile's last stages run
+        // (the A columns are free once S3' is done).  Absent rows or gates read
+        // a present row and are masked.
+        struct LoadPart {
+            uint4 ld[2][4];
+            bool keep0[2], keep1[2];
+        };
+        auto load_issue = [&](int64_t lu, int part, LoadPart& lp) {
+            const TileBase tb = tile_base<WIN>(a, lu);
             const bool has_w = a.w != nullptr;
             const int P = 2 * s + part;
-            uint4 ld[2][4];
 #pragma unroll
             for (int jh = 0; jh < 2; ++jh) {
-                const int64_t t0 = 256 * (2 * P + jh) + 8 * lane;
-                ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
-                ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
-                ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
-                ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+                // kept stage-1 index 2P + jh: its segment's rows and position
+                const int i = 2 * P + jh;
+                const PairInfo LP = pair_rows<WIN>(a, tb, q, seg_of(a, i));
+                const bool hasL = LP.o1 >= 0;
+                lp.keep0[jh] = LP.valid;
+                lp.keep1[jh] = hasL;
+                const int64_t oo1 = hasL ? LP.o1 : LP.o0;
+                const int64_t t0 = tau_of(a, i) + 8 * lane;
+                const T* pu0 = (const T*)a.u + LP.o0;
+                const T* pu1 = (const T*)a.u + oo1;
+                lp.ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
+                lp.ld[jh][1] = __ldg((const uint4*)((has_w ? (const T*)a.w + LP.o0 : pu0) + t0));
+                lp.ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
+                lp.ld[jh][3] = __ldg((const uint4*)((has_w ? (const T*)a.w + oo1 : pu1) + t0));
             }
+        };
+        auto load_finish = [&](int part, const LoadPart& lp) {
+            const bool has_w = a.w != nullptr;
+            const int P = 2 * s + part;
             float xa[2][8], xb[2][8];
 #pragma unroll
             for (int jh = 0; jh < 2; ++jh) {
-                const uint32_t ua[4] = {ld[jh][0].x, ld[jh][0].y, ld[jh][0].z, ld[jh][0].w};
-                const uint32_t wa[4] = {ld[jh][1].x, ld[jh][1].y, ld[jh][1].z, ld[jh][1].w};
-                const uint32_t ub[4] = {ld[jh][2].x, ld[jh][2].y, ld[jh][2].z, ld[jh][2].w};
-                const uint32_t wb[4] = {ld[jh][3].x, ld[jh][3].y, ld[jh][3].z, ld[jh][3].w};
+                const uint32_t ua[4] = {lp.ld[jh][0].x, lp.ld[jh][0].y, lp.ld[jh][0].z, lp.ld[jh][0].w};
+                const uint32_t wa[4] = {lp.ld[jh][1].x, lp.ld[jh][1].y, lp.ld[jh][1].z, lp.ld[jh][1].w};
+                const uint32_t ub[4] = {lp.ld[jh][2].x, lp.ld[jh][2].y, lp.ld[jh][2].z, lp.ld[jh][2].w};
+                const uint32_t wb[4] = {lp.ld[jh][3].x, lp.ld[jh][3].y, lp.ld[jh][3].z, lp.ld[jh][3].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float2 p0 = IO<T>::unpack2(ua[e]), p1 = IO<T>::unpack2(ub[e]);
@@ -475,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         const float2 g0 = IO<T>::unpack2(wa[e]), g1 = IO<T>::unpack2(wb[e]);
                         p0.x *= g0.x; p0.y *= g0.y; p1.x *= g1.x; p1.y *= g1.y;
                     }
-                    if (!LP.valid) p0 = make_float2(0.f, 0.f);
-                    if (!hasL) p1 = make_float2(0.f, 0.f);
+                    if (!lp.keep0[jh]) p0 = make_float2(0.f, 0.f);
+                    if (!lp.keep1[jh]) p1 = make_float2(0.f, 0.f);
                     xa[jh][2 * e] = p0.x; xa[jh][2 * e + 1] = p0.y;
                     xb[jh][2 * e] = p1.x; xb[jh][2 * e + 1] = p1.y;
                 }
@@ -491,6 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 if (lane == 0) mbar_arrive(bar_in);
             }
         };
+        auto load_tile = [&](int64_t lu, int part) {
+            LoadPart lp;
+            load_issue(lu, part, lp);
+            load_finish(part, lp);
+        };
 
         int iter = 0;
         bool ok = true;
@@ -500,9 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             load_tile(blockIdx.x, 1);
         }
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
-            int64_t hch;
-            const PairInfo P = pair_info<WIN>(a, unit, q, &hch);
-            const bool has1 = P.o1 >= 0;
+            const TileBase TB = tile_base<WIN>(a, unit);
+            const int64_t hch = TB.h;
             const uint32_t* Ks = (const uint32_t*)(smem + OffK);
             float kscale = __ldg(&a.Kscale[hch]);
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
@@ -624,6 +679,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             }
                         }
                     }
+                    if constexpr (BWD) {
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) kw[2 * p + 1] ^= kNegPair;   // conj(K)
+                    }
                     uint32_t h8[8];
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
@@ -676,26 +735,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             if (ok) stage_done(2);
             if (ok && unit + gridDim.x < a.nunits) load_tile(unit + gridDim.x, 1);
             // EO: lane = l; chunk 40 + k holds j3 = 2k + jl (jl = 0, 1) at
-            // columns 32 jl + PP(j1), j1 < 16.  This warp takes j1 = 4s + 2hf + jj
-            // in two halves hf: the PP words of j1 pair 2s + hf (columns
-            // 32 jl + 8s + 4hf .. + 3) of all four chunks give the eight
-            // consecutive t = 256 j1 + 8 l + j3 of each row: one 16-byte store.
-            // y = s_h v z; in a window after the first, positions t < 2048
-            // (j1 < 8: warps with s < 2) are not outputs.
+            // columns 32 jl + PP(i) for the kept stage-1 indices i < 16.  This
+            // warp takes i = 4s + 2hf + jj in two halves hf: the PP words of
+            // index pair 2s + hf (columns 32 jl + 8s + 4hf .. + 3) of all four
+            // chunks give the eight consecutive t = 256 j1 + 8 l + j3 of each
+            // row: one 16-byte store.  y = s_h v z; in a window after the
+            // first, positions t < 2048 (i < 8: warps with s < 2) are not
+            // outputs.
             {
-                const bool emit = P.valid && !(P.tail_only && s < 2);
-#pragma unroll 1
-                for (int hf = 0; hf < 2 && ok; ++hf) {
-                    const int jb = 4 * s + 2 * hf;            // this pass's first j1
-                    uint4 va[2], vb[2];
-                    {
-                        const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+                // the output gates of both halves, requested before the
+                // accumulator wait so that their latency overlaps it
+                uint4 vg[2][2][2];            // [hf][jj][row]
+                {
+                    const T* vr = a.v ? (const T*)a.v : (const T*)a.u;   // any readable row if no gate
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            const int64_t t0 = 256 * (jb + jj) + 8 * lane;
-                            va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
-                            vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                            const int i = 4 * s + 2 * hf + jj;
+                            const PairInfo Pg = pair_rows<WIN>(a, TB, q, seg_of(a, i));
+                            const int64_t tg = tau_of(a, i) + 8 * lane;
+                            vg[hf][jj][0] = __ldg((const uint4*)(vr + Pg.o0 + tg));
+                            vg[hf][jj][1] = __ldg((const uint4*)(vr + (Pg.o1 >= 0 ? Pg.o1 : Pg.o0) + tg));
                         }
+                }
+#pragma unroll
+                for (int hf = 0; hf < 2 && ok; ++hf) {
+                    const int jb = 4 * s + 2 * hf;            // this pass's first kept index
+                    PairInfo P[2];
+                    int64_t t0[2];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        P[jj] = pair_rows<WIN>(a, TB, q, seg_of(a, jb + jj));
+                        t0[jj] = tau_of(a, jb + jj) + 8 * lane;
                     }
                     if (hf == 0 && (!(ok = begin_pair(40)) || !(ok = begin_pair(42)))) break;
                     // r[cc][jl][0..3] = re(jb), re(jb+1), im(jb), im(jb+1) of j3 = 2cc + jl
@@ -709,31 +781,53 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         release(40);
                         release(42);
                     }
-                    if (emit) {
 #pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int64_t t0 = 256 * (jb + jj) + 8 * lane;
-                            const uint32_t vaw[4] = {va[jj].x, va[jj].y, va[jj].z, va[jj].w};
-                            const uint32_t vbw[4] = {vb[jj].x, vb[jj].y, vb[jj].z, vb[jj].w};
-                            uint32_t oa[4], ob[4];
+                    for (int jj = 0; jj < 2; ++jj) {
+                        if (!P[jj].valid || (P[jj].tail_only && s < 2)) continue;
+                        const bool has1 = P[jj].o1 >= 0;
+                        const uint32_t vaw[4] = {vg[hf][jj][0].x, vg[hf][jj][0].y, vg[hf][jj][0].z, vg[hf][jj][0].w};
+                        const uint32_t vbw[4] = {vg[hf][jj][1].x, vg[hf][jj][1].y, vg[hf][jj][1].z, vg[hf][jj][1].w};
+                        uint32_t oa[4], ob[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                // j3 = 2e (chunk 40 + e, jl 0) and 2e + 1 (jl 1)
-                                float a0 = __uint_as_float(r[e][0][jj]) * kscale;
-                                float a1 = __uint_as_float(r[e][1][jj]) * kscale;
-                                float b0 = __uint_as_float(r[e][0][2 + jj]) * kscale;
-                                float b1 = __uint_as_float(r[e][1][2 + jj]) * kscale;
-                                nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
-                                nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
-                                if (a.v) {
-                                    const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
-                                    a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
-                                }
-                                oa[e] = IO<T>::pack2(a0, a1);
-                                ob[e] = IO<T>::pack2(b0, b1);
+                        for (int e = 0; e < 4; ++e) {
+                            // j3 = 2e (chunk 40 + e, jl 0) and 2e + 1 (jl 1)
+                            float a0 = __uint_as_float(r[e][0][jj]) * kscale;
+                            float a1 = __uint_as_float(r[e][1][jj]) * kscale;
+                            float b0 = __uint_as_float(r[e][0][2 + jj]) * kscale;
+                            float b1 = __uint_as_float(r[e][1][2 + jj]) * kscale;
+                            nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
+                            nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
+                            if (a.v) {
+                                const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
+                                a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;
                             }
-                            *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-                            if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                            oa[e] = IO<T>::pack2(a0, a1);
+                            ob[e] = IO<T>::pack2(b0, b1);
+                        }
+                        *(uint4*)((T*)a.y + P[jj].o0 + t0[jj]) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                        if (has1) *(uint4*)((T*)a.y + P[jj].o1 + t0[jj]) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                        if constexpr (BWD) {
+                            if (a.y2) {
+                                // y2 = s_h v2 z: the same z, the second gate
+                                const uint4 ga = __ldg((const uint4*)((const T*)a.v2 + P[jj].o0 + t0[jj]));
+                                const uint4 gb = __ldg((const uint4*)((const T*)a.v2 + (has1 ? P[jj].o1 : P[jj].o0) +
+                                                                      t0[jj]));
+                                const uint32_t gaw[4] = {ga.x, ga.y, ga.z, ga.w};
+                                const uint32_t gbw[4] = {gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float a0 = __uint_as_float(r[e][0][jj]) * kscale;
+                                    const float a1 = __uint_as_float(r[e][1][jj]) * kscale;
+                                    const float b0 = __uint_as_float(r[e][0][2 + jj]) * kscale;
+                                    const float b1 = __uint_as_float(r[e][1][2 + jj]) * kscale;
+                                    const float2 g0 = IO<T>::unpack2(gaw[e]), g1 = IO<T>::unpack2(gbw[e]);
+                                    oa[e] = IO<T>::pack2(a0 * g0.x, a1 * g0.y);
+                                    ob[e] = IO<T>::pack2(b0 * g1.x, b1 * g1.y);
+                                }
+                                *(uint4*)((T*)a.y2 + P[jj].o0 + t0[jj]) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                                if (has1)
+                                    *(uint4*)((T*)a.y2 + P[jj].o1 + t0[jj]) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                            }
                         }
                     }
                 }
@@ -788,16 +882,22 @@ void put_matrix(std::vector<uint8_t>& img, size_t base, int n_out, int n_in, int
         }
 }
 
-std::vector<uint8_t> build_bimage() {
+// the stage-1 digit j1 of kept index i (< 16): the transform's inputs and the
+// kept outputs are the positions t = 256 j1 + 8 l + j3 with
+// (j1 mod 2^(lseg+1)) < 2^lseg (for N = 4096, lseg = 4: j1 < 16)
+int kept_j1(int i, int lseg) { return ((i >> lseg) << (lseg + 1)) | (i & ((1 << lseg) - 1)); }
+
+std::vector<uint8_t> build_bimage(int lseg) {
     std::vector<uint8_t> img(BImageBytes, 0);
     const double r32 = 1.0 / std::sqrt(32.0), r8 = 1.0 / std::sqrt(8.0);
     auto off = [](int o) { return (size_t)(o - OffBS1); };
     auto pp = [](int comp, int i) { return pp_index(comp, i); };
     auto pl32 = [](int comp, int i) { return pl_index(comp, i, 32); };
     std::vector<std::complex<double>> F;
-    // S1: c1 <- j1 (j1 < 16: the nonzero inputs)
+    // S1: c1 <- j1 (the 16 kept digits: the nonzero inputs)
     F.assign(32 * 16, 0);
-    for (int c = 0; c < 32; ++c) for (int j = 0; j < 16; ++j) F[c * 16 + j] = wpow((long long)c * j, 32, -1) * r32;
+    for (int c = 0; c < 32; ++c)
+        for (int j = 0; j < 16; ++j) F[c * 16 + j] = wpow((long long)c * kept_j1(j, lseg), 32, -1) * r32;
     put_matrix(img, off(OffBS1), 32, 16, 64, F, pp, pp);
     // S2: c2 <- l
     F.assign(32 * 32, 0);
@@ -819,9 +919,10 @@ std::vector<uint8_t> build_bimage() {
     F.assign(32 * 32, 0);
     for (int l = 0; l < 32; ++l) for (int c = 0; c < 32; ++c) F[l * 32 + c] = wpow((long long)c * l, 32, +1) * r32;
     put_matrix(img, off(OffBS2i), 32, 32, 64, F, pp, pp);
-    // S1': j1 <- c1 (j1 < 16: the kept outputs)
+    // S1': j1 <- c1 (the 16 kept digits: the outputs)
     F.assign(16 * 32, 0);
-    for (int j = 0; j < 16; ++j) for (int c = 0; c < 32; ++c) F[j * 32 + c] = wpow((long long)c * j, 32, +1) * r32;
+    for (int j = 0; j < 16; ++j)
+        for (int c = 0; c < 32; ++c) F[j * 32 + c] = wpow((long long)c * kept_j1(j, lseg), 32, +1) * r32;
     put_matrix(img, off(OffBS1i), 16, 32, 32, F, pl32, pp);
     return img;
 }
@@ -849,17 +950,19 @@ cudaError_t upload_vec(V** dst, const std::vector<V>& v) {
     return e;
 }
 
-template <typename T, bool WIN>
+template <typename T, bool WIN, bool BWD = false>
 void launch(const PArgs& a, int64_t grid, cudaStream_t s) {
-    tc_fftconv_planar_kernel<T, WIN><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
+    tc_fftconv_planar_kernel<T, WIN, BWD><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
 }
 
-// K_f (PP layout) -> rfft bins [0, N] of each channel
+// K_f (PP layout) -> rfft bins [0, N] of each channel's 2N-point spectrum:
+// bin f is bin f * (4096 / N) of the 8192-point spectrum of the zero-padded
+// filter (N <= 4096)
 __global__ void planar_export_kernel(const uint32_t* __restrict__ K, const float* __restrict__ scale,
-                                     float* __restrict__ out, int64_t H) {
-    const int64_t nb = kN + 1, total = H * nb;
+                                     float* __restrict__ out, int64_t H, int64_t N) {
+    const int64_t nb = N + 1, total = H * nb, stride = kN / N;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t h = i / nb, f = i % nb;
+        const int64_t h = i / nb, f = (i % nb) * stride;
         const int c1 = (int)(f & 31), c2 = (int)((f >> 5) & 31), c3 = (int)(f >> 10);
         const uint32_t* row = K + h * kM;
         const int wd = k_word(c1, c2, c3), half = c3 & 1;
@@ -872,10 +975,19 @@ __global__ void planar_export_kernel(const uint32_t* __restrict__ K, const float
 
 }  // namespace
 
+// log2(N / 256) for packed and single sequences (N <= 4096); overlap-save
+// windows (N > 4096) transform 4096 inputs each, like N = 4096
+static int plan_lseg(int64_t N) {
+    if (N > kN) return 4;
+    int l = 0;
+    while ((int64_t(256) << l) < N) ++l;
+    return l;
+}
+
 cudaError_t tc_planar_init(Plan& p) {
     Resources* r = new Resources();
     p.tcp = r;
-    cudaError_t e = upload_vec(&r->bimg, build_bimage());
+    cudaError_t e = upload_vec(&r->bimg, build_bimage(plan_lseg(p.N)));
     if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddles_h2(1024, 1024));
     if (e == cudaSuccess) e = upload_vec(&r->tw8192, twiddles_h2(kM, 256));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
@@ -891,6 +1003,12 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
     return e;
 }
 
@@ -923,8 +1041,10 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, bool windows
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H; a.N = p.N;
     a.nwin = windows ? p.N / kHop - 1 : 1;
+    a.lseg = plan_lseg(p.N);
     a.pb = (fa.B + 1) / 2;
-    a.tpc = (a.pb + 3) / 4;
+    const int64_t pairs_per_tile = int64_t(64) >> a.lseg;      // 4 rows x 4096 / N pairs
+    a.tpc = (a.pb + pairs_per_tile - 1) / pairs_per_tile;
     a.nunits = p.H * a.nwin * a.tpc;
     a.bimg = (const uint4*)r->bimg;
     a.tw1024 = r->tw1024;
@@ -941,12 +1061,42 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, bool windows
     return cudaGetLastError();
 }
 
+// Correlation pass of the backward (N <= 4096): y = v * corr(u * w, k),
+// y2 = v2 * corr(u * w, k) (y2 may be NULL), i.e. the forward kernel with the
+// product by conj(K) and a second gated output.
+cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& fa, void* y2, const void* v2, cudaStream_t s) {
+    if (p.N > kN) return cudaErrorInvalidValue;
+    const Resources* r = (const Resources*)p.tcp;
+    PArgs a{};
+    a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
+    a.y2 = y2; a.v2 = v2;
+    a.K = (const uint32_t*)fa.Kf;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.B = fa.B; a.H = p.H; a.N = p.N;
+    a.nwin = 1;
+    a.lseg = plan_lseg(p.N);
+    a.pb = (fa.B + 1) / 2;
+    const int64_t pairs_per_tile = int64_t(64) >> a.lseg;
+    a.tpc = (a.pb + pairs_per_tile - 1) / pairs_per_tile;
+    a.nunits = p.H * a.tpc;
+    a.bimg = (const uint4*)r->bimg;
+    a.tw1024 = r->tw1024;
+    a.tw8192 = r->tw8192;
+    a.status = p.status;
+    const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
+    if (p.dtype == kBF16) launch<__nv_bfloat16, false, true>(a, grid, s);
+    else launch<__half, false, true>(a, grid, s);
+    return cudaGetLastError();
+}
+
 cudaError_t tc_planar_export(const Plan& p, const void* Kf, float* out, cudaStream_t s) {
-    const int64_t total = p.H * (kN + 1);
+    if (p.N > kN) return cudaErrorInvalidValue;      // overlap-save plans store the 8192-point spectrum only
+    const int64_t total = p.H * (p.N + 1);
     int blocks = (int)((total + 255) / 256);
     if (blocks > 65535) blocks = 65535;
     planar_export_kernel<<<blocks, 256, 0, s>>>((const uint32_t*)Kf,
-                                                (const float*)((const uint8_t*)Kf + (size_t)p.H * kKBytes), out, p.H);
+                                                (const float*)((const uint8_t*)Kf + (size_t)p.H * kKBytes), out, p.H,
+                                                p.N);
     return cudaGetLastError();
 }
 

@@ -1,9 +1,10 @@
 """One process per GPU, channels sharded across ranks.
 
-Every (batch row, channel) sequence of the convolution is independent
-(FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
-Sec. 3: the convolution is applied per channel with its own filter), so a job
-of R ranks splits the channel axis: rank r owns channels [r*H, (r+1)*H), holds
+Every (batch row, channel) sequence of the convolution is independent: each
+output row depends only on its own input row and its channel's filter (the
+definition of the long convolution in "FlashFFTConv: Efficient Convolutions
+for Long Sequences with Tensor Cores", summary paragraph), so a job of R ranks
+splits the channel axis: rank r owns channels [r*H, (r+1)*H), holds
 only their filter spectra, and convolves its own inputs with no exchange on the
 data path.  The only collectives are the host plumbing around a timed region
 (a barrier and a max over ranks of the elapsed time) and an optional all-gather

@@ -59,10 +59,13 @@ def _bind(lib):
     lib.oracle_masked_filter_fft.argtypes = [dp, dp, i64, i64, i64, u8p, i64]
     lib.oracle_circular_conv_samples.argtypes = [dp, dp, dp, i64, i64, i64, dp, dp,
                                                  i64p, i64p, i64]
+    lib.oracle_conv_backward_direct.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, dp, dp, dp, dp]
+    lib.oracle_conv_backward_fft.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, dp, dp, dp, dp]
     for f in ("oracle_fft", "oracle_dft_direct", "oracle_fftconv",
               "oracle_filter_rfft", "oracle_direct_conv",
               "oracle_masked_filter_direct", "oracle_masked_filter_fft",
-              "oracle_circular_conv_samples"):
+              "oracle_circular_conv_samples", "oracle_conv_backward_direct",
+              "oracle_conv_backward_fft"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -206,6 +209,28 @@ def circular_conv_samples(u, keff, seq, ts, w=None, v=None):
                                                 _ptr(ts, ctypes.c_int64), seq.shape[0]),
            "circular_conv_samples")
     return y
+
+
+def conv_backward(u, k, dy, w=None, v=None, route="fft"):
+    """Gradients of y = v * conv(u * w, k) for the incoming gradient dy:
+    dict(du, dw, dv, dk) (dw only with w, dv only with v); dk is [H, L] summed
+    over the batch.  route "fft" (own FFT, any size) or "direct" (O(N*L)
+    sums)."""
+    u = _f64(u)
+    k = _f64(k)
+    dy = _f64(dy)
+    w = _f64(w)
+    v = _f64(v)
+    B, H, N = u.shape
+    L = k.shape[1]
+    du = np.empty((B, H, N))
+    dw = np.empty((B, H, N)) if w is not None else None
+    dv = np.empty((B, H, N)) if v is not None else None
+    dk = np.empty((H, L))
+    fn = _load().oracle_conv_backward_fft if route == "fft" else _load().oracle_conv_backward_direct
+    _check(fn(_ptr(u), _ptr(k), _ptr(w), _ptr(v), _ptr(dy), B, H, N, L, _ptr(du), _ptr(dw), _ptr(dv),
+              _ptr(dk)), "conv_backward")
+    return {"du": du, "dw": dw, "dv": dv, "dk": dk}
 
 
 def compile_variant(src_text: str, out_path: str) -> str:

@@ -396,3 +396,138 @@ int oracle_circular_conv_samples(const double* u, const double* keff, double* y,
     }
     return 0;
 }
+
+/* ------------------------------------------------------- backward pass --- */
+
+/* Gradients of the gated causal convolution, for training (page
+ * "FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores",
+ * "Key results": models trained with the convolution; the page states no
+ * backward, so these are the plain adjoints of the forward definition).
+ * With x = u*w, z[t] = sum_{s<=min(t,L-1)} k[s] x[t-s], y = v*z and the
+ * incoming gradient dy, and g = dy*v:
+ *     dv[t]  = dy[t] * z[t]
+ *     dx[t]  = sum_{s=0}^{min(L-1, N-1-t)} g[t+s] * k[s]      (correlation)
+ *     du[t]  = dx[t] * w[t],   dw[t] = dx[t] * u[t]
+ *     dk[h,s] = sum_b sum_{t=s}^{N-1} g_b[t] * x_b[t-s],   s < L
+ * Direct sums, O(N*L) per sequence.  Outputs may be NULL (not computed); dw
+ * needs w, dv needs v.  du, dw, dv: [B, H, N]; dk: [H, L].  Gates absent
+ * (NULL) are all ones. */
+int oracle_conv_backward_direct(const double* u, const double* k, const double* w,
+                                const double* v, const double* dy, int64_t B, int64_t H,
+                                int64_t N, int64_t L, double* du, double* dw, double* dv,
+                                double* dk) {
+    if (B < 0 || H <= 0 || N <= 0 || L <= 0 || L > N) return -1;
+    if ((dw && !w) || (dv && !v)) return -1;
+    double* g = (double*)malloc(sizeof(double) * (size_t)N);
+    double* x = (double*)malloc(sizeof(double) * (size_t)N);
+    if (!g || !x) { free(g); free(x); return -2; }
+    if (dk) memset(dk, 0, sizeof(double) * (size_t)(H * L));
+    for (int64_t s = 0; s < B * H; ++s) {
+        int64_t h = s % H;
+        const double* kh = k + h * L;
+        for (int64_t t = 0; t < N; ++t) {
+            x[t] = u[s * N + t] * (w ? w[s * N + t] : 1.0);
+            g[t] = dy[s * N + t] * (v ? v[s * N + t] : 1.0);
+        }
+        if (dv) {
+            for (int64_t t = 0; t < N; ++t) {
+                double z = 0.0;
+                int64_t smax = t < L - 1 ? t : L - 1;
+                for (int64_t q = 0; q <= smax; ++q) z += kh[q] * x[t - q];
+                dv[s * N + t] = dy[s * N + t] * z;
+            }
+        }
+        if (du || dw) {
+            for (int64_t t = 0; t < N; ++t) {
+                double acc = 0.0;
+                int64_t smax = (N - 1 - t) < (L - 1) ? (N - 1 - t) : (L - 1);
+                for (int64_t q = 0; q <= smax; ++q) acc += g[t + q] * kh[q];
+                if (du) du[s * N + t] = acc * (w ? w[s * N + t] : 1.0);
+                if (dw) dw[s * N + t] = acc * u[s * N + t];
+            }
+        }
+        if (dk) {
+            for (int64_t q = 0; q < L; ++q) {
+                double acc = 0.0;
+                for (int64_t t = q; t < N; ++t) acc += g[t] * x[t - q];
+                dk[h * L + q] += acc;
+            }
+        }
+    }
+    free(g); free(x);
+    return 0;
+}
+
+/* The same gradients by the FFT route (own radix-2 FFT, length M = 2N):
+ * dx = IFFT(FFT(g) * conj(FFT(k)))[:N] / M -- the circular correlation of the
+ * zero-padded g with the zero-padded k, which equals the linear correlation
+ * for t < N because the wrapped terms meet the padding -- and
+ * dk = IFFT(sum_b FFT(g_b) * conj(FFT(x_b)))[:L] / M; dv through the forward
+ * FFT route.  Usable at full sizes; pinned against the direct sums. */
+int oracle_conv_backward_fft(const double* u, const double* k, const double* w,
+                             const double* v, const double* dy, int64_t B, int64_t H,
+                             int64_t N, int64_t L, double* du, double* dw, double* dv,
+                             double* dk) {
+    if (B < 0 || H <= 0 || N <= 0 || (N & (N - 1)) || L <= 0 || L > N) return -1;
+    if ((dw && !w) || (dv && !v)) return -1;
+    int64_t M = 2 * N;
+    cplx* a = (cplx*)malloc(sizeof(cplx) * (size_t)M);
+    cplx* G = (cplx*)malloc(sizeof(cplx) * (size_t)M);
+    cplx* X = (cplx*)malloc(sizeof(cplx) * (size_t)M);
+    cplx* K = (cplx*)malloc(sizeof(cplx) * (size_t)M);
+    cplx* DK = (cplx*)malloc(sizeof(cplx) * (size_t)M);
+    cplx* twf = make_twiddles(M, -1);
+    cplx* twi = make_twiddles(M, +1);
+    int rc = 0;
+    if (!a || !G || !X || !K || !DK || !twf || !twi) { rc = -2; goto out; }
+    for (int64_t h = 0; h < H; ++h) {
+        for (int64_t t = 0; t < M; ++t) { a[t].re = (t < L) ? k[h * L + t] : 0.0; a[t].im = 0.0; }
+        fft_rec(a, K, M, 1, twf, 1);
+        for (int64_t f = 0; f < M; ++f) DK[f].re = DK[f].im = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            int64_t s = b * H + h;
+            for (int64_t t = 0; t < M; ++t) {
+                a[t].re = (t < N) ? dy[s * N + t] * (v ? v[s * N + t] : 1.0) : 0.0;
+                a[t].im = 0.0;
+            }
+            fft_rec(a, G, M, 1, twf, 1);
+            for (int64_t t = 0; t < M; ++t) {
+                a[t].re = (t < N) ? u[s * N + t] * (w ? w[s * N + t] : 1.0) : 0.0;
+                a[t].im = 0.0;
+            }
+            fft_rec(a, X, M, 1, twf, 1);
+            /* dk: accumulate G * conj(X) */
+            for (int64_t f = 0; f < M; ++f) {
+                DK[f].re += G[f].re * X[f].re + G[f].im * X[f].im;
+                DK[f].im += G[f].im * X[f].re - G[f].re * X[f].im;
+            }
+            if (dv) {   /* z = IFFT(X * K) */
+                for (int64_t f = 0; f < M; ++f) {
+                    a[f].re = X[f].re * K[f].re - X[f].im * K[f].im;
+                    a[f].im = X[f].re * K[f].im + X[f].im * K[f].re;
+                }
+                fft_rec(a, X, M, 1, twi, 1);
+                for (int64_t t = 0; t < N; ++t) dv[s * N + t] = dy[s * N + t] * X[t].re / (double)M;
+            }
+            if (du || dw) {   /* dx = IFFT(G * conj(K)) */
+                for (int64_t f = 0; f < M; ++f) {
+                    a[f].re = G[f].re * K[f].re + G[f].im * K[f].im;
+                    a[f].im = G[f].im * K[f].re - G[f].re * K[f].im;
+                }
+                fft_rec(a, G, M, 1, twi, 1);
+                for (int64_t t = 0; t < N; ++t) {
+                    double dx = G[t].re / (double)M;
+                    if (du) du[s * N + t] = dx * (w ? w[s * N + t] : 1.0);
+                    if (dw) dw[s * N + t] = dx * u[s * N + t];
+                }
+            }
+        }
+        if (dk) {
+            fft_rec(DK, a, M, 1, twi, 1);
+            for (int64_t q = 0; q < L; ++q) dk[h * L + q] = a[q].re / (double)M;
+        }
+    }
+out:
+    free(a); free(G); free(X); free(K); free(DK); free(twf); free(twi);
+    return rc;
+}

@@ -57,10 +57,18 @@ def test_small_shapes_full_compare(dtype, order, B, H, N):
 @pytest.mark.parametrize("order", [1, 4, 0])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_partial_and_masked(order, dtype, N):
+    import long_sequence_fft_b200 as lsf
     inp = _rand_inputs(3, 2, N, 300, dtype, gated=True, seed=7)
     y, _ = run_cuda(inp, dtype, order=order)
     assert_close(y, _oracle(inp), dtype, "partial L=300")
     inp = _rand_inputs(2, 3, N, N, dtype, gated=True, mask_frac=0.75, seed=8)
+    if dtype != "f32" and order == 0 and N < 4096:
+        # the tensor-core plan packs 4096 / N sequences into each transform
+        # and has no 2N-point spectrum to mask: masks need order 1 or 4
+        with pytest.raises(lsf.FFTConvError) as ei:
+            run_cuda(inp, dtype, order=order)
+        assert ei.value.status == lsf.ERR_UNSUPPORTED
+        order = 1
     y, _ = run_cuda(inp, dtype, order=order)
     assert_close(y, _oracle(inp), dtype, "masked per-channel")
     inp["mask"] = inp["mask"][:1]
@@ -259,7 +267,7 @@ def test_forward_host_pipelined_chunks_match_device_path():
     import long_sequence_fft_b200 as lsf
     import torch
     inp = _rand_inputs(19, 3, 2048, 2048, "bf16", gated=True, mask_frac=0.5, seed=11)
-    plan = lsf.Plan(2048, 3, "bf16")
+    plan = lsf.Plan(2048, 3, "bf16", order=1)         # (a masked plan at N < 4096: fp32 lanes)
     Kf = plan.precompute(to_dev(inp["k"], "bf16"))
     mask = torch.from_numpy(inp["mask"]).cuda()
     yd = plan.forward(to_dev(inp["u"], "bf16"), Kf, w=to_dev(inp["w"], "bf16"), v=to_dev(inp["v"], "bf16"),

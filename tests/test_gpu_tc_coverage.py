@@ -4,9 +4,10 @@
    of the persistent tensor-core kernel at least three tiles (148 CTAs at
    most: the "next tile loaded during the current tile's last stages" path and
    the split mode's parked z_even are exercised many times per CTA), in every
-   mode the kernel has: plain (N = 4096), overlap-save windows (partial
-   filters), the N = 8192 parity split (masked) and the staged path's row
-   pass.  The launch configuration is the plan's own, as in the benchmark.
+   mode the kernels have: plain (N = 4096), packed short sequences (N = 256 ..
+   2048, 4096 / N of them per 8192-point transform), overlap-save windows
+   (partial filters), the N = 8192 parity split (masked) and the staged path's
+   row pass.  The launch configuration is the plan's own, as in the benchmark.
 2. Closed forms the convolution must reproduce on every tensor-core mode
    (exact results of the definition "FlashFFTConv: Efficient Convolutions for
    Long Sequences with Tensor Cores", summary and "Approach", with the
@@ -72,6 +73,25 @@ def test_plain_mode_ragged_batch_many_tiles():
     _compare(_inputs(B, H, N, N, "f16", gated=False, seed=2), "f16", f"plain ragged {tiles} tiles")
 
 
+@pytest.mark.parametrize("N,B,H,L,gated,dtype", [(1024, 64, 240, 1024, True, "bf16"),
+                                                (2048, 16, 480, 2048, False, "f16"),
+                                                (512, 27, 450, 300, True, "bf16"),
+                                                (256, 33, 450, 256, False, "bf16")])
+def test_packed_mode_three_tiles_per_cta(N, B, H, L, gated, dtype):
+    pairs_per_tile = 4 * (4096 // N)
+    tiles = H * (((B + 1) // 2 + pairs_per_tile - 1) // pairs_per_tile)
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, L, dtype, gated=gated, seed=N + B), dtype, f"packed N={N} B={B} L={L} {tiles} tiles")
+
+
+def test_packed_mode_rejects_masks():
+    import long_sequence_fft_b200 as lsf
+    inp = _inputs(2, 2, 1024, 1024, "bf16", gated=False, mask_frac=0.5, seed=9)
+    with pytest.raises(lsf.FFTConvError) as ei:
+        run_cuda(inp, "bf16", order=0)
+    assert ei.value.status == lsf.ERR_UNSUPPORTED
+
+
 def test_windows_mode_three_tiles_per_cta():
     B, H, N, L = 16, 80, 8192, 2048
     tiles = H * (N // 2048 - 1) * ((B // 2 + 3) // 4)
@@ -99,6 +119,8 @@ def test_rows_mode_three_tiles_per_cta():
 
 MODES = [  # (name, N, L, order, path)
     ("plain", 4096, 4096, 0, "tc_fused"),
+    ("packed1k", 1024, 1024, 0, "tc_fused"),
+    ("packed256", 256, 256, 0, "tc_fused"),
     ("windows", 8192, 2048, 0, "tc_fused"),
     ("split", 8192, 8192, 0, "tc_fused"),
     ("rows", 16384, 16384, 5, "tc_staged"),
@@ -190,6 +212,7 @@ def _status_after(u, k, dtype, order, N, L):
 
 @pytest.mark.parametrize("name,N,L,order,path,edge,beyond", [
     ("plain", 4096, 4096, 0, "tc_fused", 90.0, 1500.0),
+    ("packed1k", 1024, 1024, 0, "tc_fused", 90.0, 6000.0),     # B = 2: one segment of 1024 per row
     ("windows", 8192, 2048, 0, "tc_fused", 90.0, 1500.0),
     ("split", 8192, 8192, 0, "tc_fused", 90.0, 3000.0),
     ("rows", 16384, 16384, 5, "tc_staged", 90.0, 2000.0),
