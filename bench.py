@@ -59,15 +59,21 @@ def mma_flops_per_elem(w: W.Workload, path: str):
     path issues, counted from the instruction shapes (complex values as real
     pairs: 2 flops per real multiply-add).  The 8192-point engine is
     32 x 32 x 8.  A zero-padded transform of 4096 inputs whose first 4096
-    outputs are kept (N = 4096, and each overlap-save window) issues
-    8*32 + 16*(32 + 8) = 896 per point of its window; a transform of all 8192
-    inputs and outputs (the N = 8192 parity split, the staged row pass)
-    16*(32 + 32 + 8) = 1152 per point.  fp32-lane paths issue none."""
+    outputs are kept (N = 4096, each overlap-save window, and a row of
+    4096/N packed shorter sequences, each in a zero-padded slot of 2N points)
+    issues 8*32 + 16*(32 + 8) = 896 per point of its window (also each block
+    of 4096 of the N = 8192 two-block mode); a transform of all 8192 inputs
+    and outputs (the N = 8192 parity split of masked calls, the staged row
+    pass) 16*(32 + 32 + 8) = 1152 per point.  fp32-lane paths issue none."""
     if path == "tc_fused":
         if w.N == 4096:
             return "32x32x8", 896.0
-        if w.N == 8192 and w.L > 2049:
-            return "32x32x8 (x2 parity halves)", 1152.0
+        if w.N < 4096:
+            return "32x32x8 (%d packed per row)" % (4096 // w.N), 896.0
+        if w.N == 8192:
+            if w.sparsity > 0:
+                return "32x32x8 (x2 parity halves)", 1152.0
+            return "32x32x8 (two blocks of 4096)", 896.0
         nwin = w.N // 2048 - 1
         return "32x32x8 windows", 896.0 * nwin * 4096 / w.N
     if path == "tc_staged":

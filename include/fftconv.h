@@ -72,8 +72,8 @@ typedef enum {
 /* Range of the 16-bit tensor-core paths (FFTCONV_PATH_TC_FUSED and
  * FFTCONV_PATH_TC_STAGED).  Their transform intermediates are fp16 (largest
  * finite value 65504); the fp32 paths (orders 1 and 4) keep fp32 throughout.
- *   - Fused kernel (N = 4096, the N = 8192 parity split, overlap-save
- *     windows): each unitary stage can grow a value by at most the number of
+ *   - Fused kernel (N <= 4096, N = 8192 as two blocks or, with a block
+ *     mask, split by bin parity, overlap-save windows): each unitary stage can grow a value by at most the number of
  *     its inputs over the square root of its length, so with max|u*w| <= 90
  *     no intermediate can overflow whatever the data and the filter.  Above
  *     that it depends on the data: a constant (DC) input overflows the forward
@@ -106,9 +106,11 @@ typedef enum {
  *   2, 3  fused: one kernel, the transform stays on chip (no intermediate in
  *         device memory).  This library's fused kernels split every transform
  *         they hold into three levels, so 2 and 3 are the same request.  They
- *         exist for N <= 8192 (tensor cores for fp16/bf16 at N = 4096 and
- *         8192; fp32 lanes otherwise) and, with filters of at most 2049 taps,
- *         for longer N as overlap-save windows of one fused transform each.
+ *         exist for N <= 8192 (tensor cores for fp16/bf16 at N = 256 ..
+ *         8192, N = 8192 as two blocks of 4096 or, for calls with a block
+ *         mask, as the 16384-point spectrum split by bin parity; fp32 lanes
+ *         otherwise) and, with filters of at most 2049 taps, for longer N as
+ *         overlap-save windows of one fused transform each.
  *         Orders 2 and 3 at N > 8192 with L > 2049 return
  *         FFTCONV_ERR_UNSUPPORTED: no fused kernel holds that transform on
  *         chip; orders 0, 4 and 5 serve it;
@@ -135,7 +137,7 @@ FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
  * partial convolution, defined as the convolution with k zero-padded to N
  * (FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
  * summary and "Approach": partial convolutions).
- * With a 16-bit dtype, N > 4096 and L <= 2049, orders 0, 2 and 3 choose the
+ * With a 16-bit dtype, N >= 16384 and L <= 2049, orders 0, 2 and 3 choose the
  * tensor-core path as overlap-save: windows of 4096 inputs with hop 2048, each
  * one 8192-point transform, N/2048 - 1 windows per sequence.  Such a plan
  * stores the 8192-point filter spectrum, so fftconv_forward rejects a

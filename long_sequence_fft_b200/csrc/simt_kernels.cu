@@ -155,9 +155,9 @@ constexpr int fused_threads() {
 
 // Stage 0 of the fused transform, reading the zero-padded input from global
 // memory: position j*S + r, j < R/2 (t < N); the upper half is zero.
-template <int LOGM, int NT, typename T>
+template <int LOGM, int NT, typename T, typename IOT = PairRows<T>>
 __device__ __forceinline__ void first_stage_global(float2* s, const float2* __restrict__ tw,
-                                                   const PairRows<T>& io, int tid) {
+                                                   const IOT& io, int tid) {
     constexpr int LB = Sched<LOGM>::bits(0);
     constexpr int R = 1 << LB;
     constexpr int S = 1 << (LOGM - LB);
@@ -356,6 +356,83 @@ simt_precompute_tc_pp_kernel(const T* __restrict__ k, int64_t L, __half* __restr
         const float2 z = s[sidx<1>(p, 0)];
         out[2 * word + (c3 & 1)] = __float2half_rn(z.x * inv);
         out[2 * word + 2 + (c3 & 1)] = __float2half_rn(z.y * inv);
+    }
+    if (tid == 0) scales[h] = sc;
+}
+
+// Filter taps of the two-block precompute as one complex row: real part
+// k[t] (t < min(L, 4096)), imaginary part k[4096 + t] (4096 + t < L).
+template <typename T>
+struct TwoBlockTaps {
+    const T* k;
+    int n0, n1;
+    __device__ __forceinline__ float2 load(int t) const {
+        return make_float2(t < n0 ? to_f32(k[t]) : 0.f, t < n1 ? to_f32(k[4096 + t]) : 0.f);
+    }
+};
+
+// Two-block filter rows of the planar tensor-core kernel (sequences of
+// 8192): with k0, k1 the taps [0, 4096) and [4096, 8192) of k,
+// G_0 = FFT_8192([k0; 0]) and G_1 = FFT_8192([k1; k0]) = H_1 + (-1)^f H_0
+// (H_b = FFT_8192([kb; 0]); the shift by 4096 is the sign (-1)^f).  One
+// transform of k0 + i k1 gives both: H_0[f] = (Z[f] + conj Z[-f]) / 2,
+// H_1[f] = (Z[f] - conj Z[-f]) / 2i.  Both rows in the PP layout of
+// simt_precompute_tc_pp_kernel, over one scale s_h = max |Re|, |Im| of G_0
+// and G_1, stored after the H row pairs.
+template <typename T>
+__global__ void __launch_bounds__(fused_threads<13>())
+simt_precompute_tc_pp2_kernel(const T* __restrict__ k, int64_t L, __half* __restrict__ Kh,
+                              float* __restrict__ scales, const float2* __restrict__ tw) {
+    constexpr int LOGM = 13;
+    constexpr int M = 1 << LOGM;
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    extern __shared__ float2 s[];
+    __shared__ float red[NT / 32];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x;
+    TwoBlockTaps<T> io;
+    io.k = k + (int64_t)h * L;
+    io.n0 = (int)(L < 4096 ? L : 4096);
+    io.n1 = (int)(L > 4096 ? L - 4096 : 0);
+    first_stage_global<LOGM, NT, T>(s, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
+    auto rows = [&](int p, int& f, float2& g0, float2& g1) {
+        f = (int)perm_to_freq(p, LOGM);
+        const int pm = (int)freq_to_perm((M - f) & (M - 1), LOGM);
+        const float2 z = s[sidx<1>(p, 0)], zm = s[sidx<1>(pm, 0)];
+        g0 = make_float2(0.5f * (z.x + zm.x), 0.5f * (z.y - zm.y));
+        const float2 h1 = make_float2(0.5f * (z.y + zm.y), -0.5f * (z.x - zm.x));
+        const float sg = (f & 1) ? -1.f : 1.f;
+        g1 = make_float2(h1.x + sg * g0.x, h1.y + sg * g0.y);
+    };
+    float m = 0.f;
+    for (int p = tid; p < M; p += NT) {
+        int f;
+        float2 g0, g1;
+        rows(p, f, g0, g1);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(g0.x), fabsf(g0.y)), fmaxf(fabsf(g1.x), fabsf(g1.y))));
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int i = 0; i < NT / 32; ++i) m = fmaxf(m, red[i]);
+    const float sc = m > 0.f ? m : 1.f;
+    const float inv = 1.f / sc;
+    __half* out0 = Kh + (int64_t)h * (4 * M);
+    __half* out1 = out0 + 2 * M;
+    for (int p = tid; p < M; p += NT) {
+        int f;
+        float2 g0, g1;
+        rows(p, f, g0, g1);
+        const int c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
+        const int word = ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + 2 * ((c3 & 3) >> 1);
+        out0[2 * word + (c3 & 1)] = __float2half_rn(g0.x * inv);
+        out0[2 * word + 2 + (c3 & 1)] = __float2half_rn(g0.y * inv);
+        out1[2 * word + (c3 & 1)] = __float2half_rn(g1.x * inv);
+        out1[2 * word + 2 + (c3 & 1)] = __float2half_rn(g1.y * inv);
     }
     if (tid == 0) scales[h] = sc;
 }
@@ -1087,6 +1164,19 @@ cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf,
         if (e != cudaSuccess) return e;
         kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>((const T*)k, p.L, (__half2*)Kf,
                                                                (float*)((uint8_t*)Kf + (size_t)p.H * (8192 * 4)), p.tw);
+        return cudaGetLastError();
+    })
+}
+
+cudaError_t simt_precompute_to_tc_pp2(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t st) {
+    if (p.L > 8192) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(float2) * smem_elems<1>(1 << 13);
+    FFTCONV_DISPATCH_T(p.dtype, {
+        auto kern = simt_precompute_tc_pp2_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>(
+            (const T*)k, p.L, (__half*)Kf, (float*)((uint8_t*)Kf + (size_t)p.H * 2 * (8192 * 4)), tw8192);
         return cudaGetLastError();
     })
 }

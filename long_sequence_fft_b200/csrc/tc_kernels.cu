@@ -1153,12 +1153,15 @@ __global__ void tc_export_kernel(const __half2* __restrict__ Kh, const float* __
     }
 }
 
-// Kernel mode of a plan: sequences of 4096 run plain; sequences of 8192 run
-// the parity split unless the filter is short enough for windows; longer
-// sequences need windows (filters of at most 2049 taps).
+// Kernel mode of a plan: sequences of 4096 run plain; sequences of 8192 carry
+// both the parity split's filter rows (calls with a frequency mask: the mask
+// acts on the 16384-point spectrum) and the two-block rows of the planar
+// kernel (every other call); longer sequences need windows (filters of at
+// most 2049 taps).
 int tc_mode(int64_t N, int64_t L) {
+    (void)L;
     if (N <= kN) return kModePlain;      // N < 4096: several sequences per transform (tc_planar.cu)
-    if (N == 2 * kN && L > kHop + 1) return kModeSplit;
+    if (N == 2 * kN) return kModeSplit;
     return kModeWindows;
 }
 
@@ -1237,6 +1240,8 @@ cudaError_t tc_plan_init(Plan& p) {
     if (e == cudaSuccess) e = set_smem_attributes<kModePlain>();
     if (e == cudaSuccess) e = set_smem_attributes<kModeWindows>();
     if (e == cudaSuccess) e = set_smem_attributes<kModeSplit>();
+    // unmasked calls run the planar kernel's two-block mode
+    if (e == cudaSuccess) e = tc_planar_init(p);
     return e;
 }
 
@@ -1257,19 +1262,31 @@ static int64_t tc_filter_rows(const Plan& p) { return tc_mode(p.N, p.L) == kMode
 
 // K_f: rows of 8192 complex fp16 (scaled so each channel's largest component
 // is 1; the split mode has two rows per channel, even and odd bins), then [H]
-// fp32 scales.
-size_t tc_filter_bytes(const Plan& p) {
+// fp32 scales; sequences of 8192 then append the two-block rows
+// (tc_planar_two_block_bytes).
+static size_t tc_split_bytes(const Plan& p) {
     return (size_t)tc_filter_rows(p) * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
+}
+size_t tc_filter_bytes(const Plan& p) {
+    return tc_split_bytes(p) + (tc_mode(p.N, p.L) == kModeSplit ? tc_planar_two_block_bytes(p) : 0);
 }
 
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
-    return tc_mode(p.N, p.L) == kModeSplit ? simt_precompute_to_tc_split(p, k, Kf, s)
-                                           : tc_planar_precompute(p, k, Kf, s);
+    if (tc_mode(p.N, p.L) != kModeSplit) return tc_planar_precompute(p, k, Kf, s);
+    cudaError_t e = simt_precompute_to_tc_split(p, k, Kf, s);
+    if (e == cudaSuccess) e = tc_planar_precompute_two_block(p, k, (uint8_t*)Kf + tc_split_bytes(p), s);
+    return e;
 }
 
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     const TcResources* r = (const TcResources*)p.tc;
-    if (r->mode != kModeSplit) return tc_planar_forward(p, fa, r->mode == kModeWindows, s);
+    if (r->mode != kModeSplit)
+        return tc_planar_forward(p, fa, r->mode == kModeWindows ? kPlanarWindows : kPlanarPlain, s);
+    if (!fa.mask) {
+        ForwardArgs two = fa;
+        two.Kf = (const uint8_t*)fa.Kf + tc_split_bytes(p);
+        return tc_planar_forward(p, two, kPlanarTwoBlock, s);
+    }
     TcArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.Kh16 = (const __half2*)fa.Kf;

@@ -1,7 +1,10 @@
 // tc_planar.cu -- tensor-core (tcgen05) fused FFT convolution with planar
 // complex data, sm_100a: sequences of 4096 (one zero-padded 8192-point
-// transform per sequence) and longer sequences with filters of at most 2049
-// taps (overlap-save windows of 4096 inputs, hop 2048).
+// transform per sequence; shorter ones packed several to a transform),
+// sequences of 8192 as two blocks of 4096 (a two-block partitioned
+// convolution: block b's output is X_b G_0 + X_{b-1} G_1 in the 8192-point
+// domain), and longer sequences with filters of at most 2049 taps
+// (overlap-save windows of 4096 inputs, hop 2048).
 //
 // FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
 // "Approach": the FFT convolution as an order-p Monarch decomposition --
@@ -58,6 +61,7 @@
 namespace fftconv {
 
 cudaError_t simt_precompute_to_tc_pp(const Plan& p, const void* k, void* Kf, cudaStream_t s);
+cudaError_t simt_precompute_to_tc_pp2(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t s);
 
 namespace {
 
@@ -88,7 +92,8 @@ constexpr int kKBytes = kM * 4;               // one filter spectrum row, 8192 c
 constexpr int OffK = OffBEnd;
 constexpr int OffTw = OffK + kKBytes;         // w8192^e, e < 256, as half2
 constexpr int OffBars = OffTw + 1024;
-constexpr int OffMisc = OffBars + 128;
+constexpr int OffXBars = OffBars + 128;       // two-block hand-over barriers [4 steps][4 slices][2]
+constexpr int OffMisc = OffXBars + 256;
 constexpr int SmemBytes = OffMisc + 64 + 1024;   // + alignment slack
 static_assert(SmemBytes <= 232448, "shared memory");
 
@@ -130,12 +135,18 @@ __device__ __forceinline__ uint32_t k_off(int m, int kbyte) {
     return swz((uint32_t)((m >> 3) * 1024 + (m & 7) * 128 + kbyte));
 }
 
+// kernel modes: one transform per row (N <= 4096, packed below), overlap-save
+// windows (N > 4096, filters of at most 2049 taps), two blocks (N = 8192)
+constexpr int kPlain = kPlanarPlain, kWin = kPlanarWindows, kTwo = kPlanarTwoBlock;
+
 struct PArgs {
     const void* u;
     const void* w;
     const void* v;
     void* y;
-    const uint32_t* K;          // [H][8192] words: the spectrum / scale, PP layout (k_word)
+    const uint32_t* K;          // [H][kstride] words: the spectrum / scale, PP layout (k_word)
+    int64_t kstride;            // words per channel: 8192, or 16384 (two-block: G_0 then G_1)
+    int g1_from_g0;             // two-block, L <= 4096: G_1 = (-1)^f G_0 (not read)
     const float* Kscale;        // [H]
     const uint8_t* mask;
     int64_t mask_h;
@@ -194,7 +205,25 @@ __device__ __forceinline__ void cmul_pp(uint32_t& xr, uint32_t& xi, uint32_t tr,
     xr = h2u(__hfma2(__hneg2(b), d, __hmul2(a, c)));
     xi = h2u(__hfma2(b, c, __hmul2(a, d)));
 }
+// (yr + i yi) += (xr + i xi) (tr + i ti), two values at once (PP words)
+__device__ __forceinline__ void cfma_pp(uint32_t& yr, uint32_t& yi, uint32_t xr, uint32_t xi, uint32_t tr,
+                                        uint32_t ti) {
+    const __half2 a = u2h(xr), b = u2h(xi), c = u2h(tr), d = u2h(ti);
+    yr = h2u(__hfma2(__hneg2(b), d, __hfma2(a, c, u2h(yr))));
+    yi = h2u(__hfma2(b, c, __hfma2(a, d, u2h(yi))));
+}
 constexpr uint32_t kNegPair = 0x80008000u;   // sign bits of both halves
+
+// Two-block hand-over slots of EK step st (byte offsets from the data
+// tiles): the bytes that E3' writes in the same step (K bytes [32 st,
+// 32 st + 32) of every row of every tile), 64 slots of 16 bytes per lane,
+// consecutive lanes on consecutive rows so that a warp's 16-byte accesses hit
+// distinct banks.  Slot z < 32: piece z % 4 of block 0's values from the warp
+// (slice s, pair pq), z = (2 s + pq) 4 + piece; slot 32 + z: the G_1 words
+// that the block-1 warp (slice s, pair pq) reads.
+__device__ __forceinline__ uint32_t xoff(int st, int z, int lane) {
+    return (uint32_t)((z >> 3) * kTile) + k_off(32 * (z & 3) + lane, 32 * st + 16 * ((z >> 2) & 1));
+}
 
 // word index of the filter spectrum value f = c1 + 32 c2 + 1024 c3 (its real
 // part; the imaginary part is the next word), and which half: 16-byte groups
@@ -225,16 +254,23 @@ struct PairInfo {
 // each pair, exactly: a filter of at most N taps reaches back at most N - 1
 // positions, into that pair's own zeros (or, for sigma = 0, around the end
 // of the row into the last pair's zeros).
+// Sequences of 8192 (two-block mode): a tile holds two pairs 2u', 2u'+1;
+// transform row q is block q >> 1 (inputs and outputs [4096 (q >> 1),
+// 4096 (q >> 1) + 4096)) of pair 2u' + (q & 1), zero-padded to 8192 points.
 struct TileBase {
     int64_t h, bp0, j;   // channel, first pair of the tile, window
 };
-template <bool WIN>
+template <int MODE>
 __device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
     TileBase t;
-    if constexpr (!WIN) {
+    if constexpr (MODE == kPlain) {
         t.h = unit / a.tpc;
         t.j = 0;
         t.bp0 = (unit - t.h * a.tpc) * (64 >> a.lseg);
+    } else if constexpr (MODE == kTwo) {
+        t.h = unit / a.tpc;
+        t.j = 0;
+        t.bp0 = (unit - t.h * a.tpc) * 2;
     } else {
         const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
         const uint32_t hh = un / per_ch, rem = un - hh * per_ch, jj = rem / tpc;
@@ -245,14 +281,14 @@ __device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
     return t;
 }
 // rows of transform row q, segment sigma of a tile
-template <bool WIN>
+template <int MODE>
 __device__ __forceinline__ PairInfo pair_rows(const PArgs& a, const TileBase& t, int q, int sigma) {
     PairInfo p;
-    const int64_t bp = t.bp0 + ((int64_t)q << (4 - a.lseg)) + sigma;
+    const int64_t bp = MODE == kTwo ? t.bp0 + (q & 1) : t.bp0 + ((int64_t)q << (4 - a.lseg)) + sigma;
     p.valid = bp < a.pb;
     p.tail_only = t.j > 0;
     const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
-    const int64_t base = WIN ? kHop * t.j : 0;
+    const int64_t base = MODE == kWin ? kHop * t.j : (MODE == kTwo ? (int64_t)kN * (q >> 1) : 0);
     p.o0 = (b0 * a.H + t.h) * a.N + base;
     p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + t.h) * a.N + base : -1;
     return p;
@@ -263,17 +299,18 @@ __device__ __forceinline__ PairInfo pair_rows(const PArgs& a, const TileBase& t,
 __device__ __forceinline__ int seg_of(const PArgs& a, int i) { return i >> a.lseg; }
 __device__ __forceinline__ int tau_of(const PArgs& a, int i) { return 256 * (i & ((1 << a.lseg) - 1)); }
 
-template <bool WIN>
+template <int MODE>
 __device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
-    if constexpr (WIN) return (int64_t)((uint32_t)u / ((uint32_t)a.nwin * (uint32_t)a.tpc));
+    if constexpr (MODE == kWin) return (int64_t)((uint32_t)u / ((uint32_t)a.nwin * (uint32_t)a.tpc));
     return u / a.tpc;
 }
 
 // BWD: the correlation of the backward pass -- the product with conj(K)
 // instead of K (the filter is real, so that is correlation with k) and the
 // second output y2.
-template <typename T, bool WIN, bool BWD = false>
+template <typename T, int MODE, bool BWD = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a) {
+    static_assert(!(BWD && MODE != kPlain), "the correlation pass runs on plain plans");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* bar = (uint64_t*)(smem + OffBars);
@@ -283,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
     uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
     uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
     uint64_t* bar_stage = bar + 11;   // [3] E2, E3', E2' done for the tile (16 epilogue warps)
+    // two-block mode: [EK step][slice][pair] block 0's spectrum values are in
+    // the hand-over slots (the 32 threads of that warp)
+    uint64_t* xfull = (uint64_t*)(smem + OffXBars);
     uint32_t* tmem_base_sh = (uint32_t*)(smem + OffMisc);
     volatile int* abort_flag = (volatile int*)(smem + OffMisc + 4);
 
@@ -303,6 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         mbar_init(bar_fin, kMmaWarps);
         mbar_init(bar_k, 1);
         for (int i = 0; i < 3; ++i) mbar_init(&bar_stage[i], kEpiWarps);
+        if constexpr (MODE == kTwo)
+            for (int i = 0; i < 32; ++i) mbar_init(&xfull[i], 32);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -362,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     // the previous tile is finished with the filter buffer (its
                     // epilogue warps arrived on bar_in after all their reads)
                     mbar_expect_tx(bar_k, kKBytes);
-                    bulk_copy_g2s(smem + OffK, a.K + unit_channel<WIN>(a, unit) * kM, kKBytes, bar_k);
+                    bulk_copy_g2s(smem + OffK, a.K + unit_channel<MODE>(a, unit) * a.kstride, kKBytes, bar_k);
                 }
                 ++k_issued;
                 __syncwarp();
@@ -415,9 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     const int64_t nu = unit + gridDim.x;
                     // (packed short sequences: the row's first segments only)
                     if (nu < a.nunits && (lane >> 3) < (16 >> a.lseg)) {
-                        const TileBase tb = tile_base<WIN>(a, nu);
+                        const TileBase tb = tile_base<MODE>(a, nu);
                         const int64_t hn = tb.h;
-                        const PairInfo Q = pair_rows<WIN>(a, tb, issuer, lane >> 3);
+                        const PairInfo Q = pair_rows<MODE>(a, tb, issuer, lane >> 3);
                         const int which = lane & 7;
                         if (Q.valid) {
                             if (which == 0) pf_src = (const T*)a.u + Q.o0;
@@ -427,7 +469,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             else if (which == 4 && Q.o1 >= 0 && a.w) pf_src = (const T*)a.w + Q.o1;
                             else if (which == 5 && Q.o1 >= 0 && a.v) pf_src = (const T*)a.v + Q.o1;
                             else if (which == 6 && issuer == 0 && (lane >> 3) == 0) {
-                                pf_src = a.K + hn * kM;
+                                pf_src = a.K + hn * a.kstride;
+                                pf_bytes = kKBytes;
+                            } else if (MODE == kTwo && which == 7 && issuer == 1 && (lane >> 3) == 0) {
+                                pf_src = a.K + hn * a.kstride + kM;     // G_1
                                 pf_bytes = kKBytes;
                             }
                         }
@@ -488,14 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             bool keep0[2], keep1[2];
         };
         auto load_issue = [&](int64_t lu, int part, LoadPart& lp) {
-            const TileBase tb = tile_base<WIN>(a, lu);
+            const TileBase tb = tile_base<MODE>(a, lu);
             const bool has_w = a.w != nullptr;
             const int P = 2 * s + part;
 #pragma unroll
             for (int jh = 0; jh < 2; ++jh) {
                 // kept stage-1 index 2P + jh: its segment's rows and position
                 const int i = 2 * P + jh;
-                const PairInfo LP = pair_rows<WIN>(a, tb, q, seg_of(a, i));
+                const PairInfo LP = pair_rows<MODE>(a, tb, q, seg_of(a, i));
                 const bool hasL = LP.o1 >= 0;
                 lp.keep0[jh] = LP.valid;
                 lp.keep1[jh] = hasL;
@@ -556,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             load_tile(blockIdx.x, 1);
         }
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
-            const TileBase TB = tile_base<WIN>(a, unit);
+            const TileBase TB = tile_base<MODE>(a, unit);
             const int64_t hch = TB.h;
             const uint32_t* Ks = (const uint32_t*)(smem + OffK);
             float kscale = __ldg(&a.Kscale[hch]);
@@ -647,24 +692,70 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             if (ok) stage_done(0);
             // EK: lane = c1; the PP columns of c3 (all eight) of c2 = 4(k+cc) + s;
             // times the filter spectrum K/scale (|K/scale| <= 1); A4 TMEM
-            // columns 8 c2 .. 8 c2 + 7 in place
+            // columns 8 c2 .. 8 c2 + 7 in place.
+            // Two-block mode: quarters 0, 1 hold block 0 (X_0) of their pair and
+            // quarters 2, 3 block 1 (X_1).  Block 0's output is X_0 G_0; block
+            // 1's is X_1 G_0 + X_0 G_1 (G_1 the spectrum of [k1; k0], which
+            // holds both the part of k that reaches from block 0 into block 1
+            // and the wrap-around of the 8192-point product).  The block-0
+            // warps hand their values over through the data tiles (free
+            // between S2 and E3'); G_1 comes from L2.
             if (ok && !(ok = wait(bar_k, iter & 1))) fail();
+            const bool x_give = MODE == kTwo && q < 2, x_take = MODE == kTwo && q >= 2;
+            const int xz = (2 * s + (q & 1)) * 4;       // this warp's slots (+ 32 for G_1)
+            uint8_t* const xs = smem + OffData;
+            if (x_take && ok && !a.g1_from_g0) {
+                // the block-1 warps fetch their G_1 words of all four steps into
+                // their slots (the data tiles are free: this warp's E2 waited for
+                // every S2 chunk)
+                const uint32_t* G1 = a.K + hch * a.kstride + kM;
+#pragma unroll
+                for (int st = 0; st < 4; ++st) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c2 = 4 * (2 * st + (e >> 1)) + s;
+                        cp_async16(xs + xoff(st, 32 + xz + e, lane), G1 + k_word(lane, c2, 4 * (e & 1)));
+                    }
+                    cp_async_commit();
+                }
+            }
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 16 + k;
+                const int st = k >> 1;
                 if (!(ok = begin_pair(c))) break;
                 uint32_t r[2][16];
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
                 tc_wait_ld();
                 release(c);
+                // h[cc]: the PP words of c2 = 4(k+cc) + s (all eight c3)
+                uint32_t h[2][8];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        h[cc][2 * p] = pk(r[cc][4 * p], r[cc][4 * p + 1]);
+                        h[cc][2 * p + 1] = pk(r[cc][4 * p + 2], r[cc][4 * p + 3]);
+                    }
+                uint64_t* xb = &xfull[(st * 4 + s) * 2 + (q & 1)];
+                if (x_give) {
+                    // hand block 0's values over before this warp's own product
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        *(uint4*)(xs + xoff(st, xz + 2 * cc, lane)) = make_uint4(h[cc][0], h[cc][1], h[cc][2], h[cc][3]);
+                        *(uint4*)(xs + xoff(st, xz + 2 * cc + 1, lane)) =
+                            make_uint4(h[cc][4], h[cc][5], h[cc][6], h[cc][7]);
+                    }
+                    mbar_arrive(xb);
+                }
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c2 = 4 * (k + cc) + s;
                     const uint4 k0 = *(const uint4*)(Ks + k_word(lane, c2, 0));
                     const uint4 k1 = *(const uint4*)(Ks + k_word(lane, c2, 4));
                     uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    if (mrow) {
+                    if (MODE != kTwo && mrow) {
                         // frequency-sparse filter: zero the masked bins (f and
                         // its mirror 8192 - f share one rfft bin)
 #pragma unroll
@@ -683,17 +774,51 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) kw[2 * p + 1] ^= kNegPair;   // conj(K)
                     }
-                    uint32_t h8[8];
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        h8[2 * p] = pk(r[cc][4 * p], r[cc][4 * p + 1]);
-                        h8[2 * p + 1] = pk(r[cc][4 * p + 2], r[cc][4 * p + 3]);
-                        cmul_pp(h8[2 * p], h8[2 * p + 1], kw[2 * p], kw[2 * p + 1]);
-                    }
-                    tmem_st8(tbase + lq + 8 * c2, h8);
+                    for (int p = 0; p < 4; ++p) cmul_pp(h[cc][2 * p], h[cc][2 * p + 1], kw[2 * p], kw[2 * p + 1]);
                 }
+                if (x_take) {
+                    // + X_0 G_1, once block 0's warp has handed X_0 over
+                    if (!(ok = wait(xb, iter & 1))) {
+                        fail();
+                        break;
+                    }
+                    if (!a.g1_from_g0) {      // this thread's G_1 copies of steps <= st have landed
+                        if (st == 0) cp_async_wait<3>();
+                        else if (st == 1) cp_async_wait<2>();
+                        else if (st == 2) cp_async_wait<1>();
+                        else cp_async_wait<0>();
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint4 x0 = *(const uint4*)(xs + xoff(st, xz + 2 * cc, lane));
+                        const uint4 x1 = *(const uint4*)(xs + xoff(st, xz + 2 * cc + 1, lane));
+                        const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                        uint32_t gw[8];
+                        if (a.g1_from_g0) {
+                            // k1 = 0: G_1 = (-1)^f G_0, and f = c1 (mod 2) = lane (mod 2)
+                            const int c2 = 4 * (k + cc) + s;
+                            const uint4 k0 = *(const uint4*)(Ks + k_word(lane, c2, 0));
+                            const uint4 k1 = *(const uint4*)(Ks + k_word(lane, c2, 4));
+                            const uint32_t sg = (lane & 1) ? kNegPair : 0u;
+                            gw[0] = k0.x ^ sg; gw[1] = k0.y ^ sg; gw[2] = k0.z ^ sg; gw[3] = k0.w ^ sg;
+                            gw[4] = k1.x ^ sg; gw[5] = k1.y ^ sg; gw[6] = k1.z ^ sg; gw[7] = k1.w ^ sg;
+                        } else {
+                            const uint4 g0 = *(const uint4*)(xs + xoff(st, 32 + xz + 2 * cc, lane));
+                            const uint4 g1 = *(const uint4*)(xs + xoff(st, 32 + xz + 2 * cc + 1, lane));
+                            gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
+                            gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
+                        }
+#pragma unroll
+                        for (int p = 0; p < 4; ++p)
+                            cfma_pp(h[cc][2 * p], h[cc][2 * p + 1], xw[2 * p], xw[2 * p + 1], gw[2 * p], gw[2 * p + 1]);
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) tmem_st8(tbase + lq + 8 * (4 * (k + cc) + s), h[cc]);
                 tc_wait_st();
             }
+            if (x_take && !a.g1_from_g0) cp_async_wait<0>();   // nothing in flight past here (also after an abort)
             // E3': lane = c1; chunk c + (s >> 1), its c2 = 4(k + cc) + cl for
             // cl < 4, j3 = 4h + jj with h = s & 1 (PP columns 16 cl + 8h ..
             // + 7); twiddle conj w8192^(c1 j3); K-major A5 tile j3, row
@@ -753,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
                             const int i = 4 * s + 2 * hf + jj;
-                            const PairInfo Pg = pair_rows<WIN>(a, TB, q, seg_of(a, i));
+                            const PairInfo Pg = pair_rows<MODE>(a, TB, q, seg_of(a, i));
                             const int64_t tg = tau_of(a, i) + 8 * lane;
                             vg[hf][jj][0] = __ldg((const uint4*)(vr + Pg.o0 + tg));
                             vg[hf][jj][1] = __ldg((const uint4*)(vr + (Pg.o1 >= 0 ? Pg.o1 : Pg.o0) + tg));
@@ -766,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     int64_t t0[2];
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
-                        P[jj] = pair_rows<WIN>(a, TB, q, seg_of(a, jb + jj));
+                        P[jj] = pair_rows<MODE>(a, TB, q, seg_of(a, jb + jj));
                         t0[jj] = tau_of(a, jb + jj) + 8 * lane;
                     }
                     if (hf == 0 && (!(ok = begin_pair(40)) || !(ok = begin_pair(42)))) break;
@@ -851,6 +976,7 @@ struct Resources {
     uint8_t* bimg = nullptr;
     uint32_t* tw1024 = nullptr;
     uint32_t* tw8192 = nullptr;
+    float2* twf8192 = nullptr;     // fp32 exp(-2 pi i e/8192), e < 8192 (two-block filter precompute)
     int num_sms = 0;
 };
 
@@ -950,9 +1076,15 @@ cudaError_t upload_vec(V** dst, const std::vector<V>& v) {
     return e;
 }
 
-template <typename T, bool WIN, bool BWD = false>
+template <typename T, int MODE, bool BWD = false>
 void launch(const PArgs& a, int64_t grid, cudaStream_t s) {
-    tc_fftconv_planar_kernel<T, WIN, BWD><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
+    tc_fftconv_planar_kernel<T, MODE, BWD><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
+}
+
+template <typename T, int MODE, bool BWD = false>
+cudaError_t allow_smem() {
+    return cudaFuncSetAttribute(tc_fftconv_planar_kernel<T, MODE, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemBytes);
 }
 
 // K_f (PP layout) -> rfft bins [0, N] of each channel's 2N-point spectrum:
@@ -991,24 +1123,22 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddles_h2(1024, 1024));
     if (e == cudaSuccess) e = upload_vec(&r->tw8192, twiddles_h2(kM, 256));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__nv_bfloat16, false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc_fftconv_planar_kernel<__half, false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
+    if (e == cudaSuccess && p.N == 2 * kN) {
+        std::vector<float2> t(kM);
+        for (int i = 0; i < kM; ++i) {
+            const std::complex<double> z = wpow(i, kM, -1);
+            t[i] = make_float2((float)z.real(), (float)z.imag());
+        }
+        e = upload_vec(&r->twf8192, t);
+    }
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kWin>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kTwo>();
+    if (e == cudaSuccess) e = allow_smem<__half, kPlain>();
+    if (e == cudaSuccess) e = allow_smem<__half, kWin>();
+    if (e == cudaSuccess) e = allow_smem<__half, kTwo>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain, true>();
+    if (e == cudaSuccess) e = allow_smem<__half, kPlain, true>();
     return e;
 }
 
@@ -1018,6 +1148,7 @@ void tc_planar_free(Plan& p) {
     cudaFree(r->bimg);
     cudaFree(r->tw1024);
     cudaFree(r->tw8192);
+    cudaFree(r->twf8192);
     delete r;
     p.tcp = nullptr;
 }
@@ -1028,22 +1159,40 @@ size_t tc_planar_filter_bytes(const Plan& p) {
     return (size_t)p.H * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
 }
 
+// Two-block K_f (sequences of 8192): per channel G_0 = FFT_8192([k0; 0]) and
+// G_1 = FFT_8192([k1; k0]) (k0, k1 the taps [0, 4096) and [4096, 8192) of k,
+// zero past L), PP layout over one common scale, then [H] fp32 scales
+size_t tc_planar_two_block_bytes(const Plan& p) {
+    return (size_t)p.H * 2 * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
+}
+
 cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
     return simt_precompute_to_tc_pp(p, k, Kf, s);
 }
 
-cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, bool windows, cudaStream_t s) {
+cudaError_t tc_planar_precompute_two_block(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
     const Resources* r = (const Resources*)p.tcp;
+    if (p.N != 2 * kN || !r->twf8192) return cudaErrorInvalidValue;
+    return simt_precompute_to_tc_pp2(p, k, Kf, r->twf8192, s);
+}
+
+// mode: kPlain (N <= 4096), kWin (overlap-save windows), kTwo (N = 8192,
+// fa.Kf the two-block filter rows)
+cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cudaStream_t s) {
+    const Resources* r = (const Resources*)p.tcp;
+    if (mode == kTwo && (p.N != 2 * kN || fa.mask)) return cudaErrorInvalidValue;
     PArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.K = (const uint32_t*)fa.Kf;
-    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.kstride = mode == kTwo ? 2 * kM : kM;
+    a.g1_from_g0 = mode == kTwo && p.L <= kN;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * (mode == kTwo ? 2 : 1) * kKBytes);
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H; a.N = p.N;
-    a.nwin = windows ? p.N / kHop - 1 : 1;
+    a.nwin = mode == kWin ? p.N / kHop - 1 : 1;
     a.lseg = plan_lseg(p.N);
     a.pb = (fa.B + 1) / 2;
-    const int64_t pairs_per_tile = int64_t(64) >> a.lseg;      // 4 rows x 4096 / N pairs
+    const int64_t pairs_per_tile = mode == kTwo ? 2 : int64_t(64) >> a.lseg;   // 4 rows x 4096 / N pairs
     a.tpc = (a.pb + pairs_per_tile - 1) / pairs_per_tile;
     a.nunits = p.H * a.nwin * a.tpc;
     a.bimg = (const uint4*)r->bimg;
@@ -1052,11 +1201,13 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, bool windows
     a.status = p.status;
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
     if (p.dtype == kBF16) {
-        if (windows) launch<__nv_bfloat16, true>(a, grid, s);
-        else launch<__nv_bfloat16, false>(a, grid, s);
+        if (mode == kWin) launch<__nv_bfloat16, kWin>(a, grid, s);
+        else if (mode == kTwo) launch<__nv_bfloat16, kTwo>(a, grid, s);
+        else launch<__nv_bfloat16, kPlain>(a, grid, s);
     } else {
-        if (windows) launch<__half, true>(a, grid, s);
-        else launch<__half, false>(a, grid, s);
+        if (mode == kWin) launch<__half, kWin>(a, grid, s);
+        else if (mode == kTwo) launch<__half, kTwo>(a, grid, s);
+        else launch<__half, kPlain>(a, grid, s);
     }
     return cudaGetLastError();
 }
@@ -1071,6 +1222,7 @@ cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& fa, void* y2, 
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.y2 = y2; a.v2 = v2;
     a.K = (const uint32_t*)fa.Kf;
+    a.kstride = kM;
     a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
     a.B = fa.B; a.H = p.H; a.N = p.N;
     a.nwin = 1;
@@ -1084,8 +1236,8 @@ cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& fa, void* y2, 
     a.tw8192 = r->tw8192;
     a.status = p.status;
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
-    if (p.dtype == kBF16) launch<__nv_bfloat16, false, true>(a, grid, s);
-    else launch<__half, false, true>(a, grid, s);
+    if (p.dtype == kBF16) launch<__nv_bfloat16, kPlain, true>(a, grid, s);
+    else launch<__half, kPlain, true>(a, grid, s);
     return cudaGetLastError();
 }
 

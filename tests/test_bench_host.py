@@ -40,11 +40,13 @@ def test_algorithmic_bytes_at_the_stored_filter_width(name, path, expected):
 # Issued MMA flops per output element, from the instruction shapes of the
 # 32 x 32 x 8 engine: 8*32 + 16*(32 + 8) = 896 for a zero-padded transform
 # with half its outputs kept; 16*(32 + 32 + 8) = 1152 for a full one; three
-# overlap-save windows of 4096 points per 8192 outputs: 896 * 3 / 2.
+# two blocks of 4096 per 8192 outputs (unmasked N = 8192) and four packed 1K
+# sequences per 8192-point row keep 4096 outputs per transform like N = 4096.
 @pytest.mark.parametrize("name,path,expected", [
     ("gated_bf16_n4k", "tc_fused", 896.0),
+    ("gated_bf16_n1k", "tc_fused", 896.0),
     ("sparse_bf16_n8k", "tc_fused", 1152.0),
-    ("partial_bf16_n8k", "tc_fused", 1344.0),
+    ("partial_bf16_n8k", "tc_fused", 896.0),
     ("fp16_n32k", "tc_staged", 1152.0),
     ("fp32_n1k", "simt_fused", 0.0),
 ])

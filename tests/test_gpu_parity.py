@@ -232,8 +232,9 @@ def test_bad_arguments_are_rejected_without_launch():
 @pytest.mark.parametrize("N,L,B", [(8192, 2048, 3), (8192, 2049, 2), (8192, 1, 1), (16384, 300, 3),
                                    (32768, 1024, 1)])
 def test_overlap_save_windows(dtype, N, L, B):
-    """Sequences longer than 4096 with filters of L <= 2049 taps run as
-    overlapping 4096-sample windows on the tensor-core kernel."""
+    """Sequences longer than 4096 with filters of L <= 2049 taps run on the
+    tensor-core kernel: as overlapping 4096-sample windows (N >= 16384) or as
+    two blocks of 4096 (N = 8192)."""
     inp = _rand_inputs(B, 2, N, L, dtype, gated=(B != 1), seed=N + L + B)
     y, plan = run_cuda(inp, dtype, order=0)
     assert plan.path_name == "tc_fused"
@@ -243,8 +244,9 @@ def test_overlap_save_windows(dtype, N, L, B):
 def test_overlap_save_limits():
     import long_sequence_fft_b200 as lsf
     import torch
-    # one tap too many for the windows: at N = 8192 the parity split serves
-    # it, longer sequences go to the SIMT path
+    # one tap too many for the windows: at N = 8192 the two-block mode (or,
+    # with a mask, the parity split) serves it, longer sequences go to the
+    # SIMT path
     assert lsf.Plan(8192, 2, "bf16", L=2050).path_name == "tc_fused"
     assert lsf.Plan(16384, 2, "bf16", L=2050).path_name != "tc_fused"
     plan = lsf.Plan(16384, 2, "bf16", L=2048)
@@ -290,8 +292,8 @@ def test_forward_host_pipelined_chunks_match_device_path():
 @pytest.mark.parametrize("B,L,gated,mask_frac", [(3, 8192, True, 0.0), (2, 8192, False, 0.75), (1, 5000, True, 0.5),
                                                  (5, 2050, True, 0.0), (4, 8192, True, 0.3)])
 def test_split_n8192_full_filters(dtype, B, L, gated, mask_frac):
-    """N = 8192 with filters longer than the windows allow: the 16384-point
-    spectrum split by bin parity, masks included."""
+    """N = 8192 with any filter length: unmasked calls run the two-block mode,
+    masked calls the 16384-point spectrum split by bin parity."""
     inp = _rand_inputs(B, 3, 8192, L, dtype, gated=gated, mask_frac=mask_frac, seed=B * 7 + L)
     y, plan = run_cuda(inp, dtype, order=0)
     assert plan.path_name == "tc_fused"

@@ -6,8 +6,9 @@
    the split mode's parked z_even are exercised many times per CTA), in every
    mode the kernels have: plain (N = 4096), packed short sequences (N = 256 ..
    2048, 4096 / N of them per 8192-point transform), overlap-save windows
-   (partial filters), the N = 8192 parity split (masked) and the staged path's
-   row pass.  The launch configuration is the plan's own, as in the benchmark.
+   (partial filters, N >= 16384), the two-block mode of N = 8192 (unmasked
+   calls), the N = 8192 parity split (masked calls) and the staged path's row
+   pass.  The launch configuration is the plan's own, as in the benchmark.
 2. Closed forms the convolution must reproduce on every tensor-core mode
    (exact results of the definition "FlashFFTConv: Efficient Convolutions for
    Long Sequences with Tensor Cores", summary and "Approach", with the
@@ -93,10 +94,23 @@ def test_packed_mode_rejects_masks():
 
 
 def test_windows_mode_three_tiles_per_cta():
-    B, H, N, L = 16, 80, 8192, 2048
+    B, H, N, L = 16, 32, 16384, 2048
     tiles = H * (N // 2048 - 1) * ((B // 2 + 3) // 4)
     assert tiles >= 3 * SMS
     _compare(_inputs(B, H, N, L, "bf16", gated=True, seed=3), "bf16", f"windows {tiles} tiles")
+
+
+@pytest.mark.parametrize("B,H,L,gated,dtype", [(16, 112, 8192, True, "bf16"),
+                                               (13, 128, 5000, False, "f16"),
+                                               (16, 112, 2048, True, "bf16"),
+                                               (15, 120, 4097, True, "f16")])
+def test_two_block_mode_three_tiles_per_cta(B, H, L, gated, dtype):
+    """N = 8192 without a mask: two pairs per tile, each as two blocks of 4096
+    (block 1 takes block 0's spectrum through shared memory)."""
+    N = 8192
+    tiles = H * (((B + 1) // 2 + 1) // 2)
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, L, dtype, gated=gated, seed=L + B), dtype, f"two-block L={L} B={B} {tiles} tiles")
 
 
 def test_split_mode_three_tiles_per_cta():
@@ -117,14 +131,22 @@ def test_rows_mode_three_tiles_per_cta():
 
 # ------------------------------------------------------- closed forms ---
 
-MODES = [  # (name, N, L, order, path)
+MODES = [  # (name, N, L, order, path); the split mode runs for masked calls
     ("plain", 4096, 4096, 0, "tc_fused"),
     ("packed1k", 1024, 1024, 0, "tc_fused"),
     ("packed256", 256, 256, 0, "tc_fused"),
-    ("windows", 8192, 2048, 0, "tc_fused"),
+    ("windows", 16384, 2048, 0, "tc_fused"),
+    ("twoblock", 8192, 8192, 0, "tc_fused"),
+    ("twoblock_partial", 8192, 3000, 0, "tc_fused"),
     ("split", 8192, 8192, 0, "tc_fused"),
     ("rows", 16384, 16384, 5, "tc_staged"),
 ]
+
+
+def _keep_all(name, N):
+    """An all-ones block mask (it selects the masked kernel, the parity split,
+    at N = 8192 and changes nothing else)."""
+    return np.ones((1, N // 32), np.uint8) if name == "split" else None
 
 
 def _run(u, k, dtype, order, path, w=None, v=None, mask=None):
@@ -145,16 +167,19 @@ def test_delta_filters_return_the_input(name, N, L, order, path, dtype):
     x = u.astype(np.float64) * w * v
     k = np.zeros((H, L), np.float32)
     k[:, 0] = 1.0
-    y = _run(u, k, dtype, order, path, w=w, v=v)
+    m = _keep_all(name, N)
+    y = _run(u, k, dtype, order, path, w=w, v=v, mask=m)
     assert_close(y, x, dtype, f"{name}: delta filter")
-    # shifted delta (a different shift per channel): y[t] = (u w)[t - d] v[t]
-    d = [min(5, L - 1), min(L - 1, 1500)]
+    # shifted delta (a different shift per channel): y[t] = (u w)[t - d] v[t];
+    # at N = 8192 one shift moves block 0 entirely into block 1 and the other
+    # gives block 1 outputs from both blocks' inputs (both two-block terms)
+    d = [min(5, L - 1), min(L - 1, 1500)] if N != 8192 else [min(L - 1, 4095), 2000]
     k = np.zeros((H, L), np.float32)
     ref = np.zeros((B, H, N))
     for h in range(H):
         k[h, d[h]] = 1.0
         ref[:, h, d[h]:] = (u[:, h, :N - d[h]].astype(np.float64) * w[:, h, :N - d[h]]) * v[:, h, d[h]:]
-    y = _run(u, k, dtype, order, path, w=w, v=v)
+    y = _run(u, k, dtype, order, path, w=w, v=v, mask=m)
     assert_close(y, ref, dtype, f"{name}: shifted delta")
 
 
@@ -166,13 +191,14 @@ def test_running_sums_of_the_filter(name, N, L, order, path):
     B, H = 2, 2
     u = np.ones((B, H, N), np.float32)
     t = np.arange(N)
+    m = _keep_all(name, N)
     k1 = np.ones((H, L), np.float32)
-    y = _run(u, k1, dtype, order, path)
+    y = _run(u, k1, dtype, order, path, mask=m)
     ref = np.broadcast_to(np.minimum(t, L - 1) + 1.0, (B, H, N))
     assert_close(y, ref, dtype, f"{name}: u = k = 1")
     r = np.array([0.999, 0.99], np.float64)
     kg = W.round_to((r[:, None] ** np.arange(L)[None, :]).astype(np.float32), dtype)
-    y = _run(u, kg, dtype, order, path)
+    y = _run(u, kg, dtype, order, path, mask=m)
     cs = np.cumsum(kg.astype(np.float64), axis=1)        # the rounded taps' running sums
     ref = np.broadcast_to(cs[:, np.minimum(t, L - 1)][None], (B, H, N))
     assert_close(y, ref, dtype, f"{name}: geometric filter")
@@ -190,6 +216,15 @@ def test_zero_and_full_masks_on_tensor_cores(name, N, order, path):
     assert np.max(np.abs(y)) == 0.0, f"{name}: all-zero mask must give exact zeros"
     inp["mask"] = np.full((2, N // 32), 9, np.uint8)     # any nonzero byte keeps the block
     y1, _ = run_cuda(inp, "bf16", order=order)
+    if name == "split":
+        # at N = 8192 an unmasked call runs the two-block kernel instead: the
+        # all-ones mask equals another all-ones mask bit for bit, and the
+        # oracle's unmasked result within the tolerance
+        inp["mask"] = np.ones((1, N // 32), np.uint8)
+        y2, _ = run_cuda(inp, "bf16", order=order)
+        assert np.array_equal(y1, y2), f"{name}: all-ones masks must agree bit for bit"
+        assert_close(y1, oracle.fftconv(inp["u"], inp["k"], w=inp["w"], v=inp["v"]), "bf16", f"{name}: all-ones")
+        return
     inp["mask"] = None
     y2, _ = run_cuda(inp, "bf16", order=order)
     assert np.array_equal(y1, y2), f"{name}: all-ones mask must equal the unmasked call"
@@ -197,13 +232,13 @@ def test_zero_and_full_masks_on_tensor_cores(name, N, order, path):
 
 # --------------------------------------------------------- fp16 range ---
 
-def _status_after(u, k, dtype, order, N, L):
+def _status_after(u, k, dtype, order, N, L, mask=None):
     import long_sequence_fft_b200 as lsf
     import torch
     from parity_util import to_dev
     plan = lsf.Plan(N, u.shape[1], dtype, order=order, L=L)
     Kf = plan.precompute(to_dev(k, dtype))
-    y = plan.forward(to_dev(u, dtype), Kf)
+    y = plan.forward(to_dev(u, dtype), Kf, mask=None if mask is None else torch.from_numpy(mask).cuda())
     torch.cuda.synchronize()
     status = lsf.library().fftconv_device_status(plan.handle, None)
     again = lsf.library().fftconv_device_status(plan.handle, None)
@@ -213,7 +248,8 @@ def _status_after(u, k, dtype, order, N, L):
 @pytest.mark.parametrize("name,N,L,order,path,edge,beyond", [
     ("plain", 4096, 4096, 0, "tc_fused", 90.0, 1500.0),
     ("packed1k", 1024, 1024, 0, "tc_fused", 90.0, 6000.0),     # B = 2: one segment of 1024 per row
-    ("windows", 8192, 2048, 0, "tc_fused", 90.0, 1500.0),
+    ("windows", 16384, 2048, 0, "tc_fused", 90.0, 1500.0),
+    ("twoblock", 8192, 8192, 0, "tc_fused", 90.0, 1500.0),
     ("split", 8192, 8192, 0, "tc_fused", 90.0, 3000.0),
     ("rows", 16384, 16384, 5, "tc_staged", 90.0, 2000.0),
 ])
@@ -224,14 +260,15 @@ def test_fp16_range_guard(name, N, L, order, path, edge, beyond):
     k[:, 0] = 1.0                                        # delta: y = u, flat spectrum
     # at the documented data-independent bound: finite, status OK, exact result
     u = np.full((B, H, N), edge, np.float32)
-    y, status, again, plan = _status_after(u, k, "bf16", order, N, L)
+    m = _keep_all(name, N)
+    y, status, again, plan = _status_after(u, k, "bf16", order, N, L, m)
     assert plan.path_name == path
     assert status == lsf.OK and np.isfinite(y).all()
     assert_close(y, u.astype(np.float64), "bf16", f"{name}: constant {edge} at the bound")
     # a constant input far beyond it overflows the fp16 forward transform: the
     # call reports FFTCONV_ERR_RANGE (and the status word resets on read)
     u = np.full((B, H, N), beyond, np.float32)
-    y, status, again, _ = _status_after(u, k, "bf16", order, N, L)
+    y, status, again, _ = _status_after(u, k, "bf16", order, N, L, m)
     assert status == lsf.ERR_RANGE, (name, status)
     assert again == lsf.OK
     assert not np.isfinite(y).all()

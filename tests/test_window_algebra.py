@@ -57,3 +57,42 @@ def test_one_tap_too_many_breaks_the_windows():
     k = rng.standard_normal((1, L))
     err = np.max(np.abs(_windows(u, k, hop) - oracle.fftconv(u, k)))
     assert err > 1e-3
+
+
+# ------------------------------------------- two-block partitioned form ---
+# Sequences of 8192 on the tensor-core kernel run as two blocks of 4096:
+# with X_b the 8192-point transform of block b (zero-padded), G_0 that of
+# [k0; 0] and G_1 that of [k1; k0] (k0, k1 the taps [0, 4096), [4096, 8192)),
+# block 0's outputs are the first 4096 of IFFT(X_0 G_0) and block 1's those
+# of IFFT(X_1 G_0 + X_0 G_1).  The filter rows come from one transform of
+# k0 + i k1: G_0 = (Z[f] + conj Z[-f]) / 2, G_1 = (Z[f] - conj Z[-f]) / 2i
+# + (-1)^f G_0, and for L <= 4096, G_1 = (-1)^f G_0.
+
+def _two_block(u, k):
+    B, H, N = u.shape
+    assert N == 8192
+    kk = np.zeros((H, 8192))
+    kk[:, :k.shape[1]] = k
+    Z = np.fft.fft(np.pad(kk[:, :4096] + 1j * kk[:, 4096:], ((0, 0), (0, 4096))), axis=-1)
+    Zm = np.conj(Z[:, (-np.arange(8192)) % 8192])
+    G0 = (Z + Zm) / 2
+    sg = np.where(np.arange(8192) % 2 == 1, -1.0, 1.0)
+    G1 = (Z - Zm) / 2j + sg * G0
+    pad = lambda x: np.pad(x.astype(np.float64), ((0, 0), (0, 0), (0, 4096)))
+    X0 = np.fft.fft(pad(u[:, :, :4096]), axis=-1)
+    X1 = np.fft.fft(pad(u[:, :, 4096:]), axis=-1)
+    y0 = np.fft.ifft(X0 * G0[None], axis=-1).real[:, :, :4096]
+    y1 = np.fft.ifft(X1 * G0[None] + X0 * G1[None], axis=-1).real[:, :, :4096]
+    return np.concatenate([y0, y1], axis=-1), G0, G1
+
+
+@pytest.mark.parametrize("L", [1, 2048, 4096, 4097, 6000, 8192])
+def test_two_block_form_equals_the_convolution(L):
+    rng = np.random.default_rng(L)
+    u = rng.standard_normal((2, 2, 8192))
+    k = rng.standard_normal((2, L)) / np.sqrt(L)
+    y, G0, G1 = _two_block(u, k)
+    ref = oracle.fftconv(u, k)
+    assert np.max(np.abs(y - ref)) <= 1e-9 * max(1.0, np.max(np.abs(ref)))
+    if L <= 4096:
+        assert np.allclose(G1, np.where(np.arange(8192) % 2 == 1, -1.0, 1.0) * G0, atol=1e-9)
