@@ -55,10 +55,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
                     "-I", os.path.join(ROOT, "include")]
     if verbose:
         flags += ["-Xptxas", "-v"]
+    # an object is rebuilt when it is older than its source, a header or
+    # this script (or on --force)
+    shared = [p for p in _inputs() if not p.endswith(".cu")]
+    newest_shared = max(os.path.getmtime(p) for p in shared)
     procs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         objs.append(obj)
+        if not force and os.path.exists(obj) and \
+                os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_shared):
+            continue
         procs.append((src, subprocess.Popen([nvcc] + flags + ["-c", src, "-o", obj],
                                             stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
     failed = []

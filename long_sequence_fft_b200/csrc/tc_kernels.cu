@@ -600,13 +600,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                     }
                 } else {
                 uint4 ld[2][4];
+                if constexpr (LY::kSplit) {
+                    // the even tile's rows are read again by the odd tile one
+                    // tile later: keep them in L2 until then
+                    const uint64_t pol = LP.odd ? l2_evict_first() : l2_evict_last();
 #pragma unroll
-                for (int jh = 0; jh < 2; ++jh) {
-                    const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
-                    ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
-                    ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
-                    ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
-                    ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
+                        ld[jh][0] = ldg_nc_hint(pu0 + t0, pol);
+                        ld[jh][1] = ldg_nc_hint(pw0 + t0, pol);
+                        ld[jh][2] = ldg_nc_hint(pu1 + t0, pol);
+                        ld[jh][3] = ldg_nc_hint(pw1 + t0, pol);
+                    }
+                } else {
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const int64_t t0 = 256 * (J * s + 2 * jp + jh) + 8 * lane;
+                        ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
+                        ld[jh][1] = __ldg((const uint4*)(pw0 + t0));
+                        ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
+                        ld[jh][3] = __ldg((const uint4*)(pw1 + t0));
+                    }
                 }
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
@@ -917,8 +931,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
                                 const int64_t t0 = 256 * (jb + jj) + 8 * lane;
-                                va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
-                                vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                                if constexpr (LY::kSplit) {     // streamed once: leave L2 to the reused rows
+                                    const uint64_t pol = l2_evict_first();
+                                    va[jj] = ldg_nc_hint(vr + P.o0 + t0, pol);
+                                    vb[jj] = ldg_nc_hint(vr + (has1 ? P.o1 : P.o0) + t0, pol);
+                                } else {
+                                    va[jj] = __ldg((const uint4*)(vr + P.o0 + t0));
+                                    vb[jj] = __ldg((const uint4*)(vr + (has1 ? P.o1 : P.o0) + t0));
+                                }
                             }
                         }
                         if (hf == 0 && (!(ok = begin_pair(c0)) || !(ok = begin_pair(c0 + 2)))) break;
@@ -944,8 +964,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                     hz[j3] = pack_h2(__uint_as_float(r[j3 >> 1][j3 & 1][2 * jj]),
                                                      __uint_as_float(r[j3 >> 1][j3 & 1][2 * jj + 1]));
                                 const int64_t t0 = 256 * (jb + jj) + 8 * lane;
-                                slot[t0 >> 2] = make_uint4(hz[0], hz[1], hz[2], hz[3]);
-                                slot[(t0 >> 2) + 1] = make_uint4(hz[4], hz[5], hz[6], hz[7]);
+                                const uint64_t pol = l2_evict_last();     // read back by the odd tile
+                                stg_hint(slot + (t0 >> 2), make_uint4(hz[0], hz[1], hz[2], hz[3]), pol);
+                                stg_hint(slot + (t0 >> 2) + 1, make_uint4(hz[4], hz[5], hz[6], hz[7]), pol);
                             }
                         }
                         if (MODE == kModeRows && emit) {
@@ -988,7 +1009,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                         const float2 w_0 = cmul(w0, a.w16k_j3[2 * e]), w_1 = cmul(w0, a.w16k_j3[2 * e + 1]);
                                         const float2 zo0 = cmulc(make_float2(a0, b0), w_0), zo1 = cmulc(make_float2(a1, b1), w_1);
                                         // z_even of t0 + 2e (+1), loaded where used
-                                        const uint2 zp = reinterpret_cast<const uint2*>(zslot)[e];
+                                        const uint2 zp = ldg2_hint(reinterpret_cast<const uint2*>(zslot) + e,
+                                                                   l2_evict_first());
                                         const float2 ze0 = __half22float2(u2h(zp.x)), ze1 = __half22float2(u2h(zp.y));
                                         a0 = ze0.x + zo0.x; b0 = ze0.y + zo0.y;
                                         a1 = ze1.x + zo1.x; b1 = ze1.y + zo1.y;
@@ -1004,8 +1026,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_n4096_kernel(TcArgs a)
                                     oa[e] = IO<T>::pack2(a0, a1);
                                     ob[e] = IO<T>::pack2(b0, b1);
                                 }
-                                *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-                                if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                                if constexpr (LY::kSplit) {
+                                    const uint64_t pol = l2_evict_first();
+                                    stg_hint((T*)a.y + P.o0 + t0, make_uint4(oa[0], oa[1], oa[2], oa[3]), pol);
+                                    if (has1) stg_hint((T*)a.y + P.o1 + t0, make_uint4(ob[0], ob[1], ob[2], ob[3]), pol);
+                                } else {
+                                    *(uint4*)((T*)a.y + P.o0 + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                                    if (has1) *(uint4*)((T*)a.y + P.o1 + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                                }
                             }
                         }
                     }

@@ -471,8 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             else if (which == 6 && issuer == 0 && (lane >> 3) == 0) {
                                 pf_src = a.K + hn * a.kstride;
                                 pf_bytes = kKBytes;
-                            } else if (MODE == kTwo && which == 7 && issuer == 1 && (lane >> 3) == 0) {
-                                pf_src = a.K + hn * a.kstride + kM;     // G_1
+                            } else if (MODE == kTwo && which == 7 && issuer == 1 && (lane >> 3) == 0 &&
+                                       !a.g1_from_g0) {
+                                pf_src = a.K + hn * a.kstride + kM;     // G_1 (read only for L > 4096)
                                 pf_bytes = kKBytes;
                             }
                         }
