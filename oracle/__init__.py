@@ -52,6 +52,8 @@ def _bind(lib):
     lib.oracle_dft_direct.argtypes = [dp, dp, dp, dp, i64, ctypes.c_int]
     lib.oracle_fftconv.argtypes = [dp, dp, dp, i64, i64, i64, i64, dp, dp,
                                    u8p, i64, ctypes.c_int, dp]
+    lib.oracle_fftconv_bins.argtypes = [dp, dp, dp, i64, i64, i64, i64, dp, dp,
+                                        u8p, i64, ctypes.c_int, dp]
     lib.oracle_filter_rfft.argtypes = [dp, dp, i64, i64, i64, u8p, i64]
     lib.oracle_direct_conv.argtypes = [dp, dp, dp, i64, i64, i64, i64, dp, dp,
                                        i64p, i64p, i64]
@@ -61,7 +63,7 @@ def _bind(lib):
                                                  i64p, i64p, i64]
     lib.oracle_conv_backward_direct.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, dp, dp, dp, dp]
     lib.oracle_conv_backward_fft.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, dp, dp, dp, dp]
-    for f in ("oracle_fft", "oracle_dft_direct", "oracle_fftconv",
+    for f in ("oracle_fft", "oracle_dft_direct", "oracle_fftconv", "oracle_fftconv_bins",
               "oracle_filter_rfft", "oracle_direct_conv",
               "oracle_masked_filter_direct", "oracle_masked_filter_fft",
               "oracle_circular_conv_samples", "oracle_conv_backward_direct",
@@ -144,6 +146,30 @@ def fftconv(u, k, w=None, v=None, mask=None, nthreads=None, return_imag_ratio=Fa
                                 _ptr(m, ctypes.c_uint8), mh, int(nthreads),
                                 ctypes.byref(ratio))
     _check(rc, "fftconv")
+    if return_imag_ratio:
+        return y, ratio.value
+    return y
+
+
+def fftconv_bins(u, k, binmask, w=None, v=None, nthreads=None, return_imag_ratio=False):
+    """FFT route with a per-bin mask of the full 2N-point filter spectrum:
+    binmask [binmask_h, 2N] (or [2N]), a zero entry zeroes that bin; keep it
+    Hermitian-symmetric (entry f == entry (2N - f) mod 2N) for a real result."""
+    u = _f64(u)
+    k = _f64(k)
+    w = _f64(w)
+    v = _f64(v)
+    B, H, N = u.shape
+    L = k.shape[1]
+    m, mh = _mask(binmask)
+    assert m.shape[1] == 2 * N
+    y = np.empty((B, H, N), dtype=np.float64)
+    ratio = ctypes.c_double(0.0)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().oracle_fftconv_bins(_ptr(u), _ptr(k), _ptr(y), B, H, N, L, _ptr(w), _ptr(v),
+                                     _ptr(m, ctypes.c_uint8), mh, int(nthreads), ctypes.byref(ratio))
+    _check(rc, "fftconv_bins")
     if return_imag_ratio:
         return y, ratio.value
     return y

@@ -129,7 +129,8 @@ typedef struct {
     /* problem */
     const double *u, *k, *w, *v;
     const uint8_t* mask;
-    int64_t B, H, N, L, mask_h;
+    const uint8_t* binmask;   /* [binmask_h, 2N] per-bin mask of the full spectrum, or NULL */
+    int64_t B, H, N, L, mask_h, binmask_h;
     double* y;
     double* max_imag_ratio;   /* per-thread self-check output */
     /* work split */
@@ -169,6 +170,12 @@ static void* conv_worker(void* arg) {
                         K[(M - g) % M].re = K[(M - g) % M].im = 0.0;
                     }
                 }
+            }
+            if (J->binmask) {
+                /* a zero byte zeroes bin f of the full M-point spectrum */
+                const uint8_t* brow = J->binmask + (J->binmask_h == 1 ? 0 : h) * M;
+                for (int64_t f = 0; f < M; ++f)
+                    if (!brow[f]) K[f].re = K[f].im = 0.0;
             }
             cached_h = h;
         }
@@ -211,13 +218,39 @@ done:
  *   mask      : [mask_h, N/32] bytes (1 = keep) or NULL
  *   imag_ratio: out, max over sequences of max|Im z| / max|z| (self-check)
  * Returns 0, or a negative code for bad arguments / allocation failure. */
+static int run_conv(const double* u, const double* k, double* y, int64_t B,
+                    int64_t H, int64_t N, int64_t L, const double* w,
+                    const double* v, const uint8_t* mask, int64_t mask_h,
+                    const uint8_t* binmask, int64_t binmask_h,
+                    int nthreads, double* imag_ratio);
+
 int oracle_fftconv(const double* u, const double* k, double* y, int64_t B,
                    int64_t H, int64_t N, int64_t L, const double* w,
                    const double* v, const uint8_t* mask, int64_t mask_h,
                    int nthreads, double* imag_ratio) {
-    if (B < 0 || H <= 0 || N <= 0 || (N & (N - 1)) || L <= 0 || L > N) return -1;
     if (mask && (mask_h != 1 && mask_h != H)) return -1;
     if (mask && N < ORACLE_BLOCK) return -1;
+    return run_conv(u, k, y, B, H, N, L, w, v, mask, mask_h, NULL, 0, nthreads, imag_ratio);
+}
+
+/* As oracle_fftconv with a per-bin mask of the full 2N-point filter spectrum:
+ * binmask is [binmask_h, 2N] bytes (binmask_h 1 or H), a zero byte zeroes
+ * that bin.  The caller keeps each row Hermitian-symmetric (binmask[f] ==
+ * binmask[(2N - f) mod 2N]) so that y stays real; imag_ratio reports it. */
+int oracle_fftconv_bins(const double* u, const double* k, double* y, int64_t B,
+                        int64_t H, int64_t N, int64_t L, const double* w,
+                        const double* v, const uint8_t* binmask, int64_t binmask_h,
+                        int nthreads, double* imag_ratio) {
+    if (!binmask || (binmask_h != 1 && binmask_h != H)) return -1;
+    return run_conv(u, k, y, B, H, N, L, w, v, NULL, 0, binmask, binmask_h, nthreads, imag_ratio);
+}
+
+static int run_conv(const double* u, const double* k, double* y, int64_t B,
+                    int64_t H, int64_t N, int64_t L, const double* w,
+                    const double* v, const uint8_t* mask, int64_t mask_h,
+                    const uint8_t* binmask, int64_t binmask_h,
+                    int nthreads, double* imag_ratio) {
+    if (B < 0 || H <= 0 || N <= 0 || (N & (N - 1)) || L <= 0 || L > N) return -1;
     int64_t S = B * H;
     if (S == 0) { if (imag_ratio) *imag_ratio = 0.0; return 0; }
     if (nthreads < 1) nthreads = 1;
@@ -229,6 +262,7 @@ int oracle_fftconv(const double* u, const double* k, double* y, int64_t B,
     for (int i = 0; i < nthreads; ++i) {
         conv_job* J = &jobs[i];
         J->u = u; J->k = k; J->w = w; J->v = v; J->mask = mask;
+        J->binmask = binmask; J->binmask_h = binmask_h;
         J->B = B; J->H = H; J->N = N; J->L = L; J->mask_h = mask_h; J->y = y;
         J->max_imag_ratio = &ratios[i];
         J->first = S * i / nthreads;
