@@ -49,7 +49,9 @@ def algorithmic_bytes(w: W.Workload, path: str = "simt_fused") -> int:
     esz = 4 if w.dtype == "f32" else 2
     per_elem = 2 * esz + (2 * esz if w.gated else 0)
     bins = (w.L + 1) if w.L < w.N else (w.N + 1)
-    if w.sparsity > 0:
+    if w.monarch_keep:
+        bins = int(round(W.monarch_kept_fraction(w) * (w.N + 1)))
+    elif w.sparsity > 0:
         bins = int(round((1 - w.sparsity) * (w.N + 1)))
     return w.elems * per_elem + w.H * bins * kf_bytes_per_bin(path)
 
@@ -66,6 +68,8 @@ def mma_flops_per_elem(w: W.Workload, path: str):
     and outputs (the N = 8192 parity split of masked calls, the staged row
     pass) 16*(32 + 32 + 8) = 1152 per point.  fp32-lane paths issue none."""
     if path == "tc_fused":
+        if w.N == 4096 and w.monarch_keep:
+            return "32x32x8, Monarch-masked c2 skipped", monarch_mma_flops_per_elem(w.monarch_keep)
         if w.N == 4096:
             return "32x32x8", 896.0
         if w.N < 4096:
@@ -79,6 +83,20 @@ def mma_flops_per_elem(w: W.Workload, path: str):
     if path == "tc_staged":
         return "columns on fp32 lanes x rows 32x32x8", 1152.0
     return "fp32 lanes", 0.0
+
+
+def monarch_mma_flops_per_elem(keep: int) -> float:
+    """Issued MMA flops per output of the N = 4096 kernel with a
+    Monarch-aligned mask, from the instructions it issues per tile (M = 128,
+    2 flops per multiply-add; a tile is 32768 outputs): S1 16 of 128x64x16,
+    S2 32 of 128x64x16, S3 and S3' one 128x16x16 per kept c2 and j3 pair
+    (8 each per c2 over the tile), S2' 8 per K step of eight c2 with any kept,
+    S1' 32 of 128x32x16.  keep = all ones gives 896."""
+    big, small, s1i = 2 * 128 * 64 * 16, 2 * 128 * 16 * 16, 2 * 128 * 32 * 16
+    kept = bin(keep & 0xFFFFFFFF).count("1")
+    ksteps = sum(1 for s in range(4) if (keep >> (8 * s)) & 0xFF)
+    per_tile = (16 + 32) * big + 2 * kept * small + 8 * ksteps * big + 32 * s1i
+    return per_tile / 32768.0
 
 
 def read_peaks():
@@ -248,7 +266,7 @@ def run_reference(args):
 # Workloads timed beside the headline (one GPU): every other configuration
 # of the hot path, each for at least about a second of steps.
 SIDE_WORKLOADS = ("fp32_n1k", "fp16_n32k", "dna_bf16_n1m", "partial_bf16_n8k", "sparse_bf16_n8k",
-                  "gated_bf16_n1k", "bf16_n1k", "dna_bf16_n4m_l1m")
+                  "monarch_bf16_n4k", "gated_bf16_n1k", "bf16_n1k", "dna_bf16_n4m_l1m")
 
 
 def roofline_entry(w: W.Workload, path: str, ms_per_step: float, hbm_peak: float, tc_peak: float):
@@ -283,25 +301,31 @@ def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: 
     Kf = plan.precompute(k)
     y = torch.empty_like(u)
     stream = torch.cuda.current_stream()
+    if w.monarch_keep:
+        fwd = lambda: plan.forward_monarch(u, Kf, w.monarch_keep, w=g, v=v, out=y)
+    else:
+        fwd = lambda: plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
     for _ in range(3):
-        plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+        fwd()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+    fwd()
     e1.record(stream)
     torch.cuda.synchronize()
     steps = int(min(20000, max(10, min_seconds / max(e0.elapsed_time(e1) * 1e-3, 1e-6))))
     with ClockSampler(torch.cuda.current_device()) as clk:
         e0.record(stream)
         for _ in range(steps):
-            plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+            fwd()
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     status = plan.device_status()
     entry = {"B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated, "io_dtype": w.dtype,
-             "sparsity": w.sparsity, "path": plan.path_name, "steps": steps, "ms_per_step": ms,
+             "sparsity": (1.0 - W.monarch_kept_fraction(w)) if w.monarch_keep else w.sparsity,
+             "monarch_keep_c2": ("0x%08X" % w.monarch_keep) if w.monarch_keep else None,
+             "path": plan.path_name, "steps": steps, "ms_per_step": ms,
              "value": w.elems / (ms * 1e-3), "unit": UNIT, "device_status": status,
              "clocks": clk.summary()}
     entry.update(roofline_entry(w, plan.path_name, ms, hbm_peak, tc_peak))
@@ -369,8 +393,12 @@ def main():
     precompute_ms = e0.elapsed_time(e1)
 
     y = torch.empty_like(u)
+    if w.monarch_keep:
+        fwd = lambda: plan.forward_monarch(u, Kf, w.monarch_keep, w=g, v=v, out=y)
+    else:
+        fwd = lambda: plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
     for _ in range(args.warmup):
-        plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+        fwd()
     torch.cuda.synchronize()
     assert plan.device_status() == 0
 
@@ -381,7 +409,7 @@ def main():
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for _ in range(args.steps):
-            plan.forward(u, Kf, w=g, v=v, mask=mask, out=y)
+            fwd()
         stop.record(stream)
         torch.cuda.synchronize()
     mg.barrier(ctx)
@@ -410,7 +438,11 @@ def main():
         return 0
 
     # end to end through the host-buffer entry point (pinned memory, copies in
-    # the timed region)
+    # the timed region); that entry point takes block masks, not Monarch keep
+    # sets, so a Monarch-masked headline has no end-to-end leg
+    if w.monarch_keep:
+        raise SystemExit("monarch_bf16_n4k is timed beside the headline (the host-buffer entry point "
+                         "has no Monarch-mask form); use --profile to time it alone")
     pin = lambda a: None if a is None else torch.from_numpy(a).to(dt).pin_memory()
     uh, gh, vh = pin(inp["u"]), pin(inp["w"]), pin(inp["v"])
     mh = torch.from_numpy(inp["mask"]).pin_memory() if inp["mask"] is not None else None

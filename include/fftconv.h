@@ -185,6 +185,27 @@ FFTCONV_API int fftconv_forward(fftconv_plan_t plan, const void* u, const void* 
                     const uint8_t* block_mask, int64_t mask_h,
                     fftconv_stream_t stream);
 
+/* fftconv_forward with a Monarch-aligned frequency mask (FlashFFTConv:
+ * Efficient Convolutions for Long Sequences with Tensor Cores, "Approach":
+ * frequency-sparse convolutions skip blocks of the Monarch matrix products;
+ * "Key results": up to 79% frequency sparsity).  For tensor-core plans with
+ * N = 4096 (fftconv_plan_path == FFTCONV_PATH_TC_FUSED): the 2N = 8192-point
+ * filter spectrum index is written f = c1 + 32 c2 + 1024 c3 (c1, c2 < 32,
+ * c3 < 8), the digits of the kernel's order-3 decomposition; bit c2 of
+ * keep_c2 keeps the bins with that middle digit.  A bin f is used only when
+ * the c2 of f and the c2 of its mirror (8192 - f) mod 8192 are both kept, so
+ * the masked spectrum stays Hermitian and y real (keep sets closed under
+ * c2 -> 31 - c2 lose only the bins f = 0 mod 32 at their edges).  The work of
+ * a masked c2 is skipped, not zeroed: its forward and inverse 8-point stage
+ * products (tcgen05 MMAs) and their epilogue work, and every K step of the
+ * 32-point inverse stage whose eight c2 are all masked.
+ *   keep_c2 : 0xffffffff is the unmasked call; 0 gives y = 0.
+ * Other arguments as fftconv_forward (no block_mask).  Other plans:
+ * FFTCONV_ERR_UNSUPPORTED.  Asynchronous on `stream`; allocates nothing. */
+FFTCONV_API int fftconv_forward_monarch(fftconv_plan_t plan, const void* u, const void* K_f, void* y,
+                            int64_t B, int64_t H, int64_t N, const void* w, const void* v,
+                            uint32_t keep_c2, fftconv_stream_t stream);
+
 /* Gradients of y = v * conv(u * w, k) for the incoming gradient dy, for
  * training (FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor
  * Cores, "Key results": the convolution inside trained models; the page gives

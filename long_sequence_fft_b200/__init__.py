@@ -47,6 +47,8 @@ _SIGNATURES = {
     "fftconv_plan_path": (ctypes.c_int, [_vp]),
     "fftconv_filter_precompute": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
     "fftconv_forward": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp]),
+    "fftconv_forward_monarch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, ctypes.c_uint32,
+                                               _vp]),
     "fftconv_forward_host_staging_bytes": (_sz, [_vp, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i64]),
     "fftconv_forward_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp,
                                             _sz, _vp]),
@@ -216,6 +218,23 @@ class Plan:
             mask_h = mask.shape[0]
         _check(_lib.fftconv_forward(self._h, _ptr(u), _ptr(Kf), _ptr(out), B, self.H, self.N, _ptr(w), _ptr(v),
                                     _ptr(mask), mask_h, _stream_handle(stream)))
+        return out
+
+    def forward_monarch(self, u, Kf, keep_c2, w=None, v=None, out=None, stream=None):
+        """forward with a Monarch-aligned frequency mask (N = 4096 tensor-core
+        plans): bit c2 of keep_c2 keeps the 8192-point spectrum bins whose
+        middle digit (f >> 5) & 31 is c2 (and whose mirror's is kept too)."""
+        import torch
+        B = u.shape[0]
+        shape = (B, self.H, self.N)
+        self._check_tensor(u, shape, "u")
+        self._check_tensor(w, shape, "w")
+        self._check_tensor(v, shape, "v")
+        if out is None:
+            out = torch.empty(shape, dtype=self.dtype, device=u.device)
+        self._check_tensor(out, shape, "out")
+        _check(_lib.fftconv_forward_monarch(self._h, _ptr(u), _ptr(Kf), _ptr(out), B, self.H, self.N, _ptr(w),
+                                            _ptr(v), int(keep_c2) & 0xffffffff, _stream_handle(stream)))
         return out
 
     def backward(self, u, Kf, dy, w=None, v=None, want_dk=True, stream=None):

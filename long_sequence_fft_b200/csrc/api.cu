@@ -350,6 +350,28 @@ int fftconv_forward(fftconv_plan_t plan, const void* u, const void* K_f, void* y
     return run_forward(p, a, (cudaStream_t)stream);
 }
 
+int fftconv_forward_monarch(fftconv_plan_t plan, const void* u, const void* K_f, void* y, int64_t B, int64_t H,
+                            int64_t N, const void* w, const void* v, uint32_t keep_c2, fftconv_stream_t stream) {
+    g_last_error.clear();
+    if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
+    const Plan& p = plan->p;
+    if (p.path != kPathTcFused || p.N != 4096)
+        return fail(FFTCONV_ERR_UNSUPPORTED,
+                    "Monarch-aligned masks act on the 8192-point spectrum of a tensor-core plan with N = 4096 "
+                    "(this plan: N=%lld, path %d)", (long long)p.N, (int)p.path);
+    int rc = validate_forward(p, u, K_f, y, B, H, N, w, v, nullptr, 0);
+    if (rc != FFTCONV_OK || B == 0) return rc;
+    cudaError_t e;
+    if (keep_c2 == 0) {
+        e = cudaMemsetAsync(y, 0, (size_t)B * (size_t)H * (size_t)N * dtype_size(p.dtype), (cudaStream_t)stream);
+    } else {
+        ForwardArgs a{u, w, v, y, K_f, nullptr, 0, B};
+        e = tc_planar_forward_monarch(p, a, keep_c2, (cudaStream_t)stream);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return FFTCONV_OK;
+}
+
 static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // extern "C"

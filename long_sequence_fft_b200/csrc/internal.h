@@ -110,13 +110,17 @@ cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cud
 // tensor-core fused kernel with planar complex data (tc_planar.cu):
 // sequences of at most 4096 (plain), of 8192 as two blocks (the filter rows
 // G_0, G_1 of tc_planar_precompute_two_block), and overlap-save windows
-enum { kPlanarPlain = 0, kPlanarWindows = 1, kPlanarTwoBlock = 2 };
+enum { kPlanarPlain = 0, kPlanarWindows = 1, kPlanarTwoBlock = 2, kPlanarMonarch = 3 };
 cudaError_t tc_planar_init(Plan& p);
 void tc_planar_free(Plan& p);
 cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 size_t tc_planar_two_block_bytes(const Plan& p);
 cudaError_t tc_planar_precompute_two_block(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& a, int mode, cudaStream_t s);
+// N = 4096 with a Monarch-aligned frequency mask: bit c2 of keep_c2 keeps the
+// spectrum bins f with (f >> 5) & 31 == c2 (f = c1 + 32 c2 + 1024 c3); the
+// stages of masked c2 are skipped
+cudaError_t tc_planar_forward_monarch(const Plan& p, const ForwardArgs& a, uint32_t keep_c2, cudaStream_t s);
 cudaError_t tc_planar_export(const Plan& p, const void* Kf, float* out, cudaStream_t s);
 // backward pass (N <= 4096): the correlation launch of the planar kernel and
 // the filter gradient on fp32 lanes (simt_kernels.cu)

@@ -111,6 +111,28 @@ __host__ __device__ __forceinline__ int chunk_stage_barrier(int c) {
     return -1;
 }
 
+// Monarch mode: bit m of empty_groups(keep) is set when the eight c2 of group m
+// (8m .. 8m + 7) are all masked; the S3 and S3' chunk pairs of such a group
+// (chunks 16 + 2m, 17 + 2m and 24 + 2m, 25 + 2m) are not run.  The ring runs
+// over the remaining chunks in order: chunk c takes slot chunk_slot(c) of the
+// tile's 44 - 4 popc(empty) slots, whose buffer is slot % 4.
+__host__ __device__ __forceinline__ uint32_t empty_groups(uint32_t keep) {
+    uint32_t e = 0;
+    for (int m = 0; m < 4; ++m)
+        if (((keep >> (8 * m)) & 0xffu) == 0) e |= 1u << m;
+    return e;
+}
+__host__ __device__ __forceinline__ int popc4(uint32_t x) { return (x & 1) + ((x >> 1) & 1) + ((x >> 2) & 1) + ((x >> 3) & 1); }
+__host__ __device__ __forceinline__ bool chunk_skipped(int c, uint32_t empty) {
+    return c >= 16 && c < 32 && ((empty >> (((c - 16) & 7) >> 1)) & 1u);
+}
+__host__ __device__ __forceinline__ int chunk_slot(int c, uint32_t empty) {
+    if (c < 16) return c;
+    if (c < 24) return c - 2 * popc4(empty & ((1u << ((c - 16) >> 1)) - 1u));
+    if (c < 32) return c - 2 * popc4(empty) - 2 * popc4(empty & ((1u << ((c - 24) >> 1)) - 1u));
+    return c - 4 * popc4(empty);
+}
+
 // fp16 element index of the real (comp 0) or imaginary (comp 1) part of
 // value i in pair-planar and planar order (n values)
 __host__ __device__ constexpr int pp_index(int comp, int i) { return 4 * (i >> 1) + 2 * comp + (i & 1); }
@@ -136,8 +158,9 @@ __device__ __forceinline__ uint32_t k_off(int m, int kbyte) {
 }
 
 // kernel modes: one transform per row (N <= 4096, packed below), overlap-save
-// windows (N > 4096, filters of at most 2049 taps), two blocks (N = 8192)
-constexpr int kPlain = kPlanarPlain, kWin = kPlanarWindows, kTwo = kPlanarTwoBlock;
+// windows (N >= 16384, filters of at most 2049 taps), two blocks (N = 8192),
+// and the plain mode with a Monarch-aligned frequency mask (N = 4096)
+constexpr int kPlain = kPlanarPlain, kWin = kPlanarWindows, kTwo = kPlanarTwoBlock, kMonarch = kPlanarMonarch;
 
 struct PArgs {
     const void* u;
@@ -147,6 +170,7 @@ struct PArgs {
     const uint32_t* K;          // [H][kstride] words: the spectrum / scale, PP layout (k_word)
     int64_t kstride;            // words per channel: 8192, or 16384 (two-block: G_0 then G_1)
     int g1_from_g0;             // two-block, L <= 4096: G_1 = (-1)^f G_0 (not read)
+    uint32_t keep_c2;           // Monarch mode: bit c2 keeps the bins with that middle digit
     const float* Kscale;        // [H]
     const uint8_t* mask;
     int64_t mask_h;
@@ -263,7 +287,7 @@ struct TileBase {
 template <int MODE>
 __device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
     TileBase t;
-    if constexpr (MODE == kPlain) {
+    if constexpr (MODE == kPlain || MODE == kMonarch) {
         t.h = unit / a.tpc;
         t.j = 0;
         t.bp0 = (unit - t.h * a.tpc) * (64 >> a.lseg);
@@ -323,6 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
     // two-block mode: [EK step][slice][pair] block 0's spectrum values are in
     // the hand-over slots (the 32 threads of that warp)
     uint64_t* xfull = (uint64_t*)(smem + OffXBars);
+    // Monarch mode (same space): [4] the EK of c2 group m is done (16 epilogue warps)
+    uint64_t* ek_done = (uint64_t*)(smem + OffXBars);
     uint32_t* tmem_base_sh = (uint32_t*)(smem + OffMisc);
     volatile int* abort_flag = (volatile int*)(smem + OffMisc + 4);
 
@@ -345,6 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         for (int i = 0; i < 3; ++i) mbar_init(&bar_stage[i], kEpiWarps);
         if constexpr (MODE == kTwo)
             for (int i = 0; i < 32; ++i) mbar_init(&xfull[i], 32);
+        if constexpr (MODE == kMonarch)
+            for (int i = 0; i < 4; ++i) mbar_init(&ek_done[i], kEpiWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -396,6 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         int k_issued = 0;
         bool ok = true;
         uint32_t g = issuer;
+        // Monarch mode: the S3 / S3' products of a masked c2 and the S2' K
+        // steps whose eight c2 are all masked are not issued (their outputs
+        // would be zero); a chunk with some kept c2 is still committed, a
+        // chunk pair whose eight c2 are all masked is not run at all
+        const uint32_t keep = MODE == kMonarch ? a.keep_c2 : 0xffffffffu;
+        const uint32_t empty = MODE == kMonarch ? empty_groups(keep) : 0u;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
             if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
             tc_fence_after();
@@ -410,12 +444,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 __syncwarp();
             }
 #pragma unroll 1
-            for (int c = issuer; c < kChunks && ok; c += kMmaWarps, g += kMmaWarps) {
+            for (int c = MODE == kMonarch ? 0 : issuer; c < kChunks && ok; c += MODE == kMonarch ? 1 : kMmaWarps) {
+                // (Monarch mode: this issuer runs the chunks whose slot is issuer mod 4)
+                if (MODE == kMonarch && (chunk_skipped(c, empty) || (chunk_slot(c, empty) & 3) != issuer)) continue;
                 const int stage = chunk_stage(c), k = chunk_index(c);
                 const uint32_t b = g % kDBuf;
                 if (g >= kDBuf && !wait(&dfree[b], ((g - kDBuf) / kDBuf) & 1)) { ok = false; fail(); break; }
-                const int sb = chunk_stage_barrier(c);
+                g += kMmaWarps;
+                int sb = chunk_stage_barrier(c);
+                if (MODE == kMonarch && stage == 2) sb = 0;      // every S3 chunk after all of E2
                 if (sb >= 0 && !wait(&bar_stage[sb], iter & 1)) { ok = false; fail(); break; }
+                // Monarch mode: an S3' chunk after the EK of its c2 group (with
+                // chunks skipped, the ring no longer orders the two)
+                if (MODE == kMonarch && stage == 3 && !wait(&ek_done[k >> 1], iter & 1)) {
+                    ok = false;
+                    fail();
+                    break;
+                }
                 tc_fence_after();
                 {
                     // the whole warp evaluates the operands; one elected lane issues
@@ -432,11 +477,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         const uint64_t db = (stage == 2 ? dS3 : dS3i) + (uint64_t)(4 * k * 32);
 #pragma unroll
                         for (int cl = 0; cl < 4; ++cl)
-                            mma_ts_warp(d + 16 * cl, tbase + 8 * (4 * k + cl), db + 32 * cl, id16, 0);
-                    } else if (stage == 4) {     // S2': K-major tile j3 = k
+                            if ((keep >> (4 * k + cl)) & 1u)
+                                mma_ts_warp(d + 16 * cl, tbase + 8 * (4 * k + cl), db + 32 * cl, id16, 0);
+                    } else if (stage == 4) {     // S2': K-major tile j3 = k, K step s = c2 8s .. 8s + 7
                         const uint64_t da = dAk + (uint64_t)(k * (kTile >> 4));
+                        uint32_t acc = 0;
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) mma_ss_warp(d, da + 2 * s, dS2i + 128 * s, id64, s);
+                        for (int s = 0; s < 4; ++s)
+                            if ((keep >> (8 * s)) & 0xffu) {
+                                mma_ss_warp(d, da + 2 * s, dS2i + 128 * s, id64, acc);
+                                acc = 1;
+                            }
                     } else {                     // S1': j3 = 2k + jl, MN-major tiles, N = 32 (16 kept j1)
 #pragma unroll
                         for (int jl = 0; jl < 2; ++jl) {
@@ -609,9 +660,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             asm volatile("mov.b32 %0, %0;" : "+f"(kscale));
             const uint8_t* mrow = a.mask ? a.mask + (a.mask_h == 1 ? 0 : hch) * nblk : nullptr;
 
+            // Monarch mode: the keep set, its empty c2 groups (their S3 and
+            // S3' chunk pairs are not run) and the ring slot of each chunk
+            const uint32_t keep = MODE == kMonarch ? a.keep_c2 : 0xffffffffu;
+            const uint32_t empty = MODE == kMonarch ? empty_groups(keep) : 0u;
+            const int slots4 = kChunks / 4 - popc4(empty);      // ring rounds per tile
             auto begin_pair = [&](int c) -> bool {
-                const uint32_t par = (uint32_t)(iter * (kChunks / 4) + (c >> 2)) & 1u;
-                if (!wait(&dfull[c & 3], par) || !wait(&dfull[(c & 3) + 1], par)) {
+                const int sl = chunk_slot(c, empty);
+                const uint32_t par = (uint32_t)(iter * slots4 + (sl >> 2)) & 1u;
+                if (!wait(&dfull[sl & 3], par) || !wait(&dfull[(sl & 3) + 1], par)) {
                     fail();
                     return false;
                 }
@@ -619,11 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 return true;
             };
             auto release = [&](int c) {
+                const int sl = chunk_slot(c, empty);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&dfree[c & 3]);
-                    mbar_arrive(&dfree[(c & 3) + 1]);
+                    mbar_arrive(&dfree[sl & 3]);
+                    mbar_arrive(&dfree[(sl & 3) + 1]);
                 }
             };
             auto stage_done = [&](int i) {
@@ -631,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_stage[i]);
             };
-            auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (c & 3); };
+            auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (chunk_slot(c, empty) & 3); };
 
             // E1 (S1 -> S2), chunks j3 = k, k+1: lane = l; PP columns of
             // c1 = 8s .. 8s+7; twiddle w1024^(c1 l); MN-major A2 tile j3,
@@ -670,11 +728,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             // E2, chunks j3 = k, k+1: lane = c1; PP columns of c2 = 8s .. 8s+7;
             // twiddle w8192^(c1 j3) (one PP pair over j3 = k, k+1); A3 TMEM
             // columns 8 c2 + k (real pair), 8 c2 + k + 1 (imaginary pair)
+            // (Monarch mode: the A3 columns of a masked c2 are not needed)
+            const uint32_t keep_e2 = (keep >> (8 * s)) & 0xffu;     // this slice's c2
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 8 + k;
                 if (!(ok = begin_pair(c))) break;
                 uint32_t r[2][16];
+                // (loads are unconditional: loads under a branch spill the array)
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
                 tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
                 const __half2 t0 = u2h(stw[lane * k]), t1 = u2h(stw[lane * (k + 1)]);
@@ -683,10 +744,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 release(c);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int ire = 4 * (i >> 1) + (i & 1);
-                    uint32_t wr = pk(r[0][ire], r[1][ire]), wi = pk(r[0][ire + 2], r[1][ire + 2]);
-                    cmul_pp(wr, wi, tr, ti);
-                    tmem_st2(tbase + lq + 8 * (8 * s + i) + k, wr, wi);
+                    if ((keep_e2 >> i) & 1u) {
+                        const int ire = 4 * (i >> 1) + (i & 1);
+                        uint32_t wr = pk(r[0][ire], r[1][ire]), wi = pk(r[0][ire + 2], r[1][ire + 2]);
+                        cmul_pp(wr, wi, tr, ti);
+                        tmem_st2(tbase + lq + 8 * (8 * s + i) + k, wr, wi);
+                    }
                 }
                 tc_wait_st();
             }
@@ -724,6 +787,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 16 + k;
                 const int st = k >> 1;
+                if (MODE == kMonarch && ((empty >> st) & 1u)) continue;     // group st: S3 not run
+                // this warp's two c2 (4k + s, 4k + 4 + s); Monarch mode skips a masked one
+                const bool kc0 = (keep >> (4 * k + s)) & 1u, kc1 = (keep >> (4 * k + 4 + s)) & 1u;
                 if (!(ok = begin_pair(c))) break;
                 uint32_t r[2][16];
                 tmem_ld16(dcol(c) + 16 * s, r[0]);
@@ -752,6 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 }
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
+                    if (!(cc ? kc1 : kc0)) continue;       // (Monarch mode) masked c2: no product
                     const int c2 = 4 * (k + cc) + s;
                     const uint4 k0 = *(const uint4*)(Ks + k_word(lane, c2, 0));
                     const uint4 k1 = *(const uint4*)(Ks + k_word(lane, c2, 4));
@@ -768,6 +835,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                                 const uint32_t keep = (c3 & 1) ? 0x0000ffffu : 0xffff0000u;
                                 kw[2 * (c3 >> 1)] &= keep;
                                 kw[2 * (c3 >> 1) + 1] &= keep;
+                            }
+                        }
+                    }
+                    if constexpr (MODE == kMonarch) {
+                        // a kept bin whose Hermitian mirror 8192 - f has a masked
+                        // c2 is zeroed too, so the spectrum stays symmetric
+#pragma unroll
+                        for (int c3 = 0; c3 < 8; ++c3) {
+                            const int f = lane + 32 * c2 + 1024 * c3;
+                            const int c2m = (((kM - f) & (kM - 1)) >> 5) & 31;
+                            if (!((keep >> c2m) & 1u)) {
+                                const uint32_t keepw = (c3 & 1) ? 0x0000ffffu : 0xffff0000u;
+                                kw[2 * (c3 >> 1)] &= keepw;
+                                kw[2 * (c3 >> 1) + 1] &= keepw;
                             }
                         }
                     }
@@ -815,9 +896,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             cfma_pp(h[cc][2 * p], h[cc][2 * p + 1], xw[2 * p], xw[2 * p + 1], gw[2 * p], gw[2 * p + 1]);
                     }
                 }
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) tmem_st8(tbase + lq + 8 * (4 * (k + cc) + s), h[cc]);
+                if (kc0) tmem_st8(tbase + lq + 8 * (4 * k + s), h[0]);
+                if (kc1) tmem_st8(tbase + lq + 8 * (4 * k + 4 + s), h[1]);
                 tc_wait_st();
+                if constexpr (MODE == kMonarch) {
+                    // this group's A4 columns are written: its S3' chunks may run
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ek_done[st]);
+                }
             }
             if (x_take && !a.g1_from_g0) cp_async_wait<0>();   // nothing in flight past here (also after an abort)
             // E3': lane = c1; chunk c + (s >> 1), its c2 = 4(k + cc) + cl for
@@ -827,13 +914,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 24 + k;
+                if (MODE == kMonarch && ((empty >> (k >> 1)) & 1u)) continue;   // S3' of this group not run
                 if (!(ok = begin_pair(c))) break;
                 const int cc = s >> 1, h = s & 1;
+                // Monarch mode: the S3' products of masked c2 were not issued,
+                // so their accumulator columns are stale: a quadruple with a
+                // masked c2 stores zeros there (S2' reads them unless its
+                // whole K step of eight c2 is masked, then nothing is stored)
+                const uint32_t kq = (keep >> (4 * (k + cc))) & 0xfu;
+                const bool kstep = (keep >> (8 * ((k + cc) >> 1))) & 0xffu;
                 uint32_t r[4][8];
 #pragma unroll
                 for (int cl = 0; cl < 4; ++cl) tmem_ld8(dcol(c + cc) + 16 * cl + 8 * h, r[cl]);
                 tc_wait_ld();
                 release(c);
+                if (!kstep) {
+                    fence_proxy_async_smem();
+                    continue;
+                }
+                if (kq != 0xfu) {
+#pragma unroll
+                    for (int cl = 0; cl < 4; ++cl)
+                        if (!((kq >> cl) & 1u))
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) r[cl][i] = 0u;
+                }
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const int j3 = 4 * h + jj;
@@ -1138,6 +1243,8 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = allow_smem<__half, kPlain>();
     if (e == cudaSuccess) e = allow_smem<__half, kWin>();
     if (e == cudaSuccess) e = allow_smem<__half, kTwo>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kMonarch>();
+    if (e == cudaSuccess) e = allow_smem<__half, kMonarch>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain, true>();
     if (e == cudaSuccess) e = allow_smem<__half, kPlain, true>();
     return e;
@@ -1210,6 +1317,31 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cu
         else if (mode == kTwo) launch<__half, kTwo>(a, grid, s);
         else launch<__half, kPlain>(a, grid, s);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_planar_forward_monarch(const Plan& p, const ForwardArgs& fa, uint32_t keep_c2, cudaStream_t s) {
+    const Resources* r = (const Resources*)p.tcp;
+    if (p.N != kN || fa.mask || keep_c2 == 0) return cudaErrorInvalidValue;
+    PArgs a{};
+    a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
+    a.K = (const uint32_t*)fa.Kf;
+    a.kstride = kM;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.keep_c2 = keep_c2;
+    a.B = fa.B; a.H = p.H; a.N = p.N;
+    a.nwin = 1;
+    a.lseg = plan_lseg(p.N);
+    a.pb = (fa.B + 1) / 2;
+    a.tpc = (a.pb + 3) / 4;
+    a.nunits = p.H * a.tpc;
+    a.bimg = (const uint4*)r->bimg;
+    a.tw1024 = r->tw1024;
+    a.tw8192 = r->tw8192;
+    a.status = p.status;
+    const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
+    if (p.dtype == kBF16) launch<__nv_bfloat16, kMonarch>(a, grid, s);
+    else launch<__half, kMonarch>(a, grid, s);
     return cudaGetLastError();
 }
 

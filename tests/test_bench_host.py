@@ -5,6 +5,7 @@ import hashlib
 import json
 import os
 
+import numpy as np
 import pytest
 
 import bench
@@ -94,3 +95,20 @@ def test_committed_traffic_entries_name_existing_sources():
         assert os.path.isfile(os.path.join(bench.ROOT, ent["source"])), key
         assert ent["bytes_per_launch"] == ent["dram_bytes_read"] + ent["dram_bytes_write"], key
         assert "--clock-control none" in ent["command"], key
+
+
+def test_monarch_flop_count_and_kept_bins():
+    """Monarch-aligned mask of the flagship shape: all c2 kept issues the dense
+    896 flops per output; keeping c2 in {0..3, 28..31} skips 24 of the 32
+    per-c2 products of S3 and S3' and two of the four K steps of S2'
+    (2 * 24 * 8 * 128*16*16 + 16 * 128*64*16*2 fewer flops per 32768-output
+    tile: 672 per output)."""
+    assert bench.monarch_mma_flops_per_elem(0xFFFFFFFF) == 896.0
+    assert bench.monarch_mma_flops_per_elem(0xF000000F) == 672.0
+    w = W.WORKLOADS["monarch_bf16_n4k"]
+    m = W.monarch_binmask(w.monarch_keep, w.N)
+    M = 2 * w.N
+    assert np.array_equal(m, m[(M - np.arange(M)) % M])          # Hermitian
+    assert abs(W.monarch_kept_fraction(w) - 0.25) < 0.01
+    assert W.make_mask(w) is None                                  # no block mask besides it
+    assert np.all(W.monarch_binmask(0xFFFFFFFF, 1024) == 1)

@@ -42,6 +42,7 @@ class Workload:
     u_kind: str = "normal"   # "normal" | "dna"
     sparsity: float = 0.0    # fraction of mask blocks zeroed (0 = no mask)
     description: str = ""
+    monarch_keep: int = 0    # Monarch-aligned mask: bit c2 keeps the middle digit c2 (0 = none)
     shard: int = 0           # channel shard (one per rank); 0 = the workload itself
 
     @property
@@ -94,6 +95,11 @@ WORKLOADS = {
                                description="gated bf16 conv B=64 H=768 N=1024"),
     "bf16_n1k": Workload("bf16_n1k", 9, 64, 768, 1024, 1024, "bf16", False, "scaled",
                          description="bf16 conv B=64 H=768 N=1024"),
+    # the flagship shape with a Monarch-aligned 75% frequency mask: the middle
+    # digits c2 in {0..3, 28..31} of the 8192-point spectrum are kept
+    "monarch_bf16_n4k": Workload("monarch_bf16_n4k", 10, 64, 768, 4096, 4096, "bf16", True, "decay:0.001",
+                                 monarch_keep=0xF000000F,
+                                 description="gated bf16 conv B=64 H=768 N=4096, Monarch-aligned 75% sparse"),
 }
 
 # The workload the benchmark times at one GPU.
@@ -176,6 +182,25 @@ def make_gates(w: Workload):
     g = round_to(_normal(_rng(w, "w"), (w.B, w.H, w.N)), w.dtype)
     v = round_to(_normal(_rng(w, "v"), (w.B, w.H, w.N)), w.dtype)
     return g, v
+
+
+def monarch_binmask(keep: int, N: int) -> np.ndarray:
+    """[2N] uint8 per-bin mask of the 2N-point spectrum that a Monarch-aligned
+    keep set selects: with f = c1 + 32 c2 + 1024 c3 (the middle digit
+    c2 = (f >> 5) & 31), bin f is kept iff the c2 of f and the c2 of its mirror
+    (2N - f) mod 2N are both in `keep` (bit c2)."""
+    M = 2 * N
+    f = np.arange(M)
+    c2 = (f >> 5) & 31
+    c2m = (((M - f) % M) >> 5) & 31
+    bit = lambda c: (np.uint64(keep) >> c.astype(np.uint64)) & np.uint64(1)
+    return (bit(c2) & bit(c2m)).astype(np.uint8)
+
+
+def monarch_kept_fraction(w: Workload) -> float:
+    """Fraction of the rfft bins [0, N] a Monarch-aligned workload keeps."""
+    m = monarch_binmask(w.monarch_keep, w.N)
+    return float(m[:w.N + 1].sum()) / (w.N + 1)
 
 
 def make_mask(w: Workload) -> Optional[np.ndarray]:
