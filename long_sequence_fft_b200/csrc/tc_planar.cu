@@ -430,6 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         // chunk pair whose eight c2 are all masked is not run at all
         const uint32_t keep = MODE == kMonarch ? a.keep_c2 : 0xffffffffu;
         const uint32_t empty = MODE == kMonarch ? empty_groups(keep) : 0u;
+        // the chunks this issuer runs (Monarch mode: the slot decides; the same every tile)
+        uint64_t mine = 0;
+        for (int c = 0; c < kChunks; ++c)
+            if (!chunk_skipped(c, empty) && (chunk_slot(c, empty) & 3) == issuer) mine |= 1ull << c;
         for (int64_t unit = blockIdx.x; unit < a.nunits && ok; unit += gridDim.x, ++iter) {
             if (!wait(bar_in, iter & 1)) { ok = false; fail(); break; }
             tc_fence_after();
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll 1
             for (int c = MODE == kMonarch ? 0 : issuer; c < kChunks && ok; c += MODE == kMonarch ? 1 : kMmaWarps) {
                 // (Monarch mode: this issuer runs the chunks whose slot is issuer mod 4)
-                if (MODE == kMonarch && (chunk_skipped(c, empty) || (chunk_slot(c, empty) & 3) != issuer)) continue;
+                if (MODE == kMonarch && !((mine >> c) & 1ull)) continue;
                 const int stage = chunk_stage(c), k = chunk_index(c);
                 const uint32_t b = g % kDBuf;
                 if (g >= kDBuf && !wait(&dfree[b], ((g - kDBuf) / kDBuf) & 1)) { ok = false; fail(); break; }
@@ -665,8 +669,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             const uint32_t keep = MODE == kMonarch ? a.keep_c2 : 0xffffffffu;
             const uint32_t empty = MODE == kMonarch ? empty_groups(keep) : 0u;
             const int slots4 = kChunks / 4 - popc4(empty);      // ring rounds per tile
-            auto begin_pair = [&](int c) -> bool {
-                const int sl = chunk_slot(c, empty);
+            const int off_late = 4 * popc4(empty);               // slot = chunk - off_late from S2' on
+            // the ring helpers take the chunk's slot (its chunk index outside
+            // the Monarch mode)
+            auto begin_pair = [&](int sl) -> bool {
                 const uint32_t par = (uint32_t)(iter * slots4 + (sl >> 2)) & 1u;
                 if (!wait(&dfull[sl & 3], par) || !wait(&dfull[(sl & 3) + 1], par)) {
                     fail();
@@ -675,8 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 tc_fence_after();
                 return true;
             };
-            auto release = [&](int c) {
-                const int sl = chunk_slot(c, empty);
+            auto release = [&](int sl) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -689,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_stage[i]);
             };
-            auto dcol = [&](int c) -> uint32_t { return tbase + lq + 256 + 64 * (chunk_slot(c, empty) & 3); };
+            auto dcol = [&](int sl) -> uint32_t { return tbase + lq + 256 + 64 * (sl & 3); };
 
             // E1 (S1 -> S2), chunks j3 = k, k+1: lane = l; PP columns of
             // c1 = 8s .. 8s+7; twiddle w1024^(c1 l); MN-major A2 tile j3,
@@ -697,12 +702,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             // E2' (S2' -> S1'): lane = c1; PP columns of l = 8s .. 8s+7;
             // twiddle conj w1024^(c1 l); MN-major A6 tile j3, rows 32q + l,
             // K = c1 and 32 + c1.  The same twiddles and the same stores.
-            auto e_transpose = [&](int c, int k, bool conj) {
+            auto e_transpose = [&](int sl, int k, bool conj) {
                 uint32_t r[2][16];
-                tmem_ld16(dcol(c) + 16 * s, r[0]);
-                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tmem_ld16(dcol(sl) + 16 * s, r[0]);
+                tmem_ld16(dcol(sl + 1) + 16 * s, r[1]);
                 tc_wait_ld();
-                release(c);
+                release(sl);
                 const uint32_t flip = conj ? kNegPair : 0u;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -788,14 +793,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 const int c = 16 + k;
                 const int st = k >> 1;
                 if (MODE == kMonarch && ((empty >> st) & 1u)) continue;     // group st: S3 not run
+                const int sl = c - 2 * popc4(empty & ((1u << st) - 1u));
                 // this warp's two c2 (4k + s, 4k + 4 + s); Monarch mode skips a masked one
                 const bool kc0 = (keep >> (4 * k + s)) & 1u, kc1 = (keep >> (4 * k + 4 + s)) & 1u;
-                if (!(ok = begin_pair(c))) break;
+                if (!(ok = begin_pair(sl))) break;
                 uint32_t r[2][16];
-                tmem_ld16(dcol(c) + 16 * s, r[0]);
-                tmem_ld16(dcol(c + 1) + 16 * s, r[1]);
+                tmem_ld16(dcol(sl) + 16 * s, r[0]);
+                tmem_ld16(dcol(sl + 1) + 16 * s, r[1]);
                 tc_wait_ld();
-                release(c);
+                release(sl);
                 // h[cc]: the PP words of c2 = 4(k+cc) + s (all eight c3)
                 uint32_t h[2][8];
 #pragma unroll
@@ -915,7 +921,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 24 + k;
                 if (MODE == kMonarch && ((empty >> (k >> 1)) & 1u)) continue;   // S3' of this group not run
-                if (!(ok = begin_pair(c))) break;
+                const int sl = c - off_late / 2 - 2 * popc4(empty & ((1u << (k >> 1)) - 1u));
+                if (!(ok = begin_pair(sl))) break;
                 const int cc = s >> 1, h = s & 1;
                 // Monarch mode: the S3' products of masked c2 were not issued,
                 // so their accumulator columns are stale: a quadruple with a
@@ -925,9 +932,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 const bool kstep = (keep >> (8 * ((k + cc) >> 1))) & 0xffu;
                 uint32_t r[4][8];
 #pragma unroll
-                for (int cl = 0; cl < 4; ++cl) tmem_ld8(dcol(c + cc) + 16 * cl + 8 * h, r[cl]);
+                for (int cl = 0; cl < 4; ++cl) tmem_ld8(dcol(sl + cc) + 16 * cl + 8 * h, r[cl]);
                 tc_wait_ld();
-                release(c);
+                release(sl);
                 if (!kstep) {
                     fence_proxy_async_smem();
                     continue;
@@ -960,8 +967,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll 1
             for (int k = 0; k < 8 && ok; k += 2) {
                 const int c = 32 + k;
-                if (!(ok = begin_pair(c))) break;
-                e_transpose(c, k, true);
+                if (!(ok = begin_pair(c - off_late))) break;
+                e_transpose(c - off_late, k, true);
             }
             if (ok) stage_done(2);
             if (ok && unit + gridDim.x < a.nunits) load_tile(unit + gridDim.x, 1);
@@ -1000,17 +1007,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         P[jj] = pair_rows<MODE>(a, TB, q, seg_of(a, jb + jj));
                         t0[jj] = tau_of(a, jb + jj) + 8 * lane;
                     }
-                    if (hf == 0 && (!(ok = begin_pair(40)) || !(ok = begin_pair(42)))) break;
+                    if (hf == 0 && (!(ok = begin_pair(40 - off_late)) || !(ok = begin_pair(42 - off_late)))) break;
                     // r[cc][jl][0..3] = re(jb), re(jb+1), im(jb), im(jb+1) of j3 = 2cc + jl
                     uint32_t r[4][2][4];
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-                        for (int jl = 0; jl < 2; ++jl) tmem_ld4(dcol(40 + cc) + 32 * jl + 2 * jb, r[cc][jl]);
+                        for (int jl = 0; jl < 2; ++jl)
+                            tmem_ld4(dcol(40 - off_late + cc) + 32 * jl + 2 * jb, r[cc][jl]);
                     tc_wait_ld();
                     if (hf == 1) {
-                        release(40);
-                        release(42);
+                        release(40 - off_late);
+                        release(42 - off_late);
                     }
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
