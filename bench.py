@@ -78,6 +78,8 @@ def mma_flops_per_elem(w: W.Workload, path: str):
             if w.sparsity > 0:
                 return "32x32x8 (x2 parity halves)", 1152.0
             return "32x32x8 (two blocks of 4096)", 896.0
+        if w.N == 16384:
+            return "32x32x8 (four blocks of 4096)", 896.0
         nwin = w.N // 2048 - 1
         return "32x32x8 windows", 896.0 * nwin * 4096 / w.N
     if path == "tc_staged":
@@ -265,7 +267,7 @@ def run_reference(args):
 
 # Workloads timed beside the headline (one GPU): every other configuration
 # of the hot path, each for at least about a second of steps.
-SIDE_WORKLOADS = ("fp32_n1k", "fp16_n32k", "dna_bf16_n1m", "partial_bf16_n8k", "sparse_bf16_n8k",
+SIDE_WORKLOADS = ("fp32_n1k", "fp16_n16k", "fp16_n32k", "dna_bf16_n1m", "partial_bf16_n8k", "sparse_bf16_n8k",
                   "monarch_bf16_n4k", "gated_bf16_n1k", "bf16_n1k", "dna_bf16_n4m_l1m")
 
 

@@ -72,8 +72,9 @@ typedef enum {
 /* Range of the 16-bit tensor-core paths (FFTCONV_PATH_TC_FUSED and
  * FFTCONV_PATH_TC_STAGED).  Their transform intermediates are fp16 (largest
  * finite value 65504); the fp32 paths (orders 1 and 4) keep fp32 throughout.
- *   - Fused kernel (N <= 4096, N = 8192 as two blocks or, with a block
- *     mask, split by bin parity, overlap-save windows): each unitary stage can grow a value by at most the number of
+ *   - Fused kernel (N <= 4096, N = 8192 and 16384 as two and four blocks
+ *     of 4096 or, N = 8192 with a block mask, split by bin parity,
+ *     overlap-save windows): each unitary stage can grow a value by at most the number of
  *     its inputs over the square root of its length, so with max|u*w| <= 90
  *     no intermediate can overflow whatever the data and the filter.  Above
  *     that it depends on the data: a constant (DC) input overflows the forward
@@ -106,12 +107,15 @@ typedef enum {
  *   2, 3  fused: one kernel, the transform stays on chip (no intermediate in
  *         device memory).  This library's fused kernels split every transform
  *         they hold into three levels, so 2 and 3 are the same request.  They
- *         exist for N <= 8192 (tensor cores for fp16/bf16 at N = 256 ..
- *         8192, N = 8192 as two blocks of 4096 or, for calls with a block
- *         mask, as the 16384-point spectrum split by bin parity; fp32 lanes
- *         otherwise) and, with filters of at most 2049 taps, for longer N as
- *         overlap-save windows of one fused transform each.
- *         Orders 2 and 3 at N > 8192 with L > 2049 return
+ *         exist for N <= 16384 (tensor cores for fp16/bf16 at N = 256 ..
+ *         16384: N = 8192 and 16384 as two and four blocks of 4096 in one
+ *         tile, N = 8192 with a block mask as the 16384-point spectrum split
+ *         by bin parity; fp32 lanes up to 8192 otherwise) and, with filters
+ *         of at most 2049 taps, for longer N as overlap-save windows of one
+ *         fused transform each.  A four-block plan (N = 16384) stores
+ *         8192-point filter rows: it rejects block masks and
+ *         fftconv_filter_to_rfft (FFTCONV_ERR_UNSUPPORTED; order 5 serves
+ *         them).  Orders 2 and 3 at N > 16384 with L > 2049 return
  *         FFTCONV_ERR_UNSUPPORTED: no fused kernel holds that transform on
  *         chip; orders 0, 4 and 5 serve it;
  *   4     staged: one intermediate pass through a plan-owned workspace in
@@ -120,7 +124,7 @@ typedef enum {
  * Two further values select an engine inside those families:
  *   1     fused on fp32 lanes (N <= 8192), whatever the dtype;
  *   5     staged, with the row pass on the tensor cores (fp16/bf16,
- *         16384 <= N <= 2^22, L > 2049).  Order 0 chooses it for those plans,
+ *         16384 <= N <= 2^22, L > 2049).  Order 0 chooses it for N >= 32768,
  *         as overlap-save windows of 2 x hop points when the filter is at most
  *         half the sequence (hop = the power of two >= max(L, 16384)); such a
  *         windowed plan rejects block masks and fftconv_filter_to_rfft with
@@ -137,7 +141,7 @@ FFTCONV_API int fftconv_plan_create(fftconv_plan_t* out, int64_t N, int64_t H,
  * partial convolution, defined as the convolution with k zero-padded to N
  * (FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
  * summary and "Approach": partial convolutions).
- * With a 16-bit dtype, N >= 16384 and L <= 2049, orders 0, 2 and 3 choose the
+ * With a 16-bit dtype, N >= 32768 and L <= 2049, orders 0, 2 and 3 choose the
  * tensor-core path as overlap-save: windows of 4096 inputs with hop 2048, each
  * one 8192-point transform, N/2048 - 1 windows per sequence.  Such a plan
  * stores the 8192-point filter spectrum, so fftconv_forward rejects a

@@ -169,7 +169,8 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         delete p;
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "order %d asks for a fused on-chip transform; none holds N=%lld with L=%lld "
-                    "(fused kernels: N <= 8192, or L <= 2049 with 16-bit data); use order 0, 4 or 5",
+                    "(fused kernels: N <= 16384 with 16-bit data, N <= 8192 in fp32, or L <= 2049 with 16-bit "
+                    "data); use order 0, 4 or 5",
                     order, (long long)N, (long long)L);
     }
 
@@ -309,10 +310,11 @@ static int validate_forward(const Plan& p, const void* u, const void* K_f, void*
                     "block masks act on the 2N-point spectrum; this tensor-core plan (N=%lld) packs %lld "
                     "sequences into one 8192-point transform: create the plan with order 1 or 4 for masks",
                     (long long)p.N, (long long)(4096 / p.N));
-    if (mask && ((p.path == kPathTcFused && tc_overlap_save(p.N, p.L)) || p.nwin > 1))
+    if (mask && ((p.path == kPathTcFused && !tc_full_spectrum(p.N, p.L)) || p.nwin > 1))
         return fail(FFTCONV_ERR_UNSUPPORTED,
-                    "block masks act on the 2N-point spectrum; this overlap-save plan (N=%lld, L=%lld) "
-                    "has none: create the plan with order 1 or 4 (or 5 for N >= 16384, L > 2049)",
+                    "block masks act on the 2N-point spectrum; this plan (N=%lld, L=%lld: overlap-save "
+                    "windows or blocks of 4096) has none: create the plan with order 1 or 4 (or 5 for "
+                    "N >= 16384, L > 2049)",
                     (long long)p.N, (long long)p.L);
     if (B > (int64_t(1) << 30) / 1) {
         if ((double)B * (double)H > 4.0e9) return fail(FFTCONV_ERR_UNSUPPORTED, "B*H too large");
@@ -544,9 +546,10 @@ int fftconv_filter_to_rfft(fftconv_plan_t plan, const void* K_f, float* out, fft
     if (!plan || !K_f || !out) return fail(FFTCONV_ERR_INVALID_ARG, "plan, K_f and out must be non-NULL");
     if (!aligned16(K_f) || ((uintptr_t)out & 7u)) return fail(FFTCONV_ERR_ALIGNMENT, "K_f/out misaligned");
     const Plan& p = plan->p;
-    if (p.path == kPathTcFused && tc_overlap_save(p.N, p.L))
+    if (p.path == kPathTcFused && !tc_full_spectrum(p.N, p.L))
         return fail(FFTCONV_ERR_UNSUPPORTED,
-                    "this overlap-save plan stores the 8192-point spectrum of k, not the 2N-point one");
+                    "this plan (overlap-save windows or blocks of 4096) stores 8192-point spectra of k, "
+                    "not the 2N-point one");
     if (p.nwin > 1)
         return fail(FFTCONV_ERR_UNSUPPORTED,
                     "this overlap-save plan stores the %lld-point spectrum of k, not the 2N-point one",

@@ -98,6 +98,7 @@ bool simt_fused_supported(int logM);
 bool tc_supported(int64_t N, int64_t L, int dtype);
 int64_t tc_windows(int64_t N);   // overlap-save windows per sequence (1: one transform)
 bool tc_overlap_save(int64_t N, int64_t L);   // the plan runs overlap-save windows
+bool tc_full_spectrum(int64_t N, int64_t L);  // the plan stores the 2N-point filter spectrum
 int64_t tc_tiles_per_pair_group(int64_t N, int64_t L);   // tiles per (channel, 4 pairs)
 cudaError_t tc_plan_init(Plan& p);
 void tc_plan_free(Plan& p);

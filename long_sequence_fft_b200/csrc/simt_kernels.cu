@@ -1168,6 +1168,95 @@ cudaError_t simt_precompute_to_tc_layout(const Plan& p, const void* k, void* Kf,
     })
 }
 
+// Four-block filter rows (sequences of 16384): G_0 = H_0 and
+// G_d = H_d + (-1)^f H_{d-1} for d = 1, 2, 3, with H_j = FFT_8192([k_j; 0])
+// (k_j the taps [4096 j, 4096 j + 4096), zero past L).  Two transforms of
+// k_0 + i k_1 and k_2 + i k_3 give the four H_j (as in the two-block
+// kernel); the rows are written in the PP layout over one scale per channel
+// (max |Re|, |Im| of all four rows), stored after the H row quartets.
+template <typename T>
+__global__ void __launch_bounds__(fused_threads<13>())
+simt_precompute_tc_pp4_kernel(const T* __restrict__ k, int64_t L, __half* __restrict__ Kh,
+                              float* __restrict__ scales, const float2* __restrict__ tw) {
+    constexpr int LOGM = 13;
+    constexpr int M = 1 << LOGM;
+    constexpr int NT = fused_threads<LOGM>();
+    constexpr int K = Sched<LOGM>::K;
+    extern __shared__ float2 s[];
+    float2* sa = s;
+    float2* sb = s + smem_elems<1>(M);
+    __shared__ float red[NT / 32];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x;
+    auto clampn = [](int64_t n) { return (int)(n < 0 ? 0 : (n > 4096 ? 4096 : n)); };
+    TwoBlockTaps<T> io;
+    io.k = k + (int64_t)h * L;
+    io.n0 = clampn(L);
+    io.n1 = clampn(L - 4096);
+    first_stage_global<LOGM, NT, T>(sa, tw, io, tid);
+    io.k = k + (int64_t)h * L + 8192;
+    io.n0 = clampn(L - 8192);
+    io.n1 = clampn(L - 12288);
+    first_stage_global<LOGM, NT, T>(sb, tw, io, tid);
+    __syncthreads();
+    fwd_stages<LOGM, 1, K, 1, NT>(sa, tw, 0, tid);
+    fwd_stages<LOGM, 1, K, 1, NT>(sb, tw, 0, tid);
+    auto rows = [&](int p, int& f, float2 (&g)[4]) {
+        f = (int)perm_to_freq(p, LOGM);
+        const int pm = (int)freq_to_perm((M - f) & (M - 1), LOGM);
+        float2 hh[4];
+        const float2 za = sa[sidx<1>(p, 0)], zam = sa[sidx<1>(pm, 0)];
+        const float2 zb = sb[sidx<1>(p, 0)], zbm = sb[sidx<1>(pm, 0)];
+        hh[0] = make_float2(0.5f * (za.x + zam.x), 0.5f * (za.y - zam.y));
+        hh[1] = make_float2(0.5f * (za.y + zam.y), -0.5f * (za.x - zam.x));
+        hh[2] = make_float2(0.5f * (zb.x + zbm.x), 0.5f * (zb.y - zbm.y));
+        hh[3] = make_float2(0.5f * (zb.y + zbm.y), -0.5f * (zb.x - zbm.x));
+        const float sg = (f & 1) ? -1.f : 1.f;
+        g[0] = hh[0];
+        for (int d = 1; d < 4; ++d) g[d] = make_float2(hh[d].x + sg * hh[d - 1].x, hh[d].y + sg * hh[d - 1].y);
+    };
+    float m = 0.f;
+    for (int p = tid; p < M; p += NT) {
+        int f;
+        float2 g[4];
+        rows(p, f, g);
+        for (int d = 0; d < 4; ++d) m = fmaxf(m, fmaxf(fabsf(g[d].x), fabsf(g[d].y)));
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+    for (int i = 0; i < NT / 32; ++i) m = fmaxf(m, red[i]);
+    const float sc = m > 0.f ? m : 1.f;
+    const float inv = 1.f / sc;
+    __half* out = Kh + (int64_t)h * (8 * M);
+    for (int p = tid; p < M; p += NT) {
+        int f;
+        float2 g[4];
+        rows(p, f, g);
+        const int c1 = f & 31, c2 = (f >> 5) & 31, c3 = f >> 10;
+        const int word = ((c2 * 2 + (c3 >> 2)) * 32 + c1) * 4 + 2 * ((c3 & 3) >> 1);
+        for (int d = 0; d < 4; ++d) {
+            out[d * 2 * M + 2 * word + (c3 & 1)] = __float2half_rn(g[d].x * inv);
+            out[d * 2 * M + 2 * word + 2 + (c3 & 1)] = __float2half_rn(g[d].y * inv);
+        }
+    }
+    if (tid == 0) scales[h] = sc;
+}
+
+cudaError_t simt_precompute_to_tc_pp4(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t st) {
+    if (p.L > 16384) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(float2) * 2 * smem_elems<1>(1 << 13);
+    FFTCONV_DISPATCH_T(p.dtype, {
+        auto kern = simt_precompute_tc_pp4_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)p.H, fused_threads<13>(), smem, st>>>(
+            (const T*)k, p.L, (__half*)Kf, (float*)((uint8_t*)Kf + (size_t)p.H * 4 * (8192 * 4)), tw8192);
+        return cudaGetLastError();
+    })
+}
+
 cudaError_t simt_precompute_to_tc_pp2(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t st) {
     if (p.L > 8192) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float2) * smem_elems<1>(1 << 13);

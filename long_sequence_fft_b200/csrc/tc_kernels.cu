@@ -97,6 +97,7 @@ constexpr int kDBuf = 4;             // accumulator ring: 4 buffers of 64 TMEM c
 // 8192-point transforms of complex workspace rows, product with that row's
 // part of the spectrum, inverse, written back in place.
 constexpr int kModePlain = 0, kModeWindows = 1, kModeSplit = 2, kModeRows = 3;
+constexpr int kModeBlocks4 = 4;     // N = 16384: four blocks of 4096 per pair (tc_planar.cu)
 
 // chunk c of a tile -> stage (0 S1, 1 S2, 2 S3, 3 S3', 4 S2', 5 S1') and index
 __host__ __device__ __forceinline__ int chunk_stage(int c) { return c < 40 ? (c >> 3) : 5; }
@@ -1190,6 +1191,7 @@ int tc_mode(int64_t N, int64_t L) {
     (void)L;
     if (N <= kN) return kModePlain;      // N < 4096: several sequences per transform (tc_planar.cu)
     if (N == 2 * kN) return kModeSplit;
+    if (N == 4 * kN) return kModeBlocks4;
     return kModeWindows;
 }
 
@@ -1197,15 +1199,19 @@ int tc_mode(int64_t N, int64_t L) {
 
 bool tc_supported(int64_t N, int64_t L, int dtype) {
     if (dtype != kF16 && dtype != kBF16) return false;
-    if (N <= kN || N == 2 * kN) return true;
+    if (N <= kN || N == 2 * kN || N == 4 * kN) return true;
     return N > kN && L <= kHop + 1;      // overlap-save windows (N a power of two)
 }
 
 int64_t tc_windows(int64_t N) { return N <= kN ? 1 : N / kHop - 1; }
 bool tc_overlap_save(int64_t N, int64_t L) { return tc_mode(N, L) == kModeWindows; }
+bool tc_full_spectrum(int64_t N, int64_t L) {
+    const int m = tc_mode(N, L);
+    return m != kModeWindows && m != kModeBlocks4;
+}
 int64_t tc_tiles_per_pair_group(int64_t N, int64_t L) {
     const int m = tc_mode(N, L);
-    return m == kModeWindows ? tc_windows(N) : (m == kModeSplit ? 2 : 1);
+    return m == kModeWindows ? tc_windows(N) : (m == kModeSplit ? 2 : (m == kModeBlocks4 ? 4 : 1));
 }
 
 namespace {
@@ -1296,10 +1302,12 @@ static size_t tc_split_bytes(const Plan& p) {
     return (size_t)tc_filter_rows(p) * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
 }
 size_t tc_filter_bytes(const Plan& p) {
+    if (tc_mode(p.N, p.L) == kModeBlocks4) return tc_planar_two_block_bytes(p);
     return tc_split_bytes(p) + (tc_mode(p.N, p.L) == kModeSplit ? tc_planar_two_block_bytes(p) : 0);
 }
 
 cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
+    if (tc_mode(p.N, p.L) == kModeBlocks4) return tc_planar_precompute_two_block(p, k, Kf, s);
     if (tc_mode(p.N, p.L) != kModeSplit) return tc_planar_precompute(p, k, Kf, s);
     cudaError_t e = simt_precompute_to_tc_split(p, k, Kf, s);
     if (e == cudaSuccess) e = tc_planar_precompute_two_block(p, k, (uint8_t*)Kf + tc_split_bytes(p), s);
@@ -1308,6 +1316,7 @@ cudaError_t tc_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s
 
 cudaError_t tc_forward(const Plan& p, const ForwardArgs& fa, cudaStream_t s) {
     const TcResources* r = (const TcResources*)p.tc;
+    if (r->mode == kModeBlocks4) return tc_planar_forward(p, fa, kPlanarTwoBlock, s);
     if (r->mode != kModeSplit)
         return tc_planar_forward(p, fa, r->mode == kModeWindows ? kPlanarWindows : kPlanarPlain, s);
     if (!fa.mask) {

@@ -62,6 +62,7 @@ namespace fftconv {
 
 cudaError_t simt_precompute_to_tc_pp(const Plan& p, const void* k, void* Kf, cudaStream_t s);
 cudaError_t simt_precompute_to_tc_pp2(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t s);
+cudaError_t simt_precompute_to_tc_pp4(const Plan& p, const void* k, void* Kf, const float2* tw8192, cudaStream_t s);
 
 namespace {
 
@@ -92,8 +93,8 @@ constexpr int kKBytes = kM * 4;               // one filter spectrum row, 8192 c
 constexpr int OffK = OffBEnd;
 constexpr int OffTw = OffK + kKBytes;         // w8192^e, e < 256, as half2
 constexpr int OffBars = OffTw + 1024;
-constexpr int OffXBars = OffBars + 128;       // two-block hand-over barriers [4 steps][4 slices][2]
-constexpr int OffMisc = OffXBars + 256;
+constexpr int OffXBars = OffBars + 128;       // block-mode hand-over barriers [4 steps][4 slices][<= 3]
+constexpr int OffMisc = OffXBars + 512;
 constexpr int SmemBytes = OffMisc + 64 + 1024;   // + alignment slack
 static_assert(SmemBytes <= 232448, "shared memory");
 
@@ -161,6 +162,15 @@ __device__ __forceinline__ uint32_t k_off(int m, int kbyte) {
 // windows (N >= 16384, filters of at most 2049 taps), two blocks (N = 8192),
 // and the plain mode with a Monarch-aligned frequency mask (N = 4096)
 constexpr int kPlain = kPlanarPlain, kWin = kPlanarWindows, kTwo = kPlanarTwoBlock, kMonarch = kPlanarMonarch;
+constexpr int kFour = 4;          // the block mode with four blocks (N = 16384)
+// block modes: P blocks of 4096 per pair, quarter q = block q >> kShift of
+// pair q & ((1 << kShift) - 1)
+template <int MODE>
+struct Blocks {
+    static constexpr bool on = MODE == kTwo || MODE == kFour;
+    static constexpr int P = MODE == kFour ? 4 : 2;
+    static constexpr int kShift = MODE == kFour ? 0 : 1;
+};
 
 struct PArgs {
     const void* u;
@@ -169,7 +179,8 @@ struct PArgs {
     void* y;
     const uint32_t* K;          // [H][kstride] words: the spectrum / scale, PP layout (k_word)
     int64_t kstride;            // words per channel: 8192, or 16384 (two-block: G_0 then G_1)
-    int g1_from_g0;             // two-block, L <= 4096: G_1 = (-1)^f G_0 (not read)
+    int g1_from_g0;             // two blocks, L <= 4096: G_1 = (-1)^f G_0 (not read)
+    int ng;                     // block mode: filter rows G_d that are not zero (d < ng)
     uint32_t keep_c2;           // Monarch mode: bit c2 keeps the bins with that middle digit
     const float* Kscale;        // [H]
     const uint8_t* mask;
@@ -291,10 +302,10 @@ __device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
         t.h = unit / a.tpc;
         t.j = 0;
         t.bp0 = (unit - t.h * a.tpc) * (64 >> a.lseg);
-    } else if constexpr (MODE == kTwo) {
+    } else if constexpr (Blocks<MODE>::on) {
         t.h = unit / a.tpc;
         t.j = 0;
-        t.bp0 = (unit - t.h * a.tpc) * 2;
+        t.bp0 = (unit - t.h * a.tpc) << Blocks<MODE>::kShift;
     } else {
         const uint32_t un = (uint32_t)unit, tpc = (uint32_t)a.tpc, per_ch = (uint32_t)a.nwin * tpc;
         const uint32_t hh = un / per_ch, rem = un - hh * per_ch, jj = rem / tpc;
@@ -308,11 +319,12 @@ __device__ __forceinline__ TileBase tile_base(const PArgs& a, int64_t unit) {
 template <int MODE>
 __device__ __forceinline__ PairInfo pair_rows(const PArgs& a, const TileBase& t, int q, int sigma) {
     PairInfo p;
-    const int64_t bp = MODE == kTwo ? t.bp0 + (q & 1) : t.bp0 + ((int64_t)q << (4 - a.lseg)) + sigma;
+    const int64_t bp = Blocks<MODE>::on ? t.bp0 + (q & ((1 << Blocks<MODE>::kShift) - 1))
+                                        : t.bp0 + ((int64_t)q << (4 - a.lseg)) + sigma;
     p.valid = bp < a.pb;
     p.tail_only = t.j > 0;
     const int64_t b0 = 2 * (p.valid ? bp : 0), b1 = b0 + 1;
-    const int64_t base = MODE == kWin ? kHop * t.j : (MODE == kTwo ? (int64_t)kN * (q >> 1) : 0);
+    const int64_t base = MODE == kWin ? kHop * t.j : (Blocks<MODE>::on ? (int64_t)kN * (q >> Blocks<MODE>::kShift) : 0);
     p.o0 = (b0 * a.H + t.h) * a.N + base;
     p.o1 = (p.valid && b1 < a.B) ? (b1 * a.H + t.h) * a.N + base : -1;
     return p;
@@ -369,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         mbar_init(bar_fin, kMmaWarps);
         mbar_init(bar_k, 1);
         for (int i = 0; i < 3; ++i) mbar_init(&bar_stage[i], kEpiWarps);
-        if constexpr (MODE == kTwo)
-            for (int i = 0; i < 32; ++i) mbar_init(&xfull[i], 32);
+        if constexpr (Blocks<MODE>::on)
+            for (int i = 0; i < 48; ++i) mbar_init(&xfull[i], 32);
         if constexpr (MODE == kMonarch)
             for (int i = 0; i < 4; ++i) mbar_init(&ek_done[i], kEpiWarps);
         *abort_flag = 0;
@@ -526,9 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             else if (which == 6 && issuer == 0 && (lane >> 3) == 0) {
                                 pf_src = a.K + hn * a.kstride;
                                 pf_bytes = kKBytes;
-                            } else if (MODE == kTwo && which == 7 && issuer == 1 && (lane >> 3) == 0 &&
-                                       !a.g1_from_g0) {
-                                pf_src = a.K + hn * a.kstride + kM;     // G_1 (read only for L > 4096)
+                            } else if (Blocks<MODE>::on && which == 7 && issuer >= 1 && issuer < a.ng &&
+                                       (lane >> 3) == 0 && !a.g1_from_g0) {
+                                pf_src = a.K + hn * a.kstride + issuer * kM;    // G_issuer (block modes)
                                 pf_bytes = kKBytes;
                             }
                         }
@@ -762,18 +774,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             // EK: lane = c1; the PP columns of c3 (all eight) of c2 = 4(k+cc) + s;
             // times the filter spectrum K/scale (|K/scale| <= 1); A4 TMEM
             // columns 8 c2 .. 8 c2 + 7 in place.
-            // Two-block mode: quarters 0, 1 hold block 0 (X_0) of their pair and
-            // quarters 2, 3 block 1 (X_1).  Block 0's output is X_0 G_0; block
-            // 1's is X_1 G_0 + X_0 G_1 (G_1 the spectrum of [k1; k0], which
-            // holds both the part of k that reaches from block 0 into block 1
-            // and the wrap-around of the 8192-point product).  The block-0
-            // warps hand their values over through the data tiles (free
-            // between S2 and E3'); G_1 comes from L2.
+            // Block mode (P = 2 or 4 blocks of 4096 per pair): quarter q holds
+            // block b = q >> blk_shift of pair q & (pairs per tile - 1).  Block
+            // b's output is sum_{j <= b} X_j G_{b-j}, G_d the spectrum of
+            // [k_d; k_{d-1}] (k_d the filter taps [4096 d, 4096 d + 4096),
+            // k_{-1} = 0): G_d holds both the taps that reach d blocks ahead
+            // and the wrap-around of the 8192-point product.  The warps of
+            // blocks b < P - 1 hand their values over through the data tiles
+            // (free between S2 and E3') before their own product; G_0 is in
+            // shared memory, G_1 of P = 2 arrives by cp.async (or is
+            // (-1)^f G_0 when k_1 = 0), the G_d of P = 4 come from L2.
             if (ok && !(ok = wait(bar_k, iter & 1))) fail();
-            const bool x_give = MODE == kTwo && q < 2, x_take = MODE == kTwo && q >= 2;
-            const int xz = (2 * s + (q & 1)) * 4;       // this warp's slots (+ 32 for G_1)
+            using BM = Blocks<MODE>;
+            const int blk = BM::on ? q >> BM::kShift : 0;
+            const int pq = BM::on ? q & ((1 << BM::kShift) - 1) : 0;
+            constexpr int np = BM::on ? (BM::P - 1) << BM::kShift : 1;      // producers per slice
+            const bool x_give = BM::on && blk < BM::P - 1, x_take = BM::on && blk > 0;
+            const int xz = (s * np + (blk << BM::kShift) + pq) * 4;   // this warp's slots when giving
+            const int xg = 32 + (2 * s + pq) * 4;                      // P = 2: the G_1 slots
+            const bool g1_async = x_take && BM::P == 2 && !a.g1_from_g0;
             uint8_t* const xs = smem + OffData;
-            if (x_take && ok && !a.g1_from_g0) {
+            if (g1_async && ok) {
                 // the block-1 warps fetch their G_1 words of all four steps into
                 // their slots (the data tiles are free: this warp's E2 waited for
                 // every S2 chunk)
@@ -783,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c2 = 4 * (2 * st + (e >> 1)) + s;
-                        cp_async16(xs + xoff(st, 32 + xz + e, lane), G1 + k_word(lane, c2, 4 * (e & 1)));
+                        cp_async16(xs + xoff(st, xg + e, lane), G1 + k_word(lane, c2, 4 * (e & 1)));
                     }
                     cp_async_commit();
                 }
@@ -811,16 +832,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         h[cc][2 * p] = pk(r[cc][4 * p], r[cc][4 * p + 1]);
                         h[cc][2 * p + 1] = pk(r[cc][4 * p + 2], r[cc][4 * p + 3]);
                     }
-                uint64_t* xb = &xfull[(st * 4 + s) * 2 + (q & 1)];
+                uint64_t* const xrow = &xfull[(st * 4 + s) * np];       // this step and slice
                 if (x_give) {
-                    // hand block 0's values over before this warp's own product
+                    // hand this block's values over before this warp's own product
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         *(uint4*)(xs + xoff(st, xz + 2 * cc, lane)) = make_uint4(h[cc][0], h[cc][1], h[cc][2], h[cc][3]);
                         *(uint4*)(xs + xoff(st, xz + 2 * cc + 1, lane)) =
                             make_uint4(h[cc][4], h[cc][5], h[cc][6], h[cc][7]);
                     }
-                    mbar_arrive(xb);
+                    mbar_arrive(&xrow[(blk << BM::kShift) + pq]);
                 }
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -829,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     const uint4 k0 = *(const uint4*)(Ks + k_word(lane, c2, 0));
                     const uint4 k1 = *(const uint4*)(Ks + k_word(lane, c2, 4));
                     uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    if (MODE != kTwo && mrow) {
+                    if (!BM::on && mrow) {
                         // frequency-sparse filter: zero the masked bins (f and
                         // its mirror 8192 - f share one rfft bin)
 #pragma unroll
@@ -865,9 +886,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
 #pragma unroll
                     for (int p = 0; p < 4; ++p) cmul_pp(h[cc][2 * p], h[cc][2 * p + 1], kw[2 * p], kw[2 * p + 1]);
                 }
-                if (x_take) {
-                    // + X_0 G_1, once block 0's warp has handed X_0 over
-                    if (!(ok = wait(xb, iter & 1))) {
+                if (BM::P == 4 && x_take) {
+                    // + X_j G_{b-j} for the earlier blocks j of this pair (G_d
+                    // words from L2, requested before the hand-over wait)
+#pragma unroll 1
+                    for (int j = 0; j < blk && ok; ++j) {
+                        const int d = blk - j;
+                        if (d >= a.ng) continue;                  // G_d = 0: the filter is shorter
+                        const uint32_t* Gd = a.K + hch * a.kstride + d * kM;
+                        uint4 gq0 = __ldg((const uint4*)(Gd + k_word(lane, 4 * k + s, 0)));
+                        uint4 gq1 = __ldg((const uint4*)(Gd + k_word(lane, 4 * k + s, 4)));
+                        if (!(ok = wait(&xrow[j], iter & 1))) {
+                            fail();
+                            break;
+                        }
+                        const int zj = (s * np + j) * 4;
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            if (cc == 1) {
+                                gq0 = __ldg((const uint4*)(Gd + k_word(lane, 4 * k + 4 + s, 0)));
+                                gq1 = __ldg((const uint4*)(Gd + k_word(lane, 4 * k + 4 + s, 4)));
+                            }
+                            const uint4 x0 = *(const uint4*)(xs + xoff(st, zj + 2 * cc, lane));
+                            const uint4 x1 = *(const uint4*)(xs + xoff(st, zj + 2 * cc + 1, lane));
+                            const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                            const uint32_t gw[8] = {gq0.x, gq0.y, gq0.z, gq0.w, gq1.x, gq1.y, gq1.z, gq1.w};
+#pragma unroll
+                            for (int p = 0; p < 4; ++p)
+                                cfma_pp(h[cc][2 * p], h[cc][2 * p + 1], xw[2 * p], xw[2 * p + 1], gw[2 * p],
+                                        gw[2 * p + 1]);
+                        }
+                    }
+                    if (!ok) break;
+                } else if (x_take) {
+                    // P = 2: + X_0 G_1, once block 0's warp has handed X_0 over
+                    if (!(ok = wait(&xrow[pq], iter & 1))) {
                         fail();
                         break;
                     }
@@ -879,8 +932,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     }
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        const uint4 x0 = *(const uint4*)(xs + xoff(st, xz + 2 * cc, lane));
-                        const uint4 x1 = *(const uint4*)(xs + xoff(st, xz + 2 * cc + 1, lane));
+                        const int z0 = (s * np + pq) * 4;              // block 0's warp of this pair
+                        const uint4 x0 = *(const uint4*)(xs + xoff(st, z0 + 2 * cc, lane));
+                        const uint4 x1 = *(const uint4*)(xs + xoff(st, z0 + 2 * cc + 1, lane));
                         const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                         uint32_t gw[8];
                         if (a.g1_from_g0) {
@@ -892,8 +946,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             gw[0] = k0.x ^ sg; gw[1] = k0.y ^ sg; gw[2] = k0.z ^ sg; gw[3] = k0.w ^ sg;
                             gw[4] = k1.x ^ sg; gw[5] = k1.y ^ sg; gw[6] = k1.z ^ sg; gw[7] = k1.w ^ sg;
                         } else {
-                            const uint4 g0 = *(const uint4*)(xs + xoff(st, 32 + xz + 2 * cc, lane));
-                            const uint4 g1 = *(const uint4*)(xs + xoff(st, 32 + xz + 2 * cc + 1, lane));
+                            const uint4 g0 = *(const uint4*)(xs + xoff(st, xg + 2 * cc, lane));
+                            const uint4 g1 = *(const uint4*)(xs + xoff(st, xg + 2 * cc + 1, lane));
                             gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
                             gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
                         }
@@ -912,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     if (lane == 0) mbar_arrive(&ek_done[st]);
                 }
             }
-            if (x_take && !a.g1_from_g0) cp_async_wait<0>();   // nothing in flight past here (also after an abort)
+            if (g1_async) cp_async_wait<0>();     // nothing in flight past here (also after an abort)
             // E3': lane = c1; chunk c + (s >> 1), its c2 = 4(k + cc) + cl for
             // cl < 4, j3 = 4h + jj with h = s & 1 (PP columns 16 cl + 8h ..
             // + 7); twiddle conj w8192^(c1 j3); K-major A5 tile j3, row
@@ -1237,7 +1291,7 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = upload_vec(&r->tw1024, twiddles_h2(1024, 1024));
     if (e == cudaSuccess) e = upload_vec(&r->tw8192, twiddles_h2(kM, 256));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&r->num_sms, cudaDevAttrMultiProcessorCount, p.device);
-    if (e == cudaSuccess && p.N == 2 * kN) {
+    if (e == cudaSuccess && (p.N == 2 * kN || p.N == 4 * kN)) {
         std::vector<float2> t(kM);
         for (int i = 0; i < kM; ++i) {
             const std::complex<double> z = wpow(i, kM, -1);
@@ -1248,9 +1302,11 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kWin>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kTwo>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kFour>();
     if (e == cudaSuccess) e = allow_smem<__half, kPlain>();
     if (e == cudaSuccess) e = allow_smem<__half, kWin>();
     if (e == cudaSuccess) e = allow_smem<__half, kTwo>();
+    if (e == cudaSuccess) e = allow_smem<__half, kFour>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kMonarch>();
     if (e == cudaSuccess) e = allow_smem<__half, kMonarch>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain, true>();
@@ -1275,11 +1331,12 @@ size_t tc_planar_filter_bytes(const Plan& p) {
     return (size_t)p.H * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
 }
 
-// Two-block K_f (sequences of 8192): per channel G_0 = FFT_8192([k0; 0]) and
-// G_1 = FFT_8192([k1; k0]) (k0, k1 the taps [0, 4096) and [4096, 8192) of k,
-// zero past L), PP layout over one common scale, then [H] fp32 scales
+// Block-mode K_f (sequences of 8192 or 16384, P = N / 4096 blocks): per
+// channel the P rows G_0 = FFT_8192([k0; 0]), G_d = FFT_8192([k_d; k_{d-1}])
+// (k_d the taps [4096 d, 4096 d + 4096) of k, zero past L), PP layout over one
+// common scale, then [H] fp32 scales
 size_t tc_planar_two_block_bytes(const Plan& p) {
-    return (size_t)p.H * 2 * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
+    return (size_t)p.H * (size_t)(p.N / kN) * kKBytes + (((size_t)p.H * 4 + 15) & ~size_t(15));
 }
 
 cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
@@ -1288,27 +1345,31 @@ cudaError_t tc_planar_precompute(const Plan& p, const void* k, void* Kf, cudaStr
 
 cudaError_t tc_planar_precompute_two_block(const Plan& p, const void* k, void* Kf, cudaStream_t s) {
     const Resources* r = (const Resources*)p.tcp;
-    if (p.N != 2 * kN || !r->twf8192) return cudaErrorInvalidValue;
-    return simt_precompute_to_tc_pp2(p, k, Kf, r->twf8192, s);
+    if ((p.N != 2 * kN && p.N != 4 * kN) || !r->twf8192) return cudaErrorInvalidValue;
+    return p.N == 2 * kN ? simt_precompute_to_tc_pp2(p, k, Kf, r->twf8192, s)
+                         : simt_precompute_to_tc_pp4(p, k, Kf, r->twf8192, s);
 }
 
 // mode: kPlain (N <= 4096), kWin (overlap-save windows), kTwo (N = 8192,
 // fa.Kf the two-block filter rows)
 cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cudaStream_t s) {
     const Resources* r = (const Resources*)p.tcp;
-    if (mode == kTwo && (p.N != 2 * kN || fa.mask)) return cudaErrorInvalidValue;
+    if (mode == kTwo && ((p.N != 2 * kN && p.N != 4 * kN) || fa.mask)) return cudaErrorInvalidValue;
     PArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.K = (const uint32_t*)fa.Kf;
-    a.kstride = mode == kTwo ? 2 * kM : kM;
-    a.g1_from_g0 = mode == kTwo && p.L <= kN;
-    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * (mode == kTwo ? 2 : 1) * kKBytes);
+    const int rows = mode == kTwo ? (int)(p.N / kN) : 1;       // filter rows per channel
+    a.kstride = (int64_t)rows * kM;
+    a.g1_from_g0 = mode == kTwo && rows == 2 && p.L <= kN;
+    a.ng = (int)((p.L + kN - 1) / kN) + 1;                      // G_d = 0 for d > ceil(L / 4096)
+    if (a.ng > rows) a.ng = rows;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * rows * kKBytes);
     a.mask = fa.mask; a.mask_h = fa.mask_h;
     a.B = fa.B; a.H = p.H; a.N = p.N;
     a.nwin = mode == kWin ? p.N / kHop - 1 : 1;
     a.lseg = plan_lseg(p.N);
     a.pb = (fa.B + 1) / 2;
-    const int64_t pairs_per_tile = mode == kTwo ? 2 : int64_t(64) >> a.lseg;   // 4 rows x 4096 / N pairs
+    const int64_t pairs_per_tile = mode == kTwo ? 4 / rows : int64_t(64) >> a.lseg;   // 4 rows x 4096 / N pairs
     a.tpc = (a.pb + pairs_per_tile - 1) / pairs_per_tile;
     a.nunits = p.H * a.nwin * a.tpc;
     a.bimg = (const uint4*)r->bimg;
@@ -1318,10 +1379,12 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cu
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
     if (p.dtype == kBF16) {
         if (mode == kWin) launch<__nv_bfloat16, kWin>(a, grid, s);
+        else if (mode == kTwo && rows == 4) launch<__nv_bfloat16, kFour>(a, grid, s);
         else if (mode == kTwo) launch<__nv_bfloat16, kTwo>(a, grid, s);
         else launch<__nv_bfloat16, kPlain>(a, grid, s);
     } else {
         if (mode == kWin) launch<__half, kWin>(a, grid, s);
+        else if (mode == kTwo && rows == 4) launch<__half, kFour>(a, grid, s);
         else if (mode == kTwo) launch<__half, kTwo>(a, grid, s);
         else launch<__half, kPlain>(a, grid, s);
     }

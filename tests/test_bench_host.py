@@ -48,6 +48,7 @@ def test_algorithmic_bytes_at_the_stored_filter_width(name, path, expected):
     ("gated_bf16_n1k", "tc_fused", 896.0),
     ("sparse_bf16_n8k", "tc_fused", 1152.0),
     ("partial_bf16_n8k", "tc_fused", 896.0),
+    ("fp16_n16k", "tc_fused", 896.0),
     ("fp16_n32k", "tc_staged", 1152.0),
     ("fp32_n1k", "simt_fused", 0.0),
 ])

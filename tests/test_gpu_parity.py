@@ -42,6 +42,7 @@ for dtype in ("f32", "f16", "bf16"):
         for (B, H, N) in ((1, 2, 256), (3, 2, 1024), (2, 3, 4096), (1, 1, 8192)):
             CASES.append((dtype, order, B, H, N))
     CASES.append((dtype, 4, 2, 2, 16384))
+    CASES.append((dtype, 0, 3, 2, 16384))
     CASES.append((dtype, 0, 3, 1, 32768))
 
 
@@ -229,12 +230,12 @@ def test_bad_arguments_are_rejected_without_launch():
 # ------------------------------------------------- overlap-save windows ---
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
-@pytest.mark.parametrize("N,L,B", [(8192, 2048, 3), (8192, 2049, 2), (8192, 1, 1), (16384, 300, 3),
+@pytest.mark.parametrize("N,L,B", [(8192, 2048, 3), (8192, 2049, 2), (8192, 1, 1), (16384, 300, 3), (32768, 300, 3),
                                    (32768, 1024, 1)])
 def test_overlap_save_windows(dtype, N, L, B):
     """Sequences longer than 4096 with filters of L <= 2049 taps run on the
-    tensor-core kernel: as overlapping 4096-sample windows (N >= 16384) or as
-    two blocks of 4096 (N = 8192)."""
+    tensor-core kernel: as overlapping 4096-sample windows (N >= 32768) or as
+    two or four blocks of 4096 (N = 8192, 16384)."""
     inp = _rand_inputs(B, 2, N, L, dtype, gated=(B != 1), seed=N + L + B)
     y, plan = run_cuda(inp, dtype, order=0)
     assert plan.path_name == "tc_fused"
@@ -244,23 +245,27 @@ def test_overlap_save_windows(dtype, N, L, B):
 def test_overlap_save_limits():
     import long_sequence_fft_b200 as lsf
     import torch
-    # one tap too many for the windows: at N = 8192 the two-block mode (or,
-    # with a mask, the parity split) serves it, longer sequences go to the
-    # SIMT path
+    # one tap too many for the windows: at N = 8192 and 16384 the block modes
+    # (at 8192 with a mask, the parity split) serve it, longer sequences go to
+    # the staged path
     assert lsf.Plan(8192, 2, "bf16", L=2050).path_name == "tc_fused"
-    assert lsf.Plan(16384, 2, "bf16", L=2050).path_name != "tc_fused"
-    plan = lsf.Plan(16384, 2, "bf16", L=2048)
-    assert plan.path_name == "tc_fused"
-    k = torch.zeros((2, 2048), dtype=torch.bfloat16, device="cuda")
-    Kf = plan.precompute(k)
-    u = torch.zeros((2, 2, 16384), dtype=torch.bfloat16, device="cuda")
-    mask = torch.ones((1, 16384 // 32), dtype=torch.uint8, device="cuda")
-    with pytest.raises(lsf.FFTConvError) as e:
-        plan.forward(u, Kf, mask=mask)
-    assert e.value.status == lsf.ERR_UNSUPPORTED
-    with pytest.raises(lsf.FFTConvError) as e:
-        plan.export_rfft(Kf)
-    assert e.value.status == lsf.ERR_UNSUPPORTED
+    assert lsf.Plan(16384, 2, "bf16", L=2050).path_name == "tc_fused"
+    assert lsf.Plan(32768, 2, "bf16", L=2050).path_name != "tc_fused"
+    # windows (N = 32768) and four blocks (N = 16384) store 8192-point spectra
+    # only: no block mask, no 2N-point export
+    for N in (32768, 16384):
+        plan = lsf.Plan(N, 2, "bf16", L=2048)
+        assert plan.path_name == "tc_fused"
+        k = torch.zeros((2, 2048), dtype=torch.bfloat16, device="cuda")
+        Kf = plan.precompute(k)
+        u = torch.zeros((2, 2, N), dtype=torch.bfloat16, device="cuda")
+        mask = torch.ones((1, N // 32), dtype=torch.uint8, device="cuda")
+        with pytest.raises(lsf.FFTConvError) as e:
+            plan.forward(u, Kf, mask=mask)
+        assert e.value.status == lsf.ERR_UNSUPPORTED
+        with pytest.raises(lsf.FFTConvError) as e:
+            plan.export_rfft(Kf)
+        assert e.value.status == lsf.ERR_UNSUPPORTED
 
 
 def test_forward_host_pipelined_chunks_match_device_path():

@@ -6,9 +6,9 @@
    the split mode's parked z_even are exercised many times per CTA), in every
    mode the kernels have: plain (N = 4096), packed short sequences (N = 256 ..
    2048, 4096 / N of them per 8192-point transform), overlap-save windows
-   (partial filters, N >= 16384), the two-block mode of N = 8192 (unmasked
-   calls), the N = 8192 parity split (masked calls) and the staged path's row
-   pass.  The launch configuration is the plan's own, as in the benchmark.
+   (partial filters, N >= 32768), the block modes of N = 8192 (two blocks of
+   4096, unmasked calls) and N = 16384 (four blocks), the N = 8192 parity
+   split (masked calls) and the staged path's row pass.  The launch configuration is the plan's own, as in the benchmark.
 2. Closed forms the convolution must reproduce on every tensor-core mode
    (exact results of the definition "FlashFFTConv: Efficient Convolutions for
    Long Sequences with Tensor Cores", summary and "Approach", with the
@@ -94,10 +94,22 @@ def test_packed_mode_rejects_masks():
 
 
 def test_windows_mode_three_tiles_per_cta():
-    B, H, N, L = 16, 32, 16384, 2048
+    B, H, N, L = 16, 16, 32768, 2048
     tiles = H * (N // 2048 - 1) * ((B // 2 + 3) // 4)
     assert tiles >= 3 * SMS
     _compare(_inputs(B, H, N, L, "bf16", gated=True, seed=3), "bf16", f"windows {tiles} tiles")
+
+
+@pytest.mark.parametrize("B,H,L,gated,dtype", [(8, 112, 16384, True, "bf16"),
+                                               (7, 128, 9000, False, "f16"),
+                                               (8, 112, 4000, True, "bf16")])
+def test_four_block_mode_three_tiles_per_cta(B, H, L, gated, dtype):
+    """N = 16384: one pair per tile as four blocks of 4096; block b adds the
+    earlier blocks' spectra times G_1 .. G_b."""
+    N = 16384
+    tiles = H * ((B + 1) // 2)
+    assert tiles >= 3 * SMS
+    _compare(_inputs(B, H, N, L, dtype, gated=gated, seed=L + B + 1), dtype, f"four-block L={L} B={B} {tiles} tiles")
 
 
 @pytest.mark.parametrize("B,H,L,gated,dtype", [(16, 112, 8192, True, "bf16"),
@@ -135,8 +147,10 @@ MODES = [  # (name, N, L, order, path); the split mode runs for masked calls
     ("plain", 4096, 4096, 0, "tc_fused"),
     ("packed1k", 1024, 1024, 0, "tc_fused"),
     ("packed256", 256, 256, 0, "tc_fused"),
-    ("windows", 16384, 2048, 0, "tc_fused"),
+    ("windows", 32768, 2048, 0, "tc_fused"),
     ("twoblock", 8192, 8192, 0, "tc_fused"),
+    ("fourblock", 16384, 16384, 0, "tc_fused"),
+    ("fourblock_partial", 16384, 6000, 0, "tc_fused"),
     ("twoblock_partial", 8192, 3000, 0, "tc_fused"),
     ("split", 8192, 8192, 0, "tc_fused"),
     ("rows", 16384, 16384, 5, "tc_staged"),
@@ -173,7 +187,7 @@ def test_delta_filters_return_the_input(name, N, L, order, path, dtype):
     # shifted delta (a different shift per channel): y[t] = (u w)[t - d] v[t];
     # at N = 8192 one shift moves block 0 entirely into block 1 and the other
     # gives block 1 outputs from both blocks' inputs (both two-block terms)
-    d = [min(5, L - 1), min(L - 1, 1500)] if N != 8192 else [min(L - 1, 4095), 2000]
+    d = {8192: [min(L - 1, 4095), 2000], 16384: [min(L - 1, 12289), 5000]}.get(N, [min(5, L - 1), min(L - 1, 1500)])
     k = np.zeros((H, L), np.float32)
     ref = np.zeros((B, H, N))
     for h in range(H):
@@ -248,7 +262,8 @@ def _status_after(u, k, dtype, order, N, L, mask=None):
 @pytest.mark.parametrize("name,N,L,order,path,edge,beyond", [
     ("plain", 4096, 4096, 0, "tc_fused", 90.0, 1500.0),
     ("packed1k", 1024, 1024, 0, "tc_fused", 90.0, 6000.0),     # B = 2: one segment of 1024 per row
-    ("windows", 16384, 2048, 0, "tc_fused", 90.0, 1500.0),
+    ("windows", 32768, 2048, 0, "tc_fused", 90.0, 1500.0),
+    ("fourblock", 16384, 16384, 0, "tc_fused", 90.0, 1500.0),
     ("twoblock", 8192, 8192, 0, "tc_fused", 90.0, 1500.0),
     ("split", 8192, 8192, 0, "tc_fused", 90.0, 3000.0),
     ("rows", 16384, 16384, 5, "tc_staged", 90.0, 2000.0),

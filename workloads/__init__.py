@@ -95,6 +95,10 @@ WORKLOADS = {
                                description="gated bf16 conv B=64 H=768 N=1024"),
     "bf16_n1k": Workload("bf16_n1k", 9, 64, 768, 1024, 1024, "bf16", False, "scaled",
                          description="bf16 conv B=64 H=768 N=1024"),
+    # sequence length 16K at cfg3's element count: the four-block fused
+    # tensor-core mode (the 32K configuration runs staged)
+    "fp16_n16k": Workload("fp16_n16k", 11, 16, 256, 16384, 16384, "f16", False, "scaled",
+                          description="fp16 conv B=16 H=256 N=16384"),
     # the flagship shape with a Monarch-aligned 75% frequency mask: the middle
     # digits c2 in {0..3, 28..31} of the 8192-point spectrum are kept
     "monarch_bf16_n4k": Workload("monarch_bf16_n4k", 10, 64, 768, 4096, 4096, "bf16", True, "decay:0.001",
