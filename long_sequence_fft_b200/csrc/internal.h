@@ -109,8 +109,9 @@ cudaError_t tc_export_rfft(const Plan& p, const void* Kf, float* out, cudaStream
 cudaError_t selftest_bounded_wait(const Plan& p, uint32_t polls, int arrive, cudaStream_t s);
 
 // tensor-core fused kernel with planar complex data (tc_planar.cu):
-// sequences of at most 4096 (plain), of 8192 as two blocks (the filter rows
-// G_0, G_1 of tc_planar_precompute_two_block), and overlap-save windows
+// sequences of at most 4096 (plain), of 8192 and 16384 as two and four blocks
+// of 4096 (kPlanarTwoBlock: the filter rows G_0 .. G_{P-1} of
+// tc_planar_precompute_two_block), and overlap-save windows
 enum { kPlanarPlain = 0, kPlanarWindows = 1, kPlanarTwoBlock = 2, kPlanarMonarch = 3 };
 cudaError_t tc_planar_init(Plan& p);
 void tc_planar_free(Plan& p);

@@ -1,10 +1,10 @@
 // tc_planar.cu -- tensor-core (tcgen05) fused FFT convolution with planar
 // complex data, sm_100a: sequences of 4096 (one zero-padded 8192-point
 // transform per sequence; shorter ones packed several to a transform),
-// sequences of 8192 as two blocks of 4096 (a two-block partitioned
-// convolution: block b's output is X_b G_0 + X_{b-1} G_1 in the 8192-point
-// domain), and longer sequences with filters of at most 2049 taps
-// (overlap-save windows of 4096 inputs, hop 2048).
+// sequences of 8192 and 16384 as two and four blocks of 4096 (a
+// block-partitioned convolution: block b's output is sum_{j <= b} X_j G_{b-j}
+// in the 8192-point domain), and longer sequences with filters of at most
+// 2049 taps (overlap-save windows of 4096 inputs, hop 2048).
 //
 // FlashFFTConv: Efficient Convolutions for Long Sequences with Tensor Cores,
 // "Approach": the FFT convolution as an order-p Monarch decomposition --
@@ -178,7 +178,7 @@ struct PArgs {
     const void* v;
     void* y;
     const uint32_t* K;          // [H][kstride] words: the spectrum / scale, PP layout (k_word)
-    int64_t kstride;            // words per channel: 8192, or 16384 (two-block: G_0 then G_1)
+    int64_t kstride;            // words per channel: 8192, or 8192 P (block modes: G_0 .. G_{P-1})
     int g1_from_g0;             // two blocks, L <= 4096: G_1 = (-1)^f G_0 (not read)
     int ng;                     // block mode: filter rows G_d that are not zero (d < ng)
     uint32_t keep_c2;           // Monarch mode: bit c2 keeps the bins with that middle digit
@@ -249,13 +249,13 @@ __device__ __forceinline__ void cfma_pp(uint32_t& yr, uint32_t& yi, uint32_t xr,
 }
 constexpr uint32_t kNegPair = 0x80008000u;   // sign bits of both halves
 
-// Two-block hand-over slots of EK step st (byte offsets from the data
+// Block-mode hand-over slots of EK step st (byte offsets from the data
 // tiles): the bytes that E3' writes in the same step (K bytes [32 st,
 // 32 st + 32) of every row of every tile), 64 slots of 16 bytes per lane,
 // consecutive lanes on consecutive rows so that a warp's 16-byte accesses hit
-// distinct banks.  Slot z < 32: piece z % 4 of block 0's values from the warp
-// (slice s, pair pq), z = (2 s + pq) 4 + piece; slot 32 + z: the G_1 words
-// that the block-1 warp (slice s, pair pq) reads.
+// distinct banks.  Slot z = (s np + i) 4 + piece: piece < 4 of the values of
+// the giving warp i (of np per slice) of slice s; with two blocks, slot
+// 32 + (2 s + pq) 4 + piece: the G_1 words the block-1 warp of pair pq reads.
 __device__ __forceinline__ uint32_t xoff(int st, int z, int lane) {
     return (uint32_t)((z >> 3) * kTile) + k_off(32 * (z & 3) + lane, 32 * st + 16 * ((z >> 2) & 1));
 }
@@ -289,9 +289,10 @@ struct PairInfo {
 // each pair, exactly: a filter of at most N taps reaches back at most N - 1
 // positions, into that pair's own zeros (or, for sigma = 0, around the end
 // of the row into the last pair's zeros).
-// Sequences of 8192 (two-block mode): a tile holds two pairs 2u', 2u'+1;
-// transform row q is block q >> 1 (inputs and outputs [4096 (q >> 1),
-// 4096 (q >> 1) + 4096)) of pair 2u' + (q & 1), zero-padded to 8192 points.
+// Sequences of 8192 and 16384 (block modes, P = N / 4096 blocks): a tile
+// holds 4 / P pairs; transform row q is block b = q >> log2(4 / P) (inputs
+// and outputs [4096 b, 4096 b + 4096)) of the tile's pair q mod (4 / P),
+// zero-padded to 8192 points.
 struct TileBase {
     int64_t h, bp0, j;   // channel, first pair of the tile, window
 };
@@ -356,8 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
     uint64_t* bar_fin = bar + 9;   // every MMA has completed (drain before exit)
     uint64_t* bar_k = bar + 10;    // the tile's filter row has landed in shared memory
     uint64_t* bar_stage = bar + 11;   // [3] E2, E3', E2' done for the tile (16 epilogue warps)
-    // two-block mode: [EK step][slice][pair] block 0's spectrum values are in
-    // the hand-over slots (the 32 threads of that warp)
+    // block modes: [EK step][slice][giving warp] that warp's spectrum values
+    // are in the hand-over slots (its 32 threads)
     uint64_t* xfull = (uint64_t*)(smem + OffXBars);
     // Monarch mode (same space): [4] the EK of c2 group m is done (16 epilogue warps)
     uint64_t* ek_done = (uint64_t*)(smem + OffXBars);
@@ -583,12 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             twi[p] = h2u(__highs2half2(t0, t1));
         }
 
-        // ---- load: x = u*w for t = 256 j1 + 8 l + j3 (l = lane), j1 in
-        // {2P, 2P+1} with P = 2s + part, into the TMEM A1 columns 16 j3 + 2P
-        // (real pair) and 16 j3 + 2P + 1 (imaginary pair: the pair's second
-        // row); part 1 then arrives on bar_in.  A tile's input is loaded while
-        // the previous tile's last stages run (the A columns are free once S3'
-        // is done).  Absent rows or gates read a present row and are masked.
         // ---- load: x = u*w for t = 256 j1 + 8 l + j3 (l = lane), j1 the kept
         // stage-1 digits of index 2P and 2P+1 with P = 2s + part, into the TMEM
         // A1 columns 16 j3 + 2P (real pair) and 16 j3 + 2P + 1 (imaginary
@@ -1350,8 +1345,8 @@ cudaError_t tc_planar_precompute_two_block(const Plan& p, const void* k, void* K
                          : simt_precompute_to_tc_pp4(p, k, Kf, r->twf8192, s);
 }
 
-// mode: kPlain (N <= 4096), kWin (overlap-save windows), kTwo (N = 8192,
-// fa.Kf the two-block filter rows)
+// mode: kPlain (N <= 4096), kWin (overlap-save windows), kTwo (block modes,
+// N = 8192 or 16384; fa.Kf the block filter rows)
 cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cudaStream_t s) {
     const Resources* r = (const Resources*)p.tcp;
     if (mode == kTwo && ((p.N != 2 * kN && p.N != 4 * kN) || fa.mask)) return cudaErrorInvalidValue;
