@@ -611,10 +611,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 const int64_t t0 = tau_of(a, i) + 8 * lane;
                 const T* pu0 = (const T*)a.u + LP.o0;
                 const T* pu1 = (const T*)a.u + oo1;
-                lp.ld[jh][0] = __ldg((const uint4*)(pu0 + t0));
-                lp.ld[jh][1] = __ldg((const uint4*)((has_w ? (const T*)a.w + LP.o0 : pu0) + t0));
-                lp.ld[jh][2] = __ldg((const uint4*)(pu1 + t0));
-                lp.ld[jh][3] = __ldg((const uint4*)((has_w ? (const T*)a.w + oo1 : pu1) + t0));
+                // read once: evict-first leaves L2 to the prefetched next rows
+                // (measured 1.3% faster on the flagship); overlap-save windows
+                // re-read half of each window and the four-block mode measured
+                // slower with it: normal policy there
+                const uint64_t pol = (MODE == kWin || MODE == kFour) ? l2_evict_normal() : l2_evict_first();
+                lp.ld[jh][0] = ldg_nc_hint(pu0 + t0, pol);
+                lp.ld[jh][1] = ldg_nc_hint((has_w ? (const T*)a.w + LP.o0 : pu0) + t0, pol);
+                lp.ld[jh][2] = ldg_nc_hint(pu1 + t0, pol);
+                lp.ld[jh][3] = ldg_nc_hint((has_w ? (const T*)a.w + oo1 : pu1) + t0, pol);
             }
         };
         auto load_finish = [&](int part, const LoadPart& lp) {
@@ -1042,8 +1047,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             const int i = 4 * s + 2 * hf + jj;
                             const PairInfo Pg = pair_rows<MODE>(a, TB, q, seg_of(a, i));
                             const int64_t tg = tau_of(a, i) + 8 * lane;
-                            vg[hf][jj][0] = __ldg((const uint4*)(vr + Pg.o0 + tg));
-                            vg[hf][jj][1] = __ldg((const uint4*)(vr + (Pg.o1 >= 0 ? Pg.o1 : Pg.o0) + tg));
+                            const uint64_t pol = l2_evict_first();      // the gate is read once
+                            vg[hf][jj][0] = ldg_nc_hint(vr + Pg.o0 + tg, pol);
+                            vg[hf][jj][1] = ldg_nc_hint(vr + (Pg.o1 >= 0 ? Pg.o1 : Pg.o0) + tg, pol);
                         }
                 }
 #pragma unroll
