@@ -225,10 +225,11 @@ FFTCONV_API int fftconv_forward_monarch(fftconv_plan_t plan, const void* u, cons
  *   dk            : [H, L] fp32 device or NULL; overwritten with the sum over
  *                   the batch (the call clears it first).
  * Outputs must not overlap each other or any input.  Supported on fp16/bf16
- * tensor-core plans with N <= 4096 (fftconv_plan_path ==
+ * tensor-core plans with N <= 8192 (fftconv_plan_path ==
  * FFTCONV_PATH_TC_FUSED); other plans return FFTCONV_ERR_UNSUPPORTED.  du and
  * dw come from one launch of the fused tensor-core kernel with the product by
- * conj(K_f) (correlation) and two gated outputs, dv from the forward kernel
+ * conj(K_f) (correlation; at N = 8192 as two blocks of 4096, block 0 adding
+ * block 1's spectrum times conj(G_1)) and two gated outputs, dv from the forward kernel
  * with dy as the output gate, dk from fp32 transforms of dy*v and u*w per
  * (channel, batch chunk).  Asynchronous on `stream`; allocates nothing.  The
  * fp16 range note above applies to du, dw, dv (FFTCONV_ERR_RANGE). */

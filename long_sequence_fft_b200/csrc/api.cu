@@ -231,7 +231,7 @@ int fftconv_plan_create_ex(fftconv_plan_t* out, int64_t N, int64_t H, fftconv_dt
         e = tc_plan_init(*p);
         p->filter_bytes = tc_filter_bytes(*p);
         // the backward pass's filter gradient transforms length 2N on fp32 lanes
-        if (e == cudaSuccess && N <= 4096) e = upload(&p->twgrad, host_twiddles(p->M, p->M, 1));
+        if (e == cudaSuccess && N <= 8192) e = upload(&p->twgrad, host_twiddles(p->M, p->M, 1));
     }
     if (e != cudaSuccess) {
         free_plan(p);
@@ -492,9 +492,9 @@ int fftconv_backward(fftconv_plan_t plan, const void* u, const void* K_f, const 
     g_last_error.clear();
     if (!plan) return fail(FFTCONV_ERR_INVALID_ARG, "plan is NULL");
     const Plan& p = plan->p;
-    if (p.path != kPathTcFused || p.N > 4096)
+    if (p.path != kPathTcFused || p.N > 8192)
         return fail(FFTCONV_ERR_UNSUPPORTED,
-                    "the backward pass runs on fp16/bf16 tensor-core plans with N <= 4096 (this plan: %s, N=%lld)",
+                    "the backward pass runs on fp16/bf16 tensor-core plans with N <= 8192 (this plan: %s, N=%lld)",
                     p.path == kPathTcFused ? "tensor-core" : "not tensor-core", (long long)p.N);
     int rc = validate_forward(p, u, K_f, du, B, H, N, w, v, nullptr, 0);
     if (rc != FFTCONV_OK) return rc;
@@ -530,9 +530,12 @@ int fftconv_backward(fftconv_plan_t plan, const void* u, const void* K_f, const 
         ForwardArgs a{u, w, dy, dv, K_f, nullptr, 0, B};
         e = tc_forward(p, a, s);
     }
-    // du = w * corr(dy * v, k), dw = u * corr(dy * v, k)
+    // du = w * corr(dy * v, k), dw = u * corr(dy * v, k) (N = 8192: on the
+    // two-block filter rows, the last part of K_f)
     if (e == cudaSuccess) {
-        ForwardArgs a{dy, v, w, du, K_f, nullptr, 0, B};
+        const void* Kc = p.N == 8192 ? (const void*)((const uint8_t*)K_f + p.filter_bytes - tc_planar_two_block_bytes(p))
+                                     : K_f;
+        ForwardArgs a{dy, v, w, du, Kc, nullptr, 0, B};
         e = tc_planar_correlate(p, a, dw, u, s);
     }
     // dk = sum_b corr(dy * v, u * w)[:L]

@@ -490,7 +490,9 @@ simt_precompute_tc_split_kernel(const T* __restrict__ k, int64_t L, __half2* __r
 // correlation, exact for s < N since the padding absorbs the wrap).  One
 // inverse transform of the sum then gives the CTA's part of dk, added to the
 // (zeroed) output with atomics.  The accumulator sits in shared memory beside
-// the transform buffer, indexed by permuted position like the spectrum.
+// the transform buffer and holds the bins [0, M/2] only (the sum is the
+// spectrum of a real sequence, so the other half is their conjugate mirror),
+// which keeps M = 16384 (N = 8192) within one CTA's shared memory.
 template <int LOGM, typename T>
 __global__ void __launch_bounds__(fused_threads<LOGM>())
 simt_filter_grad_kernel(const T* __restrict__ u, const T* __restrict__ w, const T* __restrict__ v,
@@ -501,11 +503,12 @@ simt_filter_grad_kernel(const T* __restrict__ u, const T* __restrict__ w, const 
     constexpr int M = 1 << LOGM;
     constexpr int64_t N = M / 2;
     extern __shared__ float2 s[];
+    // the summed spectrum is Hermitian (dk is real): bins [0, M/2] only
     float2* acc = s + smem_elems<1>(M);
     const int tid = threadIdx.x;
     const int64_t h = blockIdx.x;
     const int64_t b0 = (int64_t)blockIdx.y * rows, b1 = b0 + rows < B ? b0 + rows : B;
-    for (int p = tid; p < M; p += NT) acc[p] = make_float2(0.f, 0.f);
+    for (int f = tid; f <= M / 2; f += NT) acc[f] = make_float2(0.f, 0.f);
     for (int64_t b = b0; b < b1; ++b) {
         const int64_t o = (b * H + h) * N;
         PairRows<T> io;
@@ -518,18 +521,22 @@ simt_filter_grad_kernel(const T* __restrict__ u, const T* __restrict__ w, const 
         first_stage_global<LOGM, NT, T>(s, tw, io, tid);
         __syncthreads();
         fwd_stages<LOGM, 1, K, 1, NT>(s, tw, 0, tid);
-        for (int p = tid; p < M; p += NT) {
-            const int f = (int)perm_to_freq(p, LOGM);
+        for (int f = tid; f <= M / 2; f += NT) {
+            const int p = (int)freq_to_perm(f, LOGM);
             const int pm = (int)freq_to_perm((M - f) & (M - 1), LOGM);
             const float2 zf = s[sidx<1>(p, 0)], zm = s[sidx<1>(pm, 0)];
             // G = (zf + conj zm) / 2, X = (zf - conj zm) / 2i
             const float2 G = make_float2(0.5f * (zf.x + zm.x), 0.5f * (zf.y - zm.y));
             const float2 X = make_float2(0.5f * (zf.y + zm.y), 0.5f * (zm.x - zf.x));
-            acc[p] = cadd(acc[p], cmulc(G, X));
+            acc[f] = cadd(acc[f], cmulc(G, X));
         }
     }
     __syncthreads();
-    for (int p = tid; p < M; p += NT) s[sidx<1>(p, 0)] = acc[p];
+    for (int p = tid; p < M; p += NT) {
+        const int f = (int)perm_to_freq(p, LOGM);
+        const float2 z = f <= M / 2 ? acc[f] : acc[M - f];
+        s[sidx<1>(p, 0)] = f <= M / 2 ? z : make_float2(z.x, -z.y);
+    }
     __syncthreads();
     inv_stages<LOGM, 0, K, 1, NT>(s, tw, 0, tid);
     const float inv = 1.0f / (float)M;
@@ -1287,7 +1294,7 @@ template <int LOGM, typename T>
 cudaError_t launch_filter_grad(const Plan& p, const void* u, const void* w, const void* v, const void* dy,
                                int64_t B, float* dk, const float2* tw, cudaStream_t st) {
     constexpr int NT = fused_threads<LOGM>();
-    const size_t smem = sizeof(float2) * (smem_elems<1>(1 << LOGM) + (1 << LOGM));
+    const size_t smem = sizeof(float2) * (smem_elems<1>(1 << LOGM) + (1 << (LOGM - 1)) + 1);
     auto kern = simt_filter_grad_kernel<LOGM, T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -1302,7 +1309,7 @@ cudaError_t launch_filter_grad(const Plan& p, const void* u, const void* w, cons
 }
 
 // dk (fp32, [H, L]) <- the filter gradient over the batch; the plan's
-// transform length M = 2N (N <= 4096) and an exp(-2 pi i e / M) table
+// transform length M = 2N (N <= 8192) and an exp(-2 pi i e / M) table
 cudaError_t simt_filter_grad(const Plan& p, const void* u, const void* w, const void* v, const void* dy, int64_t B,
                              float* dk, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)(p.H * p.L), st);
@@ -1316,6 +1323,7 @@ cudaError_t simt_filter_grad(const Plan& p, const void* u, const void* w, const 
                 case 11: return launch_filter_grad<11, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
                 case 12: return launch_filter_grad<12, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
                 case 13: return launch_filter_grad<13, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
+                case 14: return launch_filter_grad<14, __nv_bfloat16>(p, u, w, v, dy, B, dk, tw, st);
                 default: return cudaErrorInvalidValue;
             }
         case kF16:
@@ -1325,6 +1333,7 @@ cudaError_t simt_filter_grad(const Plan& p, const void* u, const void* w, const 
                 case 11: return launch_filter_grad<11, __half>(p, u, w, v, dy, B, dk, tw, st);
                 case 12: return launch_filter_grad<12, __half>(p, u, w, v, dy, B, dk, tw, st);
                 case 13: return launch_filter_grad<13, __half>(p, u, w, v, dy, B, dk, tw, st);
+                case 14: return launch_filter_grad<14, __half>(p, u, w, v, dy, B, dk, tw, st);
                 default: return cudaErrorInvalidValue;
             }
         default: return cudaErrorInvalidValue;

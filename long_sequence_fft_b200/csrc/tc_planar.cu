@@ -347,7 +347,7 @@ __device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
 // second output y2.
 template <typename T, int MODE, bool BWD = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a) {
-    static_assert(!(BWD && MODE != kPlain), "the correlation pass runs on plain plans");
+    static_assert(!BWD || MODE == kPlain || MODE == kTwo, "the correlation pass runs on plain and two-block plans");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* bar = (uint64_t*)(smem + OffBars);
@@ -789,8 +789,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
             const int blk = BM::on ? q >> BM::kShift : 0;
             const int pq = BM::on ? q & ((1 << BM::kShift) - 1) : 0;
             constexpr int np = BM::on ? (BM::P - 1) << BM::kShift : 1;      // producers per slice
-            const bool x_give = BM::on && blk < BM::P - 1, x_take = BM::on && blk > 0;
-            const int xz = (s * np + (blk << BM::kShift) + pq) * 4;   // this warp's slots when giving
+            // (the correlation of the backward pass runs the other way: block b
+            // takes sum_{j > b} X_j conj(G_{j-b}), so the later blocks give)
+            const bool x_give = BM::on && (BWD ? blk > 0 : blk < BM::P - 1);
+            const bool x_take = BM::on && (BWD ? blk < BM::P - 1 : blk > 0);
+            const int gi = BWD ? blk - 1 : blk;                        // giving index among the blocks
+            const int xz = (s * np + (gi << BM::kShift) + pq) * 4;    // this warp's slots when giving
             const int xg = 32 + (2 * s + pq) * 4;                      // P = 2: the G_1 slots
             const bool g1_async = x_take && BM::P == 2 && !a.g1_from_g0;
             uint8_t* const xs = smem + OffData;
@@ -841,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                         *(uint4*)(xs + xoff(st, xz + 2 * cc + 1, lane)) =
                             make_uint4(h[cc][4], h[cc][5], h[cc][6], h[cc][7]);
                     }
-                    mbar_arrive(&xrow[(blk << BM::kShift) + pq]);
+                    mbar_arrive(&xrow[(gi << BM::kShift) + pq]);
                 }
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -919,7 +923,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     }
                     if (!ok) break;
                 } else if (x_take) {
-                    // P = 2: + X_0 G_1, once block 0's warp has handed X_0 over
+                    // P = 2: + X_0 G_1 (backward: + X_1 conj(G_1)), once the
+                    // other block's warp has handed its values over
                     if (!(ok = wait(&xrow[pq], iter & 1))) {
                         fail();
                         break;
@@ -932,7 +937,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                     }
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        const int z0 = (s * np + pq) * 4;              // block 0's warp of this pair
+                        const int z0 = (s * np + pq) * 4;              // the giving warp of this pair
                         const uint4 x0 = *(const uint4*)(xs + xoff(st, z0 + 2 * cc, lane));
                         const uint4 x1 = *(const uint4*)(xs + xoff(st, z0 + 2 * cc + 1, lane));
                         const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -950,6 +955,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             const uint4 g1 = *(const uint4*)(xs + xoff(st, xg + 2 * cc + 1, lane));
                             gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
                             gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
+                        }
+                        if constexpr (BWD) {
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) gw[2 * p + 1] ^= kNegPair;   // conj(G_1)
                         }
 #pragma unroll
                         for (int p = 0; p < 4; ++p)
@@ -1312,6 +1321,8 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = allow_smem<__half, kMonarch>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain, true>();
     if (e == cudaSuccess) e = allow_smem<__half, kPlain, true>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kTwo, true>();
+    if (e == cudaSuccess) e = allow_smem<__half, kTwo, true>();
     return e;
 }
 
@@ -1421,19 +1432,22 @@ cudaError_t tc_planar_forward_monarch(const Plan& p, const ForwardArgs& fa, uint
 // y2 = v2 * corr(u * w, k) (y2 may be NULL), i.e. the forward kernel with the
 // product by conj(K) and a second gated output.
 cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& fa, void* y2, const void* v2, cudaStream_t s) {
-    if (p.N > kN) return cudaErrorInvalidValue;
+    if (p.N > 2 * kN) return cudaErrorInvalidValue;
+    const bool two = p.N == 2 * kN;              // fa.Kf: the two-block rows G_0, G_1
     const Resources* r = (const Resources*)p.tcp;
     PArgs a{};
     a.u = fa.u; a.w = fa.w; a.v = fa.v; a.y = fa.y;
     a.y2 = y2; a.v2 = v2;
     a.K = (const uint32_t*)fa.Kf;
-    a.kstride = kM;
-    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * kKBytes);
+    a.kstride = two ? 2 * kM : kM;
+    a.Kscale = (const float*)((const uint8_t*)fa.Kf + (size_t)p.H * (two ? 2 : 1) * kKBytes);
+    a.g1_from_g0 = two && p.L <= kN;
+    a.ng = two ? 2 : 1;
     a.B = fa.B; a.H = p.H; a.N = p.N;
     a.nwin = 1;
     a.lseg = plan_lseg(p.N);
     a.pb = (fa.B + 1) / 2;
-    const int64_t pairs_per_tile = int64_t(64) >> a.lseg;
+    const int64_t pairs_per_tile = two ? 2 : int64_t(64) >> a.lseg;
     a.tpc = (a.pb + pairs_per_tile - 1) / pairs_per_tile;
     a.nunits = p.H * a.tpc;
     a.bimg = (const uint4*)r->bimg;
@@ -1441,8 +1455,13 @@ cudaError_t tc_planar_correlate(const Plan& p, const ForwardArgs& fa, void* y2, 
     a.tw8192 = r->tw8192;
     a.status = p.status;
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
-    if (p.dtype == kBF16) launch<__nv_bfloat16, kPlain, true>(a, grid, s);
-    else launch<__half, kPlain, true>(a, grid, s);
+    if (p.dtype == kBF16) {
+        if (two) launch<__nv_bfloat16, kTwo, true>(a, grid, s);
+        else launch<__nv_bfloat16, kPlain, true>(a, grid, s);
+    } else {
+        if (two) launch<__half, kTwo, true>(a, grid, s);
+        else launch<__half, kPlain, true>(a, grid, s);
+    }
     return cudaGetLastError();
 }
 

@@ -6,7 +6,7 @@ product by conj(K_f) and two gated outputs; the forward kernel with dy as the
 output gate) and are held to the fp16/bf16 tolerances; dk is computed on fp32
 lanes from the exactly representable inputs and summed over the batch in
 fp32, and is held to the fp32 tolerance.  Sizes include several tiles per CTA
-and packed short sequences."""
+packed short sequences and the two-block mode of N = 8192."""
 import numpy as np
 import pytest
 
@@ -46,6 +46,10 @@ def _run(u, k, dy, w, v, dtype):
     (5, 2, 1024, 1024, True, "bf16"),
     (4, 3, 256, 200, True, "f16"),
     (16, 256, 4096, 4096, True, "bf16"),      # 512 tiles: several per CTA
+    (3, 2, 8192, 8192, True, "bf16"),         # two blocks: block 0 takes block 1's spectrum
+    (2, 3, 8192, 3000, False, "f16"),         # k1 = 0: G_1 = (-1)^f G_0
+    (5, 2, 8192, 6000, True, "f16"),
+    (16, 112, 8192, 8192, True, "bf16"),      # 448 tiles
 ])
 def test_backward_matches_oracle_adjoints(B, H, N, L, gated, dtype):
     u, k, dy, w, v = _inputs(B, H, N, L, dtype, gated, seed=N + L + B)
