@@ -113,3 +113,13 @@ def test_backward_arguments():
                                         None, e.data_ptr(), None, None, dk.data_ptr(), None)
     torch.cuda.synchronize()
     assert rc == 0 and float(dk.abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("B,H,N,L", [(1, 1, 8192, 8192), (1, 2, 4096, 100)])
+def test_backward_single_row(B, H, N, L):
+    u, k, dy, w, v = _inputs(B, H, N, L, "bf16", True, seed=B + H + N + L)
+    got = _run(u, k, dy, w, v, "bf16")
+    ref = oracle.conv_backward(u, k, dy, w=w, v=v, route="fft")
+    for name in ("du", "dw", "dv"):
+        assert_close(got[name], ref[name], "bf16", f"{name} single row N={N}")
+    assert rel_l2(got["dk"], ref["dk"]) <= 1e-5

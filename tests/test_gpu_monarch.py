@@ -103,3 +103,11 @@ def test_monarch_unsupported_plans():
         with pytest.raises(lsf.FFTConvError) as e:
             plan.forward_monarch(u, Kf, 0xF000000F)
         assert e.value.status == lsf.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,H", [(1, 1), (3, 1), (2, 5)])
+def test_monarch_small_and_ragged(B, H):
+    N, keep = 4096, 0xF000000F
+    u, k, w, v = _inputs(B, H, N, "f16", gated=True, seed=B * 10 + H)
+    y, _, _ = _run(u, k, w, v, keep, "f16")
+    assert_close(y, oracle.fftconv_bins(u, k, W.monarch_binmask(keep, N), w=w, v=v), "f16", f"monarch B={B} H={H}")

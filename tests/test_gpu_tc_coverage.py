@@ -287,3 +287,26 @@ def test_fp16_range_guard(name, N, L, order, path, edge, beyond):
     assert status == lsf.ERR_RANGE, (name, status)
     assert again == lsf.OK
     assert not np.isfinite(y).all()
+
+
+# ------------------------------------------------ block-mode edge cases ---
+
+@pytest.mark.parametrize("N,B,H,L,dtype", [(8192, 1, 1, 8192, "bf16"),      # one unpaired row
+                                           (8192, 3, 1, 1, "f16"),          # L = 1, a ragged pair
+                                           (16384, 1, 2, 16384, "f16"),
+                                           (16384, 2, 1, 1, "bf16"),
+                                           (16384, 5, 3, 4097, "bf16")])    # G_2 = G_3 = 0 skipped
+def test_block_modes_small_and_ragged(N, B, H, L, dtype):
+    _compare(_inputs(B, H, N, L, dtype, gated=(B % 2 == 1), seed=N + B + L), dtype, f"blocks N={N} B={B} L={L}")
+
+
+def test_block_modes_empty_batch():
+    import torch
+    import long_sequence_fft_b200 as lsf
+    for N in (8192, 16384):
+        plan = lsf.Plan(N, 2, "bf16")
+        Kf = plan.precompute(torch.zeros((2, N), dtype=torch.bfloat16, device="cuda"))
+        u = torch.zeros((0, 2, N), dtype=torch.bfloat16, device="cuda")
+        y = plan.forward(u, Kf)
+        torch.cuda.synchronize()
+        assert y.shape == (0, 2, N) and plan.device_status() == 0
