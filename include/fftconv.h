@@ -72,22 +72,26 @@ typedef enum {
 /* Range of the 16-bit tensor-core paths (FFTCONV_PATH_TC_FUSED and
  * FFTCONV_PATH_TC_STAGED).  Their transform intermediates are fp16 (largest
  * finite value 65504); the fp32 paths (orders 1 and 4) keep fp32 throughout.
- *   - Fused kernel (N <= 4096, N = 8192 and 16384 as two and four blocks
- *     of 4096 or, N = 8192 with a block mask, split by bin parity,
- *     overlap-save windows): each unitary stage can grow a value by at most the number of
- *     its inputs over the square root of its length, so with max|u*w| <= 90
- *     no intermediate can overflow whatever the data and the filter.  Above
- *     that it depends on the data: a constant (DC) input overflows the forward
- *     transform near max|u*w| = 1450, zero-mean random data stays finite far
- *     beyond.
- *   - Staged tensor-core path (N >= 16384): no data-independent bound is
- *     useful; inputs with a large mean overflow near max|u*w| = 10^3 for
- *     R = 2N/8192 = 256 rows per column.
- * An overflow is never silent: the kernels that write y check every
- * convolution value (before the output gate v) and, if one is inf or NaN,
- * set the plan's status word to FFTCONV_ERR_RANGE, which
- * fftconv_device_status returns (and resets).  y then holds the non-finite
- * values; rerun such inputs with an fp32 plan (order 4) or rescale u. */
+ *   - Fused kernel (N <= 4096; N = 8192 and 16384 as two and four blocks
+ *     of 4096 or, N = 8192 with a block mask, split by bin parity;
+ *     overlap-save windows): each unitary stage can grow a value by at most
+ *     the number of its inputs over the square root of its length, so with
+ *     max|u*w| <= 90 no intermediate can overflow whatever the data and the
+ *     filter.  Above that it depends on the data: a constant (DC) input
+ *     overflows the forward transform near max|u*w| = 1450, zero-mean random
+ *     data stays finite far beyond.
+ *   - Staged tensor-core path (order 5 from N = 16384; N >= 32768 with
+ *     L > 2049): no data-independent bound is useful; inputs with a large
+ *     mean overflow near max|u*w| = 10^3 for R = 2N/8192 = 256 rows per
+ *     column.
+ * An overflow is never silent: the kernels that write y check the
+ * convolution values (before the output gate v; the fused tensor-core kernel
+ * checks at least, per pair of rows, the outputs at one position j1 of every
+ * residue (l, j3) of t = 256 j1 + 8 l + j3, which every fp16 overflow of its
+ * transform reaches) and, if one is inf or NaN, set the plan's status word
+ * to FFTCONV_ERR_RANGE, which fftconv_device_status returns (and resets).
+ * y then holds the non-finite values; rerun such inputs with an fp32 plan
+ * (order 4) or rescale u. */
 
 /* Kernel family a plan uses (fftconv_plan_path). */
 typedef enum {

@@ -1098,8 +1098,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                             float a1 = __uint_as_float(r[e][1][jj]) * kscale;
                             float b0 = __uint_as_float(r[e][0][2 + jj]) * kscale;
                             float b1 = __uint_as_float(r[e][1][2 + jj]) * kscale;
-                            nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
-                            nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
+                            // fp16 range (t = 256 j1 + 8 l + j3): a non-finite
+                            // value in a forward stage or the filter product
+                            // reaches every output of the transform, one after
+                            // S3' every output of its j3 and one after S2' every
+                            // j1 of its (l, j3), in the real or the imaginary
+                            // part.  So each warp checks both sequences at every
+                            // (l, j3) of its pair for one kept j1 (hf = jj = 0:
+                            // the first segment, valid whenever any is; in a
+                            // later window the warps s >= 2; the four-block
+                            // build measured faster checking every value)
+                            if (MODE == kFour || (hf == 0 && jj == 0)) {
+                                nonfinite_fold(nf, a0); nonfinite_fold(nf, a1);
+                                nonfinite_fold(nf, b0); nonfinite_fold(nf, b1);
+                            }
                             if (a.v) {
                                 const float2 g0 = IO<T>::unpack2(vaw[e]), g1 = IO<T>::unpack2(vbw[e]);
                                 a0 *= g0.x; a1 *= g0.y; b0 *= g1.x; b1 *= g1.y;

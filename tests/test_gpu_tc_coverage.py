@@ -289,6 +289,46 @@ def test_fp16_range_guard(name, N, L, order, path, edge, beyond):
     assert not np.isfinite(y).all()
 
 
+@pytest.mark.parametrize("name,N,T,amp", [("plain", 4096, 4093, 2.0e4),
+                                          ("packed1k", 1024, 1021, 4.0e4),
+                                          ("twoblock", 8192, 4093, 2.0e4)])
+def test_fp16_range_guard_inverse_stage(name, N, T, amp):
+    """An overflow that only an inverse stage meets, confined to one residue.
+
+    The fused kernel's 8192-point transform indexes time as t = 256 j1 + 8 l +
+    j3.  A linear chirp u of T samples and its matched filter k (u reversed,
+    amplitude 1) compress into one sample at t = T - 1, whose (l, j3) is
+    (31, 4) for both lengths here.  Per unit amplitude the largest forward
+    fp16 value is 2.45 (T = 4093) or 0.67 (T = 1021), the S2' output at that
+    (l, j3) 5.93 or 2.97, every other S2' value below 0.12: at `amp` the
+    forward stages stay below 49k and that one S2' value passes 65504.  Only
+    the outputs of that (l, j3) become non-finite (16 of the 4096 of a block,
+    none with j3 = 0), and the call must report FFTCONV_ERR_RANGE.  At a
+    quarter of `amp` nothing overflows and the result is the oracle's."""
+    import long_sequence_fft_b200 as lsf
+    B, H = 2, 1
+    t = np.arange(T)
+    chirp = np.cos(np.pi * t.astype(np.float64) ** 2 / (2 * T))
+    k = np.zeros((H, T), np.float32)
+    k[0] = chirp[::-1]
+    u = np.zeros((B, H, N), np.float32)
+    for scale, overflow in ((0.25, False), (1.0, True)):
+        u[0, 0, :T] = amp * scale * chirp
+        ub = W.round_to(u, "bf16")
+        kb = W.round_to(k, "bf16")
+        y, status, again, plan = _status_after(ub, kb, "bf16", 0, N, T)
+        assert plan.path_name == "tc_fused"
+        if not overflow:
+            assert status == lsf.OK and np.isfinite(y).all(), (name, status)
+            assert_close(y, oracle.fftconv(ub, kb), "bf16", f"{name}: matched chirp below the overflow")
+            continue
+        assert status == lsf.ERR_RANGE, (name, status)
+        assert again == lsf.OK
+        bad = np.nonzero(~np.isfinite(y))[-1]
+        assert bad.size > 0, name
+        assert np.all(bad % 256 == 8 * 31 + 4), (name, sorted(set((bad % 256).tolist())))
+
+
 # ------------------------------------------------ block-mode edge cases ---
 
 @pytest.mark.parametrize("N,B,H,L,dtype", [(8192, 1, 1, 8192, "bf16"),      # one unpaired row
