@@ -344,8 +344,11 @@ __device__ __forceinline__ int64_t unit_channel(const PArgs& a, int64_t u) {
 
 // BWD: the correlation of the backward pass -- the product with conj(K)
 // instead of K (the filter is real, so that is correlation with k) and the
-// second output y2.
-template <typename T, int MODE, bool BWD = false>
+// second output y2.  UNGATED: the forward build for calls without the input
+// gate w (no gate loads, normal L2 policy for u).  Against the gated build
+// given w = NULL it measured 6% faster on plain and packed sequences, 5% on
+// two blocks and 1-3% on four.
+template <typename T, int MODE, bool BWD = false, bool UNGATED = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a) {
     static_assert(!BWD || MODE == kPlain || MODE == kTwo, "the correlation pass runs on plain and two-block plans");
     extern __shared__ uint8_t smem_raw[];
@@ -597,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
         };
         auto load_issue = [&](int64_t lu, int part, LoadPart& lp) {
             const TileBase tb = tile_base<MODE>(a, lu);
-            const bool has_w = a.w != nullptr;
+            const bool has_w = !UNGATED && a.w != nullptr;
             const int P = 2 * s + part;
 #pragma unroll
             for (int jh = 0; jh < 2; ++jh) {
@@ -615,15 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fftconv_planar_kernel(PArgs a)
                 // (measured 1.3% faster on the flagship); overlap-save windows
                 // re-read half of each window and the four-block mode measured
                 // slower with it: normal policy there
-                const uint64_t pol = (MODE == kWin || MODE == kFour) ? l2_evict_normal() : l2_evict_first();
+                const uint64_t pol =
+                    (MODE == kWin || MODE == kFour || UNGATED) ? l2_evict_normal() : l2_evict_first();
                 lp.ld[jh][0] = ldg_nc_hint(pu0 + t0, pol);
-                lp.ld[jh][1] = ldg_nc_hint((has_w ? (const T*)a.w + LP.o0 : pu0) + t0, pol);
                 lp.ld[jh][2] = ldg_nc_hint(pu1 + t0, pol);
-                lp.ld[jh][3] = ldg_nc_hint((has_w ? (const T*)a.w + oo1 : pu1) + t0, pol);
+                if constexpr (UNGATED) {
+                    lp.ld[jh][1] = lp.ld[jh][3] = make_uint4(0u, 0u, 0u, 0u);
+                } else {
+                    lp.ld[jh][1] = ldg_nc_hint((has_w ? (const T*)a.w + LP.o0 : pu0) + t0, pol);
+                    lp.ld[jh][3] = ldg_nc_hint((has_w ? (const T*)a.w + oo1 : pu1) + t0, pol);
+                }
             }
         };
         auto load_finish = [&](int part, const LoadPart& lp) {
-            const bool has_w = a.w != nullptr;
+            const bool has_w = !UNGATED && a.w != nullptr;
             const int P = 2 * s + part;
             float xa[2][8], xb[2][8];
 #pragma unroll
@@ -1266,15 +1274,15 @@ cudaError_t upload_vec(V** dst, const std::vector<V>& v) {
     return e;
 }
 
-template <typename T, int MODE, bool BWD = false>
+template <typename T, int MODE, bool BWD = false, bool UNGATED = false>
 void launch(const PArgs& a, int64_t grid, cudaStream_t s) {
-    tc_fftconv_planar_kernel<T, MODE, BWD><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
+    tc_fftconv_planar_kernel<T, MODE, BWD, UNGATED><<<(unsigned)grid, kThreads, SmemBytes, s>>>(a);
 }
 
-template <typename T, int MODE, bool BWD = false>
+template <typename T, int MODE, bool BWD = false, bool UNGATED = false>
 cudaError_t allow_smem() {
-    return cudaFuncSetAttribute(tc_fftconv_planar_kernel<T, MODE, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SmemBytes);
+    return cudaFuncSetAttribute(tc_fftconv_planar_kernel<T, MODE, BWD, UNGATED>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, SmemBytes);
 }
 
 // K_f (PP layout) -> rfft bins [0, N] of each channel's 2N-point spectrum:
@@ -1335,6 +1343,12 @@ cudaError_t tc_planar_init(Plan& p) {
     if (e == cudaSuccess) e = allow_smem<__half, kPlain, true>();
     if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kTwo, true>();
     if (e == cudaSuccess) e = allow_smem<__half, kTwo, true>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kPlain, false, true>();
+    if (e == cudaSuccess) e = allow_smem<__half, kPlain, false, true>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kTwo, false, true>();
+    if (e == cudaSuccess) e = allow_smem<__half, kTwo, false, true>();
+    if (e == cudaSuccess) e = allow_smem<__nv_bfloat16, kFour, false, true>();
+    if (e == cudaSuccess) e = allow_smem<__half, kFour, false, true>();
     return e;
 }
 
@@ -1403,13 +1417,19 @@ cudaError_t tc_planar_forward(const Plan& p, const ForwardArgs& fa, int mode, cu
     const int64_t grid = a.nunits < r->num_sms ? a.nunits : r->num_sms;
     if (p.dtype == kBF16) {
         if (mode == kWin) launch<__nv_bfloat16, kWin>(a, grid, s);
+        else if (mode == kTwo && rows == 4 && !a.w) launch<__nv_bfloat16, kFour, false, true>(a, grid, s);
         else if (mode == kTwo && rows == 4) launch<__nv_bfloat16, kFour>(a, grid, s);
+        else if (mode == kTwo && !a.w) launch<__nv_bfloat16, kTwo, false, true>(a, grid, s);
         else if (mode == kTwo) launch<__nv_bfloat16, kTwo>(a, grid, s);
+        else if (!a.w) launch<__nv_bfloat16, kPlain, false, true>(a, grid, s);
         else launch<__nv_bfloat16, kPlain>(a, grid, s);
     } else {
         if (mode == kWin) launch<__half, kWin>(a, grid, s);
+        else if (mode == kTwo && rows == 4 && !a.w) launch<__half, kFour, false, true>(a, grid, s);
         else if (mode == kTwo && rows == 4) launch<__half, kFour>(a, grid, s);
+        else if (mode == kTwo && !a.w) launch<__half, kTwo, false, true>(a, grid, s);
         else if (mode == kTwo) launch<__half, kTwo>(a, grid, s);
+        else if (!a.w) launch<__half, kPlain, false, true>(a, grid, s);
         else launch<__half, kPlain>(a, grid, s);
     }
     return cudaGetLastError();

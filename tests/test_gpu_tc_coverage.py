@@ -125,6 +125,18 @@ def test_two_block_mode_three_tiles_per_cta(B, H, L, gated, dtype):
     _compare(_inputs(B, H, N, L, dtype, gated=gated, seed=L + B), dtype, f"two-block L={L} B={B} {tiles} tiles")
 
 
+@pytest.mark.parametrize("N,B,H,L,dtype", [(1024, 9, 40, 1024, "bf16"),
+                                           (4096, 5, 40, 4096, "f16"),
+                                           (8192, 7, 24, 3000, "bf16"),
+                                           (16384, 3, 16, 16384, "f16")])
+def test_output_gate_only(N, B, H, L, dtype):
+    """y = v * conv(u, k) with no input gate: calls without w run the
+    kernel's ungated build (no gate loads), with or without v."""
+    inp = _inputs(B, H, N, L, dtype, gated=True, seed=N + B)
+    inp["w"] = None
+    _compare(inp, dtype, f"v only N={N} B={B} L={L}")
+
+
 def test_split_mode_three_tiles_per_cta():
     B, H, N = 16, 128, 8192
     groups = H * ((B // 2 + 3) // 4)
