@@ -56,6 +56,16 @@ def algorithmic_bytes(w: W.Workload, path: str = "simt_fused") -> int:
     return w.elems * per_elem + w.H * bins * kf_bytes_per_bin(path)
 
 
+def backward_bytes(w: W.Workload, path: str) -> int:
+    """Compulsory HBM bytes of one backward call (fftconv_backward): read u,
+    dy (and w, v), write du (and dw, dv), read the filter spectrum once at
+    its stored width and write the fp32 filter gradient dk [H, L]."""
+    esz = 4 if w.dtype == "f32" else 2
+    per_elem = 3 * esz + (4 * esz if w.gated else 0)
+    bins = (w.L + 1) if w.L < w.N else (w.N + 1)
+    return w.elems * per_elem + w.H * bins * kf_bytes_per_bin(path) + w.H * w.L * 4
+
+
 def mma_flops_per_elem(w: W.Workload, path: str):
     """(schedule, flops per output element) of the tensor-core contractions the
     path issues, counted from the instruction shapes (complex values as real
@@ -267,6 +277,8 @@ def run_reference(args):
 
 # Workloads timed beside the headline (one GPU): every other configuration
 # of the hot path, each for at least about a second of steps.
+# backward passes timed beside the forward workloads (the workload's shape)
+BACKWARD_WORKLOADS = ("gated_bf16_n4k", "partial_bf16_n8k")
 SIDE_WORKLOADS = ("fp32_n1k", "fp16_n16k", "fp16_n32k", "dna_bf16_n1m", "partial_bf16_n8k", "sparse_bf16_n8k",
                   "monarch_bf16_n4k", "gated_bf16_n1k", "bf16_n1k", "dna_bf16_n4m_l1m")
 
@@ -336,6 +348,59 @@ def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: 
     return entry
 
 
+def time_backward(name: str, hbm_peak: float, tc_peak: float, min_seconds: float = 1.0):
+    """fftconv_backward on a workload's shape and seeded inputs (dy from its
+    own stream): du, dw, dv on the tensor cores (the forward kernel with dy as
+    output gate, then one correlation launch) and dk on fp32 lanes.  Timed
+    like the forward workloads: 3 warm-up calls, then about `min_seconds` of
+    calls into preallocated gradients, CUDA events on the launching stream."""
+    import torch
+    import long_sequence_fft_b200 as lsf
+    w = W.WORKLOADS[name]
+    inp = W.make_all(w)
+    dt = W.torch_dtype(w.dtype)
+    dev = lambda a: None if a is None else torch.from_numpy(a).to(dt).cuda()
+    u, k, g, v = dev(inp["u"]), dev(inp["k"]), dev(inp["w"]), dev(inp["v"])
+    dy = dev(W.make_grad_output(w))
+    del inp
+    plan = lsf.Plan(w.N, w.H, w.dtype, L=w.L)
+    Kf = plan.precompute(k)
+    out = plan.backward(u, Kf, dy, w=g, v=v)
+    bwd = lambda: plan.backward(u, Kf, dy, w=g, v=v, out=out)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        bwd()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    bwd()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    steps = int(min(20000, max(10, min_seconds / max(e0.elapsed_time(e1) * 1e-3, 1e-6))))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            bwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    path = plan.path_name
+    abytes = backward_bytes(w, path)
+    fpe = 2 * mma_flops_per_elem(w, path)[1]          # the dv forward and the du/dw correlation
+    t_hbm = abytes / (hbm_peak * 1e9)
+    t_mma = fpe * w.elems / (tc_peak * 1e12)
+    t = ms * 1e-3
+    entry = {"pass": "backward (du, dw, dv, dk)", "B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated,
+             "io_dtype": w.dtype, "path": path, "steps": steps, "ms_per_step": ms,
+             "value": w.elems / t, "unit": UNIT, "device_status": plan.device_status(), "clocks": clk.summary(),
+             "algorithmic_bytes": abytes, "achieved_gbs": abytes / t / 1e9, "hbm_frac": t_hbm / t,
+             "mma_flops_per_elem": fpe, "t_hbm_us": t_hbm * 1e6, "t_mma_us": t_mma * 1e6,
+             "frac": max(t_hbm, t_mma) / t, "bound": "hbm" if t_hbm >= t_mma else "tensor"}
+    del u, k, g, v, dy, out, Kf, plan
+    torch.cuda.empty_cache()
+    return entry
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -352,6 +417,8 @@ def main():
                     help="override the batch size (small cases for profiling; not a bench number)")
     ap.add_argument("--profile", action="store_true",
                     help="profiling run: skip the host-buffer, CPU-baseline and side-workload legs")
+    ap.add_argument("--backward", action="store_true",
+                    help="with --profile: run the backward pass (fftconv_backward) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -393,6 +460,29 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     precompute_ms = e0.elapsed_time(e1)
+
+    if args.backward:
+        # profiling run of the backward pass alone (the bench line times it in
+        # its workloads object)
+        if not args.profile:
+            raise SystemExit("--backward is a profiling run: add --profile")
+        dy = dev(W.make_grad_output(w))
+        grads = plan.backward(u, Kf, dy, w=g, v=v)
+        for _ in range(args.warmup):
+            plan.backward(u, Kf, dy, w=g, v=v, out=grads)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            plan.backward(u, Kf, dy, w=g, v=v, out=grads)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if plan.device_status() != 0:
+            raise SystemExit("device status after the backward passes")
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "pass": "backward", "workload": w.name, "B": w.B,
+                              "ms_per_step": e0.elapsed_time(e1) / args.steps, "path": plan.path_name}), flush=True)
+        mg.shutdown(ctx)
+        return 0
 
     y = torch.empty_like(u)
     if w.monarch_keep:
@@ -500,6 +590,8 @@ def main():
     if world == 1 and not args.no_workloads:
         line["workloads"] = {name: time_side_workload(name, hbm_peak, tc_peak) for name in SIDE_WORKLOADS
                              if name != w.name}
+        for name in BACKWARD_WORKLOADS:
+            line["workloads"]["backward_" + name] = time_backward(name, hbm_peak, tc_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, cores, sample = time_oracle(w)
         v_one, _, sample_one = time_oracle(w, target_s=8.0, cores=1, H=4)

@@ -237,19 +237,37 @@ class Plan:
                                             _ptr(v), int(keep_c2) & 0xffffffff, _stream_handle(stream)))
         return out
 
-    def backward(self, u, Kf, dy, w=None, v=None, want_dk=True, stream=None):
+    def backward(self, u, Kf, dy, w=None, v=None, want_dk=True, stream=None, out=None):
         """Gradients of y = v * conv(u * w, k) for dy: dict(du, dw, dv, dk) with
         dw only when w is given, dv only when v is given, dk an fp32 [H, L]
-        tensor (summed over the batch) when want_dk."""
+        tensor (summed over the batch) when want_dk.  `out`: an earlier
+        call's dict to write into instead of allocating."""
         import torch
         B = u.shape[0]
         shape = (B, self.H, self.N)
         for t, name in ((u, "u"), (w, "w"), (v, "v"), (dy, "dy")):
             self._check_tensor(t, shape, name)
+        if out is not None:
+            du, dw, dv, dk = out.get("du"), out.get("dw"), out.get("dv"), out.get("dk")
+            for t, name, need in ((du, "du", True), (dw, "dw", w is not None), (dv, "dv", v is not None)):
+                if need and t is None:
+                    raise ValueError(f"out[{name!r}] is missing")
+                if not need and t is not None:
+                    raise ValueError(f"out[{name!r}] given without its gate")
+                self._check_tensor(t, shape, name)
+            if want_dk and (dk is None or dk.dtype != torch.float32 or tuple(dk.shape) != (self.H, self.L)
+                            or not dk.is_contiguous()):
+                raise ValueError("out['dk'] must be a contiguous float32 [H, L] tensor")
+            if not want_dk:
+                dk = None
+            return self._backward_into(u, Kf, dy, w, v, du, dw, dv, dk, B, stream)
         du = torch.empty(shape, dtype=self.dtype, device=u.device)
         dw = torch.empty_like(du) if w is not None else None
         dv = torch.empty_like(du) if v is not None else None
         dk = torch.empty((self.H, self.L), dtype=torch.float32, device=u.device) if want_dk else None
+        return self._backward_into(u, Kf, dy, w, v, du, dw, dv, dk, B, stream)
+
+    def _backward_into(self, u, Kf, dy, w, v, du, dw, dv, dk, B, stream):
         _check(_lib.fftconv_backward(self._h, _ptr(u), _ptr(Kf), _ptr(dy), B, self.H, self.N, _ptr(w), _ptr(v),
                                      _ptr(du), _ptr(dw), _ptr(dv), _ptr(dk), _stream_handle(stream)))
         return {"du": du, "dw": dw, "dv": dv, "dk": dk}

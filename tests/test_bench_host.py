@@ -113,3 +113,18 @@ def test_monarch_flop_count_and_kept_bins():
     assert abs(W.monarch_kept_fraction(w) - 0.25) < 0.01
     assert W.make_mask(w) is None                                  # no block mask besides it
     assert np.all(W.monarch_binmask(0xFFFFFFFF, 1024) == 1)
+
+
+def test_backward_bytes_and_grad_output_stream():
+    # gated bf16 flagship shape: u, dy, w, v read and du, dw, dv written
+    # (7 x 2 B per element), K_f read once at 4 B per bin, dk written in fp32
+    w = W.WORKLOADS["gated_bf16_n4k"]
+    assert bench.backward_bytes(w, "tc_fused") == w.elems * 14 + w.H * (w.N + 1) * 4 + w.H * w.L * 4
+    p = W.WORKLOADS["partial_bf16_n8k"]
+    assert bench.backward_bytes(p, "tc_fused") == p.elems * 14 + p.H * (p.L + 1) * 4 + p.H * p.L * 4
+    small = W.Workload("t", index=99, B=2, H=3, N=64, L=64, dtype="bf16", gated=True, k_kind="scaled")
+    dy = W.make_grad_output(small)
+    assert dy.shape == (2, 3, 64) and np.array_equal(dy, W.make_grad_output(small))
+    assert not np.array_equal(dy, W.make_input(small))                     # its own stream
+    assert np.array_equal(dy, W.round_to(dy, "bf16"))
+    assert set(bench.BACKWARD_WORKLOADS) <= set(W.WORKLOADS)

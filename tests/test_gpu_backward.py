@@ -123,3 +123,30 @@ def test_backward_single_row(B, H, N, L):
     for name in ("du", "dw", "dv"):
         assert_close(got[name], ref[name], "bf16", f"{name} single row N={N}")
     assert rel_l2(got["dk"], ref["dk"]) <= 1e-5
+
+
+def test_backward_into_preallocated_gradients():
+    """Plan.backward(out=...) writes into an earlier call's tensors: du, dw, dv
+    bit for bit as the allocating call (dk up to the order of its atomic fp32
+    sums over CTAs); a missing or extra gradient tensor is rejected."""
+    import torch
+    import long_sequence_fft_b200 as lsf
+    B, H, N, L, dtype = 4, 3, 4096, 4096, "bf16"
+    u, k, dy, w, v = _inputs(B, H, N, L, dtype, True, seed=21)
+    plan = lsf.Plan(N, H, dtype, L=L)
+    Kf = plan.precompute(to_dev(k, dtype))
+    ud, dyd, wd, vd = (to_dev(a, dtype) for a in (u, dy, w, v))
+    first = plan.backward(ud, Kf, dyd, w=wd, v=vd)
+    out = {n: torch.full_like(t, float("nan")) for n, t in first.items()}
+    second = plan.backward(ud, Kf, dyd, w=wd, v=vd, out=out)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    for n in ("du", "dw", "dv", "dk"):
+        assert second[n] is out[n]
+    for n in ("du", "dw", "dv"):
+        assert torch.equal(first[n], out[n]), n
+    assert rel_l2(out["dk"].cpu().numpy().astype(np.float64), first["dk"].cpu().numpy().astype(np.float64)) <= 1e-6
+    with pytest.raises(ValueError):
+        plan.backward(ud, Kf, dyd, w=wd, v=vd, out=dict(out, dw=None))
+    with pytest.raises(ValueError):
+        plan.backward(ud, Kf, dyd, v=vd, out=out)                       # dw given without w

@@ -24,7 +24,7 @@ from typing import Optional
 
 import numpy as np
 
-TENSOR_IDS = {"u": 1, "w": 2, "v": 3, "k": 4, "mask": 5, "proj": 6, "sym": 7}
+TENSOR_IDS = {"u": 1, "w": 2, "v": 3, "k": 4, "mask": 5, "proj": 6, "sym": 7, "dy": 8}
 MASK_BLOCK = 32
 
 
@@ -218,6 +218,12 @@ def make_mask(w: Workload) -> Optional[np.ndarray]:
     m = np.ones((1, nblk), dtype=np.uint8)
     m[0, perm[:nzero]] = 0
     return m
+
+
+def make_grad_output(w: Workload) -> np.ndarray:
+    """The incoming gradient dy [B, H, N] of a backward call: standard
+    normal, rounded to the workload's dtype, from its own seeded stream."""
+    return round_to(_normal(_rng(w, "dy"), (w.B, w.H, w.N)), w.dtype)
 
 
 def make_all(w: Workload):
