@@ -297,6 +297,38 @@ def roofline_entry(w: W.Workload, path: str, ms_per_step: float, hbm_peak: float
             "frac": max(t_hbm, t_mma) / t, "bound": "hbm" if t_hbm >= t_mma else "tensor"}
 
 
+def time_in_graph(call, stream, calls: int = 100, replays: int = 50):
+    """Per-call device time of `call` replayed from a CUDA graph of `calls`
+    captured calls (after one warm-up replay); {"error": ...} when capture
+    fails, so the eager number stands alone."""
+    import torch
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            call()                              # warm-up on the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(calls):
+                call()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / (calls * replays)
+        del graph
+        return {"ms_per_call": ms, "calls_per_graph": calls, "replays": replays}
+    except Exception as exc:                    # capture is an extra view, never fatal
+        torch.cuda.synchronize()
+        return {"error": f"{type(exc).__name__}: {exc}"[:200]}
+
+
 def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: float = 1.0):
     """One configuration end to end on the device: seeded inputs copied to HBM,
     plan, filter precompute, 3 warm-up calls, then enough calls for about
@@ -335,6 +367,9 @@ def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: 
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
+    graph = None
+    if ms < 0.05:
+        graph = time_in_graph(fwd, stream)
     status = plan.device_status()
     entry = {"B": w.B, "H": w.H, "N": w.N, "L": w.L, "gated": w.gated, "io_dtype": w.dtype,
              "sparsity": (1.0 - W.monarch_kept_fraction(w)) if w.monarch_keep else w.sparsity,
@@ -343,6 +378,13 @@ def time_side_workload(name: str, hbm_peak: float, tc_peak: float, min_seconds: 
              "value": w.elems / (ms * 1e-3), "unit": UNIT, "device_status": status,
              "clocks": clk.summary()}
     entry.update(roofline_entry(w, plan.path_name, ms, hbm_peak, tc_peak))
+    if graph is not None:
+        # launch-bound calls: the same calls replayed from a CUDA graph, which
+        # removes the per-call host work (argument checks, ctypes, launch)
+        if "ms_per_call" in graph:
+            graph["value"] = w.elems / (graph["ms_per_call"] * 1e-3)
+            graph["unit"] = UNIT
+        entry["graph"] = graph
     del u, k, g, v, y, Kf, plan
     torch.cuda.empty_cache()
     return entry
