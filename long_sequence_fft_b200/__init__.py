@@ -296,9 +296,69 @@ class Plan:
         return int(_lib.fftconv_device_status(self._h, _stream_handle(stream)))
 
 
+_PLAN_CACHE = {}
+
+
+def cached_plan(N: int, H: int, dtype, L: int, order: int = 0) -> "Plan":
+    """A plan per (device, N, H, dtype, L, order), created on first use and
+    kept for the process (plans own device tables; creating one per call
+    would repeat their uploads)."""
+    import torch
+    key = (torch.cuda.current_device(), int(N), int(H), str(dtype), int(L), int(order))
+    plan = _PLAN_CACHE.get(key)
+    if plan is None:
+        plan = _PLAN_CACHE[key] = Plan(N, H, dtype, order=order, L=L)
+    return plan
+
+
+_AUTOGRAD_FN = None
+
+
+def _autograd_function():
+    """torch.autograd.Function over fftconv_forward / fftconv_backward, built
+    on first use so that importing the package does not import torch."""
+    global _AUTOGRAD_FN
+    if _AUTOGRAD_FN is not None:
+        return _AUTOGRAD_FN
+    import torch
+
+    class FFTConvFunction(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, u, k, w, v, plan):
+            Kf = plan.precompute(k)
+            ctx.plan = plan
+            ctx.k_dtype = k.dtype
+            ctx.save_for_backward(u, w, v, Kf)
+            return plan.forward(u, Kf, w=w, v=v)
+
+        @staticmethod
+        def backward(ctx, dy):
+            u, w, v, Kf = ctx.saved_tensors
+            need_u, need_k, need_w, need_v = ctx.needs_input_grad[:4]
+            g = ctx.plan.backward(u, Kf, dy.contiguous(), w=w, v=v, want_dk=need_k)
+            dk = g["dk"].to(ctx.k_dtype) if need_k else None
+            return (g["du"] if need_u else None, dk, g["dw"] if need_w else None,
+                    g["dv"] if need_v else None, None)
+
+    _AUTOGRAD_FN = FFTConvFunction
+    return _AUTOGRAD_FN
+
+
 def fftconv(u, k, w=None, v=None, mask=None, order: int = 0):
-    """One-shot convenience: plan, filter transform and forward pass."""
+    """One-shot convenience: y = v * conv(u * w, k) through a cached plan.
+
+    Differentiable when autograd is on and an input requires grad: the
+    backward pass runs fftconv_backward (fp16/bf16 tensor-core plans with
+    N <= 8192; other plans raise FFTConvError from the backward pass) and
+    returns du, dk (cast to k's dtype), dw, dv.  Block masks are forward
+    only."""
+    import torch
     H, L = k.shape
-    plan = Plan(u.shape[2], H, u.dtype, order=order, L=L)
+    plan = cached_plan(u.shape[2], H, u.dtype, L, order)
+    needs_grad = torch.is_grad_enabled() and any(t is not None and t.requires_grad for t in (u, k, w, v))
+    if needs_grad:
+        if mask is not None:
+            raise NotImplementedError("fftconv: the backward pass takes no block mask")
+        return _autograd_function().apply(u, k, w, v, plan)
     Kf = plan.precompute(k)
     return plan.forward(u, Kf, w=w, v=v, mask=mask)

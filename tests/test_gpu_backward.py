@@ -150,3 +150,29 @@ def test_backward_into_preallocated_gradients():
         plan.backward(ud, Kf, dyd, w=wd, v=vd, out=dict(out, dw=None))
     with pytest.raises(ValueError):
         plan.backward(ud, Kf, dyd, v=vd, out=out)                       # dw given without w
+
+
+def test_autograd_through_fftconv():
+    """lsf.fftconv under autograd: backward of y with incoming gradient dy
+    gives the oracle's adjoints for u, w, v and k (dk in k's dtype, so held to
+    the 16-bit tolerance); the forward value equals the call without grad; a
+    block mask with grad is refused."""
+    import torch
+    import long_sequence_fft_b200 as lsf
+    B, H, N, L, dtype = 3, 2, 4096, 4096, "bf16"
+    u, k, dy, w, v = _inputs(B, H, N, L, dtype, True, seed=31)
+    dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda().requires_grad_()
+    ut, kt, wt, vt = dev(u), dev(k), dev(w), dev(v)
+    y = lsf.fftconv(ut, kt, w=wt, v=vt)
+    y.backward(torch.from_numpy(dy).to(torch.bfloat16).cuda())
+    ref = oracle.conv_backward(u, k, dy, w=w, v=v, route="fft")
+    host = lambda t: t.float().cpu().numpy().astype(np.float64)
+    for name, t in (("du", ut), ("dw", wt), ("dv", vt), ("dk", kt)):
+        assert t.grad is not None and t.grad.dtype == torch.bfloat16, name
+        assert_close(host(t.grad), ref[name], dtype, f"autograd {name}")
+    with torch.no_grad():
+        y2 = lsf.fftconv(ut, kt, w=wt, v=vt)
+    assert torch.equal(y.detach(), y2)
+    mask = torch.ones((1, N // 32), dtype=torch.uint8, device="cuda")
+    with pytest.raises(NotImplementedError):
+        lsf.fftconv(ut, kt, w=wt, v=vt, mask=mask)
