@@ -78,3 +78,66 @@ def test_two_for_one_packing():
     ref = oracle.fftconv(u, k)
     np.testing.assert_allclose(z.real, ref[0, 0], rtol=0, atol=1e-10)
     np.testing.assert_allclose(z.imag, ref[1, 0], rtol=0, atol=1e-10)
+
+
+def _stage_values(x, K):
+    """The intermediate values of the fused kernel's 8192-point pipeline,
+    written from the three-digit split (t = 256 j1 + 8 l + j3, f = c1 + 32 c2 +
+    1024 c3, unitary factors 1/sqrt(32), 1/sqrt(32), 1/sqrt(8)): forward S1
+    (over j1, then the twiddle w8192^(c1 (8 l + j3))), S2 (over l), S3 (over j3
+    with w256^(c2 j3)), the filter product, then S3' (over c3), S2' (over c2,
+    then the conjugate twiddle) and S1' (over c1).  Returns the stages that
+    are stored as fp16 in the kernel and the output."""
+    r32, r8 = 1 / np.sqrt(32), 1 / np.sqrt(8)
+    a32 = np.arange(32)
+    a8 = np.arange(8)
+    W32 = _w(32, np.outer(a32, a32))
+    tw = _w(8192, a32[:, None, None] * (8 * a32[None, :, None] + a8[None, None, :]))    # [c1, l, j3]
+    G = _w(8, np.outer(a8, a8))[None] * _w(256, a32[:, None, None] * a8[None, None, :])  # [c2, c3, j3]
+    A1 = r32 * np.einsum("cj,jlk->clk", W32, x.reshape(32, 32, 8)) * tw
+    A2 = r32 * np.einsum("dl,clk->cdk", W32, A1)
+    X = r8 * np.einsum("dek,cdk->cde", G, A2)
+    Y = X * K.reshape(8, 32, 32).transpose(2, 1, 0)
+    P = r8 * np.einsum("dek,cde->cdk", np.conj(G), Y)
+    Q = r32 * np.einsum("dl,cdk->clk", np.conj(W32), P) * np.conj(tw)
+    z = r32 * np.einsum("cj,clk->jlk", np.conj(W32), Q).reshape(-1)
+    return {"forward": (A1, A2, X, Y), "P": P, "Q": Q, "z": z}
+
+
+def test_stage_model_is_the_circular_convolution():
+    rng = np.random.default_rng(5)
+    u, k = rng.standard_normal(8192), rng.standard_normal(8192)
+    K = np.fft.fft(k)
+    z = _stage_values(u.astype(complex), K)["z"]
+    np.testing.assert_allclose(z, np.fft.ifft(np.fft.fft(u) * K), rtol=0, atol=1e-9 * np.abs(z).max())
+
+
+@pytest.mark.parametrize("T", [4093, 1021])
+def test_matched_chirp_overflows_only_one_inverse_residue(T):
+    """The input of the GPU test of an inverse-stage fp16 overflow: a linear
+    chirp of T samples and its reversal as the filter (the kernel stores the
+    filter spectrum over s_h = max |Re|, |Im|).  Per unit amplitude the
+    largest forward value is 2.45 (T = 4093) or 0.67 (T = 1021), the S3' values
+    stay near those, and the S2' output reaches 5.93 or 2.97 at one residue
+    (l, j3) = (31, 4) while every other (l, j3) stays below 0.12: scaled by
+    2e4 (4e4 for T = 1021) only that S2' value passes fp16's 65504."""
+    t = np.arange(T)
+    chirp = np.cos(np.pi * t.astype(np.float64) ** 2 / (2 * T))
+    u = np.zeros(8192)
+    u[:T] = chirp
+    k = np.zeros(8192)
+    k[:T] = chirp[::-1]
+    K = np.fft.fft(k)
+    K = K / max(np.abs(K.real).max(), np.abs(K.imag).max())
+    S = _stage_values(u.astype(complex), K)
+    comp = lambda a: np.maximum(np.abs(a.real), np.abs(a.imag))
+    fwd = max(comp(a).max() for a in S["forward"])
+    q = comp(S["Q"]).max(axis=0)                    # [l, j3]
+    amp = 2.0e4 if T == 4093 else 4.0e4
+    assert fwd * amp < 0.8 * 65504
+    assert comp(S["P"]).max() * amp < 0.5 * 65504
+    assert q[31, 4] * amp > 1.5 * 65504
+    others = q.copy()
+    others[31, 4] = 0
+    assert others.max() * amp < 0.1 * 65504
+    assert (T - 1) % 256 == 8 * 31 + 4                # the compressed sample's (l, j3)
