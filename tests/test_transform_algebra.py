@@ -141,3 +141,33 @@ def test_matched_chirp_overflows_only_one_inverse_residue(T):
     others[31, 4] = 0
     assert others.max() * amp < 0.1 * 65504
     assert (T - 1) % 256 == 8 * 31 + 4                # the compressed sample's (l, j3)
+
+
+def test_masked_8192_in_blocks_of_4096():
+    """A masked N = 8192 call in blocks of 4096: with k_M = IFFT_16384(K M) and
+    G'_d the 8192-point spectrum of k_M's taps at lags 4096 d + m, m in
+    (-4096, 4096) (m < 0 stored at 8192 + m), y_0 = IFFT(X_0 G'_0 + X_1 G'_-1)
+    and y_1 = IFFT(X_1 G'_0 + X_0 G'_1) (first 4096 outputs each) equal
+    IFFT_16384(X K M)[:8192] for any Hermitian mask M."""
+    rng = np.random.default_rng(8)
+    N, M = 8192, 16384
+    x, k = rng.standard_normal(N), rng.standard_normal(N)
+    K = np.fft.fft(k, M)
+    mask = (rng.random(M // 32) > 0.75).repeat(32).astype(float)
+    mask = np.maximum(mask, mask[(-np.arange(M)) % M])
+    y = np.fft.ifft(np.fft.fft(x, M) * K * mask)[:N]
+    kM = np.fft.ifft(K * mask)
+    m = np.arange(4096)
+    mn = np.arange(4097, 8192)
+
+    def G(d):
+        g = np.zeros(8192, dtype=complex)
+        g[m] = kM[(4096 * d + m) % M]
+        g[mn] = kM[(4096 * d + mn - 8192) % M]
+        return np.fft.fft(g)
+
+    X0 = np.fft.fft(x[:4096], 8192)
+    X1 = np.fft.fft(x[4096:], 8192)
+    y0 = np.fft.ifft(X0 * G(0) + X1 * G(-1))[:4096]
+    y1 = np.fft.ifft(X1 * G(0) + X0 * G(1))[:4096]
+    np.testing.assert_allclose(np.r_[y0, y1], y, rtol=0, atol=1e-9 * np.abs(y).max())
