@@ -354,11 +354,11 @@ def fftconv(u, k, w=None, v=None, mask=None, order: int = 0):
     only."""
     import torch
     H, L = k.shape
-    plan = cached_plan(u.shape[2], H, u.dtype, L, order)
     needs_grad = torch.is_grad_enabled() and any(t is not None and t.requires_grad for t in (u, k, w, v))
+    if needs_grad and mask is not None:
+        raise NotImplementedError("fftconv: the backward pass takes no block mask")
+    plan = cached_plan(u.shape[2], H, u.dtype, L, order)
     if needs_grad:
-        if mask is not None:
-            raise NotImplementedError("fftconv: the backward pass takes no block mask")
         return _autograd_function().apply(u, k, w, v, plan)
     Kf = plan.precompute(k)
     return plan.forward(u, Kf, w=w, v=v, mask=mask)

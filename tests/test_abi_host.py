@@ -66,3 +66,14 @@ def test_plan_create_rejects_bad_arguments(N, H, dtype, order, L, status):
     assert rc == status
     assert not h.value
     assert lsf.library().fftconv_last_error()
+
+
+def test_fftconv_refuses_a_mask_with_grad_before_any_device_work():
+    # the backward pass takes no block mask: the refusal comes first, so it
+    # holds on tensors that never reach a plan
+    import torch
+    import long_sequence_fft_b200 as lsf
+    u = torch.zeros((2, 3, 256), requires_grad=True)
+    k = torch.zeros((3, 256))
+    with pytest.raises(NotImplementedError):
+        lsf.fftconv(u, k, mask=torch.ones((1, 8), dtype=torch.uint8))
